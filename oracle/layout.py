@@ -1,0 +1,229 @@
+"""The packed, paged cache format, written out independently of the library (oracle).
+
+The pages fix what is stored per token - b-bit centroid indices, a 16-bit norm,
+for keys m QJL sign bits and ||r|| ("TurboQuant explained", section "QJL: Inner
+Product Recovery from a Single Sign Bit": m sign bits plus 16 bits for the norm,
+no scale or zero point) - and that serving uses a packed paged cache with a page
+table ("TurboQuant" limits page, section "Operational Assumptions": vLLM-style
+packed paged decode).  How the bits are laid out is left open; this module
+states the layout the library documents in include/tq.h, reading it from the
+format description only.
+
+Format (d = 128, m = 128, P tokens per page, one block per (layer, physical
+page, kv head); the cache is [layer][physical page][kv head][block]):
+
+  region  content                               bytes
+  KN      stored ||k|| as fp16, one per token    2P
+  KR      stored ||r|| as fp16 (keys with QJL)   2P
+  VN      stored ||v|| as fp16                   2P
+  KC      key codes, b_k*d/8 bytes per token     b_k*16*P
+  KS      QJL sign bits, m/8 bytes per token     16*P   (keys with QJL)
+  VC      value codes, b_v*d/8 bytes per token   b_v*16*P
+
+Each code region is a sequence of 16-byte chunks per token, stored chunk-major:
+chunk c of token t sits at byte (c*P + t)*16 of the region.  Token t's chunks,
+concatenated, form its bit string; bit k of the bit string is bit (k mod 8) of
+byte k/8 (little endian).
+
+Stored code of a centroid index idx in [0, 2^b) ("sign-magnitude"): with
+h = 2^(b-1), the sign bit s = [idx >= h] and the rank r = idx - h if s else
+h - 1 - idx (0 = the centroid nearest zero).  Because the codebook is symmetric,
+c[idx] = (+1 if s else -1) * c[h + r].  Fields of coordinate j in the bit string:
+  b = 1:  bit j = s
+  b = 2:  bits 2j, 2j+1 = r, s
+  b = 3:  bits 2j, 2j+1 = r (2-bit rank), bit 2d + j = s
+  b = 4:  bits 4j..4j+2 = r (3-bit rank), bit 4j+3 = s
+QJL signs: bit i of the sign bit string = sigma_i = [(S r)_i >= 0].
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+
+@dataclasses.dataclass
+class Format:
+    head_dim: int = 128
+    key_bits: int = 3
+    key_qjl: bool = True
+    qjl_m: int = 128
+    value_bits: int = 3
+    page_tokens: int = 256
+
+    def regions(self) -> dict:
+        P, d, m = self.page_tokens, self.head_dim, self.qjl_m
+        sizes = [("KN", 2 * P), ("KR", 2 * P if self.key_qjl else 0), ("VN", 2 * P),
+                 ("KC", self.key_bits * d // 8 * P), ("KS", m // 8 * P if self.key_qjl else 0),
+                 ("VC", self.value_bits * d // 8 * P)]
+        out, off = {}, 0
+        for name, sz in sizes:
+            out[name] = (off, sz)
+            off += sz
+        out["total"] = (0, off)
+        return out
+
+    @property
+    def block_bytes(self) -> int:
+        return self.regions()["total"][1]
+
+
+def stored_code(idx, bits: int):
+    idx = np.asarray(idx, dtype=np.int64)
+    h = 1 << (bits - 1)
+    s = (idx >= h).astype(np.int64)
+    r = np.where(s == 1, idx - h, h - 1 - idx)
+    return s, r
+
+
+def index_from_code(s, r, bits: int):
+    h = 1 << (bits - 1)
+    s = np.asarray(s, dtype=np.int64)
+    r = np.asarray(r, dtype=np.int64)
+    return np.where(s == 1, h + r, h - 1 - r)
+
+
+def code_bits(idx, bits: int) -> np.ndarray:
+    """[N, d] indices -> [N, bits*d] uint8 bit strings."""
+    idx = np.asarray(idx, dtype=np.int64)
+    n, d = idx.shape
+    s, r = stored_code(idx, bits)
+    out = np.zeros((n, bits * d), dtype=np.uint8)
+    j = np.arange(d)
+    if bits == 1:
+        out[:, j] = s
+    elif bits == 2:
+        out[:, 2 * j] = r & 1
+        out[:, 2 * j + 1] = s
+    elif bits == 3:
+        out[:, 2 * j] = r & 1
+        out[:, 2 * j + 1] = (r >> 1) & 1
+        out[:, 2 * d + j] = s
+    elif bits == 4:
+        out[:, 4 * j] = r & 1
+        out[:, 4 * j + 1] = (r >> 1) & 1
+        out[:, 4 * j + 2] = (r >> 2) & 1
+        out[:, 4 * j + 3] = s
+    else:
+        raise ValueError("bits must be 1..4")
+    return out
+
+
+def index_from_bits(bitstr, bits: int, d: int) -> np.ndarray:
+    """[N, bits*d] bit strings -> [N, d] indices."""
+    b = np.asarray(bitstr, dtype=np.int64)
+    j = np.arange(d)
+    if bits == 1:
+        s, r = b[:, j], np.zeros_like(b[:, j])
+    elif bits == 2:
+        r, s = b[:, 2 * j], b[:, 2 * j + 1]
+    elif bits == 3:
+        r = b[:, 2 * j] | (b[:, 2 * j + 1] << 1)
+        s = b[:, 2 * d + j]
+    elif bits == 4:
+        r = b[:, 4 * j] | (b[:, 4 * j + 1] << 1) | (b[:, 4 * j + 2] << 2)
+        s = b[:, 4 * j + 3]
+    else:
+        raise ValueError("bits must be 1..4")
+    return index_from_code(s, r, bits)
+
+
+def bits_to_bytes(bitstr) -> np.ndarray:
+    return np.packbits(np.asarray(bitstr, dtype=np.uint8), axis=-1, bitorder="little")
+
+
+def bytes_to_bits(by) -> np.ndarray:
+    return np.unpackbits(np.asarray(by, dtype=np.uint8), axis=-1, bitorder="little")
+
+
+def _put_chunked(region: np.ndarray, tok_bytes: np.ndarray, t0: int, P: int):
+    """Write [n, nbytes] per-token byte strings into a chunk-major region for tokens t0.."""
+    n, nb = tok_bytes.shape
+    nch = nb // 16
+    view = region.reshape(nch, P, 16)
+    view[:, t0:t0 + n, :] = tok_bytes.reshape(n, nch, 16).transpose(1, 0, 2)
+
+
+def _get_chunked(region: np.ndarray, n: int, nb: int, P: int) -> np.ndarray:
+    nch = nb // 16
+    return region.reshape(nch, P, 16)[:, :n, :].transpose(1, 0, 2).reshape(n, nb)
+
+
+def fp16_bytes(values) -> np.ndarray:
+    return np.asarray(values, dtype=np.float64).astype(np.float16).view(np.uint8)
+
+
+def empty_cache(fmt: Format, num_pages: int, kv_heads: int, num_layers: int = 1) -> np.ndarray:
+    return np.zeros((num_layers, num_pages, kv_heads, fmt.block_bytes), dtype=np.uint8)
+
+
+def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_of_seq,
+                   kcomp, vcomp):
+    """Write one (sequence, kv head): kcomp/vcomp hold idx, norm (and rnorm, sigma for keys)
+    for its tokens 0..n-1; pages_of_seq lists the physical pages in logical order."""
+    P, d = fmt.page_tokens, fmt.head_dim
+    reg = fmt.regions()
+    n = kcomp.idx.shape[0]
+    kbytes = bits_to_bytes(code_bits(kcomp.idx, fmt.key_bits))
+    vbytes = bits_to_bytes(code_bits(vcomp.idx, fmt.value_bits))
+    sbytes = bits_to_bytes(kcomp.sigma.astype(np.uint8)) if fmt.key_qjl else None
+    for lp in range((n + P - 1) // P):
+        t0, t1 = lp * P, min(n, (lp + 1) * P)
+        blk = cache[layer, pages_of_seq[lp], head]
+
+        def region(name):
+            o, sz = reg[name]
+            return blk[o:o + sz]
+
+        region("KN")[2 * 0:2 * (t1 - t0)] = fp16_bytes(kcomp.norm[t0:t1])
+        region("VN")[0:2 * (t1 - t0)] = fp16_bytes(vcomp.norm[t0:t1])
+        if fmt.key_qjl:
+            region("KR")[0:2 * (t1 - t0)] = fp16_bytes(kcomp.rnorm[t0:t1])
+            _put_chunked(region("KS"), sbytes[t0:t1], 0, P)
+        _put_chunked(region("KC"), kbytes[t0:t1], 0, P)
+        _put_chunked(region("VC"), vbytes[t0:t1], 0, P)
+
+
+@dataclasses.dataclass
+class Unpacked:
+    k_idx: np.ndarray
+    k_norm: np.ndarray
+    v_idx: np.ndarray
+    v_norm: np.ndarray
+    k_rnorm: np.ndarray = None
+    k_sigma: np.ndarray = None
+
+
+def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_of_seq,
+                  n: int) -> Unpacked:
+    """Read tokens 0..n-1 of one (sequence, kv head) back into indices, norms and signs."""
+    P, d, m = fmt.page_tokens, fmt.head_dim, fmt.qjl_m
+    reg = fmt.regions()
+    kb, vb = fmt.key_bits * d // 8, fmt.value_bits * d // 8
+    parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc")}
+    for lp in range((n + P - 1) // P):
+        cnt = min(n, (lp + 1) * P) - lp * P
+        blk = cache[layer, pages_of_seq[lp], head]
+
+        def region(name):
+            o, sz = reg[name]
+            return blk[o:o + sz]
+
+        parts["kn"].append(region("KN")[:2 * cnt].view(np.float16).astype(np.float64))
+        parts["vn"].append(region("VN")[:2 * cnt].view(np.float16).astype(np.float64))
+        parts["kc"].append(_get_chunked(region("KC"), cnt, kb, P))
+        parts["vc"].append(_get_chunked(region("VC"), cnt, vb, P))
+        if fmt.key_qjl:
+            parts["kr"].append(region("KR")[:2 * cnt].view(np.float16).astype(np.float64))
+            parts["ks"].append(_get_chunked(region("KS"), cnt, m // 8, P))
+    cat = lambda k, w: np.concatenate(parts[k]) if parts[k] else np.zeros((0,) + w)
+    kc = cat("kc", (kb,))
+    vc = cat("vc", (vb,))
+    out = Unpacked(k_idx=index_from_bits(bytes_to_bits(kc), fmt.key_bits, d),
+                   k_norm=cat("kn", ()),
+                   v_idx=index_from_bits(bytes_to_bits(vc), fmt.value_bits, d),
+                   v_norm=cat("vn", ()))
+    if fmt.key_qjl:
+        out.k_rnorm = cat("kr", ())
+        out.k_sigma = bytes_to_bits(cat("ks", (m // 8,))).astype(bool)
+    return out
