@@ -1,0 +1,411 @@
+"""Benchmark of the TurboQuant compressed-KV hot path on B200.
+
+One step = one pass of the whole path over a Llama-3-8B-shaped model cache: for each of
+32 layers (8 KV heads x 32768 tokens, head_dim 128, fp16 K/V drawn with the config-2
+recipe) compress K (3-bit + QJL) and V (3-bit) into the packed paged cache, then run
+decode attention for 32 query heads (seq_q = 1) over every layer.  Inputs (4.3 GB of
+K/V, plus the 0.99 GB packed cache) are larger than L2, so no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own replica (the work shards by independent
+layer/head units, no data-path collective); value = all ranks' units / max-over-ranks time.
+--impl reference times the CPU oracle (double precision, numpy) on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode KV-tokens/s and achieved HBM GB/s (% of B200 roofline); keys compressed/s"
+UNIT = "KV-tokens/s"  # token x kv-head positions compressed and then scanned by decode, per second
+FALLBACK_HBM = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def workload():
+    import workloads as wl
+    return wl.config2()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "compressed_decode_attention_tq_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d[kernel]
+        if ent.get("source_hash") != kernel_hash():
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(tokens: int, heads: int):
+    """Times the oracle on `heads` KV heads of layer 0, `tokens` tokens each: compress K (3-bit
+    + QJL) and V (3-bit), pack, decode the G query heads of each KV head.  Returns
+    (token*kv-heads processed, seconds, threads)."""
+    import numpy as np
+    import workloads as wl
+    from oracle import attention as oatt, codebook as ocb, layout as olay, quant as oq, rotation as orot
+    w = workload()
+    w1 = wl.config2(max_len=tokens)
+    rin = wl.rotation_inputs(w)
+    R = orot.rotation_matrix(w.rotation, rin["signs"], rin["pi"])
+    ck, kb = ocb.codebook_f32(w.key_bits, 128)
+    cv, vb = ocb.codebook_f32(w.value_bits, 128)
+    K, V = wl.make_kv(w1, 0, heads=list(range(heads)))
+    q = wl.make_q(w1)[:, : heads * w.group]
+    fmt = olay.Format(key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits)
+    lens = np.array([tokens], dtype=np.int32)
+    npg = (tokens + 255) // 256
+    bt = np.arange(npg, dtype=np.int32)[None]
+    t0 = time.perf_counter()
+    cache = olay.empty_cache(fmt, npg, heads)
+    for h in range(heads):
+        kc = oq.compress_prod(K[0, h], R, ck, kb, rin["s"])
+        vc = oq.compress_mse(V[0, h], R, cv, vb)
+        olay.write_sequence(cache, fmt, 0, h, bt[0], kc, vc)
+    oatt.decode(cache, fmt, 0, q, bt, lens, R, ck, cv, rin["s"])
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    return tokens * heads, dt, threads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload()
+    tokens, heads = w.max_len, 1
+    for _ in range(args.warmup):
+        oracle_sample(tokens, heads)
+    tot_units, tot_s, threads = 0, 0.0, 1
+    for _ in range(args.steps):
+        u, s, threads = oracle_sample(tokens, heads)
+        tot_units += u
+        tot_s += s
+    value = tot_units / tot_s
+    sample = f"layer 0, 1 of 8 KV heads, {tokens} tokens per step (compress K/V + pack + decode 4 query heads)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args.layers),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, layers):
+    return {"workload": "llama3_8b_32k_32layers: config-2 layer (8 KV heads x 32768 tokens, 32 q heads, "
+                        "fp16 K/V Gaussian x lognormal(0,0.5) channel scales + 2% outlier channels x10) "
+                        "x 32 layers; compress K 3-bit+QJL / V 3-bit, then decode seq_q=1",
+            "model": "Llama-3-8B KV shape", "layers": layers, "global_batch": w.batch,
+            "seq_len": w.max_len, "kv_heads": w.kv_heads, "q_heads": w.q_heads, "seq_q": w.seq_q,
+            "head_dim": 128, "key_bits": w.key_bits, "key_qjl": w.key_qjl, "value_bits": w.value_bits,
+            "page_tokens": 256, "n_splits": w.n_splits, "rotation": "hadamard",
+            "l2": "inputs larger than L2 (4.3 GB K/V read + 0.99 GB packed cache per step); no flush",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import workloads as wl
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workload()
+    L = args.layers
+    rin = wl.rotation_inputs(w)
+    lens = wl.seq_lens(w)
+    bt, npages = wl.block_table(w, lens)
+    kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
+                 key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits, rotation=w.rotation,
+                 num_layers=L, signs=rin["signs"], pi=rin["pi"], s=rin["s"], device=str(dev))
+    seq = torch.as_tensor(lens, dtype=torch.int32, device=dev)
+    Ks, Vs, Qs, Outs = [], [], [], []
+    for l in range(L):
+        k, v = wl.make_kv_device(w, l, dev)
+        Ks.append(k)
+        Vs.append(v)
+        Qs.append(wl.make_q_device(w, l, dev))
+        Outs.append(torch.empty(Qs[-1].shape, dtype=torch.float32, device=dev))
+    kv.workspace(w.q_heads, w.seq_q, w.n_splits)
+    stream = torch.cuda.current_stream(dev)
+    units = L * w.batch * w.kv_heads * int(lens.sum() // w.batch)  # token x kv-head per step
+    tok_heads_layer = int(lens.sum()) * w.kv_heads
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for l in range(L):
+            kv.compress(l, Ks[l], Vs[l], seq, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        for l in range(L):
+            kv.decode(l, Qs[l], seq, w.n_splits, out=Outs[l], stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    kv.raise_on_error("warmup")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    phase_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(phase_ev[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    kv.raise_on_error("timed steps")
+    ms_step = ms / args.steps
+    comp_ms = sum(e[0].elapsed_time(e[1]) for e in phase_ev) / args.steps
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in phase_ev) / args.steps
+    value = world * units / (ms_step / 1e3)
+
+    hbm, peak_kind = peaks()
+    comp_bytes_launch = tok_heads_layer * (2 * 128 * 2 + kv.block_bytes / 256)
+    dec_bytes_launch = tok_heads_layer * (kv.block_bytes / 256) + \
+        w.batch * w.q_heads * w.seq_q * 128 * (2 + 4)
+    comp_gbs = comp_bytes_launch / (comp_ms / L / 1e3) / 1e9
+    dec_gbs = dec_bytes_launch / (dec_ms / L / 1e3) / 1e9
+    phases = {
+        "compress": {"kernel": "compress_kernel", "ms_per_step": comp_ms, "launches_per_step": L,
+                     "keys_per_s": L * tok_heads_layer / (comp_ms / 1e3),
+                     "algorithmic_bytes_per_launch": comp_bytes_launch, "achieved_gbs": comp_gbs,
+                     "frac": comp_gbs / hbm},
+        "decode": {"kernel": "prologue+split+combine", "ms_per_step": dec_ms, "launches_per_step": L,
+                   "kv_tokens_per_s": L * tok_heads_layer / (dec_ms / 1e3),
+                   "algorithmic_bytes_per_launch": dec_bytes_launch, "achieved_gbs": dec_gbs,
+                   "frac": dec_gbs / hbm},
+    }
+    dom = "compress" if comp_ms >= dec_ms else "decode"
+    ph = phases[dom]
+    roofline = {"kernel": ph["kernel"], "bound": "hbm", "achieved": ph["achieved_gbs"], "peak": hbm,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6650 GB/s", "unit": "GB/s", "frac": ph["achieved_gbs"] / hbm,
+                "traffic": traffic_for(ph["kernel"])}
+
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        e2e = run_e2e(args, kv, w, L, Ks, Vs, Qs, Outs, seq, stream, dev, units, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        u, s, threads = oracle_sample(w.max_len, 1)
+        cpu = {"value": u / s, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"layer 0, 1 of 8 KV heads, {w.max_len} tokens: compress K/V + pack + "
+                         f"decode 4 query heads ({s:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_dict(w, L), "phases": phases, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * L * 4,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, kv, w, L, Ks, Vs, Qs, Outs, seq, stream, dev, units, world):
+    """Same step through the public API starting from pinned host buffers: H2D of the step's
+    K/V/q, compress + decode, D2H of the outputs, all inside the timed region."""
+    import torch
+    hK = [torch.empty(k.shape, dtype=k.dtype, pin_memory=True) for k in Ks]
+    hV = [torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for v in Vs]
+    hQ = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for q in Qs]
+    hO = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in Outs]
+    for l in range(L):
+        hK[l].copy_(Ks[l])
+        hV[l].copy_(Vs[l])
+        hQ[l].copy_(Qs[l])
+    torch.cuda.synchronize(dev)
+    h2d = sum(t.numel() * t.element_size() for t in hK + hV + hQ)
+    d2h = sum(t.numel() * t.element_size() for t in hO)
+
+    def step():
+        for l in range(L):
+            Ks[l].copy_(hK[l], non_blocking=True)
+            Vs[l].copy_(hV[l], non_blocking=True)
+            Qs[l].copy_(hQ[l], non_blocking=True)
+            kv.compress(l, Ks[l], Vs[l], seq, stream)
+        for l in range(L):
+            kv.decode(l, Qs[l], seq, w.n_splits, out=Outs[l], stream=stream)
+            hO[l].copy_(Outs[l], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    kv.raise_on_error("e2e")
+    return {"value": world * units / (ms / args.e2e_steps / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,366 @@
+// Decode attention directly over the packed cache (split-KV, flash-decoding style).
+//
+// "turboquant_cutile" function list: asymmetric estimator = MSE dot + QJL correction;
+// full pipeline scores -> softmax -> weighted V sum; fused attention + online softmax
+// with V decompressed on chip; scores scaled by 1/sqrt(d).
+// "TurboQuant explained" (Mobilint blog), section "How is this different from
+// PolarQuant's reconstruction?": <q, Pi^T c> = <Pi q, c>, so the rotated query is
+// formed once and each cached token costs an O(d) centroid-table product; section
+// "Practical Issues Found in Implementation": dequantisation must be fused with the
+// attention, never materialising dense K/V in HBM.
+// "tq-kv" crate documentation: pre_rotate_query, fused_attention_scores.
+//
+// Kernels: prologue (R q and S q per query row), split (online softmax over one
+// contiguous range of pages, partial (m, l, acc) in rotated space), combine
+// (log-sum-exp merge, divide by l, un-rotate with R^T).
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include "tq_device.cuh"
+#include "tq_kernels.h"
+
+namespace tqk {
+
+namespace {
+
+constexpr int kRowsMax = 32;
+constexpr int kTile = 128;  // tokens per tile (half a page)
+constexpr float kInvSqrtD = 0.08838834764831845f;
+constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------
+// prologue: one warp per query row
+// ---------------------------------------------------------------------------
+__global__ void prologue_kernel(DecodeArgs a, int total_rows) {
+  __shared__ float stage[4][D];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * 4 + w;
+  if (row >= total_rows) return;
+  float x[4];
+  if (a.q_dtype == TQ_F16) {
+    const __half* q = reinterpret_cast<const __half*>(a.q) + (size_t)row * D;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = __half2float(q[lane + 32 * e]);
+  } else {
+    const float* q = reinterpret_cast<const float*>(a.q) + (size_t)row * D;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = q[lane + 32 * e];
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) stage[w][lane + 32 * e] = x[e];
+  __syncwarp();
+  float y[4];
+  if (!a.dense) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = x[e] * a.signs[lane + 32 * e];
+    fwht128_warp(y, lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] *= kInvSqrtD;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float* prow = a.pi + (size_t)(lane + 32 * e) * D;
+      float acc = 0.f;
+      for (int k = 0; k < D; ++k) acc = fmaf(prow[k], stage[w][k], acc);
+      y[e] = acc;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) a.qrot[(size_t)row * D + lane + 32 * e] = y[e];
+  if (a.qjl) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float* srow = a.s + (size_t)(lane + 32 * e) * D;
+      float acc = 0.f;
+      for (int k = 0; k < D; ++k) acc = fmaf(srow[k], stage[w][k], acc);
+      a.sq[(size_t)row * QM + lane + 32 * e] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split kernel: grid (n_splits, kv_heads, batch), 128 threads
+// ---------------------------------------------------------------------------
+struct SmemSplit {
+  float qrot[kRowsMax][D];
+  float sq[kRowsMax][QM];
+  float p[kRowsMax][kTile];
+  uint32_t vcode[kTile][17];  // up to 16 words per token (+1 pad)
+  float vnorm[kTile];
+  float kmag[8], vmag[8];
+  float sqsum[kRowsMax];
+  float m[kRowsMax], l[kRowsMax], alpha[kRowsMax];
+};
+
+template <bool kScoresOnly>
+__global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SmemSplit& sm = *reinterpret_cast<SmemSplit*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const Layout& L = a.cache.L;
+  const int R = a.rows;
+  const size_t row0 = ((size_t)b * a.q_heads + (size_t)g * a.group) * a.seq_q;
+  const int hk = 1 << (L.kbits - 1), hv = 1 << (L.vbits - 1);
+  if (tid < hk) sm.kmag[tid] = a.k_centroids[hk + tid];
+  if (tid < hv) sm.vmag[tid] = a.v_centroids[hv + tid];
+  for (int i = tid; i < R * D; i += blockDim.x) sm.qrot[i / D][i % D] = a.qrot[row0 * D + i];
+  if (L.qjl)
+    for (int i = tid; i < R * QM; i += blockDim.x) sm.sq[i / QM][i % QM] = a.sq[row0 * QM + i];
+  if (tid < R) {
+    sm.m[tid] = -CUDART_INF_F;
+    sm.l[tid] = 0.f;
+  }
+  __syncthreads();
+  if (L.qjl && tid < R) {
+    float t = 0.f;
+    for (int i = 0; i < QM; ++i) t += sm.sq[tid][i];
+    sm.sqsum[tid] = t;
+  }
+  const int len = a.seq_lens[b];
+  const bool bad_len = len < 0 || len > a.cache.max_pages * PT || (kScoresOnly && len > a.max_len);
+  if (bad_len && tid == 0 && split == 0) report(a.status, TQ_ERR_BOUNDS);
+  const int n_eff = bad_len ? 0 : len;
+  const int npages = (n_eff + PT - 1) / PT;
+  const int cp = (npages + a.n_splits - 1) / a.n_splits;
+  const int t_begin = min(n_eff, split * cp * PT);
+  const int t_end = min(n_eff, (split + 1) * cp * PT);
+  float acc[kRowsMax];
+#pragma unroll
+  for (int r = 0; r < kRowsMax; ++r) acc[r] = 0.f;
+  __syncthreads();
+
+  for (int tile0 = t_begin; tile0 < t_end; tile0 += kTile) {
+    // ---- phase A: thread = token, scores for all rows
+    const int t = tile0 + tid;
+    float vn = 0.f;
+    bool valid = t < t_end;
+    uint8_t* blk = nullptr;
+    int slot = 0;
+    if (valid) {
+      const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + t / PT];
+      if (phys < 0 || phys >= a.cache.num_pages) {
+        report(a.status, TQ_ERR_BOUNDS);
+        valid = false;
+      } else {
+        blk = a.cache.block(phys, g);
+        slot = t % PT;
+      }
+    }
+    if (valid) {
+      uint32_t kw[16];
+      for (int c = 0; c < L.kbits; ++c) {
+        const uint4 v4 = reinterpret_cast<const uint4*>(blk + L.kc)[c * PT + slot];
+        kw[4 * c] = v4.x; kw[4 * c + 1] = v4.y; kw[4 * c + 2] = v4.z; kw[4 * c + 3] = v4.w;
+      }
+      float dot[kRowsMax];
+#pragma unroll
+      for (int r = 0; r < kRowsMax; ++r) dot[r] = 0.f;
+      for (int j = 0; j < D; ++j) {
+        int s, rk;
+        code_fields(kw, L.kbits, j, s, rk);
+        const float val = s ? sm.kmag[rk] : -sm.kmag[rk];
+#pragma unroll
+        for (int r = 0; r < kRowsMax; ++r)
+          if (r < R) dot[r] = fmaf(sm.qrot[r][j], val, dot[r]);
+      }
+      const float kn = __half2float(reinterpret_cast<const __half*>(blk + L.kn)[slot]);
+      float qj[kRowsMax];
+#pragma unroll
+      for (int r = 0; r < kRowsMax; ++r) qj[r] = 0.f;
+      float rho = 0.f;
+      if (L.qjl) {
+        const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.ks)[slot];
+        const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
+        rho = __half2float(reinterpret_cast<const __half*>(blk + L.kr)[slot]);
+        for (int i = 0; i < QM; ++i) {
+          if ((sw[i >> 5] >> (i & 31)) & 1u) {
+#pragma unroll
+            for (int r = 0; r < kRowsMax; ++r)
+              if (r < R) qj[r] += sm.sq[r][i];
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kRowsMax; ++r) {
+        if (r < R) {
+          float sc = kn * dot[r];
+          if (L.qjl) sc = fmaf(rho * kQjlScale, 2.f * qj[r] - sm.sqsum[r], sc);
+          sc *= kInvSqrtD;
+          if (kScoresOnly)
+            a.scores[(row0 + r) * (size_t)a.max_len + t] = sc;
+          else
+            sm.p[r][tid] = sc;
+        }
+      }
+      if (!kScoresOnly) {
+        for (int c = 0; c < L.vbits; ++c) {
+          const uint4 v4 = reinterpret_cast<const uint4*>(blk + L.vc)[c * PT + slot];
+          sm.vcode[tid][4 * c] = v4.x; sm.vcode[tid][4 * c + 1] = v4.y;
+          sm.vcode[tid][4 * c + 2] = v4.z; sm.vcode[tid][4 * c + 3] = v4.w;
+        }
+        vn = __half2float(reinterpret_cast<const __half*>(blk + L.vn)[slot]);
+      }
+    } else if (!kScoresOnly) {
+      for (int r = 0; r < R; ++r) sm.p[r][tid] = -CUDART_INF_F;
+    }
+    if (kScoresOnly) continue;
+    sm.vnorm[tid] = valid ? vn : 0.f;
+    __syncthreads();
+    // ---- phase B: online softmax bookkeeping, warp per row
+    for (int r = warp; r < R; r += 4) {
+      float v[4], mx = -CUDART_INF_F;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[e] = sm.p[r][lane + 32 * e];
+        mx = fmaxf(mx, v[e]);
+      }
+      mx = warp_max(mx);
+      const float m_old = sm.m[r];
+      const float m_new = fmaxf(m_old, mx);
+      float ps = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p = (m_new == -CUDART_INF_F) ? 0.f : __expf(v[e] - m_new);
+        sm.p[r][lane + 32 * e] = p;
+        ps += p;
+      }
+      ps = warp_sum(ps);
+      if (lane == 0) {
+        const float al = (m_new == -CUDART_INF_F) ? 1.f : __expf(m_old - m_new);
+        sm.alpha[r] = al;
+        sm.l[r] = sm.l[r] * al + ps;
+        sm.m[r] = m_new;
+      }
+    }
+    __syncthreads();
+    // ---- phase C: thread = coordinate j, V accumulation in rotated space
+    const int j = tid;
+#pragma unroll
+    for (int r = 0; r < kRowsMax; ++r)
+      if (r < R) acc[r] *= sm.alpha[r];
+    const int nt = min(kTile, t_end - tile0);
+    for (int tt = 0; tt < nt; ++tt) {
+      int s, rk;
+      code_fields(sm.vcode[tt], L.vbits, j, s, rk);
+      const float val = (s ? sm.vmag[rk] : -sm.vmag[rk]) * sm.vnorm[tt];
+#pragma unroll
+      for (int r = 0; r < kRowsMax; ++r)
+        if (r < R) acc[r] = fmaf(sm.p[r][tt], val, acc[r]);
+    }
+    __syncthreads();
+  }
+  if (kScoresOnly) return;
+  // ---- partials
+#pragma unroll
+  for (int r = 0; r < kRowsMax; ++r) {
+    if (r < R) {
+      const size_t pr = (row0 + r) * a.n_splits + split;
+      a.part_acc[pr * D + tid] = acc[r];
+      if (tid == 0) {
+        a.part_ml[pr * 2] = sm.m[r];
+        a.part_ml[pr * 2 + 1] = sm.l[r];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// combine: one warp per query row
+// ---------------------------------------------------------------------------
+__global__ void combine_kernel(DecodeArgs a, int total_rows) {
+  __shared__ float stage[4][D];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * 4 + w;
+  if (row >= total_rows) return;
+  float M = -CUDART_INF_F;
+  for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, a.part_ml[((size_t)row * a.n_splits + s) * 2]);
+  float l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  if (M != -CUDART_INF_F) {
+    for (int s = 0; s < a.n_splits; ++s) {
+      const size_t pr = (size_t)row * a.n_splits + s;
+      const float ms = a.part_ml[pr * 2];
+      if (ms == -CUDART_INF_F) continue;
+      const float wgt = __expf(ms - M);
+      l = fmaf(wgt, a.part_ml[pr * 2 + 1], l);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] = fmaf(wgt, a.part_acc[pr * D + lane + 32 * e], o[e]);
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) o[e] *= inv;
+  float y[4];
+  if (!a.dense) {
+    // R^T = D H
+    fwht128_warp(o, lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = o[e] * kInvSqrtD * a.signs[lane + 32 * e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) stage[w][lane + 32 * e] = o[e];
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float acc = 0.f;
+      for (int i = 0; i < D; ++i) acc = fmaf(a.pi[(size_t)i * D + lane + 32 * e], stage[w][i], acc);
+      y[e] = acc;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) a.out[(size_t)row * D + lane + 32 * e] = y[e];
+}
+
+}  // namespace
+
+DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits) {
+  const size_t rows = (size_t)batch * q_heads * seq_q;
+  DecodeWorkspace w;
+  size_t off = 0;
+  w.qrot = off; off = align256(off + rows * D * sizeof(float));
+  w.sq = off; off = align256(off + rows * QM * sizeof(float));
+  w.part_acc = off; off = align256(off + rows * (size_t)n_splits * D * sizeof(float));
+  w.part_ml = off; off = align256(off + rows * (size_t)n_splits * 2 * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream, bool scores_only) {
+  const size_t smem = sizeof(SmemSplit);
+  dim3 grid(scores_only ? 1 : a.n_splits, a.cache.kv_heads, a.cache.batch);
+  if (scores_only) {
+    auto k = split_kernel<true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 128, smem, stream>>>(a);
+  } else {
+    auto k = split_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 128, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
+  prologue_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_split(a, stream, false);
+  if (e != cudaSuccess) return e;
+  combine_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream) {
+  const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
+  prologue_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_split(a, stream, true);
+}
+
+}  // namespace tqk

@@ -1,0 +1,257 @@
+// The C ABI of include/tq.h: argument checks on the host, then kernel launches.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+
+#include "tq.h"
+#include "tq_internal.h"
+#include "tq_kernels.h"
+
+namespace tqi {
+
+static thread_local char g_last_error[512] = "";
+
+tq_status fail(tq_status st, const char* msg) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+  return st;
+}
+
+void clear_error() { g_last_error[0] = 0; }
+
+static tq_status cuda_fail(cudaError_t e, const char* where) {
+  char buf[400];
+  std::snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
+  return fail(TQ_ERR_CUDA, buf);
+}
+
+static tq_status check_config(const tq_config* cfg) {
+  if (!cfg) return fail(TQ_ERR_INVALID_ARG, "config is NULL");
+  if (cfg->head_dim != tqk::D) return fail(TQ_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (cfg->qjl_m != tqk::QM) return fail(TQ_ERR_UNSUPPORTED, "qjl_m must be 128");
+  if (cfg->page_tokens != tqk::PT) return fail(TQ_ERR_UNSUPPORTED, "page_tokens must be 256");
+  if (cfg->key_bits < 1 || cfg->key_bits > 4) return fail(TQ_ERR_UNSUPPORTED, "key_bits must be in 1..4");
+  if (cfg->value_bits < 1 || cfg->value_bits > 4)
+    return fail(TQ_ERR_UNSUPPORTED, "value_bits must be in 1..4");
+  if (cfg->key_qjl != 0 && cfg->key_qjl != 1) return fail(TQ_ERR_INVALID_ARG, "key_qjl must be 0 or 1");
+  if (cfg->rotation != TQ_ROT_HADAMARD && cfg->rotation != TQ_ROT_DENSE)
+    return fail(TQ_ERR_INVALID_ARG, "unknown rotation kind");
+  return TQ_OK;
+}
+
+static tq_status check_params(const tq_config* cfg, const tq_params* p, bool need_s) {
+  if (!p) return fail(TQ_ERR_INVALID_ARG, "params is NULL");
+  if (cfg->rotation == TQ_ROT_HADAMARD && !p->signs) return fail(TQ_ERR_INVALID_ARG, "params.signs is NULL");
+  if (cfg->rotation == TQ_ROT_DENSE && !p->pi) return fail(TQ_ERR_INVALID_ARG, "params.pi is NULL");
+  if (need_s && cfg->key_qjl && !p->s) return fail(TQ_ERR_INVALID_ARG, "params.s is NULL");
+  if (!p->k_centroids || !p->v_centroids) return fail(TQ_ERR_INVALID_ARG, "centroid pointer is NULL");
+  return TQ_OK;
+}
+
+static tq_status check_cache(const tq_cache* c, int32_t layer) {
+  if (!c) return fail(TQ_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->pages || !c->block_table) return fail(TQ_ERR_INVALID_ARG, "cache.pages or block_table is NULL");
+  if (c->batch < 1 || c->kv_heads < 1 || c->num_layers < 1 || c->num_pages < 1 || c->max_pages < 1)
+    return fail(TQ_ERR_INVALID_ARG, "cache sizes must be >= 1");
+  if (layer < 0 || layer >= c->num_layers) return fail(TQ_ERR_INVALID_ARG, "layer out of range");
+  if ((size_t)c->batch * c->max_pages > (size_t)1 << 31) return fail(TQ_ERR_INVALID_ARG, "block table too large");
+  return TQ_OK;
+}
+
+static tqk::CacheRef cache_ref(const tq_config* cfg, const tq_cache* c, int32_t layer) {
+  tqk::CacheRef r;
+  r.pages = static_cast<uint8_t*>(c->pages);
+  r.block_table = c->block_table;
+  r.num_pages = c->num_pages;
+  r.max_pages = c->max_pages;
+  r.batch = c->batch;
+  r.kv_heads = c->kv_heads;
+  r.layer = layer;
+  r.L = tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits);
+  return r;
+}
+
+}  // namespace tqi
+
+using namespace tqi;
+
+extern "C" {
+
+int32_t tq_version(void) { return 100; }
+
+const char* tq_status_str(tq_status st) {
+  switch (st) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+    case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    case TQ_ERR_OVERFLOW: return "TQ_ERR_OVERFLOW";
+    case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT";
+    case TQ_ERR_BOUNDS: return "TQ_ERR_BOUNDS";
+  }
+  return "TQ_ERR_UNKNOWN";
+}
+
+const char* tq_last_error(void) { return g_last_error; }
+
+tq_status tq_validate_config(const tq_config* cfg) {
+  clear_error();
+  return check_config(cfg);
+}
+
+size_t tq_page_bytes(const tq_config* cfg) {
+  if (check_config(cfg) != TQ_OK) return 0;
+  return (size_t)tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits).bytes;
+}
+
+tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                         int32_t layer, const void* k, const void* v, int32_t in_dtype, int32_t max_len,
+                         const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  tq_status st;
+  if ((st = check_config(cfg)) != TQ_OK) return st;
+  if ((st = check_params(cfg, params, true)) != TQ_OK) return st;
+  if ((st = check_cache(cache, layer)) != TQ_OK) return st;
+  if (!params->k_boundaries || !params->v_boundaries) return fail(TQ_ERR_INVALID_ARG, "boundary pointer is NULL");
+  if (!k || !v || !seq_lens) return fail(TQ_ERR_INVALID_ARG, "k, v or seq_lens is NULL");
+  if (in_dtype != TQ_F16 && in_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "in_dtype must be TQ_F16 or TQ_F32");
+  if (max_len < 0) return fail(TQ_ERR_INVALID_ARG, "max_len must be >= 0");
+  tqk::CompressArgs a;
+  a.cache = cache_ref(cfg, cache, layer);
+  a.k = k;
+  a.v = v;
+  a.in_dtype = in_dtype;
+  a.max_len = max_len;
+  a.qjl = cfg->key_qjl;
+  a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.seq_lens = seq_lens;
+  a.signs = params->signs;
+  a.pi = params->pi;
+  a.s = params->s;
+  a.k_centroids = params->k_centroids;
+  a.k_boundaries = params->k_boundaries;
+  a.v_centroids = params->v_centroids;
+  a.v_boundaries = params->v_boundaries;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_compress(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_compress_kv launch");
+  return TQ_OK;
+}
+
+size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int32_t q_heads, int32_t seq_q,
+                                 int32_t n_splits) {
+  if (check_config(cfg) != TQ_OK || batch < 1 || q_heads < 1 || seq_q < 1 || n_splits < 1) return 0;
+  return tqk::decode_workspace(batch, q_heads, seq_q, n_splits).total;
+}
+
+static tq_status decode_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                               int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
+                               int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
+                               size_t workspace_bytes, tqk::DecodeArgs& a) {
+  tq_status st;
+  if ((st = check_config(cfg)) != TQ_OK) return st;
+  if ((st = check_params(cfg, params, true)) != TQ_OK) return st;
+  if ((st = check_cache(cache, layer)) != TQ_OK) return st;
+  if (!q || !seq_lens || !workspace) return fail(TQ_ERR_INVALID_ARG, "q, seq_lens or workspace is NULL");
+  if (q_dtype != TQ_F16 && q_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "q_dtype must be TQ_F16 or TQ_F32");
+  if (q_heads < 1 || q_heads % cache->kv_heads != 0)
+    return fail(TQ_ERR_INVALID_ARG, "q_heads must be a positive multiple of kv_heads");
+  if (seq_q < 1) return fail(TQ_ERR_INVALID_ARG, "seq_q must be >= 1");
+  const int group = q_heads / cache->kv_heads;
+  if (group * seq_q > 32) return fail(TQ_ERR_UNSUPPORTED, "q_heads/kv_heads * seq_q must be <= 32");
+  if (n_splits < 1 || n_splits > 1024) return fail(TQ_ERR_INVALID_ARG, "n_splits must be in 1..1024");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return fail(TQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const tqk::DecodeWorkspace w = tqk::decode_workspace(cache->batch, q_heads, seq_q, n_splits);
+  if (workspace_bytes < w.total) return fail(TQ_ERR_INVALID_ARG, "workspace too small");
+  char* ws = static_cast<char*>(workspace);
+  a.cache = cache_ref(cfg, cache, layer);
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.q_heads = q_heads;
+  a.seq_q = seq_q;
+  a.group = group;
+  a.rows = group * seq_q;
+  a.n_splits = n_splits;
+  a.qjl = cfg->key_qjl;
+  a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.seq_lens = seq_lens;
+  a.signs = params->signs;
+  a.pi = params->pi;
+  a.s = params->s;
+  a.k_centroids = params->k_centroids;
+  a.v_centroids = params->v_centroids;
+  a.qrot = reinterpret_cast<float*>(ws + w.qrot);
+  a.sq = reinterpret_cast<float*>(ws + w.sq);
+  a.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+  a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  a.out = nullptr;
+  a.scores = nullptr;
+  a.max_len = 0;
+  return TQ_OK;
+}
+
+tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                           int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads, int32_t seq_q,
+                           const int32_t* seq_lens, int32_t n_splits, void* workspace,
+                           size_t workspace_bytes, float* out, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  tqk::DecodeArgs a;
+  tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, n_splits,
+                               workspace, workspace_bytes, a);
+  if (st != TQ_OK) return st;
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  a.out = out;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode launch");
+  return TQ_OK;
+}
+
+tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                           int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads, int32_t seq_q,
+                           const int32_t* seq_lens, int32_t max_len, void* workspace,
+                           size_t workspace_bytes, float* scores, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  tqk::DecodeArgs a;
+  tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, 1,
+                               workspace, workspace_bytes, a);
+  if (st != TQ_OK) return st;
+  if (!scores) return fail(TQ_ERR_INVALID_ARG, "scores is NULL");
+  if (max_len < 0) return fail(TQ_ERR_INVALID_ARG, "max_len must be >= 0");
+  a.scores = scores;
+  a.max_len = max_len;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_decode_scores(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decode_scores launch");
+  return TQ_OK;
+}
+
+tq_status tq_decompress(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
+                        const int32_t* seq_lens, int32_t max_len, float* k_hat, float* v_hat,
+                        int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  tq_status st;
+  if ((st = check_config(cfg)) != TQ_OK) return st;
+  if ((st = check_params(cfg, params, false)) != TQ_OK) return st;
+  if ((st = check_cache(cache, layer)) != TQ_OK) return st;
+  if (!seq_lens) return fail(TQ_ERR_INVALID_ARG, "seq_lens is NULL");
+  if (max_len < 0) return fail(TQ_ERR_INVALID_ARG, "max_len must be >= 0");
+  tqk::DecompressArgs a;
+  a.cache = cache_ref(cfg, cache, layer);
+  a.seq_lens = seq_lens;
+  a.max_len = max_len;
+  a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.signs = params->signs;
+  a.pi = params->pi;
+  a.k_centroids = params->k_centroids;
+  a.v_centroids = params->v_centroids;
+  a.k_hat = k_hat;
+  a.v_hat = v_hat;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_decompress(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_decompress launch");
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// Kernel argument blocks and launchers (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "tq_device.cuh"
+
+namespace tqk {
+
+struct CompressArgs {
+  CacheRef cache;
+  const void* k;
+  const void* v;
+  int in_dtype, max_len, qjl, dense;
+  const int32_t* seq_lens;
+  const float *signs, *pi, *s, *k_centroids, *k_boundaries, *v_centroids, *v_boundaries;
+  int32_t* status;
+};
+
+struct DecodeArgs {
+  CacheRef cache;
+  const void* q;
+  int q_dtype, q_heads, seq_q, group, rows, n_splits, qjl, dense;
+  const int32_t* seq_lens;
+  const float *signs, *pi, *s, *k_centroids, *v_centroids;
+  float* qrot;      // [B*Hq*seq_q][D]  workspace
+  float* sq;        // [B*Hq*seq_q][QM] workspace
+  float* part_acc;  // [B*Hq*seq_q][n_splits][D] workspace
+  float* part_ml;   // [B*Hq*seq_q][n_splits][2] workspace
+  float* out;       // [B*Hq*seq_q][D]
+  float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
+  int max_len;
+  int32_t* status;
+};
+
+struct DecompressArgs {
+  CacheRef cache;
+  const int32_t* seq_lens;
+  int max_len, dense;
+  const float *signs, *pi, *k_centroids, *v_centroids;
+  float *k_hat, *v_hat;
+  int32_t* status;
+};
+
+size_t compress_smem_bytes(int qjl, int dense);
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);
+
+// Workspace layout of decode, all offsets 256-byte aligned.
+struct DecodeWorkspace {
+  size_t qrot, sq, part_acc, part_ml, total;
+};
+DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits);
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decompress(const DecompressArgs& a, cudaStream_t stream);
+
+}  // namespace tqk

@@ -1,0 +1,105 @@
+"""Device-memory plumbing around the C ABI: a paged cache plus its parameters.
+
+Owns nothing but PyTorch tensors; every computation is a call into libtq.so.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, attend_decode, codebook, compress_kv,
+               decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
+               page_bytes, status_str)
+
+
+def _f32(x, device):
+    if x is None:
+        return None
+    return torch.as_tensor(x, dtype=torch.float32).to(device).contiguous()
+
+
+class PagedKV:
+    """A packed TurboQuant cache for `num_layers` layers sharing one block table."""
+
+    def __init__(self, *, batch: int, kv_heads: int, num_pages: int, block_table, key_bits: int,
+                 key_qjl: bool, value_bits: int, rotation: int = TQ_ROT_HADAMARD,
+                 num_layers: int = 1, signs=None, pi=None, s=None, codebooks=None,
+                 device: str = "cuda"):
+        self.device = torch.device(device)
+        self.cfg = make_config(key_bits=key_bits, key_qjl=key_qjl, value_bits=value_bits,
+                               rotation=rotation)
+        self.block_bytes = page_bytes(self.cfg)
+        if self.block_bytes == 0:
+            raise TQError(2, "PagedKV", "unsupported configuration")
+        self.batch, self.kv_heads, self.num_pages, self.num_layers = batch, kv_heads, num_pages, num_layers
+        self.block_table = torch.as_tensor(block_table, dtype=torch.int32).to(self.device).contiguous()
+        self.max_pages = self.block_table.shape[1]
+        nbytes = num_layers * num_pages * kv_heads * self.block_bytes
+        self.pages = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        if codebooks is None:
+            kc, kb = codebook(key_bits)
+            vc, vb = codebook(value_bits)
+        else:
+            kc, kb, vc, vb = codebooks
+        self.tensors = {
+            "signs": _f32(signs, self.device), "pi": _f32(pi, self.device), "s": _f32(s, self.device),
+            "kc": _f32(kc, self.device), "kb": _f32(kb, self.device),
+            "vc": _f32(vc, self.device), "vb": _f32(vb, self.device),
+        }
+        t = self.tensors
+        self.params = make_params(t["signs"], t["pi"], t["s"], t["kc"], t["kb"], t["vc"], t["vb"])
+        self.cache = make_cache(self.pages, self.block_table, num_pages, self.max_pages, batch, kv_heads,
+                                num_layers)
+        self._ws = {}
+
+    # ---- calls -----------------------------------------------------------------------------
+    def compress(self, layer: int, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, stream=None):
+        compress_kv(self.cfg, self.params, self.cache, layer, k, v, seq_lens, self.status, stream)
+
+    def workspace(self, q_heads: int, seq_q: int, n_splits: int) -> torch.Tensor:
+        key = (q_heads, seq_q, n_splits)
+        if key not in self._ws:
+            nb = decode_workspace_bytes(self.cfg, self.batch, q_heads, seq_q, n_splits)
+            self._ws[key] = torch.empty(nb, dtype=torch.uint8, device=self.device)
+        return self._ws[key]
+
+    def decode(self, layer: int, q: torch.Tensor, seq_lens: torch.Tensor, n_splits: int,
+               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        ws = self.workspace(q.shape[1], q.shape[2], n_splits)
+        attend_decode(self.cfg, self.params, self.cache, layer, q, seq_lens, n_splits, ws, out,
+                      self.status, stream)
+        return out
+
+    def scores(self, layer: int, q: torch.Tensor, seq_lens: torch.Tensor, max_len: int, stream=None):
+        sc = torch.full((q.shape[0], q.shape[1], q.shape[2], max_len), float("nan"),
+                        dtype=torch.float32, device=self.device)
+        ws = self.workspace(q.shape[1], q.shape[2], 1)
+        decode_scores(self.cfg, self.params, self.cache, layer, q, seq_lens, ws, sc, self.status, stream)
+        return sc
+
+    def decompress(self, layer: int, seq_lens: torch.Tensor, max_len: int, stream=None):
+        kh = torch.zeros((self.batch, self.kv_heads, max_len, 128), dtype=torch.float32, device=self.device)
+        vh = torch.zeros_like(kh)
+        decompress(self.cfg, self.params, self.cache, layer, seq_lens, max_len, kh, vh, self.status, stream)
+        return kh, vh
+
+    def check(self) -> int:
+        """Synchronise and return the device status word (0 = ok); resets it."""
+        torch.cuda.synchronize(self.device)
+        st = int(self.status.item())
+        self.status.zero_()
+        return st
+
+    def raise_on_error(self, where: str = "device"):
+        st = self.check()
+        if st:
+            raise TQError(st, where, status_str(st))
+
+    def pages_numpy(self):
+        """Host copy of the cache as [num_layers][num_pages][kv_heads][block_bytes] uint8."""
+        return self.pages.view(self.num_layers, self.num_pages, self.kv_heads, self.block_bytes).cpu().numpy()

@@ -1,0 +1,237 @@
+/*
+ * tq.h - C ABI of the TurboQuant compressed-KV decode library for NVIDIA B200 (sm_100a).
+ *
+ * The library compresses a KV cache with TurboQuant and runs decode attention
+ * directly on the packed, paged cache.  What it computes follows these pages:
+ *
+ *   [CUTILE]  "turboquant_cutile" function list (codehub.bot, DevTechJr/turboquant_cutile):
+ *             compress K -> dict (MSE + 1-bit QJL), compress V -> dict (MSE only),
+ *             asymmetric estimator = MSE dot + QJL correction, full pipeline
+ *             scores -> softmax -> weighted V sum, decompression
+ *             indices -> centroids -> un-rotate -> rescale, codebook as sorted
+ *             float32 (centroids (2^b,), boundaries (2^b - 1,)).
+ *   [MOBILINT] "TurboQuant explained: near-optimal KV cache compression and why
+ *             the theory breaks down in practice" (Mobilint blog): sections
+ *             "How JL Matrices Evolved" (HD rotation), "QJL: Inner Product Recovery
+ *             from a Single Sign Bit", "Coordinates Become Predictable After
+ *             Rotation" (Beta density), "Designing the Optimal Codebook Without
+ *             Data" (Lloyd-Max), "Two-Stage Approach: MSE Approximation + QJL
+ *             Correction", "Practical Issues Found in Implementation" (fused
+ *             kernels, no dense K/V round trip).
+ *   [TQKV]    "tq-kv" crate documentation (docs.rs): pre-rotated query, centroid
+ *             table scoring without decompression, incremental cache.
+ *   [LIMITS]  "TurboQuant Limits And Assumptions" (ginkgoq): vLLM-style packed
+ *             paged decode; storage claims count every byte.
+ *
+ * Conventions for every call below:
+ *   - The library allocates nothing.  Every buffer is owned by the caller and
+ *     passed as a plain pointer; "device" pointers are CUDA device memory of the
+ *     current device, "host" pointers are ordinary host memory.
+ *   - Device calls are asynchronous on the given stream (a cudaStream_t; NULL is
+ *     the legacy default stream).  They return after enqueueing.
+ *   - Host-side argument errors are returned as a tq_status and nothing is
+ *     enqueued; tq_last_error() then describes the failing argument.
+ *   - Errors found on the device (norm overflow, page table out of range, a
+ *     parameter the device checks) are written to the caller's int32 dev_status
+ *     word (device memory, must start at 0): the first error code wins and the
+ *     affected output is left unspecified.  Read it after a stream sync.
+ *   - Arrays are row-major and contiguous with the shapes given.
+ *   - Supported: head_dim = 128, qjl_m = 128, page_tokens = 256, key/value
+ *     bits in 1..4.  Other values return TQ_ERR_UNSUPPORTED.
+ *
+ * Packed cache format (one block per (layer, physical page, kv head); the cache
+ * buffer is [num_layers][num_pages][kv_heads][tq_page_bytes(cfg)] bytes):
+ *
+ *   region  content                                   bytes (P = page_tokens)
+ *   KN      stored ||k|| (fp16) per token              2P
+ *   KR      stored ||r|| (fp16) per token, QJL keys    2P
+ *   VN      stored ||v|| (fp16) per token              2P
+ *   KC      key codes, key_bits*d/8 bytes per token    key_bits*16*P
+ *   KS      QJL sign bits, m/8 bytes per token          16*P   (QJL keys)
+ *   VC      value codes                               value_bits*16*P
+ *
+ *   A code region stores each token's bytes as 16-byte chunks, chunk-major:
+ *   chunk c of slot t is at region byte (c*P + t)*16.  A token's chunks,
+ *   concatenated, form its bit string; bit k is bit (k mod 8) of byte k/8.
+ *   Index idx in [0, 2^b) of coordinate j is stored in sign-magnitude form,
+ *   h = 2^(b-1): s = [idx >= h], r = idx - h if s else h - 1 - idx, so that
+ *   c[idx] = (s ? +1 : -1) * c[h + r] for the (symmetric) codebook c:
+ *     b = 1: bit j = s
+ *     b = 2: bits 2j, 2j+1 = r, s
+ *     b = 3: bits 2j, 2j+1 = r (2 bits), bit 2d + j = s
+ *     b = 4: bits 4j..4j+2 = r (3 bits), bit 4j + 3 = s
+ *   QJL sign bit i of a key = [(S r)_i >= 0] (sign(0) is stored as +1).
+ *   Slots past a sequence's length are never read and their bytes unspecified.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, without pulling in the CUDA headers. */
+typedef struct CUstream_st* tq_stream_t;
+
+typedef enum tq_status {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent sizes, bad parameter values   */
+  TQ_ERR_UNSUPPORTED = 2,  /* a size or mode outside what this build supports          */
+  TQ_ERR_CUDA = 3,         /* a CUDA runtime call or a kernel launch failed            */
+  TQ_ERR_OVERFLOW = 4,     /* a norm does not fit in fp16 (device)                     */
+  TQ_ERR_TIMEOUT = 5,      /* a bounded wait inside a kernel gave up (device)          */
+  TQ_ERR_BOUNDS = 6        /* sequence longer than its page-table row, or page id out
+                              of range (device)                                        */
+} tq_status;
+
+typedef enum tq_density { TQ_DENSITY_BETA = 0, TQ_DENSITY_GAUSS = 1 } tq_density;
+typedef enum tq_rotation_kind { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rotation_kind;
+typedef enum tq_dtype { TQ_F16 = 0, TQ_F32 = 1 } tq_dtype;
+
+/* Configuration of one cache ([TQKV] TurboQuantConfig: bits, rotation, QJL mode). */
+typedef struct tq_config {
+  int32_t head_dim;     /* d, must be 128                                             */
+  int32_t key_bits;     /* b_k: bits of the key MSE stage, 1..4                        */
+  int32_t key_qjl;      /* 1: keys carry the 1-bit QJL sketch of the residual and ||r|| */
+  int32_t qjl_m;        /* m: rows of S, must be 128                                   */
+  int32_t value_bits;   /* b_v: bits of the value MSE stage, 1..4                      */
+  int32_t page_tokens;  /* P: tokens per page, must be 256                             */
+  int32_t rotation;     /* tq_rotation_kind                                            */
+} tq_config;
+
+/* Random inputs of the method and the codebooks, all device memory, fp32.
+ * [MOBILINT] "How JL Matrices Evolved": R = H D (H the normalized Sylvester
+ * Walsh-Hadamard matrix, D a +-1 diagonal); [CUTILE]: the dense option is a
+ * Haar orthogonal Pi.  [MOBILINT] "QJL": S is an m x d Gaussian matrix. */
+typedef struct tq_params {
+  const float* signs;         /* [d] +-1 diagonal of D (TQ_ROT_HADAMARD), else unused     */
+  const float* pi;            /* [d*d] Pi, row-major, y = Pi u (TQ_ROT_DENSE), else unused */
+  const float* s;             /* [m*d] S, row-major; every entry must be exactly
+                                 representable in fp16 (checked on the device,
+                                 TQ_ERR_INVALID_ARG); unused unless key_qjl            */
+  const float* k_centroids;   /* [2^key_bits] sorted, symmetric (c_i = -c_{n-1-i})      */
+  const float* k_boundaries;  /* [2^key_bits - 1] sorted, symmetric, middle one 0        */
+  const float* v_centroids;   /* [2^value_bits]                                          */
+  const float* v_boundaries;  /* [2^value_bits - 1]                                      */
+} tq_params;
+
+/* A paged cache ([LIMITS] vLLM-style packed paged cache). */
+typedef struct tq_cache {
+  void* pages;                 /* device [num_layers][num_pages][kv_heads][page bytes]     */
+  const int32_t* block_table;  /* device [batch][max_pages]: physical page of each logical
+                                  page of each sequence                                   */
+  int32_t num_pages;           /* physical pages per layer                                */
+  int32_t max_pages;           /* length of one block-table row                           */
+  int32_t batch;
+  int32_t kv_heads;
+  int32_t num_layers;
+} tq_cache;
+
+/* Library version (major*10000 + minor*100 + patch). */
+TQ_API int32_t tq_version(void);
+
+/* Human-readable name of a status code (static string). */
+TQ_API const char* tq_status_str(tq_status st);
+
+/* Detail of the last host-side error on the calling thread (static per-thread
+ * buffer, empty string if none). */
+TQ_API const char* tq_last_error(void);
+
+/* Checks a configuration; TQ_OK if this build supports it. */
+TQ_API tq_status tq_validate_config(const tq_config* cfg);
+
+/* Bytes of one (layer, page, kv head) block for cfg; 0 if cfg is invalid. */
+TQ_API size_t tq_page_bytes(const tq_config* cfg);
+
+/* Lloyd-Max codebook ([MOBILINT] "Designing the Optimal Codebook Without Data",
+ * steps 1-3, on the density of "Coordinates Become Predictable After Rotation";
+ * [CUTILE] codebook function; [TQKV] module codebook for the Gaussian variant).
+ * HOST call, synchronous.
+ *   bits        1..8
+ *   head_dim    d >= 3; the density is f_X(t) ~ (1 - t^2)^((d-3)/2) on [-1, 1]
+ *               (TQ_DENSITY_BETA) or N(0, 1/d) (TQ_DENSITY_GAUSS)
+ *   centroids   host float[2^bits], written sorted ascending
+ *   boundaries  host float[2^bits - 1], the fp32 rounding of the midpoints of the
+ *               double-precision centroids
+ * The iteration starts from linspace(-2/sqrt(d), 2/sqrt(d), 2^bits), runs until
+ * the centroids move by less than 1e-13, and symmetrises the result. */
+TQ_API tq_status tq_codebook(int32_t bits, int32_t head_dim, int32_t density, float* centroids,
+                      float* boundaries);
+
+/* Compress K and V into the packed cache ([CUTILE] compress K (MSE + QJL) and
+ * compress V (MSE only); [MOBILINT] "Two-Stage Approach": per vector n = ||x||,
+ * u = x/n, y = R u, idx_j = #{i : beta_i < y_j}, stored fp16(n); for keys with
+ * QJL, k_mse = fp16(n) R^T c[idx], r = k - k_mse, sign bits [(S r)_i >= 0] and
+ * fp16(||r||)).
+ *   layer      0..num_layers-1
+ *   k, v       device [batch][kv_heads][max_len][d], element type in_dtype
+ *   seq_lens   device int32 [batch]; tokens 0..seq_lens[b]-1 of each (b, head) are
+ *              written to slots via the block table (logical page t/P, slot t%P)
+ *   dev_status device int32; TQ_ERR_OVERFLOW, TQ_ERR_BOUNDS, TQ_ERR_INVALID_ARG
+ * Pages not covered by a sequence are not touched. */
+TQ_API tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                         int32_t layer, const void* k, const void* v, int32_t in_dtype,
+                         int32_t max_len, const int32_t* seq_lens, int32_t* dev_status,
+                         tq_stream_t stream);
+
+/* Workspace bytes tq_attend_decode and tq_decode_scores need for these sizes. */
+TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int32_t q_heads,
+                                 int32_t seq_q, int32_t n_splits);
+
+/* Decode attention over the packed cache ([CUTILE] full pipeline with the
+ * asymmetric estimator and fused on-chip V dequantisation; [MOBILINT] "How is this
+ * different from PolarQuant's reconstruction?": <q, R^T c> = <R q, c>, so R q is
+ * formed once per query; [TQKV] pre_rotate_query / fused_attention_scores).
+ * For query row (b, h, p), kv head g = h / (q_heads / kv_heads):
+ *   score_t = ( ||k||_t <R q, c_k[idx_t]>
+ *               + [QJL] ||r||_t sqrt(pi/2)/m <S q, 2 sigma_t - 1> ) / sqrt(d)
+ *   out     = R^T sum_t softmax(score)_t ||v||_t c_v[idx_v,t]
+ * over t < seq_lens[b] (no causal mask between the seq_q rows; an empty sequence
+ * gives 0).  The sequence is cut into n_splits contiguous ranges processed in
+ * parallel and merged by their log-sum-exp.
+ *   q          device [batch][q_heads][seq_q][d], element type q_dtype
+ *   q_heads    multiple of kv_heads; q_heads/kv_heads * seq_q <= 32
+ *   n_splits   1..1024
+ *   workspace  device, >= tq_decode_workspace_bytes(...) bytes, 256-byte aligned;
+ *              scratch only, contents on return unspecified
+ *   out        device float [batch][q_heads][seq_q][d] */
+TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                           int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
+                           int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,
+                           void* workspace, size_t workspace_bytes, float* out,
+                           int32_t* dev_status, tq_stream_t stream);
+
+/* Score-only decode ([CUTILE] "Score-only kernel ... streams over KV"): writes the
+ * scaled scores score_t above for every query row and t < seq_lens[b]; entries with
+ * t >= seq_lens[b] are left untouched.
+ *   scores     device float [batch][q_heads][seq_q][max_len]
+ *   workspace  as for tq_attend_decode with n_splits = 1 */
+TQ_API tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                           int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
+                           int32_t seq_q, const int32_t* seq_lens, int32_t max_len,
+                           void* workspace, size_t workspace_bytes, float* scores,
+                           int32_t* dev_status, tq_stream_t stream);
+
+/* Decompress ([CUTILE] "indices -> centroids -> un-rotate -> rescale"):
+ * k_hat = ||k|| R^T c_k[idx] (the MSE part k_mse for QJL keys) and
+ * v_hat = ||v|| R^T c_v[idx_v], for tokens t < seq_lens[b]; rows past the
+ * length are left untouched.
+ *   k_hat, v_hat  device float [batch][kv_heads][max_len][d] (either may be NULL) */
+TQ_API tq_status tq_decompress(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                        int32_t layer, const int32_t* seq_lens, int32_t max_len, float* k_hat,
+                        float* v_hat, int32_t* dev_status, tq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

@@ -1,0 +1,150 @@
+"""Shared pieces of the GPU parity tests: run the library on a workload, run the oracle on
+the same seeded inputs, compare with the stated tolerances.
+
+Tolerances (spec contract):
+  * packed indices and QJL sign bits bit-exact, except coordinates whose rotated value
+    lies within 1e-6 of a codebook boundary, and sign bits whose projection (S r)_i lies
+    within 1e-6 * sum_j |S_ij r_j| of zero (both counted and reported);
+  * norms, scores and attention outputs |gpu - oracle| <= 1e-3 + 2e-3 |oracle|.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import workloads as wl
+from oracle import attention as oatt
+from oracle import codebook as ocb
+from oracle import layout as olay
+from oracle import quant as oq
+from oracle import rotation as orot
+
+ATOL, RTOL = 1e-3, 2e-3
+BOUNDARY_BAND = 1e-6
+SIGN_BAND = 1e-6
+
+
+def close(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return np.abs(got - ref) <= ATOL + RTOL * np.abs(ref)
+
+
+@dataclasses.dataclass
+class Run:
+    w: wl.Workload
+    lens: np.ndarray
+    bt: np.ndarray
+    npages: int
+    rin: dict
+    R: np.ndarray
+    fmt: olay.Format
+    ck: np.ndarray
+    kb: np.ndarray
+    cv: np.ndarray
+    vb: np.ndarray
+    kv: object = None
+    K: dict = None
+    V: dict = None
+
+
+def setup(w: wl.Workload, layers=(0,)):
+    """Builds the library cache for w and compresses `layers` on the GPU (inputs from workloads)."""
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+    lens = wl.seq_lens(w)
+    bt, npages = wl.block_table(w, lens)
+    rin = wl.rotation_inputs(w)
+    run = Run(w=w, lens=lens, bt=bt, npages=npages, rin=rin,
+              R=orot.rotation_matrix(w.rotation, rin["signs"], rin["pi"]),
+              fmt=olay.Format(key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits),
+              ck=None, kb=None, cv=None, vb=None)
+    run.ck, run.kb = ocb.codebook_f32(w.key_bits, 128)
+    run.cv, run.vb = ocb.codebook_f32(w.value_bits, 128)
+    run.kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
+                     key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits,
+                     rotation=w.rotation, num_layers=max(layers) + 1, signs=rin["signs"],
+                     pi=rin["pi"], s=rin["s"])
+    run.K, run.V = {}, {}
+    dt = torch.float16 if w.in_dtype == "f16" else torch.float32
+    seq = torch.as_tensor(lens, dtype=torch.int32, device="cuda")
+    for layer in layers:
+        K, V = wl.make_kv(w, layer)
+        run.K[layer], run.V[layer] = K, V
+        run.kv.compress(layer, torch.as_tensor(K, dtype=dt, device="cuda"),
+                        torch.as_tensor(V, dtype=dt, device="cuda"), seq)
+    return run
+
+
+def seq_dev(run):
+    return torch.as_tensor(run.lens, dtype=torch.int32, device="cuda")
+
+
+def q_dev(run, layer=0):
+    q = wl.make_q(run.w, layer)
+    dt = torch.float16 if run.w.in_dtype == "f16" else torch.float32
+    return q, torch.as_tensor(q, dtype=dt, device="cuda")
+
+
+@dataclasses.dataclass
+class CompressReport:
+    tokens: int = 0
+    idx_mismatch_in_band: int = 0
+    idx_mismatch_out_of_band: int = 0
+    sign_mismatch_in_band: int = 0
+    sign_mismatch_out_of_band: int = 0
+    sign_tokens_skipped: int = 0
+    norm_fail: int = 0
+
+
+def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport = None):
+    """Compares the GPU's packed (layer, b, h) against the oracle on the same inputs.
+    tokens: optional index array of positions to check (default all)."""
+    rep = rep or CompressReport()
+    n = int(run.lens[b])
+    u = olay.read_sequence(pages, run.fmt, layer, h, run.bt[b], n)
+    sel = np.arange(n) if tokens is None else np.asarray(tokens)
+    K = run.K[layer][b, h][sel]
+    V = run.V[layer][b, h][sel]
+    S = run.rin["s"]
+    kc = (oq.compress_prod(K, run.R, run.ck, run.kb, S) if run.w.key_qjl
+          else oq.compress_mse(K, run.R, run.ck, run.kb))
+    vc = oq.compress_mse(V, run.R, run.cv, run.vb)
+    rep.tokens += len(sel)
+    kmis = _check_idx(u.k_idx[sel], kc, run.kb, rep)
+    _check_idx(u.v_idx[sel], vc, run.vb, rep)
+    rep.norm_fail += int(np.sum(~close(u.k_norm[sel], kc.norm)))
+    rep.norm_fail += int(np.sum(~close(u.v_norm[sel], vc.norm)))
+    if run.w.key_qjl:
+        ok_tok = ~kmis
+        rep.sign_tokens_skipped += int(np.sum(kmis))
+        rep.norm_fail += int(np.sum(~close(u.k_rnorm[sel][ok_tok], kc.rnorm[ok_tok])))
+        diff = (u.k_sigma[sel] != kc.sigma) & ok_tok[:, None]
+        band = np.abs(kc.sr) <= SIGN_BAND * kc.sr_scale
+        rep.sign_mismatch_in_band += int(np.sum(diff & band))
+        rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
+    return rep
+
+
+def _check_idx(gpu_idx, comp, boundaries, rep):
+    diff = gpu_idx != comp.idx
+    dist = np.min(np.abs(comp.y[..., None] - boundaries.astype(np.float64)), axis=-1)
+    band = dist < BOUNDARY_BAND
+    rep.idx_mismatch_in_band += int(np.sum(diff & band))
+    rep.idx_mismatch_out_of_band += int(np.sum(diff & ~band))
+    return np.any(diff, axis=1)
+
+
+def oracle_decode(run, pages, layer, q, heads=None):
+    return oatt.decode(pages, run.fmt, layer, q, run.bt, run.lens, run.R, run.ck, run.cv,
+                       run.rin["s"] if run.w.key_qjl else None, heads=heads)
+
+
+def oracle_scores(run, pages, layer, q, b, h):
+    """Scores of query head h of sequence b over its cached tokens: [seq_q, n]."""
+    G = run.w.group
+    u = olay.read_sequence(pages, run.fmt, layer, h // G, run.bt[b], int(run.lens[b]))
+    k_mse = oq.reconstruct_mse(u.k_idx, u.k_norm, run.R, run.ck)
+    return oatt.scores_compressed(q[b, h], k_mse, u.k_rnorm, u.k_sigma,
+                                  run.rin["s"] if run.w.key_qjl else None)

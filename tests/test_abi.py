@@ -1,0 +1,119 @@
+"""CPU tests of the C ABI: the library loads, exports what include/tq.h declares, and its
+host-only logic (codebook, sizes, argument checks) behaves as documented.  No kernel runs."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def tq():
+    import compressed_decode_attention_tq_b200 as m
+    return m
+
+
+def test_every_declared_symbol_is_exported(tq):
+    declared = _declared_functions()
+    assert set(declared) == set(tq.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", tq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\b(tq_[a-z_0-9]+)\b", out))
+    assert set(declared) <= exported
+    # nothing else leaks out of the library under the tq_ prefix
+    assert exported == set(declared)
+
+
+def test_version_and_status_strings(tq):
+    assert tq.lib.tq_version() >= 100
+    assert tq.status_str(0) == "TQ_OK"
+    assert tq.status_str(6) == "TQ_ERR_BOUNDS"
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("density", [0, 1])
+def test_library_codebook_equals_oracle_codebook(tq, bits, density):
+    from oracle import codebook as ocb
+    c, b = tq.codebook(bits, 128, density)
+    oc, ob = ocb.codebook_f32(bits, 128, "beta" if density == 0 else "gauss")
+    np.testing.assert_array_equal(c, oc)
+    np.testing.assert_array_equal(b, ob)
+
+
+@pytest.mark.parametrize("d", [16, 64])
+def test_library_codebook_other_d(tq, d):
+    from oracle import codebook as ocb
+    c, b = tq.codebook(3, d, 0)
+    oc, ob = ocb.codebook_f32(3, d, "beta")
+    np.testing.assert_array_equal(c, oc)
+    np.testing.assert_array_equal(b, ob)
+
+
+def test_codebook_argument_errors(tq):
+    c = np.zeros(4, np.float32)
+    b = np.zeros(3, np.float32)
+    assert tq.lib.tq_codebook(0, 128, 0, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert "bits" in tq.last_error()
+    assert tq.lib.tq_codebook(2, 2, 0, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_codebook(2, 128, 5, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_codebook(2, 128, 0, None, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_page_bytes_match_format(tq, packing_golden):
+    g = packing_golden["c2_regions"]
+    cfg = tq.make_config(key_bits=3, key_qjl=True, value_bits=3)
+    assert tq.page_bytes(cfg) == g["total"]
+    from oracle import layout as olay
+    for kb in range(1, 5):
+        for vb in range(1, 5):
+            for qjl in (False, True):
+                cfg = tq.make_config(key_bits=kb, key_qjl=qjl, value_bits=vb)
+                fmt = olay.Format(key_bits=kb, key_qjl=qjl, value_bits=vb)
+                assert tq.page_bytes(cfg) == fmt.block_bytes
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 64, 2), ("qjl_m", 64, 2), ("page_tokens", 128, 2), ("key_bits", 5, 2),
+    ("value_bits", 0, 2), ("key_qjl", 2, 1), ("rotation", 7, 1)])
+def test_validate_config_rejects(tq, field, value, code):
+    cfg = tq.make_config()
+    assert tq.validate_config(cfg) == 0
+    setattr(cfg, field, value)
+    assert tq.validate_config(cfg) == code
+    assert tq.page_bytes(cfg) == 0
+
+
+def test_workspace_bytes(tq):
+    cfg = tq.make_config()
+    nb = tq.decode_workspace_bytes(cfg, 1, 32, 1, 16)
+    rows = 32
+    assert nb >= rows * (128 + 128 + 16 * 130) * 4
+    assert nb % 256 == 0
+    assert tq.decode_workspace_bytes(cfg, 1, 32, 1, 0) == 0
+
+
+def test_host_argument_errors_do_not_launch(tq):
+    cfg = tq.make_config()
+    params = tq.tq_params()
+    cache = tq.tq_cache()
+    by = ctypes.byref
+    # null params / cache / tensors are rejected on the host before any CUDA call
+    st = tq.lib.tq_compress_kv(by(cfg), by(params), by(cache), 0, None, None, 0, 16, None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG
+    st = tq.lib.tq_attend_decode(by(cfg), None, by(cache), 0, None, 0, 32, 1, None, 4, None, 0, None,
+                                 None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG
+    assert "params" in tq.last_error()
+    bad = tq.make_config(head_dim=96)
+    st = tq.lib.tq_decompress(by(bad), by(params), by(cache), 0, None, 0, None, None, None, None)
+    assert st == tq.TQ_ERR_UNSUPPORTED

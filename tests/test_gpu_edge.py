@@ -1,0 +1,101 @@
+"""GPU edge cases and device-side error reporting (no test faults or hangs the GPU: every
+failure is a bounds-checked condition the kernels detect and report in dev_status)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+from parity_util import close, oracle_decode, q_dev, setup
+
+
+def _run(w):
+    r = setup(w)
+    r.pages = r.kv.pages_numpy()
+    return r
+
+
+def test_empty_and_single_token_sequences():
+    w = wl.config2(batch=3, kv_heads=1, q_heads=4, max_len=300, n_splits=2)
+    lens = np.array([0, 1, 257], dtype=np.int32)
+    import parity_util as pu
+    orig = wl.seq_lens
+    try:
+        wl.seq_lens = lambda _w: lens
+        r = setup(w)
+    finally:
+        wl.seq_lens = orig
+    r.kv.raise_on_error("compress")
+    r.pages = r.kv.pages_numpy()
+    seq = torch.as_tensor(lens, device="cuda")
+    q, qd = q_dev(r)
+    out = r.kv.decode(0, qd, seq, 4).cpu().numpy()
+    r.kv.raise_on_error("decode")
+    assert np.all(out[0] == 0)
+    ref = oracle_decode(r, r.pages, 0, q)
+    assert close(out, ref).all()
+
+
+def test_sequence_longer_than_page_table_reports_bounds():
+    w = wl.config2(kv_heads=1, q_heads=4, max_len=256, n_splits=1)
+    r = _run(w)
+    r.kv.raise_on_error("compress")
+    seq = torch.tensor([600], dtype=torch.int32, device="cuda")  # 1 page in the table
+    q, qd = q_dev(r)
+    r.kv.decode(0, qd, seq, 1)
+    assert r.kv.check() == 6
+    k = torch.zeros((1, 1, 600, 128), dtype=torch.float16, device="cuda")
+    r.kv.compress(0, k, k, seq)
+    assert r.kv.check() == 6
+
+
+def test_page_id_out_of_range_reports_bounds():
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+    rin = wl.rotation_inputs(wl.config2())
+    kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[5]]), key_bits=3, key_qjl=True,
+                 value_bits=3, signs=rin["signs"], s=rin["s"])
+    k = torch.randn((1, 1, 10, 128), device="cuda").half()
+    seq = torch.tensor([10], dtype=torch.int32, device="cuda")
+    kv.compress(0, k, k, seq)
+    assert kv.check() == 6
+
+
+def test_norm_overflow_reported():
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+    rin = wl.rotation_inputs(wl.config2())
+    kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[0]]), key_bits=3, key_qjl=True,
+                 value_bits=3, signs=rin["signs"], s=rin["s"])
+    k = torch.full((1, 1, 4, 128), 7000.0, device="cuda")  # ||k|| = 79196 > fp16 max
+    seq = torch.tensor([4], dtype=torch.int32, device="cuda")
+    kv.compress(0, k, k, seq)
+    assert kv.check() == 4
+
+
+def test_non_fp16_sketch_matrix_rejected():
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+    rin = wl.rotation_inputs(wl.config2())
+    s = rin["s"].copy()
+    s[3, 5] = 0.1  # not representable in fp16
+    kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[0]]), key_bits=3, key_qjl=True,
+                 value_bits=3, signs=rin["signs"], s=s)
+    k = torch.randn((1, 1, 4, 128), device="cuda").half()
+    kv.compress(0, k, k, torch.tensor([4], dtype=torch.int32, device="cuda"))
+    assert kv.check() == 1
+
+
+def test_zero_vector_compresses_to_zero_norm():
+    from compressed_decode_attention_tq_b200.runtime import PagedKV
+    from oracle import layout as olay
+    rin = wl.rotation_inputs(wl.config2())
+    kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[0]]), key_bits=3, key_qjl=True,
+                 value_bits=2, signs=rin["signs"], s=rin["s"])
+    k = torch.zeros((1, 1, 3, 128), dtype=torch.float16, device="cuda")
+    seq = torch.tensor([3], dtype=torch.int32, device="cuda")
+    kv.compress(0, k, k, seq)
+    assert kv.check() == 0
+    u = olay.read_sequence(kv.pages_numpy(), olay.Format(key_bits=3, value_bits=2), 0, 0, [0], 3)
+    assert np.all(u.k_norm == 0) and np.all(u.v_norm == 0) and np.all(u.k_rnorm == 0)
+    # y = 0 lies on the middle boundary: index h - 1 (tie to the lower cell); sign(0) -> +1
+    assert np.all(u.k_idx == 3) and np.all(u.v_idx == 1) and np.all(u.k_sigma)

@@ -262,3 +262,47 @@ def rotation_inputs(w: Workload) -> dict:
 
 def np_dtype(w: Workload):
     return np.float16 if w.in_dtype == "f16" else np.float32
+
+
+# ---------------------------------------------------------------------------
+# large inputs drawn directly on the device (bench sizes)
+# ---------------------------------------------------------------------------
+
+def make_kv_device(w: Workload, layer: int, device, dtype=None):
+    """K, V [batch][kv_heads][max_len][d] drawn with torch on `device` (same recipe as make_kv,
+    a different random stream): Gaussian times per-(head, channel) log-normal(0, 0.5) scales,
+    optional outlier channels, or Student-t keys.  Used where the host draw would be too slow."""
+    import torch
+    dt = dtype or (torch.float16 if w.in_dtype == "f16" else torch.float32)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.data_seed) * 1000003 + layer)
+    shape = (w.batch, w.kv_heads, w.max_len, HEAD_DIM)
+    if w.kind == "student_t_keys":
+        # Student-t(3) = N / sqrt(chi2_3 / 3), chi2_3 = sum of three squared normals
+        n = torch.randn(shape, generator=g, device=device)
+        chi = sum(torch.randn(shape, generator=g, device=device) ** 2 for _ in range(3))
+        k = n / torch.sqrt(chi / 3.0)
+        v = torch.randn(shape, generator=g, device=device)
+        return k.to(dt), v.to(dt)
+    sk = torch.exp(0.5 * torch.randn((w.kv_heads, HEAD_DIM), generator=g, device=device))
+    sv = torch.exp(0.5 * torch.randn((w.kv_heads, HEAD_DIM), generator=g, device=device))
+    if w.outlier_channels:
+        for h in range(w.kv_heads):
+            ok = torch.randperm(HEAD_DIM, generator=g, device=device)[:w.outlier_channels]
+            ov = torch.randperm(HEAD_DIM, generator=g, device=device)[:w.outlier_channels]
+            sk[h, ok] *= w.outlier_scale
+            sv[h, ov] *= w.outlier_scale
+    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    k.mul_(sk[None, :, None, :])
+    k = k.to(dt)
+    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    v.mul_(sv[None, :, None, :])
+    return k, v.to(dt)
+
+
+def make_q_device(w: Workload, layer: int, device, dtype=None):
+    import torch
+    dt = dtype or (torch.float16 if w.in_dtype == "f16" else torch.float32)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.data_seed) * 7919 + layer + 17)
+    return torch.randn((w.batch, w.q_heads, w.seq_q, HEAD_DIM), generator=g, device=device).to(dt)
