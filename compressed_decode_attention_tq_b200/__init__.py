@@ -31,7 +31,7 @@ TQ_F32 = 1
 # Every function include/tq.h declares.
 EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_validate_config", "tq_page_bytes",
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
-           "tq_decode_scores", "tq_decompress")
+           "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc")
 
 
 class tq_config(ctypes.Structure):
@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "tq_attend_decode": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, SZ, P, P, P]),
         "tq_decode_scores": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, SZ, P, P, P]),
         "tq_decompress": (I32, [cfgp, parp, cachep, I32, P, I32, P, P, P, P]),
+        "tq_attend_decode_noalloc": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -174,6 +175,16 @@ def attend_decode(cfg, params, cache, layer, q, seq_lens, n_splits, workspace, o
                                 _ptr(q), dtype_code(q), q.shape[1], q.shape[2], _ptr(seq_lens),
                                 n_splits, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _ptr(out), _ptr(status), _stream(stream)), "tq_attend_decode")
+
+
+def attend_decode_noalloc(cfg, params, cache, layer, q, seq_lens, n_splits, out, status,
+                          stream=None):
+    """tq_attend_decode without a workspace: the library's built-in 8 MiB device array is
+    used instead, for callers that cannot allocate device memory (see include/tq.h)."""
+    _check(lib.tq_attend_decode_noalloc(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache),
+                                        layer, _ptr(q), dtype_code(q), q.shape[1], q.shape[2],
+                                        _ptr(seq_lens), n_splits, _ptr(out), _ptr(status),
+                                        _stream(stream)), "tq_attend_decode_noalloc")
 
 
 def decode_scores(cfg, params, cache, layer, q, seq_lens, workspace, scores, status, stream=None):

@@ -210,6 +210,28 @@ TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params,
                            void* workspace, size_t workspace_bytes, float* out,
                            int32_t* dev_status, tq_stream_t stream);
 
+/* Decode attention for callers that cannot allocate device memory (no counterpart on
+ * the source pages; it exists for users of this library).  Same computation, arguments
+ * and results as tq_attend_decode, minus the workspace: a plugin inside a runtime that
+ * owns all device memory, or a serving loop that must not call cudaMalloc mid-step, can
+ * call this instead.  The scratch lives in a built-in 8 MiB array in device global
+ * memory that every GPU loading the library holds until the process exits.
+ *   - Sizes whose tq_decode_workspace_bytes(...) exceeds 8 MiB return
+ *     TQ_ERR_UNSUPPORTED with an explanation in tq_last_error(); nothing is enqueued.
+ *   - The first call on each device looks up the array's device address on the host
+ *     (with that device current); make that first call before any stream capture
+ *     begins on the device.
+ *   - All calls on a device share the one array: calls whose kernels can overlap in
+ *     time race and give undefined results.  Order them on a single stream.
+ *   - Nothing in the array needs clearing between calls (every byte read is first
+ *     written by the same call).
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+TQ_API tq_status tq_attend_decode_noalloc(const tq_config* cfg, const tq_params* params,
+                                          const tq_cache* cache, int32_t layer, const void* q,
+                                          int32_t q_dtype, int32_t q_heads, int32_t seq_q,
+                                          const int32_t* seq_lens, int32_t n_splits, float* out,
+                                          int32_t* dev_status, tq_stream_t stream);
+
 /* Score-only decode ([CUTILE] "Score-only kernel ... streams over KV"): writes the
  * scaled scores score_t above for every query row and t < seq_lens[b]; entries with
  * t >= seq_lens[b] are left untouched.
