@@ -43,12 +43,14 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--n-splits", type=int, default=0, help="override the split count")
     return p.parse_args()
 
 
 def workload():
     import workloads as wl
-    return wl.config2()
+    # 32 splits x 8 KV heads = 256 CTAs: every SM busy (2 resident per SM), 4 pages each
+    return wl.config2(n_splits=32)
 
 
 def peaks():
@@ -233,6 +235,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = workload()
+    if args.n_splits:
+        w.n_splits = args.n_splits
     L = args.layers
     rin = wl.rotation_inputs(w)
     lens = wl.seq_lens(w)

@@ -56,7 +56,7 @@ __device__ __forceinline__ void pack_words(const int (&s)[4], const int (&r)[4],
           wout[2 * e + 1] = hi;
         }
         if (bits == 3) {
-          const uint32_t w = __ballot_sync(FULL, s[e]);
+          const uint32_t w = __reduce_or_sync(FULL, (uint32_t)s[e] << (sign_plane_pos(lane) & 31));
           if (lane == 0) wout[8 + e] = w;
         }
       }
@@ -77,16 +77,33 @@ __device__ __forceinline__ void pack_words(const int (&s)[4], const int (&r)[4],
   }
 }
 
+// Merged 3-bit key fields (r0, r1, s, sigma) as 4-bit nibbles, nibble j at bit 4j.
+__device__ __forceinline__ void pack_merged(const int (&s)[4], const int (&r)[4], const int (&sg)[4],
+                                            int lane, uint32_t* wout) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t f = (uint32_t)(r[e] | (s[e] << 2) | (sg[e] << 3));
+    const uint32_t sh = f << (4 * (lane & 7));
+    const int g = lane >> 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w = __reduce_or_sync(FULL, g == q ? sh : 0u);
+      if (lane == 0) wout[4 * e + q] = w;
+    }
+  }
+}
+
 struct VecOut {
   __half norm;
   int idx[4];
+  int s[4], r[4];
 };
 
 // norm, rotation, quantization, packing of one vector (x already loaded).
 __device__ __forceinline__ void encode_vector(const float (&x)[4], int bits, const float* cent,
                                               const float* bnd, const float* signs, const float* pi_s,
                                               float* stage, int lane, uint32_t* wbuf, VecOut& out,
-                                              int32_t* status) {
+                                              int32_t* status, bool defer_pack = false) {
   float ss = 0.f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) ss = fmaf(x[e], x[e], ss);
@@ -126,8 +143,10 @@ __device__ __forceinline__ void encode_vector(const float (&x)[4], int bits, con
     out.idx[e] = idx;
     s[e] = idx >= h;
     r[e] = s[e] ? idx - h : h - 1 - idx;
+    out.s[e] = s[e];
+    out.r[e] = r[e];
   }
-  pack_words(s, r, bits, lane, wbuf);
+  if (!defer_pack) pack_words(s, r, bits, lane, wbuf);
   (void)cent;
 }
 
@@ -195,9 +214,10 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) x[e] = ld_in<T>(kin + row + lane + 32 * e);
     VecOut ko;
-    encode_vector(x, L.kbits, sm.kc, sm.kb, sm.signs, pis, stage, lane, wbuf, ko, a.status);
+    encode_vector(x, L.kbits, sm.kc, sm.kb, sm.signs, pis, stage, lane, wbuf, ko, a.status,
+                  L.kmerged != 0);
     __syncwarp();
-    if (lane < L.kbits)
+    if (!L.kmerged && lane < L.kbits)
       reinterpret_cast<uint4*>(blk + L.kc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
     if (lane == 0) reinterpret_cast<__half*>(blk + L.kn)[slot] = ko.norm;
     if (a.qjl) {
@@ -234,19 +254,28 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) stage[lane + 32 * e] = rr[e];
       __syncwarp();
+      int sg[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float* srow = s_s + (lane + 32 * e) * kPad;
         float acc = 0.f;
         for (int k = 0; k < D; ++k) acc = fmaf(srow[k], stage[k], acc);
-        const uint32_t w = __ballot_sync(FULL, acc >= 0.f);
-        if (lane == 0) wbuf[e] = w;
+        sg[e] = acc >= 0.f;
+        if (!L.kmerged) {
+          const uint32_t w = __ballot_sync(FULL, sg[e]);
+          if (lane == 0) wbuf[e] = w;
+        }
       }
       __syncwarp();
-      if (lane == 0) {
+      if (L.kmerged) {
+        pack_merged(ko.s, ko.r, sg, lane, wbuf);
+        __syncwarp();
+        if (lane < 4)
+          reinterpret_cast<uint4*>(blk + L.kc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
+      } else if (lane == 0) {
         reinterpret_cast<uint4*>(blk + L.ks)[slot] = reinterpret_cast<const uint4*>(wbuf)[0];
-        reinterpret_cast<__half*>(blk + L.kr)[slot] = rho;
       }
+      if (lane == 0) reinterpret_cast<__half*>(blk + L.kr)[slot] = rho;
       __syncwarp();
     }
     // ---- value

@@ -31,51 +31,98 @@ constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------------------
-// prologue: one warp per query row
+// prologue: one CTA of 128 threads per query row.  Thread i owns coordinate i.
+//   qrot = R q (fp32), q8 = int8 rounding of qrot * 127 / max|qrot| (with its scale),
+//   sq = S q (fp32), sq_int = S q in 16-bit fixed point with a power-of-two scale, sum.
 // ---------------------------------------------------------------------------
-__global__ void prologue_kernel(DecodeArgs a, int total_rows) {
-  __shared__ float stage[4][D];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int row = blockIdx.x * 4 + w;
+__device__ __forceinline__ float block_max128(float v, float* red) {
+  v = warp_max(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  return m;
+}
+
+__global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_rows) {
+  // allow the dependent split kernel to start streaming pages right away
+  asm volatile("griddepcontrol.launch_dependents;");
+  __shared__ float qs[D];
+  __shared__ float red[4];
+  __shared__ int ired[4];
+  const int i = threadIdx.x;
+  const int row = blockIdx.x;
   if (row >= total_rows) return;
-  float x[4];
-  if (a.q_dtype == TQ_F16) {
-    const __half* q = reinterpret_cast<const __half*>(a.q) + (size_t)row * D;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = __half2float(q[lane + 32 * e]);
-  } else {
-    const float* q = reinterpret_cast<const float*>(a.q) + (size_t)row * D;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = q[lane + 32 * e];
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) stage[w][lane + 32 * e] = x[e];
-  __syncwarp();
-  float y[4];
+  float x;
+  if (a.q_dtype == TQ_F16)
+    x = __half2float(reinterpret_cast<const __half*>(a.q)[(size_t)row * D + i]);
+  else
+    x = reinterpret_cast<const float*>(a.q)[(size_t)row * D + i];
+  float y;
   if (!a.dense) {
+    // y = H D q / sqrt(d): butterflies in shared memory
+    qs[i] = x * a.signs[i];
+    __syncthreads();
 #pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = x[e] * a.signs[lane + 32 * e];
-    fwht128_warp(y, lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] *= kInvSqrtD;
-  } else {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float* prow = a.pi + (size_t)(lane + 32 * e) * D;
-      float acc = 0.f;
-      for (int k = 0; k < D; ++k) acc = fmaf(prow[k], stage[w][k], acc);
-      y[e] = acc;
+    for (int h = 1; h < D; h <<= 1) {
+      const float u = qs[i], v = qs[i ^ h];
+      __syncthreads();
+      qs[i] = (i & h) ? (v - u) : (u + v);
+      __syncthreads();
     }
+    y = qs[i] * kInvSqrtD;
+    __syncthreads();
+    qs[i] = x;
+    __syncthreads();
+  } else {
+    qs[i] = x;
+    __syncthreads();
+    const float4* prow = reinterpret_cast<const float4*>(a.pi + (size_t)i * D);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 p = prow[k];
+      acc = fmaf(p.x, qs[4 * k], acc);
+      acc = fmaf(p.y, qs[4 * k + 1], acc);
+      acc = fmaf(p.z, qs[4 * k + 2], acc);
+      acc = fmaf(p.w, qs[4 * k + 3], acc);
+    }
+    y = acc;
   }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) a.qrot[(size_t)row * D + lane + 32 * e] = y[e];
+  a.qrot[(size_t)row * D + i] = y;
+  const float ym = block_max128(fabsf(y), red);
+  const float lam = ym > 0.f ? 127.f / ym : 0.f;
+  a.q8[(size_t)row * D + i] = (int8_t)__float2int_rn(y * lam);
+  if (i == 0) a.q8_scale[row] = lam;
   if (a.qjl) {
+    const float4* srow = reinterpret_cast<const float4*>(a.s + (size_t)i * D);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 p = srow[k];
+      acc = fmaf(p.x, qs[4 * k], acc);
+      acc = fmaf(p.y, qs[4 * k + 1], acc);
+      acc = fmaf(p.z, qs[4 * k + 2], acc);
+      acc = fmaf(p.w, qs[4 * k + 3], acc);
+    }
+    a.sq[(size_t)row * QM + i] = acc;
+    const float mx = block_max128(fabsf(acc), red);
+    // 16-bit fixed point with a power-of-two scale: |sq_int| <= 32000
+    int ex = 0;
+    if (mx > 0.f) {
+      frexpf(32000.f / mx, &ex);
+      ex -= 1;  // 2^ex <= 32000 / mx
+    }
+    const int v = __float2int_rn(acc * ldexpf(1.f, ex));
+    a.sq_int[(size_t)row * QM + i] = (int16_t)v;
+    int sum = v;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float* srow = a.s + (size_t)(lane + 32 * e) * D;
-      float acc = 0.f;
-      for (int k = 0; k < D; ++k) acc = fmaf(srow[k], stage[w][k], acc);
-      a.sq[(size_t)row * QM + lane + 32 * e] = acc;
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
+    if ((i & 31) == 0) ired[i >> 5] = sum;
+    __syncthreads();
+    if (i == 0) {
+      a.sq_scale[row] = ldexpf(1.f, -ex);
+      a.sq_sum[row] = ired[0] + ired[1] + ired[2] + ired[3];
     }
   }
 }
@@ -151,16 +198,18 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     }
     if (valid) {
       uint32_t kw[16];
-      for (int c = 0; c < L.kbits; ++c) {
+      for (int c = 0; c < L.kchunks; ++c) {
         const uint4 v4 = reinterpret_cast<const uint4*>(blk + L.kc)[c * PT + slot];
         kw[4 * c] = v4.x; kw[4 * c + 1] = v4.y; kw[4 * c + 2] = v4.z; kw[4 * c + 3] = v4.w;
       }
       float dot[kRowsMax];
 #pragma unroll
       for (int r = 0; r < kRowsMax; ++r) dot[r] = 0.f;
+      uint32_t sw[4] = {0u, 0u, 0u, 0u};
       for (int j = 0; j < D; ++j) {
-        int s, rk;
-        code_fields(kw, L.kbits, j, s, rk);
+        int s, rk, sig;
+        key_fields(kw, L, j, s, rk, sig);
+        sw[j >> 5] |= (uint32_t)sig << (j & 31);
         const float val = s ? sm.kmag[rk] : -sm.kmag[rk];
 #pragma unroll
         for (int r = 0; r < kRowsMax; ++r)
@@ -172,8 +221,10 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       for (int r = 0; r < kRowsMax; ++r) qj[r] = 0.f;
       float rho = 0.f;
       if (L.qjl) {
-        const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.ks)[slot];
-        const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
+        if (!L.kmerged) {
+          const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.ks)[slot];
+          sw[0] = s4.x; sw[1] = s4.y; sw[2] = s4.z; sw[3] = s4.w;
+        }
         rho = __half2float(reinterpret_cast<const __half*>(blk + L.kr)[slot]);
         for (int i = 0; i < QM; ++i) {
           if ((sw[i >> 5] >> (i & 31)) & 1u) {
@@ -268,49 +319,51 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// combine: one warp per query row
+// combine: one CTA of 128 threads per query row, thread j owns coordinate j
 // ---------------------------------------------------------------------------
-__global__ void combine_kernel(DecodeArgs a, int total_rows) {
-  __shared__ float stage[4][D];
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int row = blockIdx.x * 4 + w;
+__global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int total_rows) {
+  // wait for the split kernel (launched as our programmatic predecessor) to finish
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float os[D];
+  const int j = threadIdx.x;
+  const int row = blockIdx.x;
   if (row >= total_rows) return;
+  const float* ml = a.part_ml + (size_t)row * a.n_splits * 2;
+  const float* pa = a.part_acc + (size_t)row * a.n_splits * D;
   float M = -CUDART_INF_F;
-  for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, a.part_ml[((size_t)row * a.n_splits + s) * 2]);
-  float l = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, ml[2 * s]);
+  float l = 0.f, o = 0.f;
   if (M != -CUDART_INF_F) {
     for (int s = 0; s < a.n_splits; ++s) {
-      const size_t pr = (size_t)row * a.n_splits + s;
-      const float ms = a.part_ml[pr * 2];
+      const float ms = ml[2 * s];
       if (ms == -CUDART_INF_F) continue;
       const float wgt = __expf(ms - M);
-      l = fmaf(wgt, a.part_ml[pr * 2 + 1], l);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = fmaf(wgt, a.part_acc[pr * D + lane + 32 * e], o[e]);
+      l = fmaf(wgt, ml[2 * s + 1], l);
+      o = fmaf(wgt, pa[(size_t)s * D + j], o);
     }
   }
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) o[e] *= inv;
-  float y[4];
+  o = l > 0.f ? o / l : 0.f;
+  float y;
   if (!a.dense) {
-    // R^T = D H
-    fwht128_warp(o, lane);
+    // R^T = D H: butterflies in shared memory, then the sign flips
+    os[j] = o;
+    __syncthreads();
 #pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = o[e] * kInvSqrtD * a.signs[lane + 32 * e];
-  } else {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) stage[w][lane + 32 * e] = o[e];
-    __syncwarp();
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float acc = 0.f;
-      for (int i = 0; i < D; ++i) acc = fmaf(a.pi[(size_t)i * D + lane + 32 * e], stage[w][i], acc);
-      y[e] = acc;
+    for (int h = 1; h < D; h <<= 1) {
+      const float u = os[j], v = os[j ^ h];
+      __syncthreads();
+      os[j] = (j & h) ? (v - u) : (u + v);
+      __syncthreads();
     }
+    y = os[j] * kInvSqrtD * a.signs[j];
+  } else {
+    os[j] = o;
+    __syncthreads();
+    float acc = 0.f;
+    for (int i = 0; i < D; ++i) acc = fmaf(a.pi[(size_t)i * D + j], os[i], acc);
+    y = acc;
   }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) a.out[(size_t)row * D + lane + 32 * e] = y[e];
+  a.out[(size_t)row * D + j] = y;
 }
 
 }  // namespace
@@ -323,6 +376,11 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   w.sq = off; off = align256(off + rows * QM * sizeof(float));
   w.part_acc = off; off = align256(off + rows * (size_t)n_splits * D * sizeof(float));
   w.part_ml = off; off = align256(off + rows * (size_t)n_splits * 2 * sizeof(float));
+  w.sq_int = off; off = align256(off + rows * QM * sizeof(int16_t));
+  w.sq_scale = off; off = align256(off + rows * sizeof(float));
+  w.sq_sum = off; off = align256(off + rows * sizeof(int));
+  w.q8 = off; off = align256(off + rows * D);
+  w.q8_scale = off; off = align256(off + rows * sizeof(float));
   w.total = off;
   return w;
 }
@@ -344,20 +402,40 @@ static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream, bool s
   return cudaGetLastError();
 }
 
+// Launch with programmatic stream serialization: the kernel may start while its
+// predecessor on the stream is still running and waits (griddepcontrol.wait) before it
+// reads the predecessor's results.
+template <typename... Args>
+static cudaError_t launch_pdl(void (*k)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
-  prologue_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = launch_split(a, stream, false);
+  e = fast_decode_supported(a) ? launch_fast_split(a, stream) : launch_split(a, stream, false);
   if (e != cudaSuccess) return e;
-  combine_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  e = launch_pdl(combine_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream) {
   const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
-  prologue_kernel<<<(total_rows + 3) / 4, 128, 0, stream>>>(a, total_rows);
+  prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_split(a, stream, true);

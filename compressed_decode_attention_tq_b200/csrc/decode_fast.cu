@@ -1,0 +1,647 @@
+// Tensor-core split-KV decode over the packed cache.
+//
+// Same computation as the generic split kernel in decode.cu ("turboquant_cutile" function
+// list: asymmetric estimator + online softmax + on-chip V; "TurboQuant explained",
+// section "How is this different from PolarQuant's reconstruction?": pre-rotated
+// query), organised for B200:
+//
+//  * one producer warp streams each page of the split into a 3-stage shared-memory ring
+//    with bulk asynchronous copies (cp.async.bulk, completion on mbarriers);
+//  * four consumer warps each take 16-token steps.  A lane dequantises codes straight
+//    into fp16 mma fragments with byte permutes against a centroid table held in
+//    registers; the key term  sum_j (R q)_j c[idx_j]  is an fp16 m16n8k16 mma (query in
+//    hi+lo fp16 halves, fp32 accumulation), the QJL term  sum_i (S q)_i sigma_i  an int8
+//    m16n8k32 mma on 16-bit fixed-point (S q) digits, and  sum_t p_t ||v_t|| c[idx]  an
+//    fp16 mma after an in-register 8x8 transpose (movmatrix) of the dequantised values;
+//  * online softmax per warp, then a log-sum-exp merge of the four warps; the partial
+//    (m, l, acc) per query row goes to the workspace for the combine kernel.
+//
+// Supported here: query rows per KV head R = G * seq_q <= 4, keys 3-bit + QJL (merged
+// nibbles) or 2-bit + QJL, values 3-bit or 2-bit.  Everything else uses decode.cu.
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include "tq_device.cuh"
+#include "tq_kernels.h"
+
+namespace tqk {
+
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStages = 3;
+constexpr int kChunkStride = PT * 16 + 32;  // padded so the 4 lanes of a token group hit distinct banks
+constexpr int kNormBytes = 3 * PT * 2;      // KN | KR | VN
+constexpr int kMaxKChunks = 4;
+constexpr int kMaxVChunks = 3;
+constexpr int kStageBytes = kNormBytes + (kMaxKChunks + kMaxVChunks) * kChunkStride;
+constexpr long long kWaitLimit = 1ll << 26;  // bounded mbarrier waits
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kInvSqrtD = 0.08838834764831845f;
+constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
+
+enum KPol { K3Q = 0, K2Q = 1 };
+enum VPol { V3 = 0, V2 = 1 };
+
+struct SmemFast {
+  unsigned char stage[kStages][kStageBytes];
+  unsigned long long full[kStages];
+  unsigned long long empty[kStages];
+  float wacc[kConsumerWarps][4][D];
+  float wm[kConsumerWarps][4], wl[kConsumerWarps][4];
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait on the given phase parity; false if it gave up.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  for (long long it = 0; it < kWaitLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(s));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+__device__ __forceinline__ void hmma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                     uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                     uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint16_t h_bits(float v) {
+  const __half h = __float2half_rn(v);
+  return *reinterpret_cast<const uint16_t*>(&h);
+}
+
+__device__ __forceinline__ float ld_h(const unsigned char* p) {
+  return __half2float(*reinterpret_cast<const __half*>(p));
+}
+
+// Byte tables for fp16 values: lo bytes of 4 entries in one word, hi bytes in another.
+__device__ __forceinline__ void table4(const float (&v)[4], uint32_t& lo, uint32_t& hi) {
+  lo = hi = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t b = h_bits(v[i]);
+    lo |= (uint32_t)(b & 0xff) << (8 * i);
+    hi |= (uint32_t)(b >> 8) << (8 * i);
+  }
+}
+
+// Coordinates (within the lane's quarter of 32) of crumb pair cb: (base, base + 4).
+__device__ __forceinline__ int pair_base(int cb) { return 8 * (cb >> 2) + (cb & 3); }
+
+// The two 2-bit fields of crumb pair cb of a quarter, from its crumb words c0 (coords 0..15)
+// and c1 (16..31), placed at bits 0-1 and 8-9, turned into a byte-permute selector that
+// picks [lo, hi] of entry f from a (lo-bytes, hi-bytes) table pair.
+__device__ __forceinline__ uint32_t crumb_t(uint32_t c0, uint32_t c1, int cb) {
+  const uint32_t w = (cb < 8) ? c0 : c1;
+  const int s = 2 * (cb & 3) + 16 * ((cb >> 2) & 1);
+  return (s == 0 ? w : __umulhi(w, 1u << (32 - s))) & 0x0303u;
+}
+
+__device__ __forceinline__ uint32_t crumb_sel(uint32_t c0, uint32_t c1, int cb) {
+  return crumb_t(c0, c1, cb) * 0x11u + 0x4040u;
+}
+
+// Selector of the int8 residual codes of crumb pairs n and n+1: bytes (a_n, a_n+1, b_n, b_n+1).
+__device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int n) {
+  const uint32_t t1 = crumb_t(c0, c1, n), t2 = crumb_t(c0, c1, n + 1);
+  return (t1 & 0x3u) | ((t2 & 0x3u) << 4) | (t1 & 0x300u) | ((t2 & 0x300u) << 4);
+}
+
+template <int KP, int VP>
+__global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  SmemFast& sm = *reinterpret_cast<SmemFast*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, gh = blockIdx.y, b = blockIdx.z;
+  const Layout& L = a.cache.L;
+  const int R = a.rows;
+  const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q;
+
+  const int len = a.seq_lens[b];
+  const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
+  if (bad_len && tid == 0 && split == 0) report(a.status, TQ_ERR_BOUNDS);
+  const int n_eff = bad_len ? 0 : len;
+  const int npages_all = (n_eff + PT - 1) / PT;
+  const int cp = (npages_all + a.n_splits - 1) / a.n_splits;
+  const int p_begin = min(npages_all, split * cp);
+  const int p_end = min(npages_all, (split + 1) * cp);
+  const int npages = p_end - p_begin;
+  const int t_end = min(n_eff, p_end * PT);
+
+  constexpr int kKChunks = (KP == K3Q) ? 4 : 3;  // K2Q: 2 code chunks + the KS chunk
+  constexpr int kVChunks = (VP == V3) ? 3 : 2;
+  const uint32_t page_bytes = kNormBytes + 16u * PT * (kKChunks + kVChunks);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kConsumerWarps);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      for (int i = 0; i < npages; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1)) {
+          report(a.status, TQ_ERR_TIMEOUT);
+          break;
+        }
+        int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + p_begin + i];
+        if (phys < 0 || phys >= a.cache.num_pages) {
+          report(a.status, TQ_ERR_BOUNDS);
+          phys = 0;
+        }
+        const unsigned char* blk = a.cache.block(phys, gh);
+        unsigned char* st = sm.stage[s];
+        mbar_expect_tx(&sm.full[s], page_bytes);
+        bulk_g2s(st, blk, kNormBytes, &sm.full[s]);
+        unsigned char* kc = st + kNormBytes;
+        const int kcode_chunks = (KP == K3Q) ? 4 : 2;
+        for (int c = 0; c < kcode_chunks; ++c)
+          bulk_g2s(kc + c * kChunkStride, blk + L.kc + c * PT * 16, PT * 16, &sm.full[s]);
+        if (KP == K2Q) bulk_g2s(kc + 2 * kChunkStride, blk + L.ks, PT * 16, &sm.full[s]);
+        unsigned char* vc = kc + kMaxKChunks * kChunkStride;
+        for (int c = 0; c < kVChunks; ++c)
+          bulk_g2s(vc + c * kChunkStride, blk + L.vc + c * PT * 16, PT * 16, &sm.full[s]);
+      }
+    }
+  } else {
+    // ---------------- consumers ----------------
+    const int g = lane >> 2, t4 = lane & 3;
+    // centroid tables
+    uint32_t kt_lo0 = 0, kt_lo1 = 0, kt_hi0 = 0, kt_hi1 = 0, vt_lo = 0, vt_hi = 0;
+    {
+      const int hk = 1 << (L.kbits - 1), hv = 1 << (L.vbits - 1);
+      if (KP == K3Q) {
+        // stored code (r0, r1, s) -> index r + 4 s; value s ? +a[r] : -a[r]
+        float neg[4], pos[4];
+        for (int r = 0; r < 4; ++r) {
+          pos[r] = a.k_centroids[hk + r];
+          neg[r] = -pos[r];
+        }
+        table4(neg, kt_lo0, kt_hi0);
+        table4(pos, kt_lo1, kt_hi1);
+      } else {
+        // stored code (r0, s) -> f = r0 + 2 s; value s ? +a[r0] : -a[r0]
+        float t[4] = {-a.k_centroids[hk], -a.k_centroids[hk + 1], a.k_centroids[hk], a.k_centroids[hk + 1]};
+        table4(t, kt_lo0, kt_hi0);
+      }
+      if (VP == V3) {
+        // negative magnitudes: a set sign bit (s = 1, the positive half) flips them to +a[r]
+        float t[4] = {-a.v_centroids[hv], -a.v_centroids[hv + 1], -a.v_centroids[hv + 2], -a.v_centroids[hv + 3]};
+        table4(t, vt_lo, vt_hi);
+      } else {
+        float t[4] = {-a.v_centroids[hv], -a.v_centroids[hv + 1], a.v_centroids[hv], a.v_centroids[hv + 1]};
+        table4(t, vt_lo, vt_hi);
+      }
+    }
+    // fp16 rounding residual of the key centroids, eps = c - fp16(c), as int8 codes scaled by
+    // eps_up (a power of two); the correction term sum_j q_j eps_j restores fp32 centroids
+    uint32_t et0 = 0, et1 = 0;
+    float eps_up = 1.f;
+    {
+      const int hk = 1 << (L.kbits - 1);
+      float e8[8];
+      int n = 0;
+      if (KP == K3Q) {
+        for (int i = 0; i < 8; ++i) {
+          const float c = (i >= 4) ? a.k_centroids[hk + (i & 3)] : -a.k_centroids[hk + (i & 3)];
+          e8[i] = c - __half2float(__float2half_rn(c));
+        }
+        n = 8;
+      } else {
+        const float c4[4] = {-a.k_centroids[hk], -a.k_centroids[hk + 1], a.k_centroids[hk], a.k_centroids[hk + 1]};
+        for (int i = 0; i < 4; ++i) e8[i] = c4[i] - __half2float(__float2half_rn(c4[i]));
+        for (int i = 4; i < 8; ++i) e8[i] = 0.f;
+        n = 4;
+      }
+      float emax = 0.f;
+      for (int i = 0; i < n; ++i) emax = fmaxf(emax, fabsf(e8[i]));
+      int ex = 0;
+      if (emax > 0.f) {
+        frexpf(127.f / emax, &ex);
+        ex -= 1;
+      }
+      eps_up = ldexpf(1.f, ex);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t v = (uint32_t)(__float2int_rn(e8[i] * eps_up) & 255);
+        if (i < 4) et0 |= v << (8 * i);
+        else et1 |= v << (8 * (i - 4));
+      }
+    }
+    // the prologue (our programmatic predecessor) must be done before its outputs are read
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // this lane's 32-coordinate slices of row g/2: rotated query, its int8 copy, 16-bit S q
+    const int fr = g >> 1;
+    const bool frow = fr < R;
+    float qv[32];
+    int q8v[32], sqv[32];
+    {
+      const size_t rr = row0 + (frow ? fr : 0);
+      const float4* qp = reinterpret_cast<const float4*>(a.qrot + rr * D + 32 * t4);
+      const int4* q8p = reinterpret_cast<const int4*>(a.q8 + rr * D + 32 * t4);
+      const int4* sqp = reinterpret_cast<const int4*>(a.sq_int + rr * QM + 32 * t4);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 f = frow ? qp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+        qv[4 * k] = f.x; qv[4 * k + 1] = f.y; qv[4 * k + 2] = f.z; qv[4 * k + 3] = f.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int4 v = frow ? q8p[k] : make_int4(0, 0, 0, 0);
+        const int w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int bb = 0; bb < 4; ++bb) q8v[16 * k + 4 * u + bb] = (int)(int8_t)((w4[u] >> (8 * bb)) & 255);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int4 v = frow ? sqp[k] : make_int4(0, 0, 0, 0);
+        const int w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          sqv[8 * k + 2 * u] = (int)(int16_t)(w4[u] & 0xffff);
+          sqv[8 * k + 2 * u + 1] = (int)(int16_t)((uint32_t)w4[u] >> 16);
+        }
+      }
+    }
+    // B fragments of the key term: column g = (row g/2, hi or lo half)
+    uint32_t bq[8][2];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int c;  // quarter-local coordinate of B row (ks, e)
+        if (KP == K3Q) {
+          c = 4 * ks + e;
+        } else {
+          const int n = 2 * ks + (e >> 1);  // half2 index: word n/8, pair n%8
+          c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (e & 1);
+        }
+        const float x = qv[c];
+        const float hi = __half2float(__float2half_rn(x));
+        v[e] = (g & 1) ? (x - hi) : hi;
+      }
+      bq[ks][0] = pack_h2(v[0], v[1]);
+      bq[ks][1] = pack_h2(v[2], v[3]);
+    }
+    // B fragments of the centroid correction: int8 R q in column 2r (odd columns zero)
+    uint32_t bc[4][2];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int c;  // quarter-local coordinate of byte i of correction register (w, h)
+          if (KP == K3Q) {
+            c = 8 * w + 4 * h + i;
+          } else {
+            // register (w, h) holds pairs n = 4w + 2h and 4w + 2h + 1: bytes (a1, a2, b1, b2)
+            const int n = 4 * w + 2 * h + (i & 1);
+            c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (i >> 1);
+          }
+          const int v = (g & 1) ? 0 : q8v[c];
+          word |= (uint32_t)(v & 255) << (8 * i);
+        }
+        bc[w][h] = word;
+      }
+    }
+    // B fragments of the QJL term: column g = (row g/2, digit g%2) of 16-bit (S q)
+    uint32_t bs[4][2];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          int c;  // quarter-local QJL index of byte i of register (w, h)
+          if (KP == K3Q)
+            c = 8 * w + 2 * i + h;
+          else
+            c = 8 * i + 7 - (2 * w + h);
+          const int v = sqv[c];
+          const int d0 = ((v + 128) & 255) - 128;
+          const int d1 = (v - d0) >> 8;
+          word |= (uint32_t)(((g & 1) ? d1 : d0) & 255) << (8 * i);
+        }
+        bs[w][h] = word;
+      }
+    }
+    // per-row constants of the lane's own score row t4
+    int T_row = 0;
+    float c_row_k = 0.f, c_row_q = 0.f, corr_down = 0.f;
+    if (t4 < R) {
+      T_row = a.sq_sum[row0 + t4];
+      c_row_k = kInvSqrtD * kLog2e;
+      c_row_q = kQjlScale * a.sq_scale[row0 + t4] * kInvSqrtD * kLog2e;
+      const float lam = a.q8_scale[row0 + t4];
+      corr_down = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
+    }
+
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    float acc[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+
+    for (int i = 0; i < npages; ++i) {
+      const int s = i % kStages;
+      if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
+        if (lane == 0) report(a.status, TQ_ERR_TIMEOUT);
+        break;
+      }
+      const unsigned char* st = sm.stage[s];
+      const unsigned char* kc = st + kNormBytes;
+      const unsigned char* vc = kc + kMaxKChunks * kChunkStride;
+      const int tok0 = (p_begin + i) * PT;
+      const int valid = min(PT, t_end - tok0);
+      for (int step = warp; step * 16 < valid; step += kConsumerWarps) {
+        const int ta = step * 16 + g, tb = ta + 8;
+        // ---- keys: dequantise into fp16 A fragments and int8 sign fragments
+        uint32_t ha[16], hb[16], sa[8], sb[8], ea[8], eb[8];
+        if (KP == K3Q) {
+          const uint4 wa = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + ta * 16);
+          const uint4 wb = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + tb * 16);
+          const uint32_t A4[4] = {wa.x, wa.y, wa.z, wa.w}, B4[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int side = 0; side < 2; ++side) {
+              const uint32_t W = side ? B4[w] : A4[w];
+              uint32_t* h = side ? hb : ha;
+              uint32_t* sg = side ? sb : sa;
+              uint32_t* ep = side ? eb : ea;
+              const uint32_t s0 = W & 0x7777u;
+              const uint32_t s1 = __umulhi(W, 1u << 16) & 0x7777u;
+              ep[2 * w + 0] = prmt(et0, et1, s0);
+              ep[2 * w + 1] = prmt(et0, et1, s1);
+              const uint32_t l0 = prmt(kt_lo0, kt_lo1, s0), h0 = prmt(kt_hi0, kt_hi1, s0);
+              const uint32_t l1 = prmt(kt_lo0, kt_lo1, s1), h1 = prmt(kt_hi0, kt_hi1, s1);
+              h[4 * w + 0] = prmt(l0, h0, 0x5140);
+              h[4 * w + 1] = prmt(l0, h0, 0x7362);
+              h[4 * w + 2] = prmt(l1, h1, 0x5140);
+              h[4 * w + 3] = prmt(l1, h1, 0x7362);
+              sg[2 * w + 0] = (W << 4) & 0x80808080u;
+              sg[2 * w + 1] = W & 0x80808080u;
+            }
+          }
+        } else {
+          const unsigned char* kq = kc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
+          const uint2 ca = *reinterpret_cast<const uint2*>(kq + ta * 16);
+          const uint2 cbv = *reinterpret_cast<const uint2*>(kq + tb * 16);
+          const uint32_t sA = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + ta * 16 + 4 * t4);
+          const uint32_t sB = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + tb * 16 + 4 * t4);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            ha[n] = prmt(kt_lo0, kt_hi0, crumb_sel(ca.x, ca.y, n));
+            hb[n] = prmt(kt_lo0, kt_hi0, crumb_sel(cbv.x, cbv.y, n));
+          }
+#pragma unroll
+          for (int n = 0; n < 16; n += 2) {
+            // pairs n, n+1 -> int8 residual codes (a_n, a_n+1, b_n, b_n+1)
+            ea[n >> 1] = prmt(et0, et1, crumb_pair_sel(ca.x, ca.y, n));
+            eb[n >> 1] = prmt(et0, et1, crumb_pair_sel(cbv.x, cbv.y, n));
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            sa[k] = (sA << k) & 0x80808080u;
+            sb[k] = (sB << k) & 0x80808080u;
+          }
+        }
+        float dk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
+        int dsum[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
+        int dcor[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
+        // ---- scores of row t4 for tokens ta, tb (log2 domain)
+        const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
+        const float rA = ld_h(st + 2 * PT + 2 * ta), rB = ld_h(st + 2 * PT + 2 * tb);
+        const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
+        const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
+        const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
+        float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row) * c_row_q;
+        float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row) * c_row_q;
+        if (t4 >= R || ta >= valid) sca = -CUDART_INF_F;
+        if (t4 >= R || tb >= valid) scb = -CUDART_INF_F;
+        float mx = fmaxf(sca, scb);
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+        const float m_new = fmaxf(m_run, mx);
+        float alpha = 1.f, pa = 0.f, pb = 0.f;
+        if (m_new != -CUDART_INF_F) {
+          alpha = exp2f(m_run - m_new);
+          pa = exp2f(sca - m_new);
+          pb = exp2f(scb - m_new);
+        }
+        l_run = l_run * alpha + pa + pb;
+        m_run = m_new;
+        const float vnA = ld_h(st + 4 * PT + 2 * ta), vnB = ld_h(st + 4 * PT + 2 * tb);
+        // slots past the end may hold stale bytes: force their weight to exactly 0
+        const uint32_t pk = pack_h2(ta < valid ? pa * vnA : 0.f, tb < valid ? pb * vnB : 0.f);
+        const uint32_t x1 = __shfl_sync(FULL, pk, 4 * (2 * t4) + g);
+        const uint32_t x2 = __shfl_sync(FULL, pk, 4 * (2 * t4 + 1) + g);
+        const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
+        const float al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
+        const float al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
+        // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
+        uint32_t va[16], vb[16];
+        {
+          const unsigned char* vq = vc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
+          const uint2 ca = *reinterpret_cast<const uint2*>(vq + ta * 16);
+          const uint2 cbv = *reinterpret_cast<const uint2*>(vq + tb * 16);
+          uint32_t sgA = 0, sgB = 0;
+          if (VP == V3) {
+            sgA = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + ta * 16 + 4 * t4);
+            sgB = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + tb * 16 + 4 * t4);
+          }
+#pragma unroll
+          for (int cb = 0; cb < 16; ++cb) {
+            uint32_t xa = prmt(vt_lo, vt_hi, crumb_sel(ca.x, ca.y, cb));
+            uint32_t xb = prmt(vt_lo, vt_hi, crumb_sel(cbv.x, cbv.y, cb));
+            if (VP == V3) {
+              xa ^= (sgA << (15 - cb)) & 0x80008000u;
+              xb ^= (sgB << (15 - cb)) & 0x80008000u;
+            }
+            va[cb] = movm_t(xa);
+            vb[cb] = movm_t(xb);
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          acc[mt][0] *= al0;
+          acc[mt][1] *= al1;
+          acc[mt][2] *= al0;
+          acc[mt][3] *= al1;
+          hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+    // ---- warp partial: l summed over the 8 lanes of a row, acc scattered by coordinate
+    l_run += __shfl_xor_sync(FULL, l_run, 4);
+    l_run += __shfl_xor_sync(FULL, l_run, 8);
+    l_run += __shfl_xor_sync(FULL, l_run, 16);
+    if (g == 0 && t4 < R) {
+      sm.wm[warp][t4] = m_run;
+      sm.wl[warp][t4] = l_run;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = 2 * t4 + (e & 1);
+        const int cb = 2 * mt + (e >> 1);
+        const int coord = 32 * (g >> 1) + pair_base(cb) + 4 * (g & 1);
+        if (row < R) sm.wacc[warp][row][coord] = acc[mt][e];
+      }
+    }
+  }
+  __syncthreads();
+  // ---- merge the consumer warps and write this split's partial
+  for (int idx = tid; idx < R * D; idx += blockDim.x) {
+    const int r = idx / D, j = idx % D;
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][r]);
+    float l = 0.f, o = 0.f;
+    if (M != -CUDART_INF_F) {
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float mw = sm.wm[w][r];
+        if (mw == -CUDART_INF_F) continue;
+        const float f = exp2f(mw - M);
+        l = fmaf(f, sm.wl[w][r], l);
+        o = fmaf(f, sm.wacc[w][r][j], o);
+      }
+    }
+    const size_t pr = (row0 + r) * a.n_splits + split;
+    a.part_acc[pr * D + j] = o;
+    if (j == 0) {
+      // partials are kept in the natural-log domain for the combine kernel
+      a.part_ml[pr * 2] = (M == -CUDART_INF_F) ? M : M / kLog2e;
+      a.part_ml[pr * 2 + 1] = l;
+    }
+  }
+}
+
+}  // namespace
+
+bool fast_decode_supported(const DecodeArgs& a) {
+  const Layout& L = a.cache.L;
+  if (a.rows > 4) return false;
+  const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl);
+  const bool vok = L.vbits == 3 || L.vbits == 2;
+  return kok && vok;
+}
+
+size_t fast_decode_smem_bytes() { return sizeof(SmemFast); }
+
+cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
+  const Layout& L = a.cache.L;
+  const size_t smem = sizeof(SmemFast);
+  dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch);
+  void (*k)(DecodeArgs) = nullptr;
+  if (L.kbits == 3 && L.vbits == 3) k = fast_split_kernel<K3Q, V3>;
+  if (L.kbits == 3 && L.vbits == 2) k = fast_split_kernel<K3Q, V2>;
+  if (L.kbits == 2 && L.vbits == 3) k = fast_split_kernel<K2Q, V3>;
+  if (L.kbits == 2 && L.vbits == 2) k = fast_split_kernel<K2Q, V2>;
+  if (!k) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  // programmatic launch: page streaming starts while the prologue is still running
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace tqk

@@ -15,11 +15,12 @@ namespace {
 
 constexpr float kInvSqrtD = 0.08838834764831845f;
 
-__device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, int bits, int slot,
-                              const float* cent, const float* signs, const float* pi, float* stage,
-                              int lane, float* dst) {
+__device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, int bits, int merged,
+                              int slot, const float* cent, const float* signs, const float* pi,
+                              float* stage, int lane, float* dst) {
   uint32_t w[16];
-  for (int c = 0; c < bits; ++c) {
+  const int chunks = merged ? 4 : bits;
+  for (int c = 0; c < chunks; ++c) {
     const uint4 v4 = reinterpret_cast<const uint4*>(blk + code_off)[c * PT + slot];
     w[4 * c] = v4.x; w[4 * c + 1] = v4.y; w[4 * c + 2] = v4.z; w[4 * c + 3] = v4.w;
   }
@@ -28,7 +29,14 @@ __device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, in
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     int s, r;
-    code_fields(w, bits, lane + 32 * e, s, r);
+    if (merged) {
+      const int j = lane + 32 * e;
+      const uint32_t f = (w[j >> 3] >> ((j & 7) * 4)) & 15u;
+      r = f & 3;
+      s = (f >> 2) & 1;
+    } else {
+      code_fields(w, bits, lane + 32 * e, s, r);
+    }
     z[e] = s ? cent[h + r] : -cent[h + r];
   }
   const float n = __half2float(reinterpret_cast<const __half*>(blk + norm_off)[slot]);
@@ -72,10 +80,10 @@ __global__ void decompress_kernel(DecompressArgs a) {
   const Layout& L = a.cache.L;
   const float* pi = a.dense ? a.pi : nullptr;
   if (a.k_hat)
-    decode_vector(blk, L.kc, L.kn, L.kbits, slot, a.k_centroids, a.signs, pi, stage[w], lane,
+    decode_vector(blk, L.kc, L.kn, L.kbits, L.kmerged, slot, a.k_centroids, a.signs, pi, stage[w], lane,
                   a.k_hat + row);
   if (a.v_hat)
-    decode_vector(blk, L.vc, L.vn, L.vbits, slot, a.v_centroids, a.signs, pi, stage[w], lane,
+    decode_vector(blk, L.vc, L.vn, L.vbits, 0, slot, a.v_centroids, a.signs, pi, stage[w], lane,
                   a.v_hat + row);
 }
 

@@ -185,6 +185,11 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.sq = reinterpret_cast<float*>(ws + w.sq);
   a.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
   a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  a.sq_int = reinterpret_cast<int16_t*>(ws + w.sq_int);
+  a.sq_scale = reinterpret_cast<float*>(ws + w.sq_scale);
+  a.sq_sum = reinterpret_cast<int*>(ws + w.sq_sum);
+  a.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
+  a.q8_scale = reinterpret_cast<float*>(ws + w.q8_scale);
   a.out = nullptr;
   a.scores = nullptr;
   a.max_len = 0;

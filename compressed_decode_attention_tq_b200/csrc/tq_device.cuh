@@ -18,6 +18,8 @@ constexpr unsigned FULL = 0xffffffffu;
 struct Layout {
   int kn, kr, vn, kc, ks, vc, bytes;
   int kbits, vbits, qjl;
+  int kmerged;  // 3-bit keys with QJL: one 4-bit field (r0, r1, s, sigma) per coordinate
+  int kchunks;  // 16-byte chunks of one token's key bit string
 };
 
 __host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits) {
@@ -25,15 +27,24 @@ __host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits) {
   L.kbits = kbits;
   L.vbits = vbits;
   L.qjl = qjl;
+  L.kmerged = (qjl && kbits == 3) ? 1 : 0;
+  L.kchunks = L.kmerged ? 4 : kbits;
   int off = 0;
   L.kn = off; off += 2 * PT;
   L.kr = off; off += qjl ? 2 * PT : 0;
   L.vn = off; off += 2 * PT;
-  L.kc = off; off += kbits * (D / 8) * PT;
-  L.ks = off; off += qjl ? (QM / 8) * PT : 0;
+  L.kc = off; off += L.kchunks * 16 * PT;
+  L.ks = off; off += (qjl && !L.kmerged) ? (QM / 8) * PT : 0;
   L.vc = off; off += vbits * (D / 8) * PT;
   L.bytes = off;
   return L;
+}
+
+// Position of coordinate j's sign inside the 3-bit sign plane: j = 32q + 8a + 4h + t
+// sits at 32q + 4a + t + 16h.
+__host__ __device__ __forceinline__ int sign_plane_pos(int j) {
+  const int e = j & 31;
+  return (j & ~31) + 4 * (e >> 3) + (e & 3) + 16 * ((e >> 2) & 1);
 }
 
 // Everything a kernel needs to find a block of the cache.
@@ -71,7 +82,8 @@ __device__ __forceinline__ void code_fields(const uint32_t* w, int bits, int j, 
     }
     case 3: {
       r = (w[j >> 4] >> ((j & 15) * 2)) & 3u;
-      s = (w[8 + (j >> 5)] >> (j & 31)) & 1;
+      const int p = sign_plane_pos(j);
+      s = (w[8 + (p >> 5)] >> (p & 31)) & 1;
       break;
     }
     default: {
@@ -80,6 +92,20 @@ __device__ __forceinline__ void code_fields(const uint32_t* w, int bits, int j, 
       s = f >> 3;
       break;
     }
+  }
+}
+
+// Key fields of coordinate j: merged keys carry sigma_j in the same nibble.
+__device__ __forceinline__ void key_fields(const uint32_t* w, const Layout& L, int j, int& s, int& r,
+                                           int& sigma) {
+  if (L.kmerged) {
+    const uint32_t f = (w[j >> 3] >> ((j & 7) * 4)) & 15u;
+    r = f & 3;
+    s = (f >> 2) & 1;
+    sigma = f >> 3;
+  } else {
+    code_fields(w, L.kbits, j, s, r);
+    sigma = 0;
   }
 }
 

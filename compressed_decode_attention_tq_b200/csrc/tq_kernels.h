@@ -28,6 +28,11 @@ struct DecodeArgs {
   float* sq;        // [B*Hq*seq_q][QM] workspace
   float* part_acc;  // [B*Hq*seq_q][n_splits][D] workspace
   float* part_ml;   // [B*Hq*seq_q][n_splits][2] workspace
+  int16_t* sq_int;  // [B*Hq*seq_q][QM] workspace: S q in 16-bit fixed point
+  float* sq_scale;  // [B*Hq*seq_q] workspace: S q ~= sq_int * sq_scale (a power of two)
+  int* sq_sum;      // [B*Hq*seq_q] workspace: sum_i sq_int
+  int8_t* q8;       // [B*Hq*seq_q][D] workspace: R q in int8 (scaled by q8_scale)
+  float* q8_scale;  // [B*Hq*seq_q] workspace
   float* out;       // [B*Hq*seq_q][D]
   float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
   int max_len;
@@ -48,11 +53,14 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {
-  size_t qrot, sq, part_acc, part_ml, total;
+  size_t qrot, sq, part_acc, part_ml, sq_int, sq_scale, sq_sum, q8, q8_scale, total;
 };
 DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+bool fast_decode_supported(const DecodeArgs& a);
+size_t fast_decode_smem_bytes();
+cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decompress(const DecompressArgs& a, cudaStream_t stream);
 

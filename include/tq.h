@@ -46,8 +46,8 @@
  *   KN      stored ||k|| (fp16) per token              2P
  *   KR      stored ||r|| (fp16) per token, QJL keys    2P
  *   VN      stored ||v|| (fp16) per token              2P
- *   KC      key codes, key_bits*d/8 bytes per token    key_bits*16*P
- *   KS      QJL sign bits, m/8 bytes per token          16*P   (QJL keys)
+ *   KC      key codes, key_bits*d/8 bytes per token    key_bits*16*P  (merged keys: 64*P)
+ *   KS      QJL sign bits, m/8 bytes per token          16*P   (QJL keys, not merged)
  *   VC      value codes                               value_bits*16*P
  *
  *   A code region stores each token's bytes as 16-byte chunks, chunk-major:
@@ -58,9 +58,13 @@
  *   c[idx] = (s ? +1 : -1) * c[h + r] for the (symmetric) codebook c:
  *     b = 1: bit j = s
  *     b = 2: bits 2j, 2j+1 = r, s
- *     b = 3: bits 2j, 2j+1 = r (2 bits), bit 2d + j = s
+ *     b = 3: bits 2j, 2j+1 = r (2 bits); the sign plane starts at bit 2d and,
+ *            for j = 32q + 8a + 4u + t (a < 4, u < 2, t < 4), holds s at plane bit
+ *            32q + 4a + t + 16u
  *     b = 4: bits 4j..4j+2 = r (3 bits), bit 4j + 3 = s
- *   QJL sign bit i of a key = [(S r)_i >= 0] (sign(0) is stored as +1).
+ *   Merged keys (key_bits = 3 with QJL): bits 4j..4j+3 = r0, r1, s, sigma_j, where
+ *   sigma_i = [(S r)_i >= 0] (sign(0) is stored as +1); there is no KS region.
+ *   Other QJL keys: bit i of the KS chunk = sigma_i.
  *   Slots past a sequence's length are never read and their bytes unspecified.
  */
 #ifndef TQ_H_

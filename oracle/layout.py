@@ -16,8 +16,8 @@ page, kv head); the cache is [layer][physical page][kv head][block]):
   KN      stored ||k|| as fp16, one per token    2P
   KR      stored ||r|| as fp16 (keys with QJL)   2P
   VN      stored ||v|| as fp16                   2P
-  KC      key codes, b_k*d/8 bytes per token     b_k*16*P
-  KS      QJL sign bits, m/8 bytes per token     16*P   (keys with QJL)
+  KC      key codes, b_k*d/8 bytes per token     b_k*16*P  (merged keys: 4*16*P)
+  KS      QJL sign bits, m/8 bytes per token     16*P   (keys with QJL, not merged)
   VC      value codes, b_v*d/8 bytes per token   b_v*16*P
 
 Each code region is a sequence of 16-byte chunks per token, stored chunk-major:
@@ -31,9 +31,13 @@ h - 1 - idx (0 = the centroid nearest zero).  Because the codebook is symmetric,
 c[idx] = (+1 if s else -1) * c[h + r].  Fields of coordinate j in the bit string:
   b = 1:  bit j = s
   b = 2:  bits 2j, 2j+1 = r, s
-  b = 3:  bits 2j, 2j+1 = r (2-bit rank), bit 2d + j = s
-  b = 4:  bits 4j..4j+2 = r (3-bit rank), bit 4j+3 = s
-QJL signs: bit i of the sign bit string = sigma_i = [(S r)_i >= 0].
+  b = 3:  bits 2j, 2j+1 = r (2-bit rank); the sign plane follows at bit 2d: with
+          j = 32q + 8a + 4h + t (a in 0..3, h in 0..1, t in 0..3) the sign sits at
+          bit 2d + 32q + 4a + t + 16h (a fixed permutation inside each group of 32)
+  b = 4:  bits 4j..4j+2 = r (3-bit rank), bit 4j + 3 = s
+Keys with b_k = 3 and QJL ("merged keys") store one 4-bit field per coordinate,
+bits 4j..4j+3 = r0, r1, s, sigma_j, and have no KS region; other keys with QJL keep
+the sign bits in KS, bit i = sigma_i.
 """
 from __future__ import annotations
 
@@ -51,10 +55,20 @@ class Format:
     value_bits: int = 3
     page_tokens: int = 256
 
+    @property
+    def merged_keys(self) -> bool:
+        return bool(self.key_qjl) and self.key_bits == 3
+
+    @property
+    def key_bytes(self) -> int:
+        """Bytes of one token's key bit string in KC."""
+        return (4 if self.merged_keys else self.key_bits) * self.head_dim // 8
+
     def regions(self) -> dict:
         P, d, m = self.page_tokens, self.head_dim, self.qjl_m
+        ks = m // 8 * P if (self.key_qjl and not self.merged_keys) else 0
         sizes = [("KN", 2 * P), ("KR", 2 * P if self.key_qjl else 0), ("VN", 2 * P),
-                 ("KC", self.key_bits * d // 8 * P), ("KS", m // 8 * P if self.key_qjl else 0),
+                 ("KC", self.key_bytes * P), ("KS", ks),
                  ("VC", self.value_bits * d // 8 * P)]
         out, off = {}, 0
         for name, sz in sizes:
@@ -83,6 +97,14 @@ def index_from_code(s, r, bits: int):
     return np.where(s == 1, h + r, h - 1 - r)
 
 
+def sign_plane_position(j):
+    """Bit offset inside the b = 3 sign plane of coordinate j (see the format above)."""
+    j = np.asarray(j)
+    q, e = j // 32, j % 32
+    a, h, t = e // 8, (e // 4) % 2, e % 4
+    return 32 * q + 4 * a + t + 16 * h
+
+
 def code_bits(idx, bits: int) -> np.ndarray:
     """[N, d] indices -> [N, bits*d] uint8 bit strings."""
     idx = np.asarray(idx, dtype=np.int64)
@@ -98,7 +120,7 @@ def code_bits(idx, bits: int) -> np.ndarray:
     elif bits == 3:
         out[:, 2 * j] = r & 1
         out[:, 2 * j + 1] = (r >> 1) & 1
-        out[:, 2 * d + j] = s
+        out[:, 2 * d + sign_plane_position(j)] = s
     elif bits == 4:
         out[:, 4 * j] = r & 1
         out[:, 4 * j + 1] = (r >> 1) & 1
@@ -107,6 +129,27 @@ def code_bits(idx, bits: int) -> np.ndarray:
     else:
         raise ValueError("bits must be 1..4")
     return out
+
+
+def merged_key_bits(idx, sigma) -> np.ndarray:
+    """[N, d] 3-bit indices and [N, d] QJL bits -> [N, 4d] merged key bit strings."""
+    idx = np.asarray(idx, dtype=np.int64)
+    n, d = idx.shape
+    s, r = stored_code(idx, 3)
+    out = np.zeros((n, 4 * d), dtype=np.uint8)
+    j = np.arange(d)
+    out[:, 4 * j] = r & 1
+    out[:, 4 * j + 1] = (r >> 1) & 1
+    out[:, 4 * j + 2] = s
+    out[:, 4 * j + 3] = np.asarray(sigma, dtype=np.uint8)
+    return out
+
+
+def merged_key_from_bits(bitstr, d: int):
+    b = np.asarray(bitstr, dtype=np.int64)
+    j = np.arange(d)
+    r = b[:, 4 * j] | (b[:, 4 * j + 1] << 1)
+    return index_from_code(b[:, 4 * j + 2], r, 3), b[:, 4 * j + 3].astype(bool)
 
 
 def index_from_bits(bitstr, bits: int, d: int) -> np.ndarray:
@@ -119,7 +162,7 @@ def index_from_bits(bitstr, bits: int, d: int) -> np.ndarray:
         r, s = b[:, 2 * j], b[:, 2 * j + 1]
     elif bits == 3:
         r = b[:, 2 * j] | (b[:, 2 * j + 1] << 1)
-        s = b[:, 2 * d + j]
+        s = b[:, 2 * d + sign_plane_position(j)]
     elif bits == 4:
         r = b[:, 4 * j] | (b[:, 4 * j + 1] << 1) | (b[:, 4 * j + 2] << 2)
         s = b[:, 4 * j + 3]
@@ -164,9 +207,13 @@ def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_
     P, d = fmt.page_tokens, fmt.head_dim
     reg = fmt.regions()
     n = kcomp.idx.shape[0]
-    kbytes = bits_to_bytes(code_bits(kcomp.idx, fmt.key_bits))
+    if fmt.merged_keys:
+        kbytes = bits_to_bytes(merged_key_bits(kcomp.idx, kcomp.sigma))
+        sbytes = None
+    else:
+        kbytes = bits_to_bytes(code_bits(kcomp.idx, fmt.key_bits))
+        sbytes = bits_to_bytes(kcomp.sigma.astype(np.uint8)) if fmt.key_qjl else None
     vbytes = bits_to_bytes(code_bits(vcomp.idx, fmt.value_bits))
-    sbytes = bits_to_bytes(kcomp.sigma.astype(np.uint8)) if fmt.key_qjl else None
     for lp in range((n + P - 1) // P):
         t0, t1 = lp * P, min(n, (lp + 1) * P)
         blk = cache[layer, pages_of_seq[lp], head]
@@ -179,6 +226,7 @@ def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_
         region("VN")[0:2 * (t1 - t0)] = fp16_bytes(vcomp.norm[t0:t1])
         if fmt.key_qjl:
             region("KR")[0:2 * (t1 - t0)] = fp16_bytes(kcomp.rnorm[t0:t1])
+        if sbytes is not None:
             _put_chunked(region("KS"), sbytes[t0:t1], 0, P)
         _put_chunked(region("KC"), kbytes[t0:t1], 0, P)
         _put_chunked(region("VC"), vbytes[t0:t1], 0, P)
@@ -199,7 +247,7 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
     """Read tokens 0..n-1 of one (sequence, kv head) back into indices, norms and signs."""
     P, d, m = fmt.page_tokens, fmt.head_dim, fmt.qjl_m
     reg = fmt.regions()
-    kb, vb = fmt.key_bits * d // 8, fmt.value_bits * d // 8
+    kb, vb = fmt.key_bytes, fmt.value_bits * d // 8
     parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc")}
     for lp in range((n + P - 1) // P):
         cnt = min(n, (lp + 1) * P) - lp * P
@@ -215,15 +263,19 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
         parts["vc"].append(_get_chunked(region("VC"), cnt, vb, P))
         if fmt.key_qjl:
             parts["kr"].append(region("KR")[:2 * cnt].view(np.float16).astype(np.float64))
+        if fmt.key_qjl and not fmt.merged_keys:
             parts["ks"].append(_get_chunked(region("KS"), cnt, m // 8, P))
     cat = lambda k, w: np.concatenate(parts[k]) if parts[k] else np.zeros((0,) + w)
     kc = cat("kc", (kb,))
     vc = cat("vc", (vb,))
-    out = Unpacked(k_idx=index_from_bits(bytes_to_bits(kc), fmt.key_bits, d),
-                   k_norm=cat("kn", ()),
+    if fmt.merged_keys:
+        k_idx, k_sigma = merged_key_from_bits(bytes_to_bits(kc), d)
+    else:
+        k_idx, k_sigma = index_from_bits(bytes_to_bits(kc), fmt.key_bits, d), None
+    out = Unpacked(k_idx=k_idx, k_norm=cat("kn", ()),
                    v_idx=index_from_bits(bytes_to_bits(vc), fmt.value_bits, d),
                    v_norm=cat("vn", ()))
     if fmt.key_qjl:
         out.k_rnorm = cat("kr", ())
-        out.k_sigma = bytes_to_bits(cat("ks", (m // 8,))).astype(bool)
+        out.k_sigma = k_sigma if fmt.merged_keys else bytes_to_bits(cat("ks", (m // 8,))).astype(bool)
     return out

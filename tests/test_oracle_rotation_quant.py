@@ -151,6 +151,23 @@ def test_packing_matches_hand_derived_bytes(packing_golden, name):
     np.testing.assert_array_equal(back, idx)
 
 
+def test_merged_key_packing_matches_hand_derived_bytes(packing_golden):
+    g = packing_golden["k3_qjl_merged_idx_j_mod_8_sigma_j_mod_2"]
+    j = np.arange(128)
+    idx, sigma = (j % 8)[None, :], (j % 2)[None, :]
+    got = lay.bits_to_bytes(lay.merged_key_bits(idx, sigma))[0]
+    assert got.tobytes().hex() == g["bytes_hex"]
+    bidx, bsig = lay.merged_key_from_bits(lay.bytes_to_bits(got[None]), 128)
+    np.testing.assert_array_equal(bidx, idx)
+    np.testing.assert_array_equal(bsig, sigma.astype(bool))
+
+
+def test_sign_plane_permutation_is_a_bijection():
+    pos = lay.sign_plane_position(np.arange(128))
+    assert sorted(pos.tolist()) == list(range(128))
+    assert np.all(pos // 32 == np.arange(128) // 32)
+
+
 def test_region_offsets_match_hand_derivation(packing_golden):
     g = packing_golden["c2_regions"]
     fmt = lay.Format(**g["format"])
@@ -191,7 +208,7 @@ def test_page_round_trip_with_partial_last_page():
     np.testing.assert_array_equal(u.v_norm, V.norm)
     # token 300 = page 1 (physical 0) slot 44: its second key chunk sits at (1*256+44)*16 of KC
     o, _ = fmt.regions()["KC"]
-    tok_bytes = lay.bits_to_bytes(lay.code_bits(K.idx[300:301], 3))[0]
+    tok_bytes = lay.bits_to_bytes(lay.merged_key_bits(K.idx[300:301], K.sigma[300:301]))[0]
     blk = cache[0, 0, 1]
     assert blk[o + (256 + 44) * 16: o + (256 + 44) * 16 + 16].tobytes() == tok_bytes[16:32].tobytes()
     assert not cache[0, :, 0].any()
