@@ -300,6 +300,10 @@ size_t compress_smem_bytes(int qjl, int dense) {
 }
 
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
+  if (compress_tc_supported(a)) {
+    const cudaError_t e = launch_compress_tc(a, stream);
+    if (e != cudaErrorInvalidValue) return e;  // otherwise fall through to the CUDA-core kernel
+  }
   const size_t smem = compress_smem_bytes(a.qjl, a.dense);
   dim3 grid((a.max_len + kTokPerBlock - 1) / kTokPerBlock, a.cache.kv_heads, a.cache.batch);
   if (grid.x == 0) return cudaSuccess;

@@ -50,6 +50,8 @@ struct DecompressArgs {
 
 size_t compress_smem_bytes(int qjl, int dense);
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream);
+bool compress_tc_supported(const CompressArgs& a);
+cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream);
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {
