@@ -19,12 +19,12 @@
 // sum of comparison masks (the boundaries are sorted) that also drive the centroid
 // select of the residual.
 //
-// One persistent CTA per SM: 16 compute warps and one producer warp.  Compute warp w
+// One persistent CTA per SM: 8 compute warps and a producer warpgroup.  Compute warp w
 // reads tensor-memory lane quadrant w % 4 (tokens 32 (w % 4) .. + 31) and coordinates
-// 32 (w / 4) .. + 31, so four warps share a token; their per-token sums (norms, residual
-// norm) meet in spare tensor-memory columns behind a 128-thread named barrier.  The
-// producer warp issues the TMA copies (two K/V tile stages), the MMAs and their commits;
-// the compute warps hand tensor-memory columns back through two mbarriers.
+// 64 (w / 4) .. + 63, so two warps share a token; their per-token sums (norms, residual
+// norm) meet in spare tensor-memory columns behind a 64-thread named barrier.  One thread
+// of the producer warpgroup issues the TMA copies (two K/V tile stages), the MMAs and their
+// commits; the compute warps hand tensor-memory columns back through mbarriers.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -37,27 +37,37 @@ namespace tqk {
 namespace {
 
 constexpr int TT = 128;                      // tokens per tile
-constexpr int kComputeWarps = 16;
-constexpr int kThreadsTC = (kComputeWarps + 1) * 32;
+constexpr int kComputeWarps = 8;
+constexpr int kCPT = 64;  // coordinates per compute thread
+// two compute warpgroups and one producer warpgroup (one thread of which issues the copies
+// and MMAs); registers move from the producer to the compute warpgroups after launch:
+// launched with 384 x 168, then 128 x 72 + 256 x 216 = 64512 = 384 x 168.
+constexpr int kThreadsTC = (kComputeWarps + 4) * 32;
+constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsCompute = 216;
+static_assert(128 * kRegsProducer + 32 * kComputeWarps * kRegsCompute <= kThreadsTC * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr int kTileBytes = TT * D * 2;       // one 128 x 128 fp16 operand
-// tensor-memory columns: y'_K, y'_V, A = residual hi / lo, S = sketch (and exchange slots)
-constexpr uint32_t kColK = 0, kColV = 128, kColAhi = 256, kColAlo = 320, kColS = 384;
-constexpr uint32_t kColNormX = kColS, kColRrX = kColS + 8;
+// Tensor-memory columns.  KS[0], KS[1]: y'_K of a tile, then the per-token exchange slots
+// (+0 key sums of squares, +2 residual sums), then that tile's sketch (S D H) a r_rot';
+// alternate tiles use alternate halves.  V: y'_V of a tile, then (+0) the value sums of
+// squares.  A: the residual hi (+0) / lo (+64) halves, the sketch's A operand.
+constexpr uint32_t kColKS0 = 0, kColKS1 = 128, kColV = 256, kColA = 384;
+constexpr uint32_t kXssK = 0, kXrr = 2, kXssV = 0;
 constexpr uint32_t kTmemCols = 512;
 // instruction descriptor: D f32, A and B f16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr unsigned long long kWaitNs = 1000000000ull;  // a wait gives up after 1 s
 constexpr float kSqrtD = 11.313708498984761f;
-constexpr float kResidScale = 256.f;         // residual scaled to ~O(1) before the fp16 split
 
 struct SmemTC {
   unsigned char x[2][2][kTileBytes];  // [stage][K, V] input tiles (canonical layout)
   unsigned char bhd[kTileBytes];      // B = H D
   unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part
   unsigned char bslo[kTileBytes];     // fp16 lo part
-  unsigned long long bar_load[2], bar_fwd, bar_sig, kv_free, a_ready;
+  unsigned long long bar_load[2], stage_free[2], bar_fwdk, bar_fwdv, bar_sig, ks_free, a_ready, v_free;
   uint32_t tmem_base;
   int bad_s;
+  float kpos[8], vpos[8], kmag[8], vmag[8];  // positive boundaries / centroid magnitudes
 };
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
 
@@ -84,7 +94,7 @@ __device__ __forceinline__ void bar_init(unsigned long long* b, int n) {
 __device__ __forceinline__ bool bar_try(uint32_t addr, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(done)
       : "r"(addr), "r"(parity)
@@ -98,8 +108,9 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// Wait for the phase with the given parity to complete; false after kWaitNs (or 2^24
-// polls, whichever comes first) without completion.
+// Wait for the phase with the given parity to complete (each poll may suspend the thread
+// for up to 1 ms until it does); false after kWaitNs without completion, or after 2^24
+// polls.
 __device__ __forceinline__ bool bar_wait(unsigned long long* b, uint32_t parity) {
   const uint32_t addr = s_u32(b);
   if (bar_try(addr, parity)) return true;
@@ -117,9 +128,9 @@ __device__ __forceinline__ void bar_arrive(unsigned long long* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s_u32(b)) : "memory");
 }
 
-// 128-thread barrier of the four compute warps that share a tensor-memory lane quadrant
-__device__ __forceinline__ void quad_sync(int qd) {
-  asm volatile("bar.sync %0, 128;" ::"r"(1 + qd) : "memory");
+// 64-thread barrier of the two compute warps that share a tensor-memory lane quadrant
+__device__ __forceinline__ void pair_sync(int qd) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + qd) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_tile(void* dst, const CUtensorMap* map, int row0,
@@ -170,22 +181,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
-  uint32_t r[4];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
+  uint32_t r0, r1;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
+  v[0] = __uint_as_float(r0);
+  v[1] = __uint_as_float(r1);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -197,92 +197,232 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st2(uint32_t taddr, float a, float b) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(__float_as_uint(a)),
-               "r"(__float_as_uint(b))
-               : "memory");
-}
-
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, float a) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(a))
                : "memory");
 }
 
-// all-ones when a > b (a >= b), zero otherwise and for NaN
-__device__ __forceinline__ uint32_t gt_mask(float a, float b) {
-  uint32_t m;
-  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(m) : "f"(a), "f"(b));
-  return m;
+// ---- packed fp32 pairs (two coordinates per instruction) and saturated steps ----
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float a, float b) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
 }
-__device__ __forceinline__ uint32_t ge_mask(float a, float b) {
-  uint32_t m;
-  asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(m) : "f"(a), "f"(b));
-  return m;
+__device__ __forceinline__ f2_t f2s(float a) { return f2(a, a); }
+__device__ __forceinline__ void uf2(f2_t p, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p));
+}
+__device__ __forceinline__ f2_t fma2(f2_t a, f2_t b, f2_t c) {
+  f2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2_t mul2(f2_t a, f2_t b) {
+  f2_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2_t add2(f2_t a, f2_t b) {
+  f2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// clamp(a b + c, 0, 1): a unit step of a b + c once it is scaled far past 1
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float d;
+  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
 // sum of squares of 32 values, two lanes of packed fp32 at a time
 __device__ __forceinline__ float sumsq32(const float (&v)[32]) {
-  unsigned long long acc = 0;
+  f2_t acc = 0;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    unsigned long long p;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(p) : "f"(v[i]), "f"(v[i + 1]));
-    asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(p));
+    const f2_t p = f2(v[i], v[i + 1]);
+    acc = fma2(p, p, acc);
   }
   float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc));
+  uf2(acc, lo, hi);
   return lo + hi;
+}
+
+// Integer codes are assembled in the mantissa of 2^23 + code (exact for 0 <= code < 2^23)
+// and shifted into place with an integer multiply-add; the 2^23 exponent bits each
+// coordinate drags along are subtracted up front (mod 2^32).
+constexpr float kMagic = 8388608.f;
+constexpr uint32_t kMagicBits = 0x4B000000u;
+__host__ __device__ constexpr uint32_t magic_at(int sh) {
+  return (uint32_t)(((unsigned long long)kMagicBits << sh) & 0xFFFFFFFFull);
 }
 
 // Bit of coordinate e (0..31) of a 32-coordinate group in the sign plane of 3-bit codes
 // (the permutation of sign_plane_pos, which the decode's byte tables read).
 __host__ __device__ constexpr int plane_bit(int e) { return 4 * (e >> 3) + (e & 3) + 16 * ((e >> 2) & 1); }
 
-// Thermometer masks of |y'| against the scaled positive boundaries; returns the rank
-// r = number of boundaries below |y'|.
-template <int NB>
-__device__ __forceinline__ uint32_t rank_masks(float y, const float (&thr)[8], uint32_t (&m)[8]) {
-  const float ay = fabsf(y);
-  uint32_t sum = 0;
-#pragma unroll
-  for (int k = 0; k < NB; ++k) {
-    m[k] = gt_mask(ay, thr[k]);
-    sum += m[k];
+// Where coordinate i (0..63 of this thread's coordinates) of a b-bit code lands in the
+// thread's words.  Field = r + sw * s:
+//   b = 2: 2-bit r | s << 1 (words 0..3);  b = 3: 2-bit r (words 0..3) and s in words 4, 5
+//   at the permuted sign-plane bit;  b = 4: r | s << 3 (words 0..7);  merged 3-bit key:
+//   r | s << 2 | sigma << 3 (words 0..7).
+template <int B, bool MERGED>
+struct Fields {
+  static constexpr bool nib = MERGED || B == 4;
+  static constexpr int sw = MERGED ? 4 : (B == 2 ? 2 : (B == 3 ? 0 : 8));
+  static constexpr bool plane = !MERGED && B == 3;
+  __host__ __device__ static constexpr int word(int i) { return nib ? (i >> 3) : (i >> 4); }
+  __host__ __device__ static constexpr int shift(int i) { return nib ? 4 * (i & 7) : 2 * (i & 15); }
+  // minus the magic bits the code (and, merged, sigma) adds of every coordinate of word w
+  __host__ __device__ static constexpr uint32_t init(int w) {
+    uint32_t c = 0;
+    for (int i = 0; i < kCPT; ++i) {
+      if (word(i) == w) c += magic_at(shift(i)) * (MERGED ? 2u : 1u);
+      if (plane && w == 4 + (i >> 5)) c += magic_at(plane_bit(i & 31));
+    }
+    return 0u - c;
   }
-  return 0u - sum;
-}
-
-// Code words of this thread's 32 coordinates for the b-bit field layouts without a QJL
-// sign: pack (r, s) of coordinate i into w[].
-//   b = 2: 2-bit r | s << 1, two words;  b = 3: 2-bit r in two words + one word of the
-//   permuted sign plane;  b = 4: r | s << 3, four words.
-template <int B>
-__device__ __forceinline__ void pack_plain(uint32_t (&w)[4], int i, uint32_t r, uint32_t smask) {
-  if constexpr (B == 2) {
-    w[i >> 4] += r << (2 * (i & 15));
-    w[i >> 4] |= smask & (2u << (2 * (i & 15)));
-  } else if constexpr (B == 3) {
-    w[i >> 4] += r << (2 * (i & 15));
-    w[2] |= smask & (1u << plane_bit(i));
-  } else {
-    w[i >> 3] += r << (4 * (i & 7));
-    w[i >> 3] |= smask & (8u << (4 * (i & 7)));
+  __host__ __device__ static constexpr uint32_t sig_init() {
+    uint32_t c = 0;
+    for (int i = 0; i < 32; ++i) c += magic_at(i);
+    return 0u - c;
   }
-}
+};
 
-// Store the words of pack_plain for one token slot (plane p = 16 bytes per slot; this
-// thread's coordinates 32 part .. 32 part + 31).
-template <int B>
-__device__ __forceinline__ void store_plain(uint8_t* base, int part, int slot, const uint32_t (&w)[4]) {
+// Store a thread's code words for one token slot (plane p = 16 bytes per slot; this
+// thread's coordinates 64 part .. 64 part + 63).
+template <int B, bool MERGED>
+__device__ __forceinline__ void store_words(uint8_t* base, int part, int slot, const uint32_t (&w)[8]) {
   if constexpr (B == 2) {
-    *reinterpret_cast<uint2*>(base + ((size_t)(part >> 1) * PT + slot) * 16 + 8 * (part & 1)) = make_uint2(w[0], w[1]);
-  } else if constexpr (B == 3) {
-    *reinterpret_cast<uint2*>(base + ((size_t)(part >> 1) * PT + slot) * 16 + 8 * (part & 1)) = make_uint2(w[0], w[1]);
-    *reinterpret_cast<uint32_t*>(base + ((size_t)2 * PT + slot) * 16 + 4 * part) = w[2];
-  } else {
     *reinterpret_cast<uint4*>(base + ((size_t)part * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (B == 3 && !MERGED) {
+    *reinterpret_cast<uint4*>(base + ((size_t)part * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(base + ((size_t)2 * PT + slot) * 16 + 8 * part) = make_uint2(w[4], w[5]);
+  } else {
+    *reinterpret_cast<uint4*>(base + ((size_t)(2 * part) * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(base + ((size_t)(2 * part + 1) * PT + slot) * 16) =
+        make_uint4(w[4], w[5], w[6], w[7]);
   }
 }
+
+// Boundary scales of one token: |y| > beta ||y'||  <=>  bq y'^2 - bq (beta ||y'||)^2 > 0 with
+// bq = 2^(40 - 2e) for ||y'|| ~ 2^e, so a saturated step is exact outside a 2^-40
+// relative band; bs = 2^(40 - e) makes y' bs a step for s = [y' > 0].
+struct TokScale {
+  int e;
+  float bq, bs;
+  __device__ __forceinline__ explicit TokScale(float ny) {
+    e = min(max((int)((__float_as_uint(ny) >> 23) & 0xff) - 127, -40), 40);
+    bq = __uint_as_float((uint32_t)(127 + 40 - 2 * e) << 23);
+    bs = __uint_as_float((uint32_t)(127 + 40 - e) << 23);
+  }
+};
+
+// Per-token constants of the quantiser: squared scaled boundaries, and with QJL the
+// residual scale a = 2^(8 - e) and the thermometer centroid steps a sqrt(d) fp16(||x||) dc.
+template <int NB>
+struct QuantConst {
+  TokScale ts;
+  float t2[NB > 0 ? NB : 1];
+  float alpha, inv_alpha;
+  f2_t dam[NB > 0 ? NB : 1], am0;
+  __device__ __forceinline__ QuantConst(float ny, const float* pos, const float* mag, float cnorm) : ts(ny) {
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      const float t = pos[k] * ny;
+      t2[k] = -(t * t) * ts.bq;
+    }
+    alpha = __uint_as_float((uint32_t)(127 + 8 - ts.e) << 23);
+    inv_alpha = __uint_as_float((uint32_t)(127 - 8 + ts.e) << 23);
+    const float csa = alpha * kSqrtD * cnorm;
+#pragma unroll
+    for (int k = 0; k < NB; ++k) dam[k] = f2s(csa * (mag[k + 1] - mag[k]));
+    am0 = f2s(csa * mag[0]);
+  }
+};
+
+// Codes of 32 of this thread's coordinates (OFF .. OFF + 31) of y'; with KQ also the scaled
+// residual a (y' - sqrt(d) fp16(||x||) c[idx]) split into fp16 hi / lo pairs for the
+// sketch MMAs, and its sum of squares (accumulated into rr2).
+template <int NB, class F, bool KQ, int OFF>
+__device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, uint32_t (&w)[8],
+                                           uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float y0 = y[i], y1 = y[i + 1];
+    const f2_t Y = f2(y0, y1);
+    float yb0, yb1;
+    uf2(mul2(Y, f2s(qc.ts.bq)), yb0, yb1);
+    f2_t M[NB > 0 ? NB : 1];
+    f2_t sum = f2s(kMagic);
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      M[k] = f2(fma_sat(yb0, y0, qc.t2[k]), fma_sat(yb1, y1, qc.t2[k]));
+      sum = add2(sum, M[k]);
+    }
+    const f2_t S = f2(mul_sat(y0, qc.ts.bs), mul_sat(y1, qc.ts.bs));  // s = [y' > 0]
+    if (F::sw) sum = fma2(S, f2s((float)F::sw), sum);
+    float c0, c1;
+    uf2(sum, c0, c1);
+    w[F::word(OFF + i)] += __float_as_uint(c0) << F::shift(OFF + i);
+    w[F::word(OFF + i + 1)] += __float_as_uint(c1) << F::shift(OFF + i + 1);
+    if (F::plane) {
+      uf2(add2(S, f2s(kMagic)), c0, c1);
+      w[4 + (OFF >> 5)] += __float_as_uint(c0) << plane_bit(i);
+      w[4 + (OFF >> 5)] += __float_as_uint(c1) << plane_bit(i + 1);
+    }
+    if constexpr (KQ) {
+      f2_t C = qc.am0;
+#pragma unroll
+      for (int k = 0; k < NB; ++k) C = fma2(M[k], qc.dam[k], C);
+      const f2_t negsgn = fma2(S, f2s(-2.f), f2s(1.f));  // 1 - 2 s
+      const f2_t R = fma2(Y, f2s(qc.alpha), mul2(C, negsgn));
+      rr2 = fma2(R, R, rr2);
+      float r0, r1;
+      uf2(R, r0, r1);
+      const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
+      const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+      float l0, l1;
+      uf2(fma2(f2(h0, h1), f2s(-1.f), R), l0, l1);
+      const __half2 hh = __floats2half2_rn(h0, h1);
+      const __half2 ll = __floats2half2_rn(l0, l1);
+      hi[i >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
+      lo[i >> 1] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+  }
+}
+
+// QJL signs sigma = [p >= 0] (1 also within 2^-40 below 0) of 32 of this thread's sketch
+// entries (OFF .. OFF + 31): merged into bit 3 of the key nibbles, or one sign-plane word.
+template <bool MERGED, class F, int OFF>
+__device__ __forceinline__ void sigma32(const float (&p)[32], uint32_t (&w)[8], uint32_t (&sgw)[2]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const f2_t G = f2(fma_sat(p[i], 1099511627776.f, 1.f), fma_sat(p[i + 1], 1099511627776.f, 1.f));
+    float c0, c1;
+    if constexpr (MERGED) {
+      uf2(fma2(G, f2s(8.f), f2s(kMagic)), c0, c1);
+      w[F::word(OFF + i)] += __float_as_uint(c0) << F::shift(OFF + i);
+      w[F::word(OFF + i + 1)] += __float_as_uint(c1) << F::shift(OFF + i + 1);
+    } else {
+      uf2(add2(G, f2s(kMagic)), c0, c1);
+      sgw[OFF >> 5] += __float_as_uint(c0) << i;
+      sgw[OFF >> 5] += __float_as_uint(c1) << (i + 1);
+    }
+  }
+}
+
+// The cache block and slot of the token this thread owns in tile j (blk null when the
+// token is past its sequence or its page is invalid; errors reported once, by part 0).
+struct TokRef {
+  uint8_t* blk;
+  int slot;
+};
 
 template <int KB, int KQ, int VB>
 __global__ void __launch_bounds__(kThreadsTC, 1)
@@ -292,13 +432,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const uint32_t pad = (128u - (s_u32(smem_raw) & 127u)) & 127u;
   SmemTC& sm = *reinterpret_cast<SmemTC*>(smem_raw + pad);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp == kComputeWarps;
+  const bool producer = warp >= kComputeWarps;  // the producer warpgroup
   const int qd = warp & 3;           // tensor-memory lane quadrant
-  const int part = (warp >> 2) & 3;  // coordinates 32 part .. 32 part + 31
+  const int part = (warp >> 2) & 1;  // coordinates 64 part .. 64 part + 63
   const int row = 32 * qd + lane;    // token within the tile
   const Layout& L = a.cache.L;
   constexpr int HK = 1 << (KB - 1), HV = 1 << (VB - 1);
   constexpr bool kMerged = KQ && KB == 3;
+  constexpr int kComputeThreads = kComputeWarps * 32;
 
   const int tiles_per_head = (a.max_len + TT - 1) / TT;
   const int total = a.cache.batch * a.cache.kv_heads * tiles_per_head;
@@ -329,10 +470,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (tid == 0) {
     bar_init(&sm.bar_load[0], 1);
     bar_init(&sm.bar_load[1], 1);
-    bar_init(&sm.bar_fwd, 1);
+    bar_init(&sm.stage_free[0], 1);
+    bar_init(&sm.stage_free[1], 1);
+    bar_init(&sm.bar_fwdk, 1);
+    bar_init(&sm.bar_fwdv, 1);
     bar_init(&sm.bar_sig, 1);
-    bar_init(&sm.kv_free, kComputeWarps);
+    bar_init(&sm.ks_free, kComputeWarps);
     bar_init(&sm.a_ready, kComputeWarps);
+    bar_init(&sm.v_free, kComputeWarps);
     sm.bad_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -340,7 +485,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   // tile 0 streams in while the rotation operands are built (stage 1 is set-up scratch)
-  if (producer && lane == 0 && my_tiles > 0) issue_load(0);
+  if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) issue_load(0);
   __syncwarp();
   if (tid == 0 && blockIdx.x == 0) {
     for (int i = 0; i < 2 * HK; ++i)
@@ -353,9 +498,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     for (int i = 0; i < 2 * HV - 1; ++i)
       if (a.v_boundaries[i] != -a.v_boundaries[2 * HV - 2 - i]) report(a.status, TQ_ERR_INVALID_ARG);
   }
+  if (tid < 8) {
+    sm.kpos[tid] = (tid < HK - 1) ? a.k_boundaries[HK + tid] : 0.f;
+    sm.vpos[tid] = (tid < HV - 1) ? a.v_boundaries[HV + tid] : 0.f;
+    sm.kmag[tid] = (tid < HK) ? a.k_centroids[HK + tid] : 0.f;
+    sm.vmag[tid] = (tid < HV) ? a.v_centroids[HV + tid] : 0.f;
+  }
   if (!producer) {
     // B = H D: row i, column k = (-1)^popcount(i & k) D_k
-    for (int c = tid; c < D * 16; c += kComputeWarps * 32) {
+    for (int c = tid; c < D * 16; c += kComputeThreads) {
       const int i = c & 127, ch = c >> 7;
       uint32_t w[4];
 #pragma unroll
@@ -370,62 +521,69 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       *reinterpret_cast<uint4*>(sm.bhd + canon(i, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (KQ) {
-      // B = S D H: thread (n, p) transforms coordinates 32p .. 32p + 31 of row n of S D in
+      // B = S D H: for row n of S D, coordinate block p (32 wide) is transformed in
       // registers (butterfly spans 1..16); the spans 32 and 64 meet through scratch.
-      const int n = tid & 127, p = tid >> 7;
-      float v[32];
-      const float4* srow = reinterpret_cast<const float4*>(a.s + (size_t)n * D + 32 * p);
+      float* scr = reinterpret_cast<float*>(sm.x[1][0]);  // [coordinate][n], 64 KB
+      const int n = tid & 127;
       int bad = 0;
+#pragma unroll 1
+      for (int p = tid >> 7; p < 4; p += kComputeThreads / 128) {
+        float v[32];
+        const float4* srow = reinterpret_cast<const float4*>(a.s + (size_t)n * D + 32 * p);
 #pragma unroll
-      for (int i4 = 0; i4 < 8; ++i4) {
-        const float4 q = srow[i4];
-        const float e[4] = {q.x, q.y, q.z, q.w};
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 q = srow[i4];
+          const float e[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = 4 * i4 + u;
-          if (__half2float(__float2half_rn(e[u])) != e[u]) bad = 1;
-          v[i] = e[u] * a.signs[32 * p + i];
+          for (int u = 0; u < 4; ++u) {
+            const int i = 4 * i4 + u;
+            if (__half2float(__float2half_rn(e[u])) != e[u]) bad = 1;
+            v[i] = e[u] * a.signs[32 * p + i];
+          }
         }
+#pragma unroll
+        for (int hs = 1; hs < 32; hs <<= 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i & hs) continue;
+            const float u = v[i], w = v[i + hs];
+            v[i] = u + w;
+            v[i + hs] = u - w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) scr[(32 * p + i) * 128 + n] = v[i];
       }
       if (bad) sm.bad_s = 1;
+      asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
+#pragma unroll 1
+      for (int p = tid >> 7; p < 4; p += kComputeThreads / 128) {
 #pragma unroll
-      for (int hs = 1; hs < 32; hs <<= 1) {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i & hs) continue;
-          const float u = v[i], w = v[i + hs];
-          v[i] = u + w;
-          v[i + hs] = u - w;
+          for (int e = 0; e < 4; ++e) {
+            float x2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i = 8 * c + 2 * e + u;
+              float acc = 0.f;
+#pragma unroll
+              for (int bb = 0; bb < 4; ++bb) {
+                const float t = scr[(32 * bb + i) * 128 + n];
+                acc += (__popc(p & bb) & 1) ? -t : t;
+              }
+              x2[u] = acc;
+            }
+            const __half2 h2 = __floats2half2_rn(x2[0], x2[1]);
+            const float2 hf = __half22float2(h2);
+            const __half2 l2 = __floats2half2_rn(x2[0] - hf.x, x2[1] - hf.y);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+          *reinterpret_cast<uint4*>(sm.bshi + canon(n, 32 * p + 8 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sm.bslo + canon(n, 32 * p + 8 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-      }
-      float* scr = reinterpret_cast<float*>(sm.x[1][0]);  // [coordinate][n], 64 KB
-#pragma unroll
-      for (int i = 0; i < 32; ++i) scr[(32 * p + i) * 128 + n] = v[i];
-      asm volatile("bar.sync 5, 512;" ::: "memory");  // the 16 compute warps
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float acc = 0.f;
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const float t = scr[(32 * bb + i) * 128 + n];
-          acc += (__popc(p & bb) & 1) ? -t : t;
-        }
-        v[i] = acc;
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = v[8 * c + 2 * e], x1 = v[8 * c + 2 * e + 1];
-          const __half2 h2 = __floats2half2_rn(x0, x1);
-          const float2 hf = __half22float2(h2);
-          const __half2 l2 = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-          hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
-          lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
-        }
-        *reinterpret_cast<uint4*>(sm.bshi + canon(n, 32 * p + 8 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sm.bslo + canon(n, 32 * p + 8 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -435,233 +593,258 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const uint32_t tmem = sm.tmem_base;
 
   if (producer) {
-    // ---------------- producer: copies and MMAs ----------------
-    if (lane == 0 && my_tiles > 0) {
-      if (my_tiles > 1) issue_load(1);
-      int loads_issued = my_tiles > 1 ? 2 : 1, loads_done = 0;
-      int fwd_issued = 0, fwd_done = 0;
-      bool ok = true;
-      for (int j = 0; j < my_tiles; ++j) {
-        const int st = j & 1;
-        ok = bar_wait(&sm.bar_load[st], (j >> 1) & 1);
-        if (!ok) break;
-        ++loads_done;
-        if (j > 0) {
-          ok = bar_wait(&sm.kv_free, (j - 1) & 1);
-          if (!ok) break;
-        }
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+    // ---------------- producer: MMAs (warp 8) and copies (warp 9) ----------------
+    // MMAs of tile j: forward K into KS[j & 1] once KS[(j - 2) & 1] is released (its sketch
+    // read, or without QJL its exchange done); the sketch into KS[j & 1] once the compute
+    // warps have written A; forward V into V once the previous y'_V is read.  Copies: tile
+    // j + 2 into stage j & 1 as soon as both forward MMAs of tile j have read it.  Each wait's
+    // phase is one the other side cannot run two phases past.
+    if (warp == kComputeWarps && lane == 0 && my_tiles > 0) {
+      auto fwd = [&](int j, uint32_t dcol, int kv) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + dcol, smem_desc(sm.x[j & 1][kv], ks), smem_desc(sm.bhd, ks), ks > 0);
+      };
+      bool ok = bar_wait(&sm.bar_load[0], 0);
+      if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + kColK, smem_desc(sm.x[st][0], ks), smem_desc(sm.bhd, ks), ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + kColV, smem_desc(sm.x[st][1], ks), smem_desc(sm.bhd, ks), ks > 0);
-        mma_commit(&sm.bar_fwd);
-        ++fwd_issued;
-        ok = bar_wait(&sm.bar_fwd, j & 1);
-        if (!ok) break;
-        ++fwd_done;
-        // stage st is consumed: stream tile j + 2 into it
-        if (j + 2 < my_tiles) {
-          issue_load(j + 2);
-          ++loads_issued;
+        fwd(0, kColKS0, 0);
+        mma_commit(&sm.bar_fwdk);
+        fwd(0, kColV, 1);
+        mma_commit(&sm.bar_fwdv);
+        mma_commit(&sm.stage_free[0]);
+      }
+      for (int j = 0; j < my_tiles && ok; ++j) {
+        const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
+        if (j + 1 < my_tiles) {
+          // phase j of ks_free arrives in tile j, after every compute warp has waited for
+          // y'_K of tile j: with QJL once tile j - 1's sketch in KS[(j + 1) & 1] is read
+          // (in tile 0 right after the wait), without QJL once tile j's exchange is done
+          if (!(ok = bar_wait(&sm.ks_free, j & 1))) break;
+          if (!(ok = bar_wait(&sm.bar_load[(j + 1) & 1], ((j + 1) >> 1) & 1))) break;
+          tc_fence_after();
+          fwd(j + 1, (j & 1) ? kColKS0 : kColKS1, 0);
+          mma_commit(&sm.bar_fwdk);
         }
         if (KQ) {
-          ok = bar_wait(&sm.a_ready, j & 1);
-          if (!ok) break;
+          if (!(ok = bar_wait(&sm.a_ready, j & 1))) break;
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            mma_ts(tmem + kColS, tmem + kColAhi + 8 * ks, smem_desc(sm.bshi, ks), ks > 0);
-            mma_ts(tmem + kColS, tmem + kColAhi + 8 * ks, smem_desc(sm.bslo, ks), 1);
-            mma_ts(tmem + kColS, tmem + kColAlo + 8 * ks, smem_desc(sm.bshi, ks), 1);
+            mma_ts(tmem + ks_j, tmem + kColA + 8 * ks, smem_desc(sm.bshi, ks), ks > 0);
+            mma_ts(tmem + ks_j, tmem + kColA + 8 * ks, smem_desc(sm.bslo, ks), 1);
+            mma_ts(tmem + ks_j, tmem + kColA + 64 + 8 * ks, smem_desc(sm.bshi, ks), 1);
           }
-          mma_commit(&sm.bar_sig);  // the compute warps wait for this one
+          mma_commit(&sm.bar_sig);
+        }
+        if (j + 1 < my_tiles) {
+          if (!(ok = bar_wait(&sm.v_free, j & 1))) break;
+          tc_fence_after();
+          fwd(j + 1, kColV, 1);
+          mma_commit(&sm.bar_fwdv);
+          mma_commit(&sm.stage_free[(j + 1) & 1]);
         }
       }
-      if (!ok) {
-        report(a.status, TQ_ERR_TIMEOUT);
-        // drain what is still in flight before the shared and tensor memory go away
-        while (loads_done < loads_issued) {
-          bar_wait(&sm.bar_load[loads_done & 1], (loads_done >> 1) & 1);
-          ++loads_done;
-        }
-        if (fwd_done < fwd_issued) bar_wait(&sm.bar_fwd, fwd_done & 1);
+      if (!ok) report(a.status, TQ_ERR_TIMEOUT);
+    } else if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) {
+      int issued = 1;  // tile 0 went out before the set-up
+      if (my_tiles > 1) {
+        issue_load(1);
+        issued = 2;
       }
+      bool ok = true;
+      for (int i = 0; i + 2 < my_tiles; ++i) {
+        // phase i >> 1 of stage_free[i & 1]: the forward MMAs of tile i are done with it
+        if (!(ok = bar_wait(&sm.stage_free[i & 1], (i >> 1) & 1))) break;
+        issue_load(i + 2);
+        issued = i + 3;
+      }
+      if (!ok) report(a.status, TQ_ERR_TIMEOUT);
+      // the last copy into each stage is that stage's final phase: wait (bounded) for both to
+      // land so that no copy is still in flight when the shared memory goes away
+      for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) bar_wait(&sm.bar_load[i & 1], (i >> 1) & 1);
     }
     __syncwarp();
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
     // ---------------- compute warps ----------------
-    float kpos[8], vpos[8], kmag[8], vmag[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      kpos[i] = (i < HK - 1) ? a.k_boundaries[HK + i] : 0.f;
-      vpos[i] = (i < HV - 1) ? a.v_boundaries[HV + i] : 0.f;
-      kmag[i] = (i < HK) ? a.k_centroids[HK + i] : 0.f;
-      vmag[i] = (i < HV) ? a.v_centroids[HV + i] : 0.f;
-    }
+    typedef Fields<KB, kMerged> FK;
+    typedef Fields<VB, false> FV;
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    bool failed = false;
-    for (int j = 0; j < my_tiles; ++j) {
+    auto token_ref = [&](int j) -> TokRef {
       int b, h, t0;
       tile_coords(j, b, h, t0);
       const int len = a.seq_lens[b];
       const int tok = t0 + row;
       const bool bad_len = len < 0 || len > a.max_len || len > a.cache.max_pages * PT;
-      bool valid = !bad_len && tok < len;
       if (bad_len && tid == 0 && t0 == 0) report(a.status, TQ_ERR_BOUNDS);
-      uint8_t* blk = nullptr;
-      const int slot = tok % PT;
-      if (valid) {
+      TokRef r{nullptr, tok % PT};
+      if (!bad_len && tok < len) {
         const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + tok / PT];
         if (phys < 0 || phys >= a.cache.num_pages) {
           if (part == 0) report(a.status, TQ_ERR_BOUNDS);
-          valid = false;
         } else {
-          blk = a.cache.block(phys, h);
+          r.blk = a.cache.block(phys, h);
         }
       }
-
-      // ---- forward result, per-token norms ----
-      if (!failed && !bar_wait(&sm.bar_fwd, j & 1)) failed = true;
-      __syncwarp();
-      tc_fence_after();
-      float y[32];
-      tmem_ld32(tmem + lane_base + kColK + 32 * part, y);
-      float z[32];
-      tmem_ld32(tmem + lane_base + kColV + 32 * part, z);
-      tmem_wait_ld();
-      const float ssk = sumsq32(y), ssv = sumsq32(z);
-      // every warp of the quadrant is past its reads of the previous tile's sketch
-      tc_fence_before();
-      quad_sync(qd);
-      tc_fence_after();
-      tmem_st2(tmem + lane_base + kColNormX + 2 * part, ssk, ssv);
+      return r;
+    };
+    // per-token sum over the two warps of the quadrant: each writes its part, then reads both
+    auto pair_sum = [&](uint32_t col, float v) -> float {
+      tmem_st1(tmem + lane_base + col + part, v);
       tmem_wait_st();
       tc_fence_before();
-      quad_sync(qd);
+      pair_sync(qd);
       tc_fence_after();
-      float nx[8];
-      tmem_ld8(tmem + lane_base + kColNormX, nx);
+      float x[2];
+      tmem_ld2(tmem + lane_base + col, x);
       tmem_wait_ld();
-      const float nyk = sqrtf((nx[0] + nx[2]) + (nx[4] + nx[6]));  // ||y'_K|| = sqrt(d) ||k||
-      const float nyv = sqrtf((nx[1] + nx[3]) + (nx[5] + nx[7]));
+      return x[0] + x[1];
+    };
+    // key words of the previous tile, completed by its sketch signs one tile later
+    TokRef prev{nullptr, 0};
+    uint32_t pkw[8];
+    uint32_t pnorms = 0;  // fp16 ||k|| | fp16 rho << 16
+    auto finish_keys = [&](const float (&s0)[32], const float (&s1)[32]) {
+      constexpr uint32_t sg0 = FK::sig_init();
+      uint32_t sgw[2] = {sg0, sg0};
+      sigma32<kMerged, FK, 0>(s0, pkw, sgw);
+      sigma32<kMerged, FK, 32>(s1, pkw, sgw);
+      if (prev.blk != nullptr) {
+        store_words<KB, kMerged>(prev.blk + L.kc, part, prev.slot, pkw);
+        if (!kMerged)
+          *reinterpret_cast<uint2*>(prev.blk + L.ks + (size_t)prev.slot * 16 + 8 * part) = make_uint2(sgw[0], sgw[1]);
+        if (part == 0) {
+          reinterpret_cast<uint16_t*>(prev.blk + L.kn)[prev.slot] = (uint16_t)(pnorms & 0xffff);
+          reinterpret_cast<uint16_t*>(prev.blk + L.kr)[prev.slot] = (uint16_t)(pnorms >> 16);
+        }
+      }
+    };
+    bool failed = false;
+    for (int j = 0; j < my_tiles; ++j) {
+      const TokRef cur = token_ref(j);
+      const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
+      const uint32_t ks_p = (j & 1) ? kColKS0 : kColKS1;
 
-      // ---- keys ----
-      const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
-      if (valid && part == 0 && __hisinf(nk16)) report(a.status, TQ_ERR_OVERFLOW);
-      float thr[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) thr[k] = kpos[k] * nyk;
-      const float alpha = nyk > 0.f ? kResidScale / nyk : 1.f;
-      float am[8];
-      const float csa = alpha * kSqrtD * __half2float(nk16);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) am[k] = csa * kmag[k];
-      uint32_t kw[4] = {0, 0, 0, 0};
-      float rr = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        uint32_t m[8];
-        const uint32_t r = rank_masks<HK - 1>(y[i], thr, m);
-        const uint32_t smask = gt_mask(y[i], 0.f);
-        if constexpr (kMerged) {
-          kw[i >> 3] += r << (4 * (i & 7));
-          kw[i >> 3] |= smask & (4u << (4 * (i & 7)));
-        } else {
-          pack_plain<KB>(kw, i, r, smask);
-        }
-        if constexpr (KQ) {
-          // signed centroid a cs c[idx] from the masks, then the scaled residual
-          uint32_t c = __float_as_uint(am[0]);
-#pragma unroll
-          for (int k = 1; k < HK; ++k) c = (m[k - 1] & __float_as_uint(am[k])) | (~m[k - 1] & c);
-          c ^= ~smask & 0x80000000u;
-          const float rv = fmaf(y[i], alpha, -__uint_as_float(c));
-          y[i] = rv;
-          rr = fmaf(rv, rv, rr);
-        }
-      }
-      float rho = 0.f;
-      if constexpr (KQ) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float r0 = y[2 * i], r1 = y[2 * i + 1];
-          const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
-          const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
-          const __half2 hh = __floats2half2_rn(h0, h1);
-          const __half2 ll = __floats2half2_rn(r0 - h0, r1 - h1);
-          hi[i] = *reinterpret_cast<const uint32_t*>(&hh);
-          lo[i] = *reinterpret_cast<const uint32_t*>(&ll);
-        }
-        tmem_st16(tmem + lane_base + kColAhi + 16 * part, hi);
-        tmem_st16(tmem + lane_base + kColAlo + 16 * part, lo);
-        tmem_st1(tmem + lane_base + kColRrX + part, rr);
-        tmem_wait_st();
-        tc_fence_before();
-        quad_sync(qd);
-        tc_fence_after();
-        float rx[4];
-        tmem_ld4(tmem + lane_base + kColRrX, rx);
-        tmem_wait_ld();
-        rho = sqrtf((rx[0] + rx[1]) + (rx[2] + rx[3])) / (alpha * kSqrtD);
-      }
-      // ---- values: re-read y'_V (its columns are released after this) ----
-      tmem_ld32(tmem + lane_base + kColV + 32 * part, z);
+      // ---- y'_K and the key norm ----
+      if (!failed && !bar_wait(&sm.bar_fwdk, j & 1)) failed = true;
+      __syncwarp();
+      tc_fence_after();
+      float y0[32], y1[32];
+      tmem_ld32(tmem + lane_base + ks_j + kCPT * part, y0);
+      tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32, y1);
       tmem_wait_ld();
+      const float ssk = sumsq32(y0) + sumsq32(y1);
+      tc_fence_before();
+      pair_sync(qd);  // the quadrant's y'_K is read: its first columns take the exchange
+      tc_fence_after();
+      const float nyk = sqrtf(pair_sum(ks_j + kXssK, ssk));  // ||y'_K|| = sqrt(d) ||k||
+      if (!KQ || j == 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&sm.ks_free);
+      }
+      const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
+      if (cur.blk && part == 0 && __hisinf(nk16)) report(a.status, TQ_ERR_OVERFLOW);
+
+      // ---- keys: codes and (with QJL) the split residual ----
+      constexpr uint32_t kwi[8] = {FK::init(0), FK::init(1), FK::init(2), FK::init(3),
+                                   FK::init(4), FK::init(5), FK::init(6), FK::init(7)};
+      uint32_t kw[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kw[i] = kwi[i];
+      {
+        const QuantConst<HK - 1> qc(nyk, sm.kpos, sm.kmag, __half2float(nk16));
+        uint32_t hi0[16], lo0[16], hi1[16], lo1[16];
+        f2_t rr2 = 0;
+        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qc, kw, hi0, lo0, rr2);
+        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qc, kw, hi1, lo1, rr2);
+        if constexpr (KQ) {
+          // A (and the residual norm) once the previous sketch is done with A
+          if (j > 0 && !failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
+          __syncwarp();
+          tc_fence_after();
+          tmem_st16(tmem + lane_base + kColA + 32 * part, hi0);
+          tmem_st16(tmem + lane_base + kColA + 32 * part + 16, hi1);
+          tmem_st16(tmem + lane_base + kColA + 64 + 32 * part, lo0);
+          tmem_st16(tmem + lane_base + kColA + 64 + 32 * part + 16, lo1);
+          float ra, rb;
+          uf2(rr2, ra, rb);
+          const float rho = sqrtf(pair_sum(ks_j + kXrr, ra + rb)) * qc.inv_alpha * (1.0f / kSqrtD);
+          // ... and the previous tile's signs, which that sketch produced
+          if (j > 0) {
+            tmem_ld32(tmem + lane_base + ks_p + kCPT * part, y0);
+            tmem_ld32(tmem + lane_base + ks_p + kCPT * part + 32, y1);
+            tmem_wait_ld();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            bar_arrive(&sm.a_ready);
+            if (j > 0) bar_arrive(&sm.ks_free);
+          }
+          if (j > 0) {
+            if (failed) prev.blk = nullptr;
+            finish_keys(y0, y1);
+          }
+          prev = failed ? TokRef{nullptr, 0} : cur;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) pkw[i] = kw[i];
+          pnorms = (uint32_t)__half_as_ushort(nk16) | ((uint32_t)__half_as_ushort(__float2half_rn(rho)) << 16);
+        } else if (cur.blk && !failed) {
+          store_words<KB, false>(cur.blk + L.kc, part, cur.slot, kw);
+          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+        }
+      }
+
+      // ---- y'_V, the value norm, value codes ----
+      if (!failed && !bar_wait(&sm.bar_fwdv, j & 1)) failed = true;
+      __syncwarp();
+      tc_fence_after();
+      tmem_ld32(tmem + lane_base + kColV + kCPT * part, y0);
+      tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32, y1);
+      tmem_wait_ld();
+      const float ssv = sumsq32(y0) + sumsq32(y1);
+      tc_fence_before();
+      pair_sync(qd);  // the quadrant's y'_V is read: its first columns take the exchange
+      tc_fence_after();
+      const float nyv = sqrtf(pair_sum(kColV + kXssV, ssv));
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        bar_arrive(&sm.kv_free);
-        if (KQ) bar_arrive(&sm.a_ready);
-      }
+      if (lane == 0) bar_arrive(&sm.v_free);
       const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
-      if (valid && part == 0 && __hisinf(nv16)) report(a.status, TQ_ERR_OVERFLOW);
+      if (cur.blk && part == 0 && __hisinf(nv16)) report(a.status, TQ_ERR_OVERFLOW);
+      {
+        constexpr uint32_t vwi[8] = {FV::init(0), FV::init(1), FV::init(2), FV::init(3),
+                                     FV::init(4), FV::init(5), FV::init(6), FV::init(7)};
+        uint32_t vw[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) thr[k] = vpos[k] * nyv;
-      uint32_t vw[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        uint32_t m[8];
-        const uint32_t r = rank_masks<HV - 1>(z[i], thr, m);
-        pack_plain<VB>(vw, i, r, gt_mask(z[i], 0.f));
+        for (int i = 0; i < 8; ++i) vw[i] = vwi[i];
+        const QuantConst<HV - 1> qc(nyv, sm.vpos, sm.vmag, 0.f);
+        uint32_t dh[16], dl[16];
+        f2_t drr = 0;
+        quantise32<HV - 1, FV, false, 0>(y0, qc, vw, dh, dl, drr);
+        quantise32<HV - 1, FV, false, 32>(y1, qc, vw, dh, dl, drr);
+        if (cur.blk && !failed) {
+          store_words<VB, false>(cur.blk + L.vc, part, cur.slot, vw);
+          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+        }
       }
-      if (valid && !failed) {
-        store_plain<VB>(blk + L.vc, part, slot, vw);
-        if (part == 0) reinterpret_cast<__half*>(blk + L.vn)[slot] = nv16;
-      }
-
-      // ---- QJL signs, then the key words ----
-      uint32_t sgw = 0;
-      if constexpr (KQ) {
-        if (!failed && !bar_wait(&sm.bar_sig, j & 1)) failed = true;
+    }
+    if constexpr (KQ) {
+      // the last tile's signs
+      if (my_tiles > 0) {
+        if (!failed && !bar_wait(&sm.bar_sig, (my_tiles - 1) & 1)) failed = true;
         __syncwarp();
         tc_fence_after();
-        tmem_ld32(tmem + lane_base + kColS + 32 * part, z);
+        const uint32_t ks_l = ((my_tiles - 1) & 1) ? kColKS1 : kColKS0;
+        float s0[32], s1[32];
+        tmem_ld32(tmem + lane_base + ks_l + kCPT * part, s0);
+        tmem_ld32(tmem + lane_base + ks_l + kCPT * part + 32, s1);
         tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint32_t sg = ge_mask(z[i], 0.f);
-          if constexpr (kMerged)
-            kw[i >> 3] |= sg & (8u << (4 * (i & 7)));
-          else
-            sgw |= sg & (1u << i);
-        }
-      }
-      if (valid && !failed) {
-        if constexpr (kMerged) {
-          *reinterpret_cast<uint4*>(blk + L.kc + ((size_t)part * PT + slot) * 16) =
-              make_uint4(kw[0], kw[1], kw[2], kw[3]);
-        } else {
-          store_plain<KB>(blk + L.kc, part, slot, kw);
-          if (KQ) *reinterpret_cast<uint32_t*>(blk + L.ks + (size_t)slot * 16 + 4 * part) = sgw;
-        }
-        if (part == 0) {
-          reinterpret_cast<__half*>(blk + L.kn)[slot] = nk16;
-          if (KQ) reinterpret_cast<__half*>(blk + L.kr)[slot] = __float2half_rn(rho);
-        }
+        if (failed) prev.blk = nullptr;
+        finish_keys(s0, s1);
       }
     }
     if (failed && lane == 0) report(a.status, TQ_ERR_TIMEOUT);
@@ -715,6 +898,11 @@ bool make_tile_map(CUtensorMap* m, const void* base, size_t rows) {
 template <int KB, int KQ, int VB>
 cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
   auto k = compress_tc_kernel<KB, KQ, VB>;
+  // the register hand-over inside the kernel assumes the launch allocation it was built for
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != kRegsLaunch ||
+      fa.maxThreadsPerBlock < kThreadsTC)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemTC);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;

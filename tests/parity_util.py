@@ -98,6 +98,27 @@ class CompressReport:
     norm_fail: int = 0
 
 
+def compare_compress_rows(fmt, u, K, V, R, ck, kb, cv, vb, S, rep: CompressReport):
+    """Compares unpacked GPU codes u (tokens in the order of the rows) with the oracle's
+    compression of the same float64 rows K, V [n][d]."""
+    kc = (oq.compress_prod(K, R, ck, kb, S) if fmt.key_qjl else oq.compress_mse(K, R, ck, kb))
+    vc = oq.compress_mse(V, R, cv, vb)
+    rep.tokens += K.shape[0]
+    kmis = _check_idx(u.k_idx, kc, kb, rep)
+    _check_idx(u.v_idx, vc, vb, rep)
+    rep.norm_fail += int(np.sum(~close(u.k_norm, kc.norm)))
+    rep.norm_fail += int(np.sum(~close(u.v_norm, vc.norm)))
+    if fmt.key_qjl:
+        ok_tok = ~kmis
+        rep.sign_tokens_skipped += int(np.sum(kmis))
+        rep.norm_fail += int(np.sum(~close(u.k_rnorm[ok_tok], kc.rnorm[ok_tok])))
+        diff = (u.k_sigma != kc.sigma) & ok_tok[:, None]
+        band = np.abs(kc.sr) <= SIGN_BAND * kc.sr_scale
+        rep.sign_mismatch_in_band += int(np.sum(diff & band))
+        rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
+    return rep
+
+
 def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport = None):
     """Compares the GPU's packed (layer, b, h) against the oracle on the same inputs.
     tokens: optional index array of positions to check (default all)."""
