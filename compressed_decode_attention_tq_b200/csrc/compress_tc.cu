@@ -60,14 +60,15 @@ constexpr unsigned long long kWaitNs = 1000000000ull;  // a wait gives up after 
 constexpr float kSqrtD = 11.313708498984761f;
 
 struct SmemTC {
-  unsigned char x[2][2][kTileBytes];  // [stage][K, V] input tiles (canonical layout)
+  unsigned char x[2][2][kTileBytes];  // [stage][K, V] input tiles (canonical layout); S at set-up
   unsigned char bhd[kTileBytes];      // B = H D
   unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part
   unsigned char bslo[kTileBytes];     // fp16 lo part
-  unsigned long long bar_load[2], stage_free[2], bar_fwdk, bar_fwdv, bar_sig, ks_free, a_ready, v_free;
+  unsigned long long bar_load[2], stage_free[2], bar_fwdk, bar_fwdv, bar_sig, ks_free, a_ready, v_free, bar_setup;
   uint32_t tmem_base;
   int bad_s;
-  float kpos[8], vpos[8], kmag[8], vmag[8];  // positive boundaries / centroid magnitudes
+  float signs[D];                        // D of the rotation
+  float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
 };
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
 
@@ -478,6 +479,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     bar_init(&sm.ks_free, kComputeWarps);
     bar_init(&sm.a_ready, kComputeWarps);
     bar_init(&sm.v_free, kComputeWarps);
+    bar_init(&sm.bar_setup, 1);
     sm.bad_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -487,32 +489,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // tile 0 streams in while the rotation operands are built (stage 1 is set-up scratch)
   if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) issue_load(0);
   __syncwarp();
-  if (tid == 0 && blockIdx.x == 0) {
-    for (int i = 0; i < 2 * HK; ++i)
-      if (a.k_centroids[i] != -a.k_centroids[2 * HK - 1 - i]) report(a.status, TQ_ERR_INVALID_ARG);
-    for (int i = 0; i < 2 * HV; ++i)
-      if (a.v_centroids[i] != -a.v_centroids[2 * HV - 1 - i]) report(a.status, TQ_ERR_INVALID_ARG);
-    // the rank rule reads only the positive boundaries: they must mirror, middle one 0
-    for (int i = 0; i < 2 * HK - 1; ++i)
-      if (a.k_boundaries[i] != -a.k_boundaries[2 * HK - 2 - i]) report(a.status, TQ_ERR_INVALID_ARG);
-    for (int i = 0; i < 2 * HV - 1; ++i)
-      if (a.v_boundaries[i] != -a.v_boundaries[2 * HV - 2 - i]) report(a.status, TQ_ERR_INVALID_ARG);
-  }
-  if (tid < 8) {
-    sm.kpos[tid] = (tid < HK - 1) ? a.k_boundaries[HK + tid] : 0.f;
-    sm.vpos[tid] = (tid < HV - 1) ? a.v_boundaries[HV + tid] : 0.f;
-    sm.kmag[tid] = (tid < HK) ? a.k_centroids[HK + tid] : 0.f;
-    sm.vmag[tid] = (tid < HV) ? a.v_centroids[HV + tid] : 0.f;
-  }
   if (!producer) {
+    // small inputs once into shared memory, one load per thread
+    if (tid < D) sm.signs[tid] = a.signs[tid];
+    if (tid < 16) {
+      sm.kc[tid] = tid < 2 * HK ? a.k_centroids[tid] : 0.f;
+      sm.kb[tid] = tid < 2 * HK - 1 ? a.k_boundaries[tid] : 0.f;
+      sm.vc[tid] = tid < 2 * HV ? a.v_centroids[tid] : 0.f;
+      sm.vb[tid] = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
+    }
+    asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
+    if (tid == 0 && blockIdx.x == 0) {
+      bool sym = true;
+      for (int i = 0; i < 2 * HK; ++i) sym &= sm.kc[i] == -sm.kc[2 * HK - 1 - i];
+      for (int i = 0; i < 2 * HV; ++i) sym &= sm.vc[i] == -sm.vc[2 * HV - 1 - i];
+      // the rank rule reads only the positive boundaries: they must mirror, middle one 0
+      for (int i = 0; i < 2 * HK - 1; ++i) sym &= sm.kb[i] == -sm.kb[2 * HK - 2 - i];
+      for (int i = 0; i < 2 * HV - 1; ++i) sym &= sm.vb[i] == -sm.vb[2 * HV - 2 - i];
+      if (!sym) report(a.status, TQ_ERR_INVALID_ARG);
+    }
     // B = H D: row i, column k = (-1)^popcount(i & k) D_k
-    for (int c = tid; c < D * 16; c += kComputeThreads) {
+#pragma unroll
+    for (int it = 0; it < D * 16 / kComputeThreads; ++it) {
+      const int c = tid + it * kComputeThreads;
       const int i = c & 127, ch = c >> 7;
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k0 = ch * 8 + 2 * e;
-        const float s0 = a.signs[k0], s1 = a.signs[k0 + 1];
+        const float s0 = sm.signs[k0], s1 = sm.signs[k0 + 1];
         const float v0 = (__popc(i & k0) & 1) ? -s0 : s0;
         const float v1 = (__popc(i & (k0 + 1)) & 1) ? -s1 : s1;
         const __half2 h = __floats2half2_rn(v0, v1);
@@ -521,70 +526,28 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       *reinterpret_cast<uint4*>(sm.bhd + canon(i, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (KQ) {
-      // B = S D H: for row n of S D, coordinate block p (32 wide) is transformed in
-      // registers (butterfly spans 1..16); the spans 32 and 64 meet through scratch.
-      float* scr = reinterpret_cast<float*>(sm.x[1][0]);  // [coordinate][n], 64 KB
-      const int n = tid & 127;
+      // S (fp16-exact by contract) as an fp16 A operand in stage 1; S D H = S (H D)^T is then
+      // one MMA against the B = H D operand above
+      unsigned char* sa = sm.x[1][0];
       int bad = 0;
-#pragma unroll 1
-      for (int p = tid >> 7; p < 4; p += kComputeThreads / 128) {
-        float v[32];
-        const float4* srow = reinterpret_cast<const float4*>(a.s + (size_t)n * D + 32 * p);
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 q = srow[i4];
-          const float e[4] = {q.x, q.y, q.z, q.w};
+      for (int it = 0; it < QM * 16 / kComputeThreads; ++it) {
+        const int c = tid + it * kComputeThreads;
+        const int m = c & 127, ch = c >> 7;
+        const float4* src = reinterpret_cast<const float4*>(a.s + (size_t)m * D + 8 * ch);
+        const float4 q0 = src[0], q1 = src[1];
+        const float e[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint32_t w[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int i = 4 * i4 + u;
-            if (__half2float(__float2half_rn(e[u])) != e[u]) bad = 1;
-            v[i] = e[u] * a.signs[32 * p + i];
-          }
+        for (int u = 0; u < 4; ++u) {
+          const __half2 h = __floats2half2_rn(e[2 * u], e[2 * u + 1]);
+          const float2 hf = __half22float2(h);
+          if (hf.x != e[2 * u] || hf.y != e[2 * u + 1]) bad = 1;
+          w[u] = *reinterpret_cast<const uint32_t*>(&h);
         }
-#pragma unroll
-        for (int hs = 1; hs < 32; hs <<= 1) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i & hs) continue;
-            const float u = v[i], w = v[i + hs];
-            v[i] = u + w;
-            v[i + hs] = u - w;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) scr[(32 * p + i) * 128 + n] = v[i];
+        *reinterpret_cast<uint4*>(sa + canon(m, 8 * ch)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (bad) sm.bad_s = 1;
-      asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
-#pragma unroll 1
-      for (int p = tid >> 7; p < 4; p += kComputeThreads / 128) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float x2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int i = 8 * c + 2 * e + u;
-              float acc = 0.f;
-#pragma unroll
-              for (int bb = 0; bb < 4; ++bb) {
-                const float t = scr[(32 * bb + i) * 128 + n];
-                acc += (__popc(p & bb) & 1) ? -t : t;
-              }
-              x2[u] = acc;
-            }
-            const __half2 h2 = __floats2half2_rn(x2[0], x2[1]);
-            const float2 hf = __half22float2(h2);
-            const __half2 l2 = __floats2half2_rn(x2[0] - hf.x, x2[1] - hf.y);
-            hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
-            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
-          }
-          *reinterpret_cast<uint4*>(sm.bshi + canon(n, 32 * p + 8 * c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(sm.bslo + canon(n, 32 * p + 8 * c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
-      }
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -600,6 +563,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // warps have written A; forward V into V once the previous y'_V is read.  Copies: tile
     // j + 2 into stage j & 1 as soon as both forward MMAs of tile j have read it.  Each wait's
     // phase is one the other side cannot run two phases past.
+    if (warp == kComputeWarps && lane == 0 && KQ) {
+      // S D H into KS[1] (free until tile 1): read out by the compute warps before tile 0
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + kColKS1, smem_desc(sm.x[1][0], ks), smem_desc(sm.bhd, ks), ks > 0);
+      mma_commit(&sm.bar_setup);
+    }
     if (warp == kComputeWarps && lane == 0 && my_tiles > 0) {
       auto fwd = [&](int j, uint32_t dcol, int kv) {
 #pragma unroll
@@ -649,12 +619,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (!ok) report(a.status, TQ_ERR_TIMEOUT);
     } else if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) {
       int issued = 1;  // tile 0 went out before the set-up
-      if (my_tiles > 1) {
+      bool ok = true;
+      // stage 1 holds S until the S D H MMA has read it
+      if (KQ && !(ok = bar_wait(&sm.bar_setup, 0))) report(a.status, TQ_ERR_TIMEOUT);
+      if (ok && my_tiles > 1) {
         issue_load(1);
         issued = 2;
       }
-      bool ok = true;
-      for (int i = 0; i + 2 < my_tiles; ++i) {
+      for (int i = 0; ok && i + 2 < my_tiles; ++i) {
         // phase i >> 1 of stage_free[i & 1]: the forward MMAs of tile i are done with it
         if (!(ok = bar_wait(&sm.stage_free[i & 1], (i >> 1) & 1))) break;
         issue_load(i + 2);
@@ -722,6 +694,37 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
     };
     bool failed = false;
+    if constexpr (KQ) {
+      // S D H (fp32 in KS[1], row = sketch index) split into the fp16 hi / lo B operands
+      if (!bar_wait(&sm.bar_setup, 0)) failed = true;
+      __syncwarp();
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + kColKS1 + kCPT * part + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
+            const __half2 h2 = __floats2half2_rn(x0, x1);
+            const float2 hf = __half22float2(h2);
+            const __half2 l2 = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+            hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+          }
+          const int k = kCPT * part + 32 * c + 8 * g;
+          *reinterpret_cast<uint4*>(sm.bshi + canon(row, k)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sm.bslo + canon(row, k)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+      // visible to the sketch MMAs, which wait for a_ready after these writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+    }
     for (int j = 0; j < my_tiles; ++j) {
       const TokRef cur = token_ref(j);
       const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
@@ -755,7 +758,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) kw[i] = kwi[i];
       {
-        const QuantConst<HK - 1> qc(nyk, sm.kpos, sm.kmag, __half2float(nk16));
+        const QuantConst<HK - 1> qc(nyk, sm.kb + HK, sm.kc + HK, __half2float(nk16));
         uint32_t hi0[16], lo0[16], hi1[16], lo1[16];
         f2_t rr2 = 0;
         quantise32<HK - 1, FK, KQ != 0, 0>(y0, qc, kw, hi0, lo0, rr2);
@@ -821,7 +824,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         uint32_t vw[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) vw[i] = vwi[i];
-        const QuantConst<HV - 1> qc(nyv, sm.vpos, sm.vmag, 0.f);
+        const QuantConst<HV - 1> qc(nyv, sm.vb + HV, sm.vc + HV, 0.f);
         uint32_t dh[16], dl[16];
         f2_t drr = 0;
         quantise32<HV - 1, FV, false, 0>(y0, qc, vw, dh, dl, drr);
