@@ -237,6 +237,9 @@ def run_ours(args, rank, world, local_rank):
     w = workload()
     if args.n_splits:
         w.n_splits = args.n_splits
+    else:
+        from compressed_decode_attention_tq_b200.runtime import default_splits
+        w.n_splits = default_splits(w.batch, w.kv_heads, local_rank)
     L = args.layers
     rin = wl.rotation_inputs(w)
     lens = wl.seq_lens(w)

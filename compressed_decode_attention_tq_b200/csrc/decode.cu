@@ -47,36 +47,32 @@ __device__ __forceinline__ float block_max128(float v, float* red) {
 __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_rows) {
   // allow the dependent split kernel to start streaming pages right away
   asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float qs[D];
-  __shared__ float red[4];
+  __shared__ float qs[D], ys[D];
+  __shared__ float red[2][4];
   __shared__ int ired[4];
-  const int i = threadIdx.x;
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   const int row = blockIdx.x;
   if (row >= total_rows) return;
-  float x;
-  if (a.q_dtype == TQ_F16)
-    x = __half2float(reinterpret_cast<const __half*>(a.q)[(size_t)row * D + i]);
-  else
-    x = reinterpret_cast<const float*>(a.q)[(size_t)row * D + i];
+  // the merge counters of the fused split kernel start every call at zero
+  if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads) a.counter[row] = 0u;
+  const float x = a.q_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.q)[(size_t)row * D + i])
+                                      : reinterpret_cast<const float*>(a.q)[(size_t)row * D + i];
+  qs[i] = x;
+  __syncthreads();
   float y;
   if (!a.dense) {
-    // y = H D q / sqrt(d): butterflies in shared memory
-    qs[i] = x * a.signs[i];
-    __syncthreads();
+    // y = H D q / sqrt(d): the warp-level transform in warp 0
+    if (warp == 0) {
+      float v[4];
 #pragma unroll
-    for (int h = 1; h < D; h <<= 1) {
-      const float u = qs[i], v = qs[i ^ h];
-      __syncthreads();
-      qs[i] = (i & h) ? (v - u) : (u + v);
-      __syncthreads();
+      for (int e = 0; e < 4; ++e) v[e] = qs[lane + 32 * e] * a.signs[lane + 32 * e];
+      fwht128_warp(v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ys[lane + 32 * e] = v[e] * kInvSqrtD;
     }
-    y = qs[i] * kInvSqrtD;
     __syncthreads();
-    qs[i] = x;
-    __syncthreads();
+    y = ys[i];
   } else {
-    qs[i] = x;
-    __syncthreads();
     const float4* prow = reinterpret_cast<const float4*>(a.pi + (size_t)i * D);
     float acc = 0.f;
 #pragma unroll 8
@@ -90,35 +86,55 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
     y = acc;
   }
   a.qrot[(size_t)row * D + i] = y;
-  const float ym = block_max128(fabsf(y), red);
+  float sq = 0.f;
+  if (a.qjl) {
+    // (S q)_o for the 32 outputs o of this warp: lanes read 4 consecutive entries of row o
+    // (coalesced), then a warp sum; all 32 row loads are in flight together
+    const float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
+    float4 p[32];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) p[u] = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      float t = p[u].x * q4.x;
+      t = fmaf(p[u].y, q4.y, t);
+      t = fmaf(p[u].z, q4.z, t);
+      t = fmaf(p[u].w, q4.w, t);
+      t = warp_sum(t);
+      if (lane == u) sq = t;
+    }
+    a.sq[(size_t)row * QM + 32 * warp + lane] = sq;
+  }
+  // maxima of |R q| and |S q| over the row
+  float my = fabsf(y), ms = fabsf(sq);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    my = fmaxf(my, __shfl_xor_sync(FULL, my, o));
+    ms = fmaxf(ms, __shfl_xor_sync(FULL, ms, o));
+  }
+  if (lane == 0) {
+    red[0][warp] = my;
+    red[1][warp] = ms;
+  }
+  __syncthreads();
+  const float ym = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
   const float lam = ym > 0.f ? 127.f / ym : 0.f;
   a.q8[(size_t)row * D + i] = (int8_t)__float2int_rn(y * lam);
   if (i == 0) a.q8_scale[row] = lam;
   if (a.qjl) {
-    const float4* srow = reinterpret_cast<const float4*>(a.s + (size_t)i * D);
-    float acc = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < D / 4; ++k) {
-      const float4 p = srow[k];
-      acc = fmaf(p.x, qs[4 * k], acc);
-      acc = fmaf(p.y, qs[4 * k + 1], acc);
-      acc = fmaf(p.z, qs[4 * k + 2], acc);
-      acc = fmaf(p.w, qs[4 * k + 3], acc);
-    }
-    a.sq[(size_t)row * QM + i] = acc;
-    const float mx = block_max128(fabsf(acc), red);
+    const float mx = fmaxf(fmaxf(red[1][0], red[1][1]), fmaxf(red[1][2], red[1][3]));
     // 16-bit fixed point with a power-of-two scale: |sq_int| <= 32000
     int ex = 0;
     if (mx > 0.f) {
       frexpf(32000.f / mx, &ex);
       ex -= 1;  // 2^ex <= 32000 / mx
     }
-    const int v = __float2int_rn(acc * ldexpf(1.f, ex));
-    a.sq_int[(size_t)row * QM + i] = (int16_t)v;
+    const int v = __float2int_rn(sq * ldexpf(1.f, ex));
+    a.sq_int[(size_t)row * QM + 32 * warp + lane] = (int16_t)v;
     int sum = v;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
-    if ((i & 31) == 0) ired[i >> 5] = sum;
+    if (lane == 0) ired[warp] = sum;
     __syncthreads();
     if (i == 0) {
       a.sq_scale[row] = ldexpf(1.f, -ex);
@@ -381,6 +397,8 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   w.sq_sum = off; off = align256(off + rows * sizeof(int));
   w.q8 = off; off = align256(off + rows * D);
   w.q8_scale = off; off = align256(off + rows * sizeof(float));
+  // one counter per (sequence, kv head); kv_heads divides q_heads, so batch * q_heads bounds it
+  w.counter = off; off = align256(off + (size_t)batch * q_heads * sizeof(unsigned int));
   w.total = off;
   return w;
 }
@@ -423,10 +441,18 @@ static cudaError_t launch_pdl(void (*k)(Args...), dim3 grid, dim3 block, size_t 
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
+  if (fast_decode_supported(a)) {
+    // query transforms (and zeroed merge counters), then the split kernel, whose last
+    // split per (sequence, kv head) merges the partials: two launches
+    prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_fast_split(a, stream);
+  }
   prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = fast_decode_supported(a) ? launch_fast_split(a, stream) : launch_split(a, stream, false);
+  e = launch_split(a, stream, false);
   if (e != cudaSuccess) return e;
   e = launch_pdl(combine_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
   if (e != cudaSuccess) return e;

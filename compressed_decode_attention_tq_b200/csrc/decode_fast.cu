@@ -5,8 +5,9 @@
 // section "How is this different from PolarQuant's reconstruction?": pre-rotated
 // query), organised for B200:
 //
-//  * one producer warp streams each page of the split into a 3-stage shared-memory ring
-//    with bulk asynchronous copies (cp.async.bulk, completion on mbarriers);
+//  * one producer warp streams the split's half pages (128 tokens; the splits are dealt
+//    contiguous runs of half pages, so they stay balanced) into a 3-stage shared-memory
+//    ring with bulk asynchronous copies (cp.async.bulk, completion on mbarriers);
 //  * four consumer warps each take 16-token steps.  A lane dequantises codes straight
 //    into fp16 mma fragments with byte permutes against a centroid table held in
 //    registers; the key term  sum_j (R q)_j c[idx_j]  is an fp16 m16n8k16 mma (query in
@@ -14,7 +15,9 @@
 //    m16n8k32 mma on 16-bit fixed-point (S q) digits, and  sum_t p_t ||v_t|| c[idx]  an
 //    fp16 mma after an in-register 8x8 transpose (movmatrix) of the dequantised values;
 //  * online softmax per warp, then a log-sum-exp merge of the four warps; the partial
-//    (m, l, acc) per query row goes to the workspace for the combine kernel.
+//    (m, l, acc) per query row goes to the workspace, and the last split of each
+//    (sequence, kv head) to finish (a counter the prologue zeroes) merges all partials
+//    and applies R^T.
 //
 // Supported here: query rows per KV head R = G * seq_q <= 4, keys 3-bit + QJL (merged
 // nibbles) or 2-bit + QJL, values 3-bit or 2-bit.  Everything else uses decode.cu.
@@ -31,8 +34,10 @@ namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStages = 3;
-constexpr int kChunkStride = PT * 16 + 32;  // padded so the 4 lanes of a token group hit distinct banks
-constexpr int kNormBytes = 3 * PT * 2;      // KN | KR | VN
+constexpr int kUnit = PT / 2;                  // tokens per copy unit: half a page
+constexpr int kUnitsPerPage = PT / kUnit;
+constexpr int kChunkStride = kUnit * 16 + 32;  // padded so the 4 lanes of a token group hit distinct banks
+constexpr int kNormBytes = 3 * kUnit * 2;      // KN | KR | VN of the unit
 constexpr int kMaxKChunks = 4;
 constexpr int kMaxVChunks = 3;
 constexpr int kStageBytes = kNormBytes + (kMaxKChunks + kMaxVChunks) * kChunkStride;
@@ -50,6 +55,7 @@ struct SmemFast {
   unsigned long long empty[kStages];
   float wacc[kConsumerWarps][4][D];
   float wm[kConsumerWarps][4], wl[kConsumerWarps][4];
+  int last;
 };
 
 // ---------------------------------------------------------------------------
@@ -187,16 +193,17 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
   if (bad_len && tid == 0 && split == 0) report(a.status, TQ_ERR_BOUNDS);
   const int n_eff = bad_len ? 0 : len;
-  const int npages_all = (n_eff + PT - 1) / PT;
-  const int cp = (npages_all + a.n_splits - 1) / a.n_splits;
-  const int p_begin = min(npages_all, split * cp);
-  const int p_end = min(npages_all, (split + 1) * cp);
-  const int npages = p_end - p_begin;
-  const int t_end = min(n_eff, p_end * PT);
+  // the sequence in half-page units, dealt to the splits in contiguous runs
+  const int units_all = (n_eff + kUnit - 1) / kUnit;
+  const int cu = (units_all + a.n_splits - 1) / a.n_splits;
+  const int u_begin = min(units_all, split * cu);
+  const int u_end = min(units_all, (split + 1) * cu);
+  const int nunits = u_end - u_begin;
+  const int t_end = min(n_eff, u_end * kUnit);
 
   constexpr int kKChunks = (KP == K3Q) ? 4 : 3;  // K2Q: 2 code chunks + the KS chunk
   constexpr int kVChunks = (VP == V3) ? 3 : 2;
-  const uint32_t page_bytes = kNormBytes + 16u * PT * (kKChunks + kVChunks);
+  const uint32_t unit_bytes = kNormBytes + 16u * kUnit * (kKChunks + kVChunks);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -210,29 +217,33 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
     if (lane == 0) {
-      for (int i = 0; i < npages; ++i) {
+      for (int i = 0; i < nunits; ++i) {
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1)) {
           report(a.status, TQ_ERR_TIMEOUT);
           break;
         }
-        int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + p_begin + i];
+        const int u = u_begin + i, half = u % kUnitsPerPage;
+        int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + u / kUnitsPerPage];
         if (phys < 0 || phys >= a.cache.num_pages) {
           report(a.status, TQ_ERR_BOUNDS);
           phys = 0;
         }
         const unsigned char* blk = a.cache.block(phys, gh);
         unsigned char* st = sm.stage[s];
-        mbar_expect_tx(&sm.full[s], page_bytes);
-        bulk_g2s(st, blk, kNormBytes, &sm.full[s]);
+        const uint32_t hb2 = half * kUnit * 2, hb16 = half * kUnit * 16;
+        mbar_expect_tx(&sm.full[s], unit_bytes);
+        bulk_g2s(st, blk + L.kn + hb2, kUnit * 2, &sm.full[s]);
+        bulk_g2s(st + kUnit * 2, blk + L.kr + hb2, kUnit * 2, &sm.full[s]);
+        bulk_g2s(st + kUnit * 4, blk + L.vn + hb2, kUnit * 2, &sm.full[s]);
         unsigned char* kc = st + kNormBytes;
         const int kcode_chunks = (KP == K3Q) ? 4 : 2;
         for (int c = 0; c < kcode_chunks; ++c)
-          bulk_g2s(kc + c * kChunkStride, blk + L.kc + c * PT * 16, PT * 16, &sm.full[s]);
-        if (KP == K2Q) bulk_g2s(kc + 2 * kChunkStride, blk + L.ks, PT * 16, &sm.full[s]);
+          bulk_g2s(kc + c * kChunkStride, blk + L.kc + c * PT * 16 + hb16, kUnit * 16, &sm.full[s]);
+        if (KP == K2Q) bulk_g2s(kc + 2 * kChunkStride, blk + L.ks + hb16, kUnit * 16, &sm.full[s]);
         unsigned char* vc = kc + kMaxKChunks * kChunkStride;
         for (int c = 0; c < kVChunks; ++c)
-          bulk_g2s(vc + c * kChunkStride, blk + L.vc + c * PT * 16, PT * 16, &sm.full[s]);
+          bulk_g2s(vc + c * kChunkStride, blk + L.vc + c * PT * 16 + hb16, kUnit * 16, &sm.full[s]);
       }
     }
   } else {
@@ -420,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
 
-    for (int i = 0; i < npages; ++i) {
+    for (int i = 0; i < nunits; ++i) {
       const int s = i % kStages;
       if (!mbar_wait(&sm.full[s], (i / kStages) & 1)) {
         if (lane == 0) report(a.status, TQ_ERR_TIMEOUT);
@@ -429,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       const unsigned char* st = sm.stage[s];
       const unsigned char* kc = st + kNormBytes;
       const unsigned char* vc = kc + kMaxKChunks * kChunkStride;
-      const int tok0 = (p_begin + i) * PT;
-      const int valid = min(PT, t_end - tok0);
+      const int tok0 = (u_begin + i) * kUnit;
+      const int valid = min(kUnit, t_end - tok0);
       for (int step = warp; step * 16 < valid; step += kConsumerWarps) {
         const int ta = step * 16 + g, tb = ta + 8;
         // ---- keys: dequantise into fp16 A fragments and int8 sign fragments
@@ -484,18 +495,31 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             sb[k] = (sB << k) & 0x80808080u;
           }
         }
-        float dk[4] = {0.f, 0.f, 0.f, 0.f};
+        // two accumulators per term halve the dependent mma chains
+        float dk[4] = {0.f, 0.f, 0.f, 0.f}, dk2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
-        int dsum[4] = {0, 0, 0, 0};
+        for (int ks = 0; ks < 8; ks += 2) {
+          hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
+          hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[ks + 1][0], bq[ks + 1][1]);
+        }
+        int dsum[4] = {0, 0, 0, 0}, dsum2[4] = {0, 0, 0, 0};
+        int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
-        int dcor[4] = {0, 0, 0, 0};
+        for (int w = 0; w < 4; w += 2) {
+          imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
+          imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
+          imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
+          imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[w + 1][0], bc[w + 1][1]);
+        }
 #pragma unroll
-        for (int w = 0; w < 4; ++w) imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
+        for (int e = 0; e < 4; ++e) {
+          dk[e] += dk2[e];
+          dsum[e] += dsum2[e];
+          dcor[e] += dcor2[e];
+        }
         // ---- scores of row t4 for tokens ta, tb (log2 domain)
         const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
-        const float rA = ld_h(st + 2 * PT + 2 * ta), rB = ld_h(st + 2 * PT + 2 * tb);
+        const float rA = ld_h(st + 2 * kUnit + 2 * ta), rB = ld_h(st + 2 * kUnit + 2 * tb);
         const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
         const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
         const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
@@ -508,22 +532,27 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
         const float m_new = fmaxf(m_run, mx);
+        // the running sums are rescaled only in steps where some row maximum grew
+        const bool grow = __any_sync(FULL, m_new > m_run);
         float alpha = 1.f, pa = 0.f, pb = 0.f;
         if (m_new != -CUDART_INF_F) {
-          alpha = exp2f(m_run - m_new);
+          if (grow) alpha = exp2f(m_run - m_new);
           pa = exp2f(sca - m_new);
           pb = exp2f(scb - m_new);
         }
         l_run = l_run * alpha + pa + pb;
         m_run = m_new;
-        const float vnA = ld_h(st + 4 * PT + 2 * ta), vnB = ld_h(st + 4 * PT + 2 * tb);
+        const float vnA = ld_h(st + 4 * kUnit + 2 * ta), vnB = ld_h(st + 4 * kUnit + 2 * tb);
         // slots past the end may hold stale bytes: force their weight to exactly 0
         const uint32_t pk = pack_h2(ta < valid ? pa * vnA : 0.f, tb < valid ? pb * vnB : 0.f);
         const uint32_t x1 = __shfl_sync(FULL, pk, 4 * (2 * t4) + g);
         const uint32_t x2 = __shfl_sync(FULL, pk, 4 * (2 * t4 + 1) + g);
         const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
-        const float al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
-        const float al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
+        float al0 = 1.f, al1 = 1.f;
+        if (grow) {
+          al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
+          al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
+        }
         // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
         uint32_t va[16], vb[16];
         {
@@ -547,14 +576,17 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             vb[cb] = movm_t(xb);
           }
         }
+        if (grow) {
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          acc[mt][0] *= al0;
-          acc[mt][1] *= al1;
-          acc[mt][2] *= al0;
-          acc[mt][3] *= al1;
-          hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+          for (int mt = 0; mt < 8; ++mt) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
+          }
         }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
@@ -597,9 +629,50 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     const size_t pr = (row0 + r) * a.n_splits + split;
     a.part_acc[pr * D + j] = o;
     if (j == 0) {
-      // partials are kept in the natural-log domain for the combine kernel
+      // partials are kept in the natural-log domain for the merge
       a.part_ml[pr * 2] = (M == -CUDART_INF_F) ? M : M / kLog2e;
       a.part_ml[pr * 2 + 1] = l;
+    }
+  }
+  // ---- the last split of this (sequence, kv head) to finish merges all of them ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned int done = atomicAdd(&a.counter[(size_t)b * a.cache.kv_heads + gh], 1u);
+    sm.last = done == (unsigned int)a.n_splits - 1;
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  if (warp < R) {
+    // log-sum-exp merge of the splits' (m, l, acc), then out = R^T o / l = D H o / (sqrt(d) l)
+    const size_t rowq = row0 + warp;
+    const float* ml = a.part_ml + rowq * a.n_splits * 2;
+    const float* pa = a.part_acc + rowq * a.n_splits * D;
+    float M = -CUDART_INF_F;
+    for (int sp = lane; sp < a.n_splits; sp += 32) M = fmaxf(M, __ldcg(ml + 2 * sp));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
+    float l = 0.f, o4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (M != -CUDART_INF_F) {
+#pragma unroll 4
+      for (int sp = 0; sp < a.n_splits; ++sp) {
+        const float msp = __ldcg(ml + 2 * sp);
+        if (msp == -CUDART_INF_F) continue;
+        const float wgt = __expf(msp - M);
+        l = fmaf(wgt, __ldcg(ml + 2 * sp + 1), l);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o4[e] = fmaf(wgt, __ldcg(pa + (size_t)sp * D + lane + 32 * e), o4[e]);
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o4[e] *= inv;
+    fwht128_warp(o4, lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int jj = lane + 32 * e;
+      a.out[rowq * D + jj] = o4[e] * kInvSqrtD * a.signs[jj];
     }
   }
 }

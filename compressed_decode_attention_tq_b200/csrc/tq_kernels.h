@@ -33,6 +33,7 @@ struct DecodeArgs {
   int* sq_sum;      // [B*Hq*seq_q] workspace: sum_i sq_int
   int8_t* q8;       // [B*Hq*seq_q][D] workspace: R q in int8 (scaled by q8_scale)
   float* q8_scale;  // [B*Hq*seq_q] workspace
+  unsigned int* counter;  // [B*Hkv] workspace (sized B*Hq): finished splits per (sequence, kv head)
   float* out;       // [B*Hq*seq_q][D]
   float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
   int max_len;
@@ -55,7 +56,7 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream);
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {
-  size_t qrot, sq, part_acc, part_ml, sq_int, sq_scale, sq_sum, q8, q8_scale, total;
+  size_t qrot, sq, part_acc, part_ml, sq_int, sq_scale, sq_sum, q8, q8_scale, counter, total;
 };
 DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits);
 

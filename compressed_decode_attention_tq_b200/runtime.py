@@ -20,6 +20,13 @@ def _f32(x, device):
     return torch.as_tensor(x, dtype=torch.float32).to(device).contiguous()
 
 
+def default_splits(batch: int, kv_heads: int, device=None) -> int:
+    """Split count that fills the GPU once: the fast decode kernel keeps two CTAs per SM,
+    one CTA per (split, kv head, sequence)."""
+    sms = torch.cuda.get_device_properties(device if device is not None else 0).multi_processor_count
+    return max(1, min(1024, (2 * sms) // max(1, batch * kv_heads)))
+
+
 class PagedKV:
     """A packed TurboQuant cache for `num_layers` layers sharing one block table."""
 
