@@ -36,7 +36,7 @@ FALLBACK_HBM = 6650.0
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--layers", type=int, default=32)
@@ -63,10 +63,17 @@ def peaks():
         return FALLBACK_HBM, "fallback"
 
 
-def kernel_hash() -> str:
+# the sources each timed kernel is built from (its traffic entry is void once any changes)
+KERNEL_SOURCES = {
+    "compress_tc_kernel": ("compress_tc.cu", "tq_device.cuh", "tq_kernels.h"),
+    "fast_split_kernel": ("decode_fast.cu", "decode.cu", "tq_device.cuh", "tq_kernels.h"),
+}
+
+
+def kernel_hash(kernel: str) -> str:
     h = hashlib.sha256()
     src = os.path.join(ROOT, "compressed_decode_attention_tq_b200", "csrc")
-    for name in sorted(os.listdir(src)):
+    for name in KERNEL_SOURCES.get(kernel, tuple(sorted(os.listdir(src)))):
         with open(os.path.join(src, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -80,7 +87,7 @@ def traffic_for(kernel: str):
         with open(path) as f:
             d = json.load(f)
         ent = d[kernel]
-        if ent.get("source_hash") != kernel_hash():
+        if ent.get("source_hash") != kernel_hash(kernel):
             return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:
@@ -103,7 +110,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -306,11 +313,12 @@ def run_ours(args, rank, world, local_rank):
     comp_gbs = comp_bytes_launch / (comp_ms / L / 1e3) / 1e9
     dec_gbs = dec_bytes_launch / (dec_ms / L / 1e3) / 1e9
     phases = {
-        "compress": {"kernel": "compress_kernel", "ms_per_step": comp_ms, "launches_per_step": L,
+        "compress": {"kernel": "compress_tc_kernel", "ms_per_step": comp_ms, "launches_per_step": L,
                      "keys_per_s": L * tok_heads_layer / (comp_ms / 1e3),
                      "algorithmic_bytes_per_launch": comp_bytes_launch, "achieved_gbs": comp_gbs,
                      "frac": comp_gbs / hbm},
-        "decode": {"kernel": "prologue+split+combine", "ms_per_step": dec_ms, "launches_per_step": L,
+        "decode": {"kernel": "fast_split_kernel", "ms_per_step": dec_ms, "launches_per_step": 2 * L,
+                   "kernels": "prologue_kernel + fast_split_kernel",
                    "kv_tokens_per_s": L * tok_heads_layer / (dec_ms / 1e3),
                    "algorithmic_bytes_per_launch": dec_bytes_launch, "achieved_gbs": dec_gbs,
                    "frac": dec_gbs / hbm},
@@ -339,7 +347,9 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(w, L), "phases": phases, "roofline": roofline,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps * L * 4,
+            "cpu_baseline": cpu, "e2e": e2e,
+            # per layer: compress_tc_kernel, then prologue_kernel + fast_split_kernel
+            "gpu_launches": args.steps * L * 3,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
