@@ -55,6 +55,12 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
   if (row >= total_rows) return;
   // the merge counters of the fused split kernel start every call at zero
   if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads) a.counter[row] = 0u;
+  // the rows of S this warp needs, requested before the query (they do not depend on it)
+  float4 p[32];
+  if (a.qjl) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) p[u] = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
+  }
   const float x = a.q_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.q)[(size_t)row * D + i])
                                       : reinterpret_cast<const float*>(a.q)[(size_t)row * D + i];
   qs[i] = x;
@@ -91,9 +97,6 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
     // (S q)_o for the 32 outputs o of this warp: lanes read 4 consecutive entries of row o
     // (coalesced), then a warp sum; all 32 row loads are in flight together
     const float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
-    float4 p[32];
-#pragma unroll
-    for (int u = 0; u < 32; ++u) p[u] = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
 #pragma unroll
     for (int u = 0; u < 32; ++u) {
       float t = p[u].x * q4.x;

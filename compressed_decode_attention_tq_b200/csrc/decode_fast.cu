@@ -635,45 +635,63 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     }
   }
   // ---- the last split of this (sequence, kv head) to finish merges all of them ----
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
+    // the CTA's partial writes are ordered before the count by the barrier and this fence
+    __threadfence();
     const unsigned int done = atomicAdd(&a.counter[(size_t)b * a.cache.kv_heads + gh], 1u);
     sm.last = done == (unsigned int)a.n_splits - 1;
   }
   __syncthreads();
   if (!sm.last) return;
   __threadfence();
-  if (warp < R) {
-    // log-sum-exp merge of the splits' (m, l, acc), then out = R^T o / l = D H o / (sqrt(d) l)
-    const size_t rowq = row0 + warp;
-    const float* ml = a.part_ml + rowq * a.n_splits * 2;
-    const float* pa = a.part_acc + rowq * a.n_splits * D;
-    float M = -CUDART_INF_F;
-    for (int sp = lane; sp < a.n_splits; sp += 32) M = fmaxf(M, __ldcg(ml + 2 * sp));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
-    float l = 0.f, o4[4] = {0.f, 0.f, 0.f, 0.f};
-    if (M != -CUDART_INF_F) {
-#pragma unroll 4
-      for (int sp = 0; sp < a.n_splits; ++sp) {
-        const float msp = __ldcg(ml + 2 * sp);
-        if (msp == -CUDART_INF_F) continue;
-        const float wgt = __expf(msp - M);
-        l = fmaf(wgt, __ldcg(ml + 2 * sp + 1), l);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o4[e] = fmaf(wgt, __ldcg(pa + (size_t)sp * D + lane + 32 * e), o4[e]);
-      }
+  const int ns = a.n_splits;
+  if (tid < 32 * R) {
+    // thread (row r, float4 c4) of the output: online log-sum-exp over the splits'
+    // (m, l, acc), sixteen splits' loads in flight at a time
+    const int r = tid >> 5, c4 = tid & 31;
+    const size_t rowq = row0 + r;
+    const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * ns * 2);
+    const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
+    float M = -CUDART_INF_F, l = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 16
+    for (int sp = 0; sp < ns; ++sp) {
+      const float2 m2 = __ldcg(ml2 + sp);
+      const float4 v = __ldcg(pa4 + (size_t)sp * (D / 4));
+      // branch-free update (the loads of later splits do not wait on it)
+      const float Mn = fmaxf(M, m2.x);
+      const bool live = Mn != -CUDART_INF_F;
+      const float f = live ? __expf(M - Mn) : 1.f;
+      const float wgt = live ? __expf(m2.x - Mn) : 0.f;
+      l = fmaf(wgt, m2.y, l * f);
+      o.x = fmaf(wgt, v.x, o.x * f);
+      o.y = fmaf(wgt, v.y, o.y * f);
+      o.z = fmaf(wgt, v.z, o.z * f);
+      o.w = fmaf(wgt, v.w, o.w * f);
+      M = Mn;
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o4[e] *= inv;
-    fwht128_warp(o4, lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int jj = lane + 32 * e;
-      a.out[rowq * D + jj] = o4[e] * kInvSqrtD * a.signs[jj];
+    // out = D H (o / l) / sqrt(d): H over coordinates 4 c4 + e, spans 1 and 2 in the
+    // thread, spans 4..64 across the row's 32 lanes
+    float x[4] = {o.x * inv, o.y * inv, o.z * inv, o.w * inv};
+    {
+      const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
+      x[0] = a0 + a2;
+      x[1] = a1 + a3;
+      x[2] = a0 - a2;
+      x[3] = a1 - a3;
     }
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float y = __shfl_xor_sync(FULL, x[e], h);
+        x[e] = (c4 & h) ? (y - x[e]) : (x[e] + y);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a.out[rowq * D + 4 * c4 + e] = x[e] * kInvSqrtD * a.signs[4 * c4 + e];
   }
 }
 
