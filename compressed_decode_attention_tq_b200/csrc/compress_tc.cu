@@ -15,9 +15,9 @@
 //    well; three MMAs (hi.hi, hi.lo, lo.hi) give the projections to ~2^-22 relative.
 //
 // Quantisation works on y' directly: |y| > beta  <=>  |y'| > beta ||y'||, so each token
-// scales its boundaries once instead of normalising every coordinate, and the rank is a
-// sum of comparison masks (the boundaries are sorted) that also drive the centroid
-// select of the residual.
+// scales its boundaries once instead of normalising every coordinate; the rank is a sum
+// of saturated unit steps (the boundaries are sorted), and the residual's centroid is read
+// from a table by the code field just formed.
 //
 // One persistent CTA per SM: 8 compute warps and a producer warpgroup.  Compute warp w
 // reads tensor-memory lane quadrant w % 4 (tokens 32 (w % 4) .. + 31) and coordinates
@@ -69,6 +69,7 @@ struct SmemTC {
   int bad_s;
   float signs[D];                        // D of the rotation
   float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
+  float kcode_c[8];                      // c[idx] of a key code field r + sw s
 };
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
 
@@ -311,78 +312,64 @@ __device__ __forceinline__ void store_words(uint8_t* base, int part, int slot, c
   }
 }
 
-// Boundary scales of one token: |y| > beta ||y'||  <=>  bq y'^2 - bq (beta ||y'||)^2 > 0 with
-// bq = 2^(40 - 2e) for ||y'|| ~ 2^e, so a saturated step is exact outside a 2^-40
-// relative band; bs = 2^(40 - e) makes y' bs a step for s = [y' > 0].
+// Boundary scales of one token: |y| > beta ||y'||  <=>  bs |y'| - bs beta ||y'|| > 0 with
+// bs = 2^(40 - e) for ||y'|| ~ 2^e: one fused multiply-add of |y'| (exact product, one
+// rounding, so the sign is exact), saturated to [0, 1], is a unit step outside a 2^-40
+// relative band; bs y' saturated is the step s = [y' > 0].
 struct TokScale {
   int e;
-  float bq, bs;
+  float bs;
   __device__ __forceinline__ explicit TokScale(float ny) {
     e = min(max((int)((__float_as_uint(ny) >> 23) & 0xff) - 127, -40), 40);
-    bq = __uint_as_float((uint32_t)(127 + 40 - 2 * e) << 23);
     bs = __uint_as_float((uint32_t)(127 + 40 - e) << 23);
   }
 };
 
-// Per-token constants of the quantiser: squared scaled boundaries, and with QJL the
-// residual scale a = 2^(8 - e) and the thermometer centroid steps a sqrt(d) fp16(||x||) dc.
+// Per-token constants of the quantiser: the scaled boundaries, and with QJL the residual
+// scale a = 2^(8 - e) and a sqrt(d) fp16(||x||).
 template <int NB>
 struct QuantConst {
   TokScale ts;
-  float t2[NB > 0 ? NB : 1];
-  float alpha, inv_alpha;
-  f2_t dam[NB > 0 ? NB : 1], am0;
-  __device__ __forceinline__ QuantConst(float ny, const float* pos, const float* mag, float cnorm) : ts(ny) {
+  float tb[NB > 0 ? NB : 1];  // -bs beta_k ||y'||
+  float alpha, inv_alpha, csa;
+  __device__ __forceinline__ QuantConst(float ny, const float* pos, float cnorm) : ts(ny) {
 #pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      const float t = pos[k] * ny;
-      t2[k] = -(t * t) * ts.bq;
-    }
+    for (int k = 0; k < NB; ++k) tb[k] = -(pos[k] * ny) * ts.bs;
     alpha = __uint_as_float((uint32_t)(127 + 8 - ts.e) << 23);
     inv_alpha = __uint_as_float((uint32_t)(127 - 8 + ts.e) << 23);
-    const float csa = alpha * kSqrtD * cnorm;
-#pragma unroll
-    for (int k = 0; k < NB; ++k) dam[k] = f2s(csa * (mag[k + 1] - mag[k]));
-    am0 = f2s(csa * mag[0]);
+    csa = alpha * kSqrtD * cnorm;
   }
 };
 
 // Codes of 32 of this thread's coordinates (OFF .. OFF + 31) of y'; with KQ also the scaled
-// residual a (y' - sqrt(d) fp16(||x||) c[idx]) split into fp16 hi / lo pairs for the
-// sketch MMAs, and its sum of squares (accumulated into rr2).
+// residual a y' - a sqrt(d) fp16(||x||) c[idx] (c[idx] read from the table of signed
+// centroids by the code just formed) split into fp16 hi / lo pairs for the sketch MMAs, and
+// its sum of squares (accumulated into rr2).
 template <int NB, class F, bool KQ, int OFF>
-__device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, uint32_t (&w)[8],
-                                           uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
+__device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, const float* ctab,
+                                           uint32_t (&w)[8], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float y0 = y[i], y1 = y[i + 1];
-    const f2_t Y = f2(y0, y1);
-    float yb0, yb1;
-    uf2(mul2(Y, f2s(qc.ts.bq)), yb0, yb1);
-    f2_t M[NB > 0 ? NB : 1];
     f2_t sum = f2s(kMagic);
 #pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      M[k] = f2(fma_sat(yb0, y0, qc.t2[k]), fma_sat(yb1, y1, qc.t2[k]));
-      sum = add2(sum, M[k]);
-    }
+    for (int k = 0; k < NB; ++k)
+      sum = add2(sum, f2(fma_sat(fabsf(y0), qc.ts.bs, qc.tb[k]), fma_sat(fabsf(y1), qc.ts.bs, qc.tb[k])));
     const f2_t S = f2(mul_sat(y0, qc.ts.bs), mul_sat(y1, qc.ts.bs));  // s = [y' > 0]
     if (F::sw) sum = fma2(S, f2s((float)F::sw), sum);
     float c0, c1;
     uf2(sum, c0, c1);
-    w[F::word(OFF + i)] += __float_as_uint(c0) << F::shift(OFF + i);
-    w[F::word(OFF + i + 1)] += __float_as_uint(c1) << F::shift(OFF + i + 1);
+    const uint32_t code0 = __float_as_uint(c0), code1 = __float_as_uint(c1);
+    w[F::word(OFF + i)] += code0 << F::shift(OFF + i);
+    w[F::word(OFF + i + 1)] += code1 << F::shift(OFF + i + 1);
     if (F::plane) {
       uf2(add2(S, f2s(kMagic)), c0, c1);
       w[4 + (OFF >> 5)] += __float_as_uint(c0) << plane_bit(i);
       w[4 + (OFF >> 5)] += __float_as_uint(c1) << plane_bit(i + 1);
     }
     if constexpr (KQ) {
-      f2_t C = qc.am0;
-#pragma unroll
-      for (int k = 0; k < NB; ++k) C = fma2(M[k], qc.dam[k], C);
-      const f2_t negsgn = fma2(S, f2s(-2.f), f2s(1.f));  // 1 - 2 s
-      const f2_t R = fma2(Y, f2s(qc.alpha), mul2(C, negsgn));
+      const f2_t C = f2(ctab[code0 & 7], ctab[code1 & 7]);
+      const f2_t R = fma2(C, f2s(-qc.csa), mul2(f2(y0, y1), f2s(qc.alpha)));
       rr2 = fma2(R, R, rr2);
       float r0, r1;
       uf2(R, r0, r1);
@@ -499,6 +486,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       sm.vb[tid] = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
     }
     asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
+    if (tid < 8) {
+      // code field f = r + sw s (merged keys: r + 4 s; 2-bit: r + 2 s) -> c[s ? h + r : h - 1 - r]
+      constexpr int sw = Fields<KB, kMerged>::sw > 0 ? Fields<KB, kMerged>::sw : HK;
+      const int r = tid % sw, sg = tid / sw;
+      sm.kcode_c[tid] = (sg <= 1 && r < HK) ? sm.kc[sg ? HK + r : HK - 1 - r] : 0.f;
+    }
     if (tid == 0 && blockIdx.x == 0) {
       bool sym = true;
       for (int i = 0; i < 2 * HK; ++i) sym &= sm.kc[i] == -sm.kc[2 * HK - 1 - i];
@@ -758,11 +751,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) kw[i] = kwi[i];
       {
-        const QuantConst<HK - 1> qc(nyk, sm.kb + HK, sm.kc + HK, __half2float(nk16));
+        const QuantConst<HK - 1> qc(nyk, sm.kb + HK, __half2float(nk16));
         uint32_t hi0[16], lo0[16], hi1[16], lo1[16];
         f2_t rr2 = 0;
-        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qc, kw, hi0, lo0, rr2);
-        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qc, kw, hi1, lo1, rr2);
+        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qc, sm.kcode_c, kw, hi0, lo0, rr2);
+        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qc, sm.kcode_c, kw, hi1, lo1, rr2);
         if constexpr (KQ) {
           // A (and the residual norm) once the previous sketch is done with A
           if (j > 0 && !failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
@@ -824,11 +817,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         uint32_t vw[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) vw[i] = vwi[i];
-        const QuantConst<HV - 1> qc(nyv, sm.vb + HV, sm.vc + HV, 0.f);
+        const QuantConst<HV - 1> qc(nyv, sm.vb + HV, 0.f);
         uint32_t dh[16], dl[16];
         f2_t drr = 0;
-        quantise32<HV - 1, FV, false, 0>(y0, qc, vw, dh, dl, drr);
-        quantise32<HV - 1, FV, false, 32>(y1, qc, vw, dh, dl, drr);
+        quantise32<HV - 1, FV, false, 0>(y0, qc, sm.kcode_c, vw, dh, dl, drr);
+        quantise32<HV - 1, FV, false, 32>(y1, qc, sm.kcode_c, vw, dh, dl, drr);
         if (cur.blk && !failed) {
           store_words<VB, false>(cur.blk + L.vc, part, cur.slot, vw);
           if (part == 0) reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
