@@ -477,6 +477,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) issue_load(0);
   __syncwarp();
   if (!producer) {
+    // S (fp16-exact by contract) is requested first: lanes read consecutive 16-byte pieces
+    // of a row (coalesced); it is converted and stored once the small tables are in
+    constexpr int kSIter = QM * 16 / kComputeThreads;
+    float4 sraw[KQ ? 2 * kSIter : 1];
+    if (KQ) {
+#pragma unroll
+      for (int it = 0; it < kSIter; ++it) {
+        const int c = tid + it * kComputeThreads;
+        const float4* src = reinterpret_cast<const float4*>(a.s + (size_t)(c >> 4) * D + 8 * (c & 15));
+        sraw[2 * it] = src[0];
+        sraw[2 * it + 1] = src[1];
+      }
+    }
     // small inputs once into shared memory, one load per thread
     if (tid < D) sm.signs[tid] = a.signs[tid];
     if (tid < 16) {
@@ -519,16 +532,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       *reinterpret_cast<uint4*>(sm.bhd + canon(i, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (KQ) {
-      // S (fp16-exact by contract) as an fp16 A operand in stage 1; S D H = S (H D)^T is then
-      // one MMA against the B = H D operand above
+      // S as an fp16 A operand in stage 1; S D H = S (H D)^T is then one MMA against the
+      // B = H D operand above
       unsigned char* sa = sm.x[1][0];
       int bad = 0;
 #pragma unroll
-      for (int it = 0; it < QM * 16 / kComputeThreads; ++it) {
+      for (int it = 0; it < kSIter; ++it) {
         const int c = tid + it * kComputeThreads;
-        const int m = c & 127, ch = c >> 7;
-        const float4* src = reinterpret_cast<const float4*>(a.s + (size_t)m * D + 8 * ch);
-        const float4 q0 = src[0], q1 = src[1];
+        const int m = c >> 4, ch = c & 15;
+        const float4 q0 = sraw[2 * it], q1 = sraw[2 * it + 1];
         const float e[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         uint32_t w[4];
 #pragma unroll
