@@ -48,11 +48,11 @@ static_assert(128 * kRegsProducer + 32 * kComputeWarps * kRegsCompute <= kThread
               "register split exceeds the launch allocation");
 constexpr int kTileBytes = TT * D * 2;       // one 128 x 128 fp16 operand
 // Tensor-memory columns.  KS[0], KS[1]: y'_K of a tile, then the per-token exchange slots
-// (+0 key sums of squares, +2 residual sums), then that tile's sketch (S D H) a r_rot';
-// alternate tiles use alternate halves.  V: y'_V of a tile, then (+0) the value sums of
-// squares.  A: the residual hi (+0) / lo (+64) halves, the sketch's A operand.
+// (+0..3 key and value sums of squares, +4..5 residual sums), then that tile's sketch
+// (S D H) a r_rot'; alternate tiles use alternate halves.  V: y'_V of a tile.  A: the
+// residual hi (+0) / lo (+64) halves, the sketch's A operand.
 constexpr uint32_t kColKS0 = 0, kColKS1 = 128, kColV = 256, kColA = 384;
-constexpr uint32_t kXssK = 0, kXrr = 2, kXssV = 0;
+constexpr uint32_t kXss = 0, kXrr = 4;
 constexpr uint32_t kTmemCols = 512;
 // instruction descriptor: D f32, A and B f16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -183,6 +183,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
   uint32_t r0, r1;
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
@@ -197,6 +206,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, float a, float b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(__float_as_uint(a)),
+               "r"(__float_as_uint(b))
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, float a) {
@@ -593,14 +608,21 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int j = 0; j < my_tiles && ok; ++j) {
         const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
         if (j + 1 < my_tiles) {
+          // y'_V of tile j is in the compute warps' registers (v_free phase j arrives after
+          // each warp has waited for it): the next one may land
+          if (!(ok = bar_wait(&sm.v_free, j & 1))) break;
+          if (!(ok = bar_wait(&sm.bar_load[(j + 1) & 1], ((j + 1) >> 1) & 1))) break;
+          tc_fence_after();
+          fwd(j + 1, kColV, 1);
+          mma_commit(&sm.bar_fwdv);
           // phase j of ks_free arrives in tile j, after every compute warp has waited for
           // y'_K of tile j: with QJL once tile j - 1's sketch in KS[(j + 1) & 1] is read
-          // (in tile 0 right after the wait), without QJL once tile j's exchange is done
+          // (in tile 0 right after the norms), without QJL once tile j's exchange is done
           if (!(ok = bar_wait(&sm.ks_free, j & 1))) break;
-          if (!(ok = bar_wait(&sm.bar_load[(j + 1) & 1], ((j + 1) >> 1) & 1))) break;
           tc_fence_after();
           fwd(j + 1, (j & 1) ? kColKS0 : kColKS1, 0);
           mma_commit(&sm.bar_fwdk);
+          mma_commit(&sm.stage_free[(j + 1) & 1]);  // both forward MMAs of tile j + 1 read it
         }
         if (KQ) {
           if (!(ok = bar_wait(&sm.a_ready, j & 1))) break;
@@ -612,13 +634,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             mma_ts(tmem + ks_j, tmem + kColA + 64 + 8 * ks, smem_desc(sm.bshi, ks), 1);
           }
           mma_commit(&sm.bar_sig);
-        }
-        if (j + 1 < my_tiles) {
-          if (!(ok = bar_wait(&sm.v_free, j & 1))) break;
-          tc_fence_after();
-          fwd(j + 1, kColV, 1);
-          mma_commit(&sm.bar_fwdv);
-          mma_commit(&sm.stage_free[(j + 1) & 1]);
         }
       }
       if (!ok) report(a.status, TQ_ERR_TIMEOUT);
@@ -735,39 +750,66 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
       const uint32_t ks_p = (j & 1) ? kColKS0 : kColKS1;
 
-      // ---- y'_K and the key norm ----
+      // ---- y'_K and y'_V of the tile, both norms in one exchange ----
       if (!failed && !bar_wait(&sm.bar_fwdk, j & 1)) failed = true;
+      if (!failed && !bar_wait(&sm.bar_fwdv, j & 1)) failed = true;
       __syncwarp();
       tc_fence_after();
-      float y0[32], y1[32];
+      float y0[32], y1[32], z0[32], z1[32];
       tmem_ld32(tmem + lane_base + ks_j + kCPT * part, y0);
       tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32, y1);
+      tmem_ld32(tmem + lane_base + kColV + kCPT * part, z0);
+      tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32, z1);
       tmem_wait_ld();
-      const float ssk = sumsq32(y0) + sumsq32(y1);
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(&sm.v_free);  // y'_V is in registers: the next one may land
+      const float ssk = sumsq32(y0) + sumsq32(y1), ssv = sumsq32(z0) + sumsq32(z1);
       pair_sync(qd);  // the quadrant's y'_K is read: its first columns take the exchange
       tc_fence_after();
-      const float nyk = sqrtf(pair_sum(ks_j + kXssK, ssk));  // ||y'_K|| = sqrt(d) ||k||
+      tmem_st2(tmem + lane_base + ks_j + kXss + 2 * part, ssk, ssv);
+      tmem_wait_st();
+      tc_fence_before();
+      pair_sync(qd);
+      tc_fence_after();
+      float xs[4];
+      tmem_ld4(tmem + lane_base + ks_j + kXss, xs);
+      tmem_wait_ld();
       if (!KQ || j == 0) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) bar_arrive(&sm.ks_free);
       }
+      const float nyk = sqrtf(xs[0] + xs[2]);  // ||y'_K|| = sqrt(d) ||k||
+      const float nyv = sqrtf(xs[1] + xs[3]);
       const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
-      if (cur.blk && part == 0 && __hisinf(nk16)) report(a.status, TQ_ERR_OVERFLOW);
+      const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
+      if (cur.blk && part == 0 && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
 
-      // ---- keys: codes and (with QJL) the split residual ----
+      // ---- values and keys, chunk by chunk (independent work side by side) ----
       constexpr uint32_t kwi[8] = {FK::init(0), FK::init(1), FK::init(2), FK::init(3),
                                    FK::init(4), FK::init(5), FK::init(6), FK::init(7)};
-      uint32_t kw[8];
+      constexpr uint32_t vwi[8] = {FV::init(0), FV::init(1), FV::init(2), FV::init(3),
+                                   FV::init(4), FV::init(5), FV::init(6), FV::init(7)};
+      uint32_t kw[8], vw[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) kw[i] = kwi[i];
+      for (int i = 0; i < 8; ++i) {
+        kw[i] = kwi[i];
+        vw[i] = vwi[i];
+      }
       {
-        const QuantConst<HK - 1> qc(nyk, sm.kb + HK, __half2float(nk16));
-        uint32_t hi0[16], lo0[16], hi1[16], lo1[16];
-        f2_t rr2 = 0;
-        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qc, sm.kcode_c, kw, hi0, lo0, rr2);
-        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qc, sm.kcode_c, kw, hi1, lo1, rr2);
+        const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
+        const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
+        uint32_t hi0[16], lo0[16], hi1[16], lo1[16], dh[16], dl[16];
+        f2_t rr2 = 0, drr = 0;
+        quantise32<HV - 1, FV, false, 0>(z0, qv, sm.kcode_c, vw, dh, dl, drr);
+        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qk, sm.kcode_c, kw, hi0, lo0, rr2);
+        quantise32<HV - 1, FV, false, 32>(z1, qv, sm.kcode_c, vw, dh, dl, drr);
+        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qk, sm.kcode_c, kw, hi1, lo1, rr2);
+        if (cur.blk && !failed) {
+          store_words<VB, false>(cur.blk + L.vc, part, cur.slot, vw);
+          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+        }
         if constexpr (KQ) {
           // A (and the residual norm) once the previous sketch is done with A
           if (j > 0 && !failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
@@ -779,7 +821,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           tmem_st16(tmem + lane_base + kColA + 64 + 32 * part + 16, lo1);
           float ra, rb;
           uf2(rr2, ra, rb);
-          const float rho = sqrtf(pair_sum(ks_j + kXrr, ra + rb)) * qc.inv_alpha * (1.0f / kSqrtD);
+          const float rho = sqrtf(pair_sum(ks_j + kXrr, ra + rb)) * qk.inv_alpha * (1.0f / kSqrtD);
           // ... and the previous tile's signs, which that sketch produced
           if (j > 0) {
             tmem_ld32(tmem + lane_base + ks_p + kCPT * part, y0);
@@ -803,40 +845,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         } else if (cur.blk && !failed) {
           store_words<KB, false>(cur.blk + L.kc, part, cur.slot, kw);
           if (part == 0) reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
-        }
-      }
-
-      // ---- y'_V, the value norm, value codes ----
-      if (!failed && !bar_wait(&sm.bar_fwdv, j & 1)) failed = true;
-      __syncwarp();
-      tc_fence_after();
-      tmem_ld32(tmem + lane_base + kColV + kCPT * part, y0);
-      tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32, y1);
-      tmem_wait_ld();
-      const float ssv = sumsq32(y0) + sumsq32(y1);
-      tc_fence_before();
-      pair_sync(qd);  // the quadrant's y'_V is read: its first columns take the exchange
-      tc_fence_after();
-      const float nyv = sqrtf(pair_sum(kColV + kXssV, ssv));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(&sm.v_free);
-      const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
-      if (cur.blk && part == 0 && __hisinf(nv16)) report(a.status, TQ_ERR_OVERFLOW);
-      {
-        constexpr uint32_t vwi[8] = {FV::init(0), FV::init(1), FV::init(2), FV::init(3),
-                                     FV::init(4), FV::init(5), FV::init(6), FV::init(7)};
-        uint32_t vw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) vw[i] = vwi[i];
-        const QuantConst<HV - 1> qc(nyv, sm.vb + HV, 0.f);
-        uint32_t dh[16], dl[16];
-        f2_t drr = 0;
-        quantise32<HV - 1, FV, false, 0>(y0, qc, sm.kcode_c, vw, dh, dl, drr);
-        quantise32<HV - 1, FV, false, 32>(y1, qc, sm.kcode_c, vw, dh, dl, drr);
-        if (cur.blk && !failed) {
-          store_words<VB, false>(cur.blk + L.vc, part, cur.slot, vw);
-          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
         }
       }
     }
