@@ -745,8 +745,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
     }
+    // the token address of the next tile is looked up one tile ahead (its global loads
+    // overlap this tile's work)
+    TokRef next = my_tiles > 0 ? token_ref(0) : TokRef{nullptr, 0};
     for (int j = 0; j < my_tiles; ++j) {
-      const TokRef cur = token_ref(j);
+      const TokRef cur = next;
+      if (j + 1 < my_tiles) next = token_ref(j + 1);
       const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
       const uint32_t ks_p = (j & 1) ? kColKS0 : kColKS1;
 
