@@ -47,12 +47,12 @@ constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsCompute = 216;
 static_assert(128 * kRegsProducer + 32 * kComputeWarps * kRegsCompute <= kThreadsTC * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr int kTileBytes = TT * D * 2;       // one 128 x 128 fp16 operand
-// Tensor-memory columns.  KS[0], KS[1]: y'_K of a tile, then the per-token exchange slots
-// (+0..3 key and value sums of squares, +4..5 residual sums), then that tile's sketch
-// (S D H) a r_rot'; alternate tiles use alternate halves.  V: y'_V of a tile.  A: the
-// residual hi (+0) / lo (+64) halves, the sketch's A operand.
-constexpr uint32_t kColKS0 = 0, kColKS1 = 128, kColV = 256, kColA = 384;
-constexpr uint32_t kXss = 0, kXrr = 4;
+// Tensor-memory columns.  KS[0], KS[1]: y'_K of a tile (alternate tiles, alternate
+// blocks); as each 32-coordinate chunk of it is read, the chunk's scaled residual is
+// written in its place as fp16 hi (first 16 columns) and lo (next 16): the sketch's A
+// operand.  V: y'_V of a tile.  X: the sketch (S D H) a r_rot' of a tile, then (+0, +1) the
+// residual sums of the two warps of a token.
+constexpr uint32_t kColKS0 = 0, kColKS1 = 128, kColV = 256, kColX = 384;
 constexpr uint32_t kTmemCols = 512;
 // instruction descriptor: D f32, A and B f16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -67,9 +67,9 @@ struct SmemTC {
   unsigned long long bar_load[2], stage_free[2], bar_fwdk, bar_fwdv, bar_sig, ks_free, a_ready, v_free, bar_setup;
   uint32_t tmem_base;
   int bad_s;
-  float signs[D];                        // D of the rotation
   float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
   float kcode_c[8];                      // c[idx] of a key code field r + sw s
+  float2 red[TT][2];                     // per-token sums of the two warps of a token
 };
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
 
@@ -283,11 +283,11 @@ __host__ __device__ constexpr uint32_t magic_at(int sh) {
 // (the permutation of sign_plane_pos, which the decode's byte tables read).
 __host__ __device__ constexpr int plane_bit(int e) { return 4 * (e >> 3) + (e & 3) + 16 * ((e >> 2) & 1); }
 
-// Where coordinate i (0..63 of this thread's coordinates) of a b-bit code lands in the
-// thread's words.  Field = r + sw * s:
-//   b = 2: 2-bit r | s << 1 (words 0..3);  b = 3: 2-bit r (words 0..3) and s in words 4, 5
-//   at the permuted sign-plane bit;  b = 4: r | s << 3 (words 0..7);  merged 3-bit key:
-//   r | s << 2 | sigma << 3 (words 0..7).
+// Where coordinate i (0..31 of one 32-coordinate chunk) of a b-bit code lands in the
+// chunk's four words.  Field = r + sw * s:
+//   b = 2: 2-bit r | s << 1 (words 0, 1);  b = 3: 2-bit r (words 0, 1) and s in word 2 at
+//   the permuted sign-plane bit;  b = 4: r | s << 3 (words 0..3);  merged 3-bit key:
+//   r | s << 2 | sigma << 3 (words 0..3).
 template <int B, bool MERGED>
 struct Fields {
   static constexpr bool nib = MERGED || B == 4;
@@ -298,9 +298,9 @@ struct Fields {
   // minus the magic bits the code (and, merged, sigma) adds of every coordinate of word w
   __host__ __device__ static constexpr uint32_t init(int w) {
     uint32_t c = 0;
-    for (int i = 0; i < kCPT; ++i) {
+    for (int i = 0; i < 32; ++i) {
       if (word(i) == w) c += magic_at(shift(i)) * (MERGED ? 2u : 1u);
-      if (plane && w == 4 + (i >> 5)) c += magic_at(plane_bit(i & 31));
+      if (plane && w == 2) c += magic_at(plane_bit(i));
     }
     return 0u - c;
   }
@@ -311,19 +311,15 @@ struct Fields {
   }
 };
 
-// Store a thread's code words for one token slot (plane p = 16 bytes per slot; this
-// thread's coordinates 64 part .. 64 part + 63).
+// Store the words of one chunk (coordinates 64 part + 32 c .. + 31) of a token slot
+// (plane p = 16 bytes per slot).
 template <int B, bool MERGED>
-__device__ __forceinline__ void store_words(uint8_t* base, int part, int slot, const uint32_t (&w)[8]) {
-  if constexpr (B == 2) {
-    *reinterpret_cast<uint4*>(base + ((size_t)part * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else if constexpr (B == 3 && !MERGED) {
-    *reinterpret_cast<uint4*>(base + ((size_t)part * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint2*>(base + ((size_t)2 * PT + slot) * 16 + 8 * part) = make_uint2(w[4], w[5]);
+__device__ __forceinline__ void store_chunk(uint8_t* base, int part, int c, int slot, const uint4& w) {
+  if constexpr (B == 2 || (B == 3 && !MERGED)) {
+    *reinterpret_cast<uint2*>(base + ((size_t)part * PT + slot) * 16 + 8 * c) = make_uint2(w.x, w.y);
+    if constexpr (B == 3) *reinterpret_cast<uint32_t*>(base + ((size_t)2 * PT + slot) * 16 + 4 * (2 * part + c)) = w.z;
   } else {
-    *reinterpret_cast<uint4*>(base + ((size_t)(2 * part) * PT + slot) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(base + ((size_t)(2 * part + 1) * PT + slot) * 16) =
-        make_uint4(w[4], w[5], w[6], w[7]);
+    *reinterpret_cast<uint4*>(base + ((size_t)(2 * part + c) * PT + slot) * 16) = w;
   }
 }
 
@@ -356,13 +352,13 @@ struct QuantConst {
   }
 };
 
-// Codes of 32 of this thread's coordinates (OFF .. OFF + 31) of y'; with KQ also the scaled
+// Codes of one 32-coordinate chunk of y' into the chunk's words w; with KQ also the scaled
 // residual a y' - a sqrt(d) fp16(||x||) c[idx] (c[idx] read from the table of signed
 // centroids by the code just formed) split into fp16 hi / lo pairs for the sketch MMAs, and
 // its sum of squares (accumulated into rr2).
-template <int NB, class F, bool KQ, int OFF>
+template <int NB, class F, bool KQ>
 __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, const float* ctab,
-                                           uint32_t (&w)[8], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
+                                           uint32_t (&w)[4], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float y0 = y[i], y1 = y[i + 1];
@@ -375,12 +371,12 @@ __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantCons
     float c0, c1;
     uf2(sum, c0, c1);
     const uint32_t code0 = __float_as_uint(c0), code1 = __float_as_uint(c1);
-    w[F::word(OFF + i)] += code0 << F::shift(OFF + i);
-    w[F::word(OFF + i + 1)] += code1 << F::shift(OFF + i + 1);
+    w[F::word(i)] += code0 << F::shift(i);
+    w[F::word(i + 1)] += code1 << F::shift(i + 1);
     if (F::plane) {
       uf2(add2(S, f2s(kMagic)), c0, c1);
-      w[4 + (OFF >> 5)] += __float_as_uint(c0) << plane_bit(i);
-      w[4 + (OFF >> 5)] += __float_as_uint(c1) << plane_bit(i + 1);
+      w[2] += __float_as_uint(c0) << plane_bit(i);
+      w[2] += __float_as_uint(c1) << plane_bit(i + 1);
     }
     if constexpr (KQ) {
       const f2_t C = f2(ctab[code0 & 7], ctab[code1 & 7]);
@@ -400,24 +396,26 @@ __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantCons
   }
 }
 
-// QJL signs sigma = [p >= 0] (1 also within 2^-40 below 0) of 32 of this thread's sketch
-// entries (OFF .. OFF + 31): merged into bit 3 of the key nibbles, or one sign-plane word.
-template <bool MERGED, class F, int OFF>
-__device__ __forceinline__ void sigma32(const float (&p)[32], uint32_t (&w)[8], uint32_t (&sgw)[2]) {
+// QJL signs sigma = [p >= 0] (1 also within 2^-40 below 0) of one 32-entry chunk of the
+// sketch: merged into bit 3 of the chunk's key nibbles, or one sign-plane word.
+template <bool MERGED, class F>
+__device__ __forceinline__ void sigma32(const float (&p)[32], uint4& w, uint32_t& sgw) {
+  uint32_t wa[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const f2_t G = f2(fma_sat(p[i], 1099511627776.f, 1.f), fma_sat(p[i + 1], 1099511627776.f, 1.f));
     float c0, c1;
     if constexpr (MERGED) {
       uf2(fma2(G, f2s(8.f), f2s(kMagic)), c0, c1);
-      w[F::word(OFF + i)] += __float_as_uint(c0) << F::shift(OFF + i);
-      w[F::word(OFF + i + 1)] += __float_as_uint(c1) << F::shift(OFF + i + 1);
+      wa[F::word(i)] += __float_as_uint(c0) << F::shift(i);
+      wa[F::word(i + 1)] += __float_as_uint(c1) << F::shift(i + 1);
     } else {
       uf2(add2(G, f2s(kMagic)), c0, c1);
-      sgw[OFF >> 5] += __float_as_uint(c0) << i;
-      sgw[OFF >> 5] += __float_as_uint(c1) << (i + 1);
+      sgw += __float_as_uint(c0) << i;
+      sgw += __float_as_uint(c1) << (i + 1);
     }
   }
+  w = make_uint4(wa[0], wa[1], wa[2], wa[3]);
 }
 
 // The cache block and slot of the token this thread owns in tile j (blk null when the
@@ -506,7 +504,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
     }
     // small inputs once into shared memory, one load per thread
-    if (tid < D) sm.signs[tid] = a.signs[tid];
+    // D of the rotation, for the set-up only (in the space of the S D H operand, filled later)
+    float* signs = reinterpret_cast<float*>(sm.bshi);
+    if (tid < D) signs[tid] = a.signs[tid];
     if (tid < 16) {
       sm.kc[tid] = tid < 2 * HK ? a.k_centroids[tid] : 0.f;
       sm.kb[tid] = tid < 2 * HK - 1 ? a.k_boundaries[tid] : 0.f;
@@ -538,7 +538,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int k0 = ch * 8 + 2 * e;
-        const float s0 = sm.signs[k0], s1 = sm.signs[k0 + 1];
+        const float s0 = signs[k0], s1 = signs[k0 + 1];
         const float v0 = (__popc(i & k0) & 1) ? -s0 : s0;
         const float v1 = (__popc(i & (k0 + 1)) & 1) ? -s1 : s1;
         const __half2 h = __floats2half2_rn(v0, v1);
@@ -608,16 +608,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int j = 0; j < my_tiles && ok; ++j) {
         const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
         if (j + 1 < my_tiles) {
-          // y'_V of tile j is in the compute warps' registers (v_free phase j arrives after
-          // each warp has waited for it): the next one may land
+          // y'_V of tile j has been read (v_free phase j arrives after each compute warp has
+          // waited for it and read it): the next one may land
           if (!(ok = bar_wait(&sm.v_free, j & 1))) break;
           if (!(ok = bar_wait(&sm.bar_load[(j + 1) & 1], ((j + 1) >> 1) & 1))) break;
           tc_fence_after();
           fwd(j + 1, kColV, 1);
           mma_commit(&sm.bar_fwdv);
-          // phase j of ks_free arrives in tile j, after every compute warp has waited for
-          // y'_K of tile j: with QJL once tile j - 1's sketch in KS[(j + 1) & 1] is read
-          // (in tile 0 right after the norms), without QJL once tile j's exchange is done
+          // KS[(j + 1) & 1] holds tile j - 1's A: its sketch must be done with it (this thread
+          // issued it and consumes each sketch commit in turn); ks_free phase j arrives after
+          // every compute warp has waited for y'_K of tile j
+          if (KQ && j >= 1 && !(ok = bar_wait(&sm.bar_sig, (j - 1) & 1))) break;
           if (!(ok = bar_wait(&sm.ks_free, j & 1))) break;
           tc_fence_after();
           fwd(j + 1, (j & 1) ? kColKS0 : kColKS1, 0);
@@ -625,18 +626,26 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mma_commit(&sm.stage_free[(j + 1) & 1]);  // both forward MMAs of tile j + 1 read it
         }
         if (KQ) {
+          // A of tile j is in KS[j & 1] and X is free (the previous sketch was read)
           if (!(ok = bar_wait(&sm.a_ready, j & 1))) break;
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            mma_ts(tmem + ks_j, tmem + kColA + 8 * ks, smem_desc(sm.bshi, ks), ks > 0);
-            mma_ts(tmem + ks_j, tmem + kColA + 8 * ks, smem_desc(sm.bslo, ks), 1);
-            mma_ts(tmem + ks_j, tmem + kColA + 64 + 8 * ks, smem_desc(sm.bshi, ks), 1);
+            // coordinates 16 ks ..: part ks / 4, chunk (ks / 2) % 2, half ks % 2
+            const uint32_t ahi = tmem + ks_j + 64 * (ks >> 2) + 32 * ((ks >> 1) & 1) + 8 * (ks & 1);
+            mma_ts(tmem + kColX, ahi, smem_desc(sm.bshi, ks), ks > 0);
+            mma_ts(tmem + kColX, ahi, smem_desc(sm.bslo, ks), 1);
+            mma_ts(tmem + kColX, ahi + 16, smem_desc(sm.bshi, ks), 1);
           }
           mma_commit(&sm.bar_sig);
         }
       }
-      if (!ok) report(a.status, TQ_ERR_TIMEOUT);
+      if (!ok) {
+        report(a.status, TQ_ERR_TIMEOUT);
+        // let the MMAs already issued finish (bounded) before tensor memory is freed
+        mma_commit(&sm.bar_setup);
+        bar_wait(&sm.bar_setup, KQ ? 1 : 0);
+      }
     } else if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) {
       int issued = 1;  // tile 0 went out before the set-up
       bool ok = true;
@@ -682,35 +691,37 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       return r;
     };
-    // per-token sum over the two warps of the quadrant: each writes its part, then reads both
-    auto pair_sum = [&](uint32_t col, float v) -> float {
-      tmem_st1(tmem + lane_base + col + part, v);
-      tmem_wait_st();
-      tc_fence_before();
+    // per-token sum over the two warps of a token, through shared memory; the barrier
+    // before the write keeps the partner's reads of the previous use ahead of it
+    auto pair_sum2 = [&](float u, float v) -> float2 {
       pair_sync(qd);
-      tc_fence_after();
-      float x[2];
-      tmem_ld2(tmem + lane_base + col, x);
-      tmem_wait_ld();
-      return x[0] + x[1];
+      sm.red[row][part] = make_float2(u, v);
+      pair_sync(qd);
+      const float2 a0 = sm.red[row][0], a1 = sm.red[row][1];
+      return make_float2(a0.x + a1.x, a0.y + a1.y);
     };
     // key words of the previous tile, completed by its sketch signs one tile later
     TokRef prev{nullptr, 0};
-    uint32_t pkw[8];
+    uint4 pk[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     uint32_t pnorms = 0;  // fp16 ||k|| | fp16 rho << 16
-    auto finish_keys = [&](const float (&s0)[32], const float (&s1)[32]) {
-      constexpr uint32_t sg0 = FK::sig_init();
-      uint32_t sgw[2] = {sg0, sg0};
-      sigma32<kMerged, FK, 0>(s0, pkw, sgw);
-      sigma32<kMerged, FK, 32>(s1, pkw, sgw);
-      if (prev.blk != nullptr) {
-        store_words<KB, kMerged>(prev.blk + L.kc, part, prev.slot, pkw);
-        if (!kMerged)
-          *reinterpret_cast<uint2*>(prev.blk + L.ks + (size_t)prev.slot * 16 + 8 * part) = make_uint2(sgw[0], sgw[1]);
-        if (part == 0) {
-          reinterpret_cast<uint16_t*>(prev.blk + L.kn)[prev.slot] = (uint16_t)(pnorms & 0xffff);
-          reinterpret_cast<uint16_t*>(prev.blk + L.kr)[prev.slot] = (uint16_t)(pnorms >> 16);
+    // the previous tile's signs from X, chunk by chunk, and its key words stored
+    auto finish_keys = [&]() {
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float sk[32];
+        tmem_ld32(tmem + lane_base + kColX + kCPT * part + 32 * c, sk);
+        tmem_wait_ld();
+        uint4 w = c ? pk[1] : pk[0];
+        uint32_t sgw = FK::sig_init();
+        sigma32<kMerged, FK>(sk, w, sgw);
+        if (prev.blk != nullptr) {
+          store_chunk<KB, kMerged>(prev.blk + L.kc, part, c, prev.slot, w);
+          if (!kMerged) *reinterpret_cast<uint32_t*>(prev.blk + L.ks + (size_t)prev.slot * 16 + 4 * (2 * part + c)) = sgw;
         }
+      }
+      if (prev.blk != nullptr && part == 0) {
+        reinterpret_cast<uint16_t*>(prev.blk + L.kn)[prev.slot] = (uint16_t)(pnorms & 0xffff);
+        reinterpret_cast<uint16_t*>(prev.blk + L.kr)[prev.slot] = (uint16_t)(pnorms >> 16);
       }
     };
     bool failed = false;
@@ -719,7 +730,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (!bar_wait(&sm.bar_setup, 0)) failed = true;
       __syncwarp();
       tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_base + kColKS1 + kCPT * part + 32 * c, v);
@@ -745,111 +756,92 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
     }
-    // the token address of the next tile is looked up one tile ahead (its global loads
-    // overlap this tile's work)
+    // the token address of the next tile is looked up one tile ahead
     TokRef next = my_tiles > 0 ? token_ref(0) : TokRef{nullptr, 0};
     for (int j = 0; j < my_tiles; ++j) {
       const TokRef cur = next;
       if (j + 1 < my_tiles) next = token_ref(j + 1);
       const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
-      const uint32_t ks_p = (j & 1) ? kColKS0 : kColKS1;
 
-      // ---- y'_K and y'_V of the tile, both norms in one exchange ----
+      // ---- norms of y'_K and y'_V ----
       if (!failed && !bar_wait(&sm.bar_fwdk, j & 1)) failed = true;
       if (!failed && !bar_wait(&sm.bar_fwdv, j & 1)) failed = true;
       __syncwarp();
       tc_fence_after();
-      float y0[32], y1[32], z0[32], z1[32];
-      tmem_ld32(tmem + lane_base + ks_j + kCPT * part, y0);
-      tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32, y1);
-      tmem_ld32(tmem + lane_base + kColV + kCPT * part, z0);
-      tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32, z1);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(&sm.v_free);  // y'_V is in registers: the next one may land
-      const float ssk = sumsq32(y0) + sumsq32(y1), ssv = sumsq32(z0) + sumsq32(z1);
-      pair_sync(qd);  // the quadrant's y'_K is read: its first columns take the exchange
-      tc_fence_after();
-      tmem_st2(tmem + lane_base + ks_j + kXss + 2 * part, ssk, ssv);
-      tmem_wait_st();
-      tc_fence_before();
-      pair_sync(qd);
-      tc_fence_after();
-      float xs[4];
-      tmem_ld4(tmem + lane_base + ks_j + kXss, xs);
-      tmem_wait_ld();
-      if (!KQ || j == 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) bar_arrive(&sm.ks_free);
+      if (lane == 0) bar_arrive(&sm.ks_free);  // this warp is past its wait for y'_K of tile j
+      float ssk = 0.f, ssv = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float y[32], z[32];
+        tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32 * c, y);
+        tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32 * c, z);
+        tmem_wait_ld();
+        ssk += sumsq32(y);
+        ssv += sumsq32(z);
       }
-      const float nyk = sqrtf(xs[0] + xs[2]);  // ||y'_K|| = sqrt(d) ||k||
-      const float nyv = sqrtf(xs[1] + xs[3]);
+      const float2 ss = pair_sum2(ssk, ssv);
+      const float nyk = sqrtf(ss.x);  // ||y'_K|| = sqrt(d) ||k||
+      const float nyv = sqrtf(ss.y);
       const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
       const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
       if (cur.blk && part == 0 && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
 
-      // ---- values and keys, chunk by chunk (independent work side by side) ----
-      constexpr uint32_t kwi[8] = {FK::init(0), FK::init(1), FK::init(2), FK::init(3),
-                                   FK::init(4), FK::init(5), FK::init(6), FK::init(7)};
-      constexpr uint32_t vwi[8] = {FV::init(0), FV::init(1), FV::init(2), FV::init(3),
-                                   FV::init(4), FV::init(5), FV::init(6), FV::init(7)};
-      uint32_t kw[8], vw[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        kw[i] = kwi[i];
-        vw[i] = vwi[i];
-      }
-      {
-        const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
-        const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
-        uint32_t hi0[16], lo0[16], hi1[16], lo1[16], dh[16], dl[16];
-        f2_t rr2 = 0, drr = 0;
-        quantise32<HV - 1, FV, false, 0>(z0, qv, sm.kcode_c, vw, dh, dl, drr);
-        quantise32<HK - 1, FK, KQ != 0, 0>(y0, qk, sm.kcode_c, kw, hi0, lo0, rr2);
-        quantise32<HV - 1, FV, false, 32>(z1, qv, sm.kcode_c, vw, dh, dl, drr);
-        quantise32<HK - 1, FK, KQ != 0, 32>(y1, qk, sm.kcode_c, kw, hi1, lo1, rr2);
-        if (cur.blk && !failed) {
-          store_words<VB, false>(cur.blk + L.vc, part, cur.slot, vw);
-          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
-        }
+      // ---- values and keys, chunk by chunk; the keys' residual goes to TMEM in place ----
+      const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
+      const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
+      f2_t rr2 = 0;
+      uint4 kwc[2];
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float y[32], z[32];
+        tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32 * c, y);
+        tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32 * c, z);
+        tmem_wait_ld();
+        constexpr uint32_t vw0 = FV::init(0), vw1 = FV::init(1), vw2 = FV::init(2), vw3 = FV::init(3);
+        constexpr uint32_t kw0 = FK::init(0), kw1 = FK::init(1), kw2 = FK::init(2), kw3 = FK::init(3);
+        uint32_t vw[4] = {vw0, vw1, vw2, vw3}, kw[4] = {kw0, kw1, kw2, kw3};
+        uint32_t hi[16], lo[16], dh[16], dl[16];
+        f2_t drr = 0;
+        quantise32<HV - 1, FV, false>(z, qv, sm.kcode_c, vw, dh, dl, drr);
+        quantise32<HK - 1, FK, KQ != 0>(y, qk, sm.kcode_c, kw, hi, lo, rr2);
+        if (cur.blk && !failed) store_chunk<VB, false>(cur.blk + L.vc, part, c, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
+        const uint4 kq = make_uint4(kw[0], kw[1], kw[2], kw[3]);
         if constexpr (KQ) {
-          // A (and the residual norm) once the previous sketch is done with A
-          if (j > 0 && !failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
+          tmem_st16(tmem + lane_base + ks_j + kCPT * part + 32 * c, hi);
+          tmem_st16(tmem + lane_base + ks_j + kCPT * part + 32 * c + 16, lo);
+          if (c) kwc[1] = kq; else kwc[0] = kq;
+        } else if (cur.blk && !failed) {
+          store_chunk<KB, false>(cur.blk + L.kc, part, c, cur.slot, kq);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(&sm.v_free);  // y'_V of tile j is read
+      if (cur.blk && !failed && part == 0) {
+        reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+        if (!KQ) reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+      }
+
+      if constexpr (KQ) {
+        // the previous tile's sketch (in X) is done: its signs complete that tile's keys
+        tmem_wait_st();
+        if (j > 0) {
+          if (!failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
           __syncwarp();
           tc_fence_after();
-          tmem_st16(tmem + lane_base + kColA + 32 * part, hi0);
-          tmem_st16(tmem + lane_base + kColA + 32 * part + 16, hi1);
-          tmem_st16(tmem + lane_base + kColA + 64 + 32 * part, lo0);
-          tmem_st16(tmem + lane_base + kColA + 64 + 32 * part + 16, lo1);
-          float ra, rb;
-          uf2(rr2, ra, rb);
-          const float rho = sqrtf(pair_sum(ks_j + kXrr, ra + rb)) * qk.inv_alpha * (1.0f / kSqrtD);
-          // ... and the previous tile's signs, which that sketch produced
-          if (j > 0) {
-            tmem_ld32(tmem + lane_base + ks_p + kCPT * part, y0);
-            tmem_ld32(tmem + lane_base + ks_p + kCPT * part + 32, y1);
-            tmem_wait_ld();
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            bar_arrive(&sm.a_ready);
-            if (j > 0) bar_arrive(&sm.ks_free);
-          }
-          if (j > 0) {
-            if (failed) prev.blk = nullptr;
-            finish_keys(y0, y1);
-          }
-          prev = failed ? TokRef{nullptr, 0} : cur;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) pkw[i] = kw[i];
-          pnorms = (uint32_t)__half_as_ushort(nk16) | ((uint32_t)__half_as_ushort(__float2half_rn(rho)) << 16);
-        } else if (cur.blk && !failed) {
-          store_words<KB, false>(cur.blk + L.kc, part, cur.slot, kw);
-          if (part == 0) reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+          if (failed) prev.blk = nullptr;
+          finish_keys();
         }
+        float ra, rb;
+        uf2(rr2, ra, rb);
+        const float rho = sqrtf(pair_sum2(ra + rb, 0.f).x) * qk.inv_alpha * (1.0f / kSqrtD);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&sm.a_ready);  // A of tile j is written and X is free
+        prev = failed ? TokRef{nullptr, 0} : cur;
+        pk[0] = kwc[0];
+        pk[1] = kwc[1];
+        pnorms = (uint32_t)__half_as_ushort(nk16) | ((uint32_t)__half_as_ushort(__float2half_rn(rho)) << 16);
       }
     }
     if constexpr (KQ) {
@@ -858,13 +850,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (!failed && !bar_wait(&sm.bar_sig, (my_tiles - 1) & 1)) failed = true;
         __syncwarp();
         tc_fence_after();
-        const uint32_t ks_l = ((my_tiles - 1) & 1) ? kColKS1 : kColKS0;
-        float s0[32], s1[32];
-        tmem_ld32(tmem + lane_base + ks_l + kCPT * part, s0);
-        tmem_ld32(tmem + lane_base + ks_l + kCPT * part + 32, s1);
-        tmem_wait_ld();
         if (failed) prev.blk = nullptr;
-        finish_keys(s0, s1);
+        finish_keys();
       }
     }
     if (failed && lane == 0) report(a.status, TQ_ERR_TIMEOUT);
