@@ -54,7 +54,7 @@ struct SmemFast {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   float wacc[kConsumerWarps][4][D];
-  float wm[kConsumerWarps][4], wl[kConsumerWarps][4];
+  float wm[kConsumerWarps][4], wl[kConsumerWarps][4], wf[kConsumerWarps][4];
   int last;
 };
 
@@ -442,141 +442,121 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       const unsigned char* vc = kc + kMaxKChunks * kChunkStride;
       const int tok0 = (u_begin + i) * kUnit;
       const int valid = min(kUnit, t_end - tok0);
-      for (int step = warp; step * 16 < valid; step += kConsumerWarps) {
-        const int ta = step * 16 + g, tb = ta + 8;
-        // ---- keys: dequantise into fp16 A fragments and int8 sign fragments
-        uint32_t ha[16], hb[16], sa[8], sb[8], ea[8], eb[8];
-        if (KP == K3Q) {
-          const uint4 wa = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + ta * 16);
-          const uint4 wb = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + tb * 16);
-          const uint32_t A4[4] = {wa.x, wa.y, wa.z, wa.w}, B4[4] = {wb.x, wb.y, wb.z, wb.w};
+      // two 16-token steps per iteration: their key and value work interleave, and one
+      // joint running maximum (one rescale) serves both
+      for (int pr = warp; pr * 32 < valid; pr += kConsumerWarps) {
+        float sc[2][2];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int side = 0; side < 2; ++side) {
-              const uint32_t W = side ? B4[w] : A4[w];
-              uint32_t* h = side ? hb : ha;
-              uint32_t* sg = side ? sb : sa;
-              uint32_t* ep = side ? eb : ea;
-              const uint32_t s0 = W & 0x7777u;
-              const uint32_t s1 = __umulhi(W, 1u << 16) & 0x7777u;
-              ep[2 * w + 0] = prmt(et0, et1, s0);
-              ep[2 * w + 1] = prmt(et0, et1, s1);
-              const uint32_t l0 = prmt(kt_lo0, kt_lo1, s0), h0 = prmt(kt_hi0, kt_hi1, s0);
-              const uint32_t l1 = prmt(kt_lo0, kt_lo1, s1), h1 = prmt(kt_hi0, kt_hi1, s1);
-              h[4 * w + 0] = prmt(l0, h0, 0x5140);
-              h[4 * w + 1] = prmt(l0, h0, 0x7362);
-              h[4 * w + 2] = prmt(l1, h1, 0x5140);
-              h[4 * w + 3] = prmt(l1, h1, 0x7362);
-              sg[2 * w + 0] = (W << 4) & 0x80808080u;
-              sg[2 * w + 1] = W & 0x80808080u;
+        for (int u = 0; u < 2; ++u) {
+          const int step = 2 * pr + u;
+            const int ta = step * 16 + g, tb = ta + 8;
+            // ---- keys: dequantise into fp16 A fragments and int8 sign fragments
+            uint32_t ha[16], hb[16], sa[8], sb[8], ea[8], eb[8];
+            if (KP == K3Q) {
+              const uint4 wa = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + ta * 16);
+              const uint4 wb = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + tb * 16);
+              const uint32_t A4[4] = {wa.x, wa.y, wa.z, wa.w}, B4[4] = {wb.x, wb.y, wb.z, wb.w};
+    #pragma unroll
+              for (int w = 0; w < 4; ++w) {
+    #pragma unroll
+                for (int side = 0; side < 2; ++side) {
+                  const uint32_t W = side ? B4[w] : A4[w];
+                  uint32_t* h = side ? hb : ha;
+                  uint32_t* sg = side ? sb : sa;
+                  uint32_t* ep = side ? eb : ea;
+                  const uint32_t s0 = W & 0x7777u;
+                  const uint32_t s1 = __umulhi(W, 1u << 16) & 0x7777u;
+                  ep[2 * w + 0] = prmt(et0, et1, s0);
+                  ep[2 * w + 1] = prmt(et0, et1, s1);
+                  const uint32_t l0 = prmt(kt_lo0, kt_lo1, s0), h0 = prmt(kt_hi0, kt_hi1, s0);
+                  const uint32_t l1 = prmt(kt_lo0, kt_lo1, s1), h1 = prmt(kt_hi0, kt_hi1, s1);
+                  h[4 * w + 0] = prmt(l0, h0, 0x5140);
+                  h[4 * w + 1] = prmt(l0, h0, 0x7362);
+                  h[4 * w + 2] = prmt(l1, h1, 0x5140);
+                  h[4 * w + 3] = prmt(l1, h1, 0x7362);
+                  sg[2 * w + 0] = (W << 4) & 0x80808080u;
+                  sg[2 * w + 1] = W & 0x80808080u;
+                }
+              }
+            } else {
+              const unsigned char* kq = kc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
+              const uint2 ca = *reinterpret_cast<const uint2*>(kq + ta * 16);
+              const uint2 cbv = *reinterpret_cast<const uint2*>(kq + tb * 16);
+              const uint32_t sA = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + ta * 16 + 4 * t4);
+              const uint32_t sB = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + tb * 16 + 4 * t4);
+    #pragma unroll
+              for (int n = 0; n < 16; ++n) {
+                ha[n] = prmt(kt_lo0, kt_hi0, crumb_sel(ca.x, ca.y, n));
+                hb[n] = prmt(kt_lo0, kt_hi0, crumb_sel(cbv.x, cbv.y, n));
+              }
+    #pragma unroll
+              for (int n = 0; n < 16; n += 2) {
+                // pairs n, n+1 -> int8 residual codes (a_n, a_n+1, b_n, b_n+1)
+                ea[n >> 1] = prmt(et0, et1, crumb_pair_sel(ca.x, ca.y, n));
+                eb[n >> 1] = prmt(et0, et1, crumb_pair_sel(cbv.x, cbv.y, n));
+              }
+    #pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                sa[k] = (sA << k) & 0x80808080u;
+                sb[k] = (sB << k) & 0x80808080u;
+              }
             }
-          }
-        } else {
-          const unsigned char* kq = kc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
-          const uint2 ca = *reinterpret_cast<const uint2*>(kq + ta * 16);
-          const uint2 cbv = *reinterpret_cast<const uint2*>(kq + tb * 16);
-          const uint32_t sA = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + ta * 16 + 4 * t4);
-          const uint32_t sB = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + tb * 16 + 4 * t4);
-#pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            ha[n] = prmt(kt_lo0, kt_hi0, crumb_sel(ca.x, ca.y, n));
-            hb[n] = prmt(kt_lo0, kt_hi0, crumb_sel(cbv.x, cbv.y, n));
-          }
-#pragma unroll
-          for (int n = 0; n < 16; n += 2) {
-            // pairs n, n+1 -> int8 residual codes (a_n, a_n+1, b_n, b_n+1)
-            ea[n >> 1] = prmt(et0, et1, crumb_pair_sel(ca.x, ca.y, n));
-            eb[n >> 1] = prmt(et0, et1, crumb_pair_sel(cbv.x, cbv.y, n));
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            sa[k] = (sA << k) & 0x80808080u;
-            sb[k] = (sB << k) & 0x80808080u;
-          }
+            // two accumulators per term halve the dependent mma chains
+            float dk[4] = {0.f, 0.f, 0.f, 0.f}, dk2[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+            for (int ks = 0; ks < 8; ks += 2) {
+              hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
+              hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[ks + 1][0], bq[ks + 1][1]);
+            }
+            int dsum[4] = {0, 0, 0, 0}, dsum2[4] = {0, 0, 0, 0};
+            int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
+    #pragma unroll
+            for (int w = 0; w < 4; w += 2) {
+              imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
+              imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
+              imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
+              imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[w + 1][0], bc[w + 1][1]);
+            }
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dk[e] += dk2[e];
+              dsum[e] += dsum2[e];
+              dcor[e] += dcor2[e];
+            }
+            // ---- scores of row t4 for tokens ta, tb (log2 domain)
+            const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
+            const float rA = ld_h(st + 2 * kUnit + 2 * ta), rB = ld_h(st + 2 * kUnit + 2 * tb);
+            const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
+            const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
+            const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
+            float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row) * c_row_q;
+            float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row) * c_row_q;
+            if (t4 >= R || ta >= valid) sca = -CUDART_INF_F;
+            if (t4 >= R || tb >= valid) scb = -CUDART_INF_F;
+          sc[u][0] = sca;
+          sc[u][1] = scb;
         }
-        // two accumulators per term halve the dependent mma chains
-        float dk[4] = {0.f, 0.f, 0.f, 0.f}, dk2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 8; ks += 2) {
-          hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
-          hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[ks + 1][0], bq[ks + 1][1]);
-        }
-        int dsum[4] = {0, 0, 0, 0}, dsum2[4] = {0, 0, 0, 0};
-        int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int w = 0; w < 4; w += 2) {
-          imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
-          imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
-          imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
-          imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[w + 1][0], bc[w + 1][1]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          dk[e] += dk2[e];
-          dsum[e] += dsum2[e];
-          dcor[e] += dcor2[e];
-        }
-        // ---- scores of row t4 for tokens ta, tb (log2 domain)
-        const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
-        const float rA = ld_h(st + 2 * kUnit + 2 * ta), rB = ld_h(st + 2 * kUnit + 2 * tb);
-        const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
-        const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
-        const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
-        float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row) * c_row_q;
-        float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row) * c_row_q;
-        if (t4 >= R || ta >= valid) sca = -CUDART_INF_F;
-        if (t4 >= R || tb >= valid) scb = -CUDART_INF_F;
-        float mx = fmaxf(sca, scb);
+        float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
         const float m_new = fmaxf(m_run, mx);
-        // the running sums are rescaled only in steps where some row maximum grew
+        // the running sums are rescaled only when some row maximum grew
         const bool grow = __any_sync(FULL, m_new > m_run);
-        float alpha = 1.f, pa = 0.f, pb = 0.f;
+        float alpha = 1.f, p[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         if (m_new != -CUDART_INF_F) {
           if (grow) alpha = exp2f(m_run - m_new);
-          pa = exp2f(sca - m_new);
-          pb = exp2f(scb - m_new);
-        }
-        l_run = l_run * alpha + pa + pb;
-        m_run = m_new;
-        const float vnA = ld_h(st + 4 * kUnit + 2 * ta), vnB = ld_h(st + 4 * kUnit + 2 * tb);
-        // slots past the end may hold stale bytes: force their weight to exactly 0
-        const uint32_t pk = pack_h2(ta < valid ? pa * vnA : 0.f, tb < valid ? pb * vnB : 0.f);
-        const uint32_t x1 = __shfl_sync(FULL, pk, 4 * (2 * t4) + g);
-        const uint32_t x2 = __shfl_sync(FULL, pk, 4 * (2 * t4 + 1) + g);
-        const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
-        float al0 = 1.f, al1 = 1.f;
-        if (grow) {
-          al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
-          al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
-        }
-        // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
-        uint32_t va[16], vb[16];
-        {
-          const unsigned char* vq = vc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
-          const uint2 ca = *reinterpret_cast<const uint2*>(vq + ta * 16);
-          const uint2 cbv = *reinterpret_cast<const uint2*>(vq + tb * 16);
-          uint32_t sgA = 0, sgB = 0;
-          if (VP == V3) {
-            sgA = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + ta * 16 + 4 * t4);
-            sgB = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + tb * 16 + 4 * t4);
-          }
 #pragma unroll
-          for (int cb = 0; cb < 16; ++cb) {
-            uint32_t xa = prmt(vt_lo, vt_hi, crumb_sel(ca.x, ca.y, cb));
-            uint32_t xb = prmt(vt_lo, vt_hi, crumb_sel(cbv.x, cbv.y, cb));
-            if (VP == V3) {
-              xa ^= (sgA << (15 - cb)) & 0x80008000u;
-              xb ^= (sgB << (15 - cb)) & 0x80008000u;
-            }
-            va[cb] = movm_t(xa);
-            vb[cb] = movm_t(xb);
+          for (int u = 0; u < 2; ++u) {
+            p[u][0] = exp2f(sc[u][0] - m_new);
+            p[u][1] = exp2f(sc[u][1] - m_new);
           }
         }
+        l_run = l_run * alpha + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        m_run = m_new;
         if (grow) {
+          const float al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
+          const float al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             acc[mt][0] *= al0;
@@ -586,7 +566,41 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
           }
         }
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+        for (int u = 0; u < 2; ++u) {
+          const int step = 2 * pr + u;
+          const int ta = step * 16 + g, tb = ta + 8;
+          const float vnA = ld_h(st + 4 * kUnit + 2 * ta), vnB = ld_h(st + 4 * kUnit + 2 * tb);
+          // slots past the end may hold stale bytes: force their weight to exactly 0
+          const uint32_t pk = pack_h2(ta < valid ? p[u][0] * vnA : 0.f, tb < valid ? p[u][1] * vnB : 0.f);
+          const uint32_t x1 = __shfl_sync(FULL, pk, 4 * (2 * t4) + g);
+          const uint32_t x2 = __shfl_sync(FULL, pk, 4 * (2 * t4 + 1) + g);
+          const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
+            // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
+            uint32_t va[16], vb[16];
+            {
+              const unsigned char* vq = vc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
+              const uint2 ca = *reinterpret_cast<const uint2*>(vq + ta * 16);
+              const uint2 cbv = *reinterpret_cast<const uint2*>(vq + tb * 16);
+              uint32_t sgA = 0, sgB = 0;
+              if (VP == V3) {
+                sgA = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + ta * 16 + 4 * t4);
+                sgB = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + tb * 16 + 4 * t4);
+              }
+    #pragma unroll
+              for (int cb = 0; cb < 16; ++cb) {
+                uint32_t xa = prmt(vt_lo, vt_hi, crumb_sel(ca.x, ca.y, cb));
+                uint32_t xb = prmt(vt_lo, vt_hi, crumb_sel(cbv.x, cbv.y, cb));
+                if (VP == V3) {
+                  xa ^= (sgA << (15 - cb)) & 0x80008000u;
+                  xb ^= (sgB << (15 - cb)) & 0x80008000u;
+                }
+                va[cb] = movm_t(xa);
+                vb[cb] = movm_t(xb);
+              }
+            }
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
@@ -612,39 +626,45 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   }
   __syncthreads();
   // ---- merge the consumer warps and write this split's partial
+  // per row: the maximum over the warps, each warp's factor, the sum (natural-log domain
+  // for the merge across splits)
+  if (tid < R) {
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][tid]);
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float f = (M == -CUDART_INF_F || sm.wm[w][tid] == -CUDART_INF_F) ? 0.f : exp2f(sm.wm[w][tid] - M);
+      sm.wf[w][tid] = f;
+      l = fmaf(f, sm.wl[w][tid], l);
+    }
+    const size_t pr = (row0 + tid) * a.n_splits + split;
+    a.part_ml[pr * 2] = (M == -CUDART_INF_F) ? M : M / kLog2e;
+    a.part_ml[pr * 2 + 1] = l;
+  }
+  __syncthreads();
   for (int idx = tid; idx < R * D; idx += blockDim.x) {
     const int r = idx / D, j = idx % D;
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][r]);
-    float l = 0.f, o = 0.f;
-    if (M != -CUDART_INF_F) {
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mw = sm.wm[w][r];
-        if (mw == -CUDART_INF_F) continue;
-        const float f = exp2f(mw - M);
-        l = fmaf(f, sm.wl[w][r], l);
-        o = fmaf(f, sm.wacc[w][r][j], o);
-      }
-    }
-    const size_t pr = (row0 + r) * a.n_splits + split;
-    a.part_acc[pr * D + j] = o;
-    if (j == 0) {
-      // partials are kept in the natural-log domain for the merge
-      a.part_ml[pr * 2] = (M == -CUDART_INF_F) ? M : M / kLog2e;
-      a.part_ml[pr * 2 + 1] = l;
-    }
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm.wf[w][r], sm.wacc[w][r][j], o);
+    a.part_acc[((row0 + r) * a.n_splits + split) * D + j] = o;
   }
   // ---- the last split of this (sequence, kv head) to finish merges all of them ----
   __syncthreads();
   if (tid == 0) {
-    // the CTA's partial writes are ordered before the count by the barrier and this fence
-    __threadfence();
-    const unsigned int done = atomicAdd(&a.counter[(size_t)b * a.cache.kv_heads + gh], 1u);
+    // release: the CTA's partial writes (ordered before this by the barrier) are visible to
+    // whoever reads the count after it; acquire: the last one sees all the others' partials
+    unsigned int done;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
+                 : "=r"(done)
+                 : "l"(&a.counter[(size_t)b * a.cache.kv_heads + gh])
+                 : "memory");
     sm.last = done == (unsigned int)a.n_splits - 1;
   }
   __syncthreads();
   if (!sm.last) return;
-  __threadfence();
   const int ns = a.n_splits;
   if (tid < 32 * R) {
     // thread (row r, float4 c4) of the output: online log-sum-exp over the splits'
@@ -655,10 +675,15 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    // every partial this thread needs, requested into L1 at once (no registers held)
+    for (int sp = 0; sp < ns; ++sp) {
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(pa4 + (size_t)sp * (D / 4)));
+      if (c4 == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(ml2 + sp));
+    }
 #pragma unroll 16
     for (int sp = 0; sp < ns; ++sp) {
-      const float2 m2 = __ldcg(ml2 + sp);
-      const float4 v = __ldcg(pa4 + (size_t)sp * (D / 4));
+      const float2 m2 = ml2[sp];
+      const float4 v = pa4[(size_t)sp * (D / 4)];
       // branch-free update (the loads of later splits do not wait on it)
       const float Mn = fmaxf(M, m2.x);
       const bool live = Mn != -CUDART_INF_F;
