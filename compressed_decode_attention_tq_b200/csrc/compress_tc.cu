@@ -19,12 +19,13 @@
 // of saturated unit steps (the boundaries are sorted), and the residual's centroid is read
 // from a table by the code field just formed.
 //
-// One persistent CTA per SM: 8 compute warps and a producer warpgroup.  Compute warp w
-// reads tensor-memory lane quadrant w % 4 (tokens 32 (w % 4) .. + 31) and coordinates
-// 64 (w / 4) .. + 63, so two warps share a token; their per-token sums (norms, residual
-// norm) meet in spare tensor-memory columns behind a 64-thread named barrier.  One thread
-// of the producer warpgroup issues the TMA copies (two K/V tile stages), the MMAs and their
-// commits; the compute warps hand tensor-memory columns back through mbarriers.
+// One persistent CTA per SM: two compute groups of four warps and a producer warpgroup.
+// Group g takes the CTA's tiles g, g + 2, ... (ping-pong), so that one group's waits for
+// its MMAs are covered by the other group's CUDA-core work.  Each thread owns one token
+// (a tensor-memory lane: warp w reads lane quadrant w % 4) and all 128 of its coordinates,
+// so no per-token sum crosses threads.  Each group has its own tensor-memory columns
+// (y'_K, then the sketch's A operand in place; y'_V, then the sketch output) and its own
+// MMA-issuing thread; one more producer thread issues the TMA copies into two stages.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -38,21 +39,24 @@ namespace {
 
 constexpr int TT = 128;                      // tokens per tile
 constexpr int kComputeWarps = 8;
-constexpr int kCPT = 64;  // coordinates per compute thread
-// two compute warpgroups and one producer warpgroup (one thread of which issues the copies
-// and MMAs); registers move from the producer to the compute warpgroups after launch:
-// launched with 384 x 168, then 128 x 72 + 256 x 216 = 64512 = 384 x 168.
+constexpr int kGroupWarps = 4;  // warps of one compute group (one tile)
+// producer warpgroup: the MMA issuers of groups 0 and 1 and the copy issuer
+constexpr int kIssuerWarp0 = kComputeWarps, kLoaderWarp = kComputeWarps + 1, kIssuerWarp1 = kComputeWarps + 2;
+// two compute warpgroups and one producer warpgroup; registers move from the producer to
+// the compute warpgroups after launch: launched with 384 x 168, then 128 x 96 + 256 x 200
+// = 63488 <= 384 x 168.
 constexpr int kThreadsTC = (kComputeWarps + 4) * 32;
-constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsCompute = 216;
+constexpr int kRegsLaunch = 168, kRegsProducer = 96, kRegsCompute = 200;
+static_assert(kComputeWarps == 2 * kGroupWarps && kGroupWarps == 4, "two groups of four lane quadrants");
 static_assert(128 * kRegsProducer + 32 * kComputeWarps * kRegsCompute <= kThreadsTC * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr int kTileBytes = TT * D * 2;       // one 128 x 128 fp16 operand
-// Tensor-memory columns.  KS[0], KS[1]: y'_K of a tile (alternate tiles, alternate
-// blocks); as each 32-coordinate chunk of it is read, the chunk's scaled residual is
-// written in its place as fp16 hi (first 16 columns) and lo (next 16): the sketch's A
-// operand.  V: y'_V of a tile.  X: the sketch (S D H) a r_rot' of a tile, then (+0, +1) the
-// residual sums of the two warps of a token.
-constexpr uint32_t kColKS0 = 0, kColKS1 = 128, kColV = 256, kColX = 384;
+// Tensor-memory columns of group g, from kColGroup g: +0 y'_K of the group's tile; as each
+// 32-coordinate chunk of it is read, the chunk's scaled residual is written in its place as
+// fp16 hi (first 16 columns) and lo (next 16): the sketch's A operand.  +kColV: y'_V, then
+// the sketch (S D H) a r_rot' once y'_V has been read.  At set-up S D H lands in group 1's
+// y'_K columns.
+constexpr uint32_t kColGroup = 256, kColV = 128;
 constexpr uint32_t kTmemCols = 512;
 // instruction descriptor: D f32, A and B f16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -64,12 +68,14 @@ struct SmemTC {
   unsigned char bhd[kTileBytes];      // B = H D
   unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part
   unsigned char bslo[kTileBytes];     // fp16 lo part
-  unsigned long long bar_load[2], stage_free[2], bar_fwdk, bar_fwdv, bar_sig, ks_free, a_ready, v_free, bar_setup;
+  // [stage]: tile landed / read by its forward MMAs; [group]: forward MMAs done, A written
+  // (and y'_V read), sketch done, tensor-memory columns released, error drain
+  unsigned long long bar_load[2], stage_free[2], fwd_done[2], a_ready[2], sig_done[2], tm_free[2], bar_drain[2];
+  unsigned long long bar_setup, setup_read;  // S D H MMA done / read out into bshi, bslo
   uint32_t tmem_base;
   int bad_s;
   float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
-  float kcode_c[8];                      // c[idx] of a key code field r + sw s
-  float2 red[TT][2];                     // per-token sums of the two warps of a token
+  float kmag[8];                         // |c| of a key's magnitude rank r: c[h + r]
 };
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
 
@@ -130,11 +136,6 @@ __device__ __forceinline__ void bar_arrive(unsigned long long* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s_u32(b)) : "memory");
 }
 
-// 64-thread barrier of the two compute warps that share a tensor-memory lane quadrant
-__device__ __forceinline__ void pair_sync(int qd) {
-  asm volatile("bar.sync %0, 64;" ::"r"(1 + qd) : "memory");
-}
-
 __device__ __forceinline__ void tma_load_tile(void* dst, const CUtensorMap* map, int row0,
                                               unsigned long long* bar) {
   asm volatile(
@@ -183,22 +184,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
-  uint32_t r[4];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
-  uint32_t r0, r1;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(taddr));
-  v[0] = __uint_as_float(r0);
-  v[1] = __uint_as_float(r1);
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -206,17 +191,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
-}
-
-__device__ __forceinline__ void tmem_st2(uint32_t taddr, float a, float b) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(__float_as_uint(a)),
-               "r"(__float_as_uint(b))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, float a) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(a))
-               : "memory");
 }
 
 // ---- packed fp32 pairs (two coordinates per instruction) and saturated steps ----
@@ -251,11 +225,6 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-__device__ __forceinline__ float mul_sat(float a, float b) {
-  float d;
-  asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-  return d;
-}
 
 // sum of squares of 32 values, two lanes of packed fp32 at a time
 __device__ __forceinline__ float sumsq32(const float (&v)[32]) {
@@ -270,46 +239,61 @@ __device__ __forceinline__ float sumsq32(const float (&v)[32]) {
   return lo + hi;
 }
 
-// Integer codes are assembled in the mantissa of 2^23 + code (exact for 0 <= code < 2^23)
-// and shifted into place with an integer multiply-add; the 2^23 exponent bits each
-// coordinate drags along are subtracted up front (mod 2^32).
-constexpr float kMagic = 8388608.f;
-constexpr uint32_t kMagicBits = 0x4B000000u;
-__host__ __device__ constexpr uint32_t magic_at(int sh) {
-  return (uint32_t)(((unsigned long long)kMagicBits << sh) & 0xFFFFFFFFull);
-}
+// Magnitude ranks are assembled in the mantissa of a power of two plus the rank (exact
+// for small integers) and shifted into place with an integer multiply-add; the exponent
+// bits each coordinate drags along are subtracted up front (mod 2^32).  With 2^23 the rank
+// sits at mantissa bit 0; with 2^21 (ulp 1/4) at bit 2, which is directly the byte offset
+// of its entry in a table of fp32 centroids.
+constexpr float kMagic23 = 8388608.f, kMagic21 = 2097152.f;
+__host__ __device__ constexpr uint32_t magic_bits(int ms) { return ms == 2 ? 0x4A000000u : 0x4B000000u; }
+// x << k for k >= 0, x >> -k otherwise
+__host__ __device__ constexpr uint32_t shl(uint32_t x, int k) { return k >= 0 ? x << k : x >> -k; }
 
 // Bit of coordinate e (0..31) of a 32-coordinate group in the sign plane of 3-bit codes
 // (the permutation of sign_plane_pos, which the decode's byte tables read).
 __host__ __device__ constexpr int plane_bit(int e) { return 4 * (e >> 3) + (e & 3) + 16 * ((e >> 2) & 1); }
 
 // Where coordinate i (0..31 of one 32-coordinate chunk) of a b-bit code lands in the
-// chunk's four words.  Field = r + sw * s:
-//   b = 2: 2-bit r | s << 1 (words 0, 1);  b = 3: 2-bit r (words 0, 1) and s in word 2 at
-//   the permuted sign-plane bit;  b = 4: r | s << 3 (words 0..3);  merged 3-bit key:
-//   r | s << 2 | sigma << 3 (words 0..3).
+// chunk's four words.  Field = r | s << (b - 1) with r the magnitude rank and s = [y' > 0]:
+//   b = 2: 2-bit fields (words 0, 1);  b = 3: 2-bit r (words 0, 1) and s in word 2 at the
+//   permuted sign-plane bit;  b = 4: nibbles (words 0..3);  merged 3-bit key: nibbles
+//   r | s << 2 | sigma << 3 (words 0..3), or for other keys sigma in a word of its own.
+// Sign bits are placed two at a time (coordinates i and i + pair, which land in different
+// bytes of the same word).
 template <int B, bool MERGED>
 struct Fields {
   static constexpr bool nib = MERGED || B == 4;
-  static constexpr int sw = MERGED ? 4 : (B == 2 ? 2 : (B == 3 ? 0 : 8));
   static constexpr bool plane = !MERGED && B == 3;
   __host__ __device__ static constexpr int word(int i) { return nib ? (i >> 3) : (i >> 4); }
   __host__ __device__ static constexpr int shift(int i) { return nib ? 4 * (i & 7) : 2 * (i & 15); }
-  // minus the magic bits the code (and, merged, sigma) adds of every coordinate of word w
-  __host__ __device__ static constexpr uint32_t init(int w) {
-    uint32_t c = 0;
-    for (int i = 0; i < 32; ++i) {
-      if (word(i) == w) c += magic_at(shift(i)) * (MERGED ? 2u : 1u);
-      if (plane && w == 2) c += magic_at(plane_bit(i));
-    }
-    return 0u - c;
+  __host__ __device__ static constexpr int sword(int i) { return plane ? 2 : word(i); }
+  __host__ __device__ static constexpr int spos(int i) {
+    return plane ? plane_bit(i) : shift(i) + (MERGED ? 2 : (B == 2 ? 1 : 3));
   }
-  __host__ __device__ static constexpr uint32_t sig_init() {
+  __host__ __device__ static constexpr int spair() { return nib ? 2 : 4; }
+  __host__ __device__ static constexpr int sigpos(int i) { return MERGED ? shift(i) + 3 : i; }
+  __host__ __device__ static constexpr int sigpair() { return MERGED ? 2 : 8; }
+  // minus the magic bits the ranks (at mantissa bit ms) add to word w
+  __host__ __device__ static constexpr uint32_t init(int w, int ms) {
     uint32_t c = 0;
-    for (int i = 0; i < 32; ++i) c += magic_at(i);
+    for (int i = 0; i < 32; ++i)
+      if (word(i) == w) c += shl(magic_bits(ms), shift(i) - ms);
     return 0u - c;
   }
 };
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+// The sign bits of a and b at bits pa and pb (in different bytes), all other bits 0: prmt
+// with the sign-replicating selector (8 | byte) copies the top byte's sign over a whole
+// byte, and the mask keeps one bit of each.
+__device__ __forceinline__ uint32_t sign_bits(float a, float b, int pa, int pb) {
+  const uint32_t sel = (0xBu << (4 * (pa >> 3))) | (0xFu << (4 * (pb >> 3)));
+  return prmt(__float_as_uint(a), __float_as_uint(b), sel) & ((1u << pa) | (1u << pb));
+}
 
 // Store the words of one chunk (coordinates 64 part + 32 c .. + 31) of a token slot
 // (plane p = 16 bytes per slot).
@@ -326,7 +310,7 @@ __device__ __forceinline__ void store_chunk(uint8_t* base, int part, int c, int 
 // Boundary scales of one token: |y| > beta ||y'||  <=>  bs |y'| - bs beta ||y'|| > 0 with
 // bs = 2^(40 - e) for ||y'|| ~ 2^e: one fused multiply-add of |y'| (exact product, one
 // rounding, so the sign is exact), saturated to [0, 1], is a unit step outside a 2^-40
-// relative band; bs y' saturated is the step s = [y' > 0].
+// relative band.
 struct TokScale {
   int e;
   float bs;
@@ -336,50 +320,66 @@ struct TokScale {
   }
 };
 
-// Per-token constants of the quantiser: the scaled boundaries, and with QJL the residual
-// scale a = 2^(8 - e) and a sqrt(d) fp16(||x||).
+// Per-token constants of the quantiser: the scaled positive boundaries tb[k] = -bs beta_k
+// ||y'|| (and for three of them tb[2] - tb[0], which selects the last step's boundary from
+// the middle one's outcome), and with QJL the residual scale a = 2^(8 - e) and
+// a sqrt(d) fp16(||x||).
 template <int NB>
 struct QuantConst {
   TokScale ts;
-  float tb[NB > 0 ? NB : 1];  // -bs beta_k ||y'||
+  float tb[NB > 0 ? NB : 1];
+  float d20;
   float alpha, inv_alpha, csa;
   __device__ __forceinline__ QuantConst(float ny, const float* pos, float cnorm) : ts(ny) {
 #pragma unroll
     for (int k = 0; k < NB; ++k) tb[k] = -(pos[k] * ny) * ts.bs;
+    d20 = NB == 3 ? tb[NB == 3 ? 2 : 0] - tb[0] : 0.f;
     alpha = __uint_as_float((uint32_t)(127 + 8 - ts.e) << 23);
     inv_alpha = __uint_as_float((uint32_t)(127 - 8 + ts.e) << 23);
     csa = alpha * kSqrtD * cnorm;
   }
 };
 
-// Codes of one 32-coordinate chunk of y' into the chunk's words w; with KQ also the scaled
-// residual a y' - a sqrt(d) fp16(||x||) c[idx] (c[idx] read from the table of signed
-// centroids by the code just formed) split into fp16 hi / lo pairs for the sketch MMAs, and
-// its sum of squares (accumulated into rr2).
+// Codes of one 32-coordinate chunk of y' into the chunk's words w.  The magnitude rank is
+// the number of positive boundaries below |y'|: with three boundaries a binary search (is
+// it above the middle one; then above the upper or the lower one), otherwise a sum of unit
+// steps.  s = [y' > 0] is the sign bit of tiny - y' (exact at +-0).  With KQ also the scaled
+// residual a y' - a sqrt(d) fp16(||x||) c[idx] (|c| read from a table by the rank, signed
+// by s) split into fp16 hi / lo pairs for the sketch MMAs, and its sum of squares (into rr2).
+constexpr float kTiny = 1.40129846e-45f;  // 2^-149
 template <int NB, class F, bool KQ>
-__device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, const float* ctab,
+__device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, const float* cmag,
                                            uint32_t (&w)[4], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
+  constexpr int MS = KQ ? 2 : 0;
+  const f2_t magic = f2s(KQ ? kMagic21 : kMagic23);
+  float u[32];
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
     const float y0 = y[i], y1 = y[i + 1];
-    f2_t sum = f2s(kMagic);
+    f2_t sum;
+    if constexpr (NB == 3) {
+      const f2_t s2 = f2(fma_sat(fabsf(y0), qc.ts.bs, qc.tb[1]), fma_sat(fabsf(y1), qc.ts.bs, qc.tb[1]));
+      float t0, t1;
+      uf2(fma2(s2, f2s(qc.d20), f2s(qc.tb[0])), t0, t1);
+      const f2_t b0 = f2(fma_sat(fabsf(y0), qc.ts.bs, t0), fma_sat(fabsf(y1), qc.ts.bs, t1));
+      sum = add2(fma2(s2, f2s(2.f), magic), b0);
+    } else {
+      sum = magic;
 #pragma unroll
-    for (int k = 0; k < NB; ++k)
-      sum = add2(sum, f2(fma_sat(fabsf(y0), qc.ts.bs, qc.tb[k]), fma_sat(fabsf(y1), qc.ts.bs, qc.tb[k])));
-    const f2_t S = f2(mul_sat(y0, qc.ts.bs), mul_sat(y1, qc.ts.bs));  // s = [y' > 0]
-    if (F::sw) sum = fma2(S, f2s((float)F::sw), sum);
+      for (int k = 0; k < NB; ++k)
+        sum = add2(sum, f2(fma_sat(fabsf(y0), qc.ts.bs, qc.tb[k]), fma_sat(fabsf(y1), qc.ts.bs, qc.tb[k])));
+    }
     float c0, c1;
     uf2(sum, c0, c1);
     const uint32_t code0 = __float_as_uint(c0), code1 = __float_as_uint(c1);
-    w[F::word(i)] += code0 << F::shift(i);
-    w[F::word(i + 1)] += code1 << F::shift(i + 1);
-    if (F::plane) {
-      uf2(add2(S, f2s(kMagic)), c0, c1);
-      w[2] += __float_as_uint(c0) << plane_bit(i);
-      w[2] += __float_as_uint(c1) << plane_bit(i + 1);
-    }
+    w[F::word(i)] += shl(code0, F::shift(i) - MS);
+    w[F::word(i + 1)] += shl(code1, F::shift(i + 1) - MS);
+    uf2(fma2(f2(y0, y1), f2s(-1.f), f2s(kTiny)), u[i], u[i + 1]);
     if constexpr (KQ) {
-      const f2_t C = f2(ctab[code0 & 7], ctab[code1 & 7]);
+      const uint32_t m0 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + (code0 & 0xCu));
+      const uint32_t m1 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + (code1 & 0xCu));
+      const f2_t C = f2(__uint_as_float(m0 | (~__float_as_uint(u[i]) & 0x80000000u)),
+                        __uint_as_float(m1 | (~__float_as_uint(u[i + 1]) & 0x80000000u)));
       const f2_t R = fma2(C, f2s(-qc.csa), mul2(f2(y0, y1), f2s(qc.alpha)));
       rr2 = fma2(R, R, rr2);
       float r0, r1;
@@ -394,32 +394,34 @@ __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantCons
       lo[i >> 1] = *reinterpret_cast<const uint32_t*>(&ll);
     }
   }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i & F::spair()) continue;
+    const int j = i + F::spair();
+    w[F::sword(i)] |= sign_bits(u[i], u[j], F::spos(i), F::spos(j));
+  }
 }
 
-// QJL signs sigma = [p >= 0] (1 also within 2^-40 below 0) of one 32-entry chunk of the
-// sketch: merged into bit 3 of the chunk's key nibbles, or one sign-plane word.
+// QJL signs sigma = [p >= 0] (the complement of p's sign bit) of one 32-entry chunk of the
+// sketch: into bit 3 of the chunk's key nibbles, or into a sign-plane word of their own.
 template <bool MERGED, class F>
 __device__ __forceinline__ void sigma32(const float (&p)[32], uint4& w, uint32_t& sgw) {
   uint32_t wa[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const f2_t G = f2(fma_sat(p[i], 1099511627776.f, 1.f), fma_sat(p[i + 1], 1099511627776.f, 1.f));
-    float c0, c1;
-    if constexpr (MERGED) {
-      uf2(fma2(G, f2s(8.f), f2s(kMagic)), c0, c1);
-      wa[F::word(i)] += __float_as_uint(c0) << F::shift(i);
-      wa[F::word(i + 1)] += __float_as_uint(c1) << F::shift(i + 1);
-    } else {
-      uf2(add2(G, f2s(kMagic)), c0, c1);
-      sgw += __float_as_uint(c0) << i;
-      sgw += __float_as_uint(c1) << (i + 1);
-    }
+  for (int i = 0; i < 32; ++i) {
+    if (i & F::sigpair()) continue;
+    const int j = i + F::sigpair();
+    const int pa = F::sigpos(i), pb = F::sigpos(j);
+    const uint32_t sel = (0xBu << (4 * (pa >> 3))) | (0xFu << (4 * (pb >> 3)));
+    const uint32_t m = ~prmt(__float_as_uint(p[i]), __float_as_uint(p[j]), sel) & ((1u << pa) | (1u << pb));
+    if constexpr (MERGED) wa[F::word(i)] |= m;
+    else sgw |= m;
   }
   w = make_uint4(wa[0], wa[1], wa[2], wa[3]);
 }
 
 // The cache block and slot of the token this thread owns in tile j (blk null when the
-// token is past its sequence or its page is invalid; errors reported once, by part 0).
+// token is past its sequence or its page is invalid).
 struct TokRef {
   uint8_t* blk;
   int slot;
@@ -435,7 +437,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool producer = warp >= kComputeWarps;  // the producer warpgroup
   const int qd = warp & 3;           // tensor-memory lane quadrant
-  const int part = (warp >> 2) & 1;  // coordinates 64 part .. 64 part + 63
   const int row = 32 * qd + lane;    // token within the tile
   const Layout& L = a.cache.L;
   constexpr int HK = 1 << (KB - 1), HV = 1 << (VB - 1);
@@ -469,17 +470,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    bar_init(&sm.bar_load[0], 1);
-    bar_init(&sm.bar_load[1], 1);
-    bar_init(&sm.stage_free[0], 1);
-    bar_init(&sm.stage_free[1], 1);
-    bar_init(&sm.bar_fwdk, 1);
-    bar_init(&sm.bar_fwdv, 1);
-    bar_init(&sm.bar_sig, 1);
-    bar_init(&sm.ks_free, kComputeWarps);
-    bar_init(&sm.a_ready, kComputeWarps);
-    bar_init(&sm.v_free, kComputeWarps);
+    for (int g = 0; g < 2; ++g) {
+      bar_init(&sm.bar_load[g], 1);
+      bar_init(&sm.stage_free[g], 1);
+      bar_init(&sm.fwd_done[g], 1);
+      bar_init(&sm.a_ready[g], kGroupWarps);
+      bar_init(&sm.sig_done[g], 1);
+      bar_init(&sm.tm_free[g], kGroupWarps);
+      bar_init(&sm.bar_drain[g], 1);
+    }
     bar_init(&sm.bar_setup, 1);
+    bar_init(&sm.setup_read, kGroupWarps);
     sm.bad_s = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   // tile 0 streams in while the rotation operands are built (stage 1 is set-up scratch)
-  if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) issue_load(0);
+  if (warp == kLoaderWarp && lane == 0 && my_tiles > 0) issue_load(0);
   __syncwarp();
   if (!producer) {
     // S (fp16-exact by contract) is requested first: lanes read consecutive 16-byte pieces
@@ -514,12 +515,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       sm.vb[tid] = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
     }
     asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
-    if (tid < 8) {
-      // code field f = r + sw s (merged keys: r + 4 s; 2-bit: r + 2 s) -> c[s ? h + r : h - 1 - r]
-      constexpr int sw = Fields<KB, kMerged>::sw > 0 ? Fields<KB, kMerged>::sw : HK;
-      const int r = tid % sw, sg = tid / sw;
-      sm.kcode_c[tid] = (sg <= 1 && r < HK) ? sm.kc[sg ? HK + r : HK - 1 - r] : 0.f;
-    }
+    if (tid < 8) sm.kmag[tid] = tid < HK ? sm.kc[HK + tid] : 0.f;
     if (tid == 0 && blockIdx.x == 0) {
       bool sym = true;
       for (int i = 0; i < 2 * HK; ++i) sym &= sm.kc[i] == -sm.kc[2 * HK - 1 - i];
@@ -577,76 +573,61 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   if (producer) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
-    // ---------------- producer: MMAs (warp 8) and copies (warp 9) ----------------
-    // MMAs of tile j: forward K into KS[j & 1] once KS[(j - 2) & 1] is released (its sketch
-    // read, or without QJL its exchange done); the sketch into KS[j & 1] once the compute
-    // warps have written A; forward V into V once the previous y'_V is read.  Copies: tile
-    // j + 2 into stage j & 1 as soon as both forward MMAs of tile j have read it.  Each wait's
-    // phase is one the other side cannot run two phases past.
-    if (warp == kComputeWarps && lane == 0 && KQ) {
-      // S D H into KS[1] (free until tile 1): read out by the compute warps before tile 0
-      tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) mma_ss(tmem + kColKS1, smem_desc(sm.x[1][0], ks), smem_desc(sm.bhd, ks), ks > 0);
-      mma_commit(&sm.bar_setup);
-    }
-    if (warp == kComputeWarps && lane == 0 && my_tiles > 0) {
-      auto fwd = [&](int j, uint32_t dcol, int kv) {
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + dcol, smem_desc(sm.x[j & 1][kv], ks), smem_desc(sm.bhd, ks), ks > 0);
-      };
-      bool ok = bar_wait(&sm.bar_load[0], 0);
-      if (ok) {
+    // ---------------- producer: one MMA issuer per group, one copy issuer ----------------
+    // Group g owns tiles j = g, g + 2, ... and the tensor-memory columns K[g], V[g].  For its
+    // n-th tile its issuer waits until the group has released K[g] / V[g] (tile n - 1 read
+    // out) and the tile has landed in stage g, issues the forward MMAs (y'_K -> K[g],
+    // y'_V -> V[g]), and with QJL waits for the group's A (in place in K[g]) before issuing
+    // the sketch into V[g].  The copy issuer refills stage s with the next tile of that
+    // stage once both forward MMAs of the previous one have read it.  Each wait's phase is
+    // one the other side cannot run two phases past.
+    if ((warp == kIssuerWarp0 || warp == kIssuerWarp1) && lane == 0) {
+      const int g = warp == kIssuerWarp0 ? 0 : 1;
+      const uint32_t colK = tmem + kColGroup * g, colV = colK + kColV;
+      bool ok = true;
+      if (KQ && g == 1) {
+        // S D H into K[1] (free until tile 1): read out by group 1 before its first tile
         tc_fence_after();
-        fwd(0, kColKS0, 0);
-        mma_commit(&sm.bar_fwdk);
-        fwd(0, kColV, 1);
-        mma_commit(&sm.bar_fwdv);
-        mma_commit(&sm.stage_free[0]);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_ss(colK, smem_desc(sm.x[1][0], ks), smem_desc(sm.bhd, ks), ks > 0);
+        mma_commit(&sm.bar_setup);
       }
-      for (int j = 0; j < my_tiles && ok; ++j) {
-        const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
-        if (j + 1 < my_tiles) {
-          // y'_V of tile j has been read (v_free phase j arrives after each compute warp has
-          // waited for it and read it): the next one may land
-          if (!(ok = bar_wait(&sm.v_free, j & 1))) break;
-          if (!(ok = bar_wait(&sm.bar_load[(j + 1) & 1], ((j + 1) >> 1) & 1))) break;
-          tc_fence_after();
-          fwd(j + 1, kColV, 1);
-          mma_commit(&sm.bar_fwdv);
-          // KS[(j + 1) & 1] holds tile j - 1's A: its sketch must be done with it (this thread
-          // issued it and consumes each sketch commit in turn); ks_free phase j arrives after
-          // every compute warp has waited for y'_K of tile j
-          if (KQ && j >= 1 && !(ok = bar_wait(&sm.bar_sig, (j - 1) & 1))) break;
-          if (!(ok = bar_wait(&sm.ks_free, j & 1))) break;
-          tc_fence_after();
-          fwd(j + 1, (j & 1) ? kColKS0 : kColKS1, 0);
-          mma_commit(&sm.bar_fwdk);
-          mma_commit(&sm.stage_free[(j + 1) & 1]);  // both forward MMAs of tile j + 1 read it
-        }
+      // S D H read out of K[1]: group 1's first tile may land there
+      if (KQ && g == 1 && my_tiles > 1) ok = bar_wait(&sm.setup_read, 0);
+      for (int n = 0, j = g; ok && j < my_tiles; ++n, j += 2) {
+        if (n > 0 && !(ok = bar_wait(&sm.tm_free[g], (n - 1) & 1))) break;
+        if (!(ok = bar_wait(&sm.bar_load[g], n & 1))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_ss(colK, smem_desc(sm.x[g][0], ks), smem_desc(sm.bhd, ks), ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) mma_ss(colV, smem_desc(sm.x[g][1], ks), smem_desc(sm.bhd, ks), ks > 0);
+        mma_commit(&sm.fwd_done[g]);
+        mma_commit(&sm.stage_free[g]);  // both forward MMAs of tile j have read stage g
         if (KQ) {
-          // A of tile j is in KS[j & 1] and X is free (the previous sketch was read)
-          if (!(ok = bar_wait(&sm.a_ready, j & 1))) break;
+          // A of tile j is in K[g] and y'_V is read: the sketch goes into V[g]; its B
+          // operands (S D H hi / lo) are in shared memory once group 1 has read them out
+          if (g == 0 && n == 0 && !(ok = bar_wait(&sm.setup_read, 0))) break;
+          if (!(ok = bar_wait(&sm.a_ready[g], n & 1))) break;
           tc_fence_after();
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            // coordinates 16 ks ..: part ks / 4, chunk (ks / 2) % 2, half ks % 2
-            const uint32_t ahi = tmem + ks_j + 64 * (ks >> 2) + 32 * ((ks >> 1) & 1) + 8 * (ks & 1);
-            mma_ts(tmem + kColX, ahi, smem_desc(sm.bshi, ks), ks > 0);
-            mma_ts(tmem + kColX, ahi, smem_desc(sm.bslo, ks), 1);
-            mma_ts(tmem + kColX, ahi + 16, smem_desc(sm.bshi, ks), 1);
+            // coordinates 16 ks ..: chunk ks / 2, half ks % 2 (hi at +0, lo at +16)
+            const uint32_t ahi = colK + 32 * (ks >> 1) + 8 * (ks & 1);
+            mma_ts(colV, ahi, smem_desc(sm.bshi, ks), ks > 0);
+            mma_ts(colV, ahi, smem_desc(sm.bslo, ks), 1);
+            mma_ts(colV, ahi + 16, smem_desc(sm.bshi, ks), 1);
           }
-          mma_commit(&sm.bar_sig);
+          mma_commit(&sm.sig_done[g]);
         }
       }
       if (!ok) {
         report(a.status, TQ_ERR_TIMEOUT);
         // let the MMAs already issued finish (bounded) before tensor memory is freed
-        mma_commit(&sm.bar_setup);
-        bar_wait(&sm.bar_setup, KQ ? 1 : 0);
+        mma_commit(&sm.bar_drain[g]);
+        bar_wait(&sm.bar_drain[g], 0);
       }
-    } else if (warp == kComputeWarps + 1 && lane == 0 && my_tiles > 0) {
+    } else if (warp == kLoaderWarp && lane == 0 && my_tiles > 0) {
       int issued = 1;  // tile 0 went out before the set-up
       bool ok = true;
       // stage 1 holds S until the S D H MMA has read it
@@ -669,189 +650,170 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     __syncwarp();
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
-    // ---------------- compute warps ----------------
+    // ---------------- compute groups ----------------
     typedef Fields<KB, kMerged> FK;
     typedef Fields<VB, false> FV;
+    const int g = warp / kGroupWarps;  // tiles g, g + 2, ...
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+    const uint32_t colK = tmem + lane_base + kColGroup * g, colV = colK + kColV;
     auto token_ref = [&](int j) -> TokRef {
       int b, h, t0;
       tile_coords(j, b, h, t0);
       const int len = a.seq_lens[b];
       const int tok = t0 + row;
       const bool bad_len = len < 0 || len > a.max_len || len > a.cache.max_pages * PT;
-      if (bad_len && tid == 0 && t0 == 0) report(a.status, TQ_ERR_BOUNDS);
+      if (bad_len && row == 0 && t0 == 0) report(a.status, TQ_ERR_BOUNDS);
       TokRef r{nullptr, tok % PT};
       if (!bad_len && tok < len) {
         const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + tok / PT];
         if (phys < 0 || phys >= a.cache.num_pages) {
-          if (part == 0) report(a.status, TQ_ERR_BOUNDS);
+          report(a.status, TQ_ERR_BOUNDS);
         } else {
           r.blk = a.cache.block(phys, h);
         }
       }
       return r;
     };
-    // per-token sum over the two warps of a token, through shared memory; the barrier
-    // before the write keeps the partner's reads of the previous use ahead of it
-    auto pair_sum2 = [&](float u, float v) -> float2 {
-      pair_sync(qd);
-      sm.red[row][part] = make_float2(u, v);
-      pair_sync(qd);
-      const float2 a0 = sm.red[row][0], a1 = sm.red[row][1];
-      return make_float2(a0.x + a1.x, a0.y + a1.y);
-    };
-    // key words of the previous tile, completed by its sketch signs one tile later
-    TokRef prev{nullptr, 0};
-    uint4 pk[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-    uint32_t pnorms = 0;  // fp16 ||k|| | fp16 rho << 16
-    // the previous tile's signs from X, chunk by chunk, and its key words stored
-    auto finish_keys = [&]() {
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        float sk[32];
-        tmem_ld32(tmem + lane_base + kColX + kCPT * part + 32 * c, sk);
-        tmem_wait_ld();
-        uint4 w = c ? pk[1] : pk[0];
-        uint32_t sgw = FK::sig_init();
-        sigma32<kMerged, FK>(sk, w, sgw);
-        if (prev.blk != nullptr) {
-          store_chunk<KB, kMerged>(prev.blk + L.kc, part, c, prev.slot, w);
-          if (!kMerged) *reinterpret_cast<uint32_t*>(prev.blk + L.ks + (size_t)prev.slot * 16 + 4 * (2 * part + c)) = sgw;
-        }
-      }
-      if (prev.blk != nullptr && part == 0) {
-        reinterpret_cast<uint16_t*>(prev.blk + L.kn)[prev.slot] = (uint16_t)(pnorms & 0xffff);
-        reinterpret_cast<uint16_t*>(prev.blk + L.kr)[prev.slot] = (uint16_t)(pnorms >> 16);
-      }
-    };
     bool failed = false;
-    if constexpr (KQ) {
-      // S D H (fp32 in KS[1], row = sketch index) split into the fp16 hi / lo B operands
+    if (KQ && g == 1) {
+      // S D H (fp32 in K[1], row = sketch index) split into the fp16 hi / lo B operands
       if (!bar_wait(&sm.bar_setup, 0)) failed = true;
       __syncwarp();
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_base + kColKS1 + kCPT * part + 32 * c, v);
+        tmem_ld32(colK + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int q = 0; q < 4; ++q) {
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
+            const float x0 = v[8 * q + 2 * e], x1 = v[8 * q + 2 * e + 1];
             const __half2 h2 = __floats2half2_rn(x0, x1);
             const float2 hf = __half22float2(h2);
             const __half2 l2 = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
             hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
             lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
           }
-          const int k = kCPT * part + 32 * c + 8 * g;
+          const int k = 32 * c + 8 * q;
           *reinterpret_cast<uint4*>(sm.bshi + canon(row, k)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(sm.bslo + canon(row, k)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
-      // visible to the sketch MMAs, which wait for a_ready after these writes
+      // visible to the sketch MMAs, which wait for setup_read after these writes
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(&sm.setup_read);
     }
-    // the token address of the next tile is looked up one tile ahead
-    TokRef next = my_tiles > 0 ? token_ref(0) : TokRef{nullptr, 0};
-    for (int j = 0; j < my_tiles; ++j) {
+    // the token address of the group's next tile is looked up one tile ahead
+    TokRef next = g < my_tiles ? token_ref(g) : TokRef{nullptr, 0};
+    for (int n = 0, j = g; j < my_tiles; ++n, j += 2) {
       const TokRef cur = next;
-      if (j + 1 < my_tiles) next = token_ref(j + 1);
-      const uint32_t ks_j = (j & 1) ? kColKS1 : kColKS0;
+      if (j + 2 < my_tiles) next = token_ref(j + 2);
 
       // ---- norms of y'_K and y'_V ----
-      if (!failed && !bar_wait(&sm.bar_fwdk, j & 1)) failed = true;
-      if (!failed && !bar_wait(&sm.bar_fwdv, j & 1)) failed = true;
+      if (!failed && !bar_wait(&sm.fwd_done[g], n & 1)) failed = true;
       __syncwarp();
       tc_fence_after();
-      if (lane == 0) bar_arrive(&sm.ks_free);  // this warp is past its wait for y'_K of tile j
       float ssk = 0.f, ssv = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float y[32], z[32];
-        tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32 * c, y);
-        tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32 * c, z);
+        tmem_ld32(colK + 32 * c, y);
+        tmem_ld32(colV + 32 * c, z);
         tmem_wait_ld();
         ssk += sumsq32(y);
         ssv += sumsq32(z);
       }
-      const float2 ss = pair_sum2(ssk, ssv);
-      const float nyk = sqrtf(ss.x);  // ||y'_K|| = sqrt(d) ||k||
-      const float nyv = sqrtf(ss.y);
+      const float nyk = sqrtf(ssk);  // ||y'_K|| = sqrt(d) ||k||
+      const float nyv = sqrtf(ssv);
       const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
       const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
-      if (cur.blk && part == 0 && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
+      if (cur.blk && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
 
       // ---- values and keys, chunk by chunk; the keys' residual goes to TMEM in place ----
       const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
       const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
       f2_t rr2 = 0;
-      uint4 kwc[2];
+      // key words of the four chunks (completed by the signs)
+      uint4 kw0 = make_uint4(0, 0, 0, 0), kw1 = kw0, kw2 = kw0, kw3 = kw0;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float y[32], z[32];
-        tmem_ld32(tmem + lane_base + ks_j + kCPT * part + 32 * c, y);
-        tmem_ld32(tmem + lane_base + kColV + kCPT * part + 32 * c, z);
+        tmem_ld32(colK + 32 * c, y);
+        tmem_ld32(colV + 32 * c, z);
         tmem_wait_ld();
-        constexpr uint32_t vw0 = FV::init(0), vw1 = FV::init(1), vw2 = FV::init(2), vw3 = FV::init(3);
-        constexpr uint32_t kw0 = FK::init(0), kw1 = FK::init(1), kw2 = FK::init(2), kw3 = FK::init(3);
-        uint32_t vw[4] = {vw0, vw1, vw2, vw3}, kw[4] = {kw0, kw1, kw2, kw3};
+        constexpr int kMS = KQ ? 2 : 0;  // key ranks at mantissa bit 2 (table offsets), value ranks at 0
+        constexpr uint32_t vw0 = FV::init(0, 0), vw1 = FV::init(1, 0), vw2 = FV::init(2, 0), vw3 = FV::init(3, 0);
+        constexpr uint32_t kwi0 = FK::init(0, kMS), kwi1 = FK::init(1, kMS), kwi2 = FK::init(2, kMS),
+                           kwi3 = FK::init(3, kMS);
+        uint32_t vw[4] = {vw0, vw1, vw2, vw3}, kw[4] = {kwi0, kwi1, kwi2, kwi3};
         uint32_t hi[16], lo[16], dh[16], dl[16];
         f2_t drr = 0;
-        quantise32<HV - 1, FV, false>(z, qv, sm.kcode_c, vw, dh, dl, drr);
-        quantise32<HK - 1, FK, KQ != 0>(y, qk, sm.kcode_c, kw, hi, lo, rr2);
-        if (cur.blk && !failed) store_chunk<VB, false>(cur.blk + L.vc, part, c, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
+        quantise32<HV - 1, FV, false>(z, qv, sm.kmag, vw, dh, dl, drr);
+        quantise32<HK - 1, FK, KQ != 0>(y, qk, sm.kmag, kw, hi, lo, rr2);
+        if (cur.blk && !failed)
+          store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
         const uint4 kq = make_uint4(kw[0], kw[1], kw[2], kw[3]);
         if constexpr (KQ) {
-          tmem_st16(tmem + lane_base + ks_j + kCPT * part + 32 * c, hi);
-          tmem_st16(tmem + lane_base + ks_j + kCPT * part + 32 * c + 16, lo);
-          if (c) kwc[1] = kq; else kwc[0] = kq;
+          tmem_st16(colK + 32 * c, hi);
+          tmem_st16(colK + 32 * c + 16, lo);
+          kw0 = c == 0 ? kq : kw0;
+          kw1 = c == 1 ? kq : kw1;
+          kw2 = c == 2 ? kq : kw2;
+          kw3 = c == 3 ? kq : kw3;
         } else if (cur.blk && !failed) {
-          store_chunk<KB, false>(cur.blk + L.kc, part, c, cur.slot, kq);
+          store_chunk<KB, false>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, kq);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) bar_arrive(&sm.v_free);  // y'_V of tile j is read
-      if (cur.blk && !failed && part == 0) {
-        reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
-        if (!KQ) reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
-      }
-
       if constexpr (KQ) {
-        // the previous tile's sketch (in X) is done: its signs complete that tile's keys
+        // A of tile j is written and y'_V is read: the sketch may overwrite V[g]
         tmem_wait_st();
-        if (j > 0) {
-          if (!failed && !bar_wait(&sm.bar_sig, (j - 1) & 1)) failed = true;
-          __syncwarp();
-          tc_fence_after();
-          if (failed) prev.blk = nullptr;
-          finish_keys();
-        }
-        float ra, rb;
-        uf2(rr2, ra, rb);
-        const float rho = sqrtf(pair_sum2(ra + rb, 0.f).x) * qk.inv_alpha * (1.0f / kSqrtD);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) bar_arrive(&sm.a_ready);  // A of tile j is written and X is free
-        prev = failed ? TokRef{nullptr, 0} : cur;
-        pk[0] = kwc[0];
-        pk[1] = kwc[1];
-        pnorms = (uint32_t)__half_as_ushort(nk16) | ((uint32_t)__half_as_ushort(__float2half_rn(rho)) << 16);
-      }
-    }
-    if constexpr (KQ) {
-      // the last tile's signs
-      if (my_tiles > 0) {
-        if (!failed && !bar_wait(&sm.bar_sig, (my_tiles - 1) & 1)) failed = true;
+        if (lane == 0) bar_arrive(&sm.a_ready[g]);
+        float ra, rb;
+        uf2(rr2, ra, rb);
+        const float rho = sqrtf(ra + rb) * qk.inv_alpha * (1.0f / kSqrtD);
+        if (cur.blk && !failed) {
+          reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+          reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+          reinterpret_cast<__half*>(cur.blk + L.kr)[cur.slot] = __float2half_rn(rho);
+        }
+        // the sketch's signs complete the key words
+        if (!failed && !bar_wait(&sm.sig_done[g], n & 1)) failed = true;
         __syncwarp();
         tc_fence_after();
-        if (failed) prev.blk = nullptr;
-        finish_keys();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float sk[32];
+          tmem_ld32(colV + 32 * c, sk);
+          tmem_wait_ld();
+          if (c == 3) {
+            // K[g] and V[g] are read out: the group's next tile may land in them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) bar_arrive(&sm.tm_free[g]);
+          }
+          uint4 w = c == 0 ? kw0 : (c == 1 ? kw1 : (c == 2 ? kw2 : kw3));
+          uint32_t sgw = 0;
+          sigma32<kMerged, FK>(sk, w, sgw);
+          if (cur.blk && !failed) {
+            store_chunk<KB, kMerged>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, w);
+            if (!kMerged) *reinterpret_cast<uint32_t*>(cur.blk + L.ks + (size_t)cur.slot * 16 + 4 * c) = sgw;
+          }
+        }
+      } else {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&sm.tm_free[g]);
+        if (cur.blk && !failed) {
+          reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+          reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+        }
       }
     }
     if (failed && lane == 0) report(a.status, TQ_ERR_TIMEOUT);
