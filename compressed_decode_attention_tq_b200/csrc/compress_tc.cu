@@ -43,10 +43,10 @@ constexpr int kGroupWarps = 4;  // warps of one compute group (one tile)
 // producer warpgroup: the MMA issuers of groups 0 and 1 and the copy issuer
 constexpr int kIssuerWarp0 = kComputeWarps, kLoaderWarp = kComputeWarps + 1, kIssuerWarp1 = kComputeWarps + 2;
 // two compute warpgroups and one producer warpgroup; registers move from the producer to
-// the compute warpgroups after launch: launched with 384 x 168, then 128 x 96 + 256 x 200
-// = 63488 <= 384 x 168.
+// the compute warpgroups after launch: launched with 384 x 168, then 128 x 72 + 256 x 216
+// = 64512 = 384 x 168.
 constexpr int kThreadsTC = (kComputeWarps + 4) * 32;
-constexpr int kRegsLaunch = 168, kRegsProducer = 96, kRegsCompute = 200;
+constexpr int kRegsLaunch = 168, kRegsProducer = 72, kRegsCompute = 216;
 static_assert(kComputeWarps == 2 * kGroupWarps && kGroupWarps == 4, "two groups of four lane quadrants");
 static_assert(128 * kRegsProducer + 32 * kComputeWarps * kRegsCompute <= kThreadsTC * kRegsLaunch,
               "register split exceeds the launch allocation");
@@ -68,9 +68,10 @@ struct SmemTC {
   unsigned char bhd[kTileBytes];      // B = H D
   unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part
   unsigned char bslo[kTileBytes];     // fp16 lo part
-  // [stage]: tile landed / read by its forward MMAs; [group]: forward MMAs done, A written
-  // (and y'_V read), sketch done, tensor-memory columns released, error drain
-  unsigned long long bar_load[2], stage_free[2], fwd_done[2], a_ready[2], sig_done[2], tm_free[2], bar_drain[2];
+  // [stage]: tile landed / read by its forward MMAs; [group]: forward MMAs done, A of key
+  // chunk c written (y'_V read before the first), sketch done, tensor-memory columns
+  // released, error drain
+  unsigned long long bar_load[2], stage_free[2], fwd_done[2], a_chunk[2][4], sig_done[2], tm_free[2], bar_drain[2];
   unsigned long long bar_setup, setup_read;  // S D H MMA done / read out into bshi, bslo
   uint32_t tmem_base;
   int bad_s;
@@ -228,15 +229,17 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
 
 // sum of squares of 32 values, two lanes of packed fp32 at a time
 __device__ __forceinline__ float sumsq32(const float (&v)[32]) {
-  f2_t acc = 0;
+  f2_t acc0 = 0, acc1 = 0;
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const f2_t p = f2(v[i], v[i + 1]);
-    acc = fma2(p, p, acc);
+  for (int i = 0; i < 32; i += 4) {
+    const f2_t p = f2(v[i], v[i + 1]), q = f2(v[i + 2], v[i + 3]);
+    acc0 = fma2(p, p, acc0);
+    acc1 = fma2(q, q, acc1);
   }
-  float lo, hi;
-  uf2(acc, lo, hi);
-  return lo + hi;
+  float a, b, c, d;
+  uf2(acc0, a, b);
+  uf2(acc1, c, d);
+  return (a + b) + (c + d);
 }
 
 // Magnitude ranks are assembled in the mantissa of a power of two plus the rank (exact
@@ -474,7 +477,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bar_init(&sm.bar_load[g], 1);
       bar_init(&sm.stage_free[g], 1);
       bar_init(&sm.fwd_done[g], 1);
-      bar_init(&sm.a_ready[g], kGroupWarps);
+      for (int c = 0; c < 4; ++c) bar_init(&sm.a_chunk[g][c], kGroupWarps);
       bar_init(&sm.sig_done[g], 1);
       bar_init(&sm.tm_free[g], kGroupWarps);
       bar_init(&sm.bar_drain[g], 1);
@@ -594,31 +597,57 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       // S D H read out of K[1]: group 1's first tile may land there
       if (KQ && g == 1 && my_tiles > 1) ok = bar_wait(&sm.setup_read, 0);
+      // MMA issue is not on any critical path: the loops stay rolled to keep the producer's
+      // registers few
+      auto fwd = [&](int kv, uint32_t dcol) {
+#pragma unroll 1
+        for (int ks = 0; ks < 8; ++ks) mma_ss(dcol, smem_desc(sm.x[g][kv], ks), smem_desc(sm.bhd, ks), ks > 0);
+      };
+      bool k_issued = false;  // y'_K of the group's next tile already requested
       for (int n = 0, j = g; ok && j < my_tiles; ++n, j += 2) {
-        if (n > 0 && !(ok = bar_wait(&sm.tm_free[g], (n - 1) & 1))) break;
-        if (!(ok = bar_wait(&sm.bar_load[g], n & 1))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(colK, smem_desc(sm.x[g][0], ks), smem_desc(sm.bhd, ks), ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) mma_ss(colV, smem_desc(sm.x[g][1], ks), smem_desc(sm.bhd, ks), ks > 0);
+        if (!k_issued) {
+          if (n > 0 && !(ok = bar_wait(&sm.tm_free[g], (n - 1) & 1))) break;
+          if (!(ok = bar_wait(&sm.bar_load[g], n & 1))) break;
+          tc_fence_after();
+          fwd(0, colK);
+        } else {
+          // y'_V of the previous tile, then the sketch output, read out of V[g]
+          if (!(ok = bar_wait(&sm.tm_free[g], (n - 1) & 1))) break;
+          tc_fence_after();
+        }
+        fwd(1, colV);
         mma_commit(&sm.fwd_done[g]);
         mma_commit(&sm.stage_free[g]);  // both forward MMAs of tile j have read stage g
+        k_issued = false;
         if (KQ) {
-          // A of tile j is in K[g] and y'_V is read: the sketch goes into V[g]; its B
-          // operands (S D H hi / lo) are in shared memory once group 1 has read them out
+          // The sketch goes into V[g] (y'_V is read before the first key chunk is released),
+          // chunk by chunk as the group writes A into K[g]; its B operands (S D H hi / lo) are
+          // in shared memory once group 1 has read them out
           if (g == 0 && n == 0 && !(ok = bar_wait(&sm.setup_read, 0))) break;
-          if (!(ok = bar_wait(&sm.a_ready[g], n & 1))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            // coordinates 16 ks ..: chunk ks / 2, half ks % 2 (hi at +0, lo at +16)
-            const uint32_t ahi = colK + 32 * (ks >> 1) + 8 * (ks & 1);
-            mma_ts(colV, ahi, smem_desc(sm.bshi, ks), ks > 0);
-            mma_ts(colV, ahi, smem_desc(sm.bslo, ks), 1);
-            mma_ts(colV, ahi + 16, smem_desc(sm.bshi, ks), 1);
+#pragma unroll 1
+          for (int c = 0; c < 4 && ok; ++c) {
+            if (!(ok = bar_wait(&sm.a_chunk[g][c], n & 1))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+              // coordinates 16 ks ..: chunk c, half h (hi at +0, lo at +16)
+              const int ks = 2 * c + h;
+              const uint32_t ahi = colK + 32 * c + 8 * h;
+              mma_ts(colV, ahi, smem_desc(sm.bshi, ks), ks > 0);
+              mma_ts(colV, ahi, smem_desc(sm.bslo, ks), 1);
+              mma_ts(colV, ahi + 16, smem_desc(sm.bshi, ks), 1);
+            }
           }
+          if (!ok) break;
           mma_commit(&sm.sig_done[g]);
+          // once the sketch is done with A, K[g] takes y'_K of the group's next tile
+          if (j + 2 < my_tiles) {
+            if (!(ok = bar_wait(&sm.sig_done[g], n & 1))) break;
+            if (!(ok = bar_wait(&sm.bar_load[g], (n + 1) & 1))) break;
+            tc_fence_after();
+            fwd(0, colK);
+            k_issued = true;
+          }
         }
       }
       if (!ok) {
@@ -656,20 +685,28 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int g = warp / kGroupWarps;  // tiles g, g + 2, ...
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
     const uint32_t colK = tmem + lane_base + kColGroup * g, colV = colK + kColV;
-    auto token_ref = [&](int j) -> TokRef {
+    // The sequence length and the page entry of the token this thread owns in tile j: two
+    // independent loads, issued one group tile ahead and checked when the tile starts.
+    struct TokLoad {
+      int len, phys, t0, h;
+    };
+    auto token_load = [&](int j) -> TokLoad {
       int b, h, t0;
       tile_coords(j, b, h, t0);
-      const int len = a.seq_lens[b];
-      const int tok = t0 + row;
-      const bool bad_len = len < 0 || len > a.max_len || len > a.cache.max_pages * PT;
-      if (bad_len && row == 0 && t0 == 0) report(a.status, TQ_ERR_BOUNDS);
+      const int page = (t0 + row) / PT;
+      return TokLoad{a.seq_lens[b],
+                     page < a.cache.max_pages ? a.cache.block_table[(size_t)b * a.cache.max_pages + page] : -1, t0, h};
+    };
+    auto token_ref = [&](const TokLoad& l) -> TokRef {
+      const int tok = l.t0 + row;
+      const bool bad_len = l.len < 0 || l.len > a.max_len || l.len > a.cache.max_pages * PT;
+      if (bad_len && row == 0 && l.t0 == 0) report(a.status, TQ_ERR_BOUNDS);
       TokRef r{nullptr, tok % PT};
-      if (!bad_len && tok < len) {
-        const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + tok / PT];
-        if (phys < 0 || phys >= a.cache.num_pages) {
+      if (!bad_len && tok < l.len) {
+        if (l.phys < 0 || l.phys >= a.cache.num_pages) {
           report(a.status, TQ_ERR_BOUNDS);
         } else {
-          r.blk = a.cache.block(phys, h);
+          r.blk = a.cache.block(l.phys, l.h);
         }
       }
       return r;
@@ -708,11 +745,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(&sm.setup_read);
     }
-    // the token address of the group's next tile is looked up one tile ahead
-    TokRef next = g < my_tiles ? token_ref(g) : TokRef{nullptr, 0};
+    TokLoad next = g < my_tiles ? token_load(g) : TokLoad{0, -1, 0, 0};
     for (int n = 0, j = g; j < my_tiles; ++n, j += 2) {
-      const TokRef cur = next;
-      if (j + 2 < my_tiles) next = token_ref(j + 2);
+      const TokRef cur = token_ref(next);
+      if (j + 2 < my_tiles) next = token_load(j + 2);
 
       // ---- norms of y'_K and y'_V ----
       if (!failed && !bar_wait(&sm.fwd_done[g], n & 1)) failed = true;
@@ -734,29 +770,42 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
       if (cur.blk && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
 
-      // ---- values and keys, chunk by chunk; the keys' residual goes to TMEM in place ----
+      // ---- values, then keys chunk by chunk; the keys' residual goes to TMEM in place and each
+      // chunk is released to the sketch MMAs while the next chunk's load is in flight ----
       const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
       const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float z[32];
+        tmem_ld32(colV + 32 * c, z);
+        tmem_wait_ld();
+        constexpr uint32_t vw0 = FV::init(0, 0), vw1 = FV::init(1, 0), vw2 = FV::init(2, 0), vw3 = FV::init(3, 0);
+        uint32_t vw[4] = {vw0, vw1, vw2, vw3}, dh[16], dl[16];
+        f2_t drr = 0;
+        quantise32<HV - 1, FV, false>(z, qv, sm.kmag, vw, dh, dl, drr);
+        if (cur.blk && !failed)
+          store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
+      }
       f2_t rr2 = 0;
       // key words of the four chunks (completed by the signs)
       uint4 kw0 = make_uint4(0, 0, 0, 0), kw1 = kw0, kw2 = kw0, kw3 = kw0;
+      auto release = [&](int c) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&sm.a_chunk[g][c]);
+      };
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
-        float y[32], z[32];
+        float y[32];
         tmem_ld32(colK + 32 * c, y);
-        tmem_ld32(colV + 32 * c, z);
+        if (KQ && c > 0) release(c - 1);
         tmem_wait_ld();
-        constexpr int kMS = KQ ? 2 : 0;  // key ranks at mantissa bit 2 (table offsets), value ranks at 0
-        constexpr uint32_t vw0 = FV::init(0, 0), vw1 = FV::init(1, 0), vw2 = FV::init(2, 0), vw3 = FV::init(3, 0);
+        constexpr int kMS = KQ ? 2 : 0;  // key ranks at mantissa bit 2 (table offsets)
         constexpr uint32_t kwi0 = FK::init(0, kMS), kwi1 = FK::init(1, kMS), kwi2 = FK::init(2, kMS),
                            kwi3 = FK::init(3, kMS);
-        uint32_t vw[4] = {vw0, vw1, vw2, vw3}, kw[4] = {kwi0, kwi1, kwi2, kwi3};
-        uint32_t hi[16], lo[16], dh[16], dl[16];
-        f2_t drr = 0;
-        quantise32<HV - 1, FV, false>(z, qv, sm.kmag, vw, dh, dl, drr);
+        uint32_t kw[4] = {kwi0, kwi1, kwi2, kwi3}, hi[16], lo[16];
         quantise32<HK - 1, FK, KQ != 0>(y, qk, sm.kmag, kw, hi, lo, rr2);
-        if (cur.blk && !failed)
-          store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
         const uint4 kq = make_uint4(kw[0], kw[1], kw[2], kw[3]);
         if constexpr (KQ) {
           tmem_st16(colK + 32 * c, hi);
@@ -770,11 +819,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
       if constexpr (KQ) {
-        // A of tile j is written and y'_V is read: the sketch may overwrite V[g]
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) bar_arrive(&sm.a_ready[g]);
+        release(3);
         float ra, rb;
         uf2(rr2, ra, rb);
         const float rho = sqrtf(ra + rb) * qk.inv_alpha * (1.0f / kSqrtD);
@@ -787,25 +832,28 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (!failed && !bar_wait(&sm.sig_done[g], n & 1)) failed = true;
         __syncwarp();
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float sk[32];
-          tmem_ld32(colV + 32 * c, sk);
-          tmem_wait_ld();
-          if (c == 3) {
-            // K[g] and V[g] are read out: the group's next tile may land in them
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) bar_arrive(&sm.tm_free[g]);
-          }
-          uint4 w = c == 0 ? kw0 : (c == 1 ? kw1 : (c == 2 ? kw2 : kw3));
+        float sk0[32], sk1[32], sk2[32], sk3[32];
+        tmem_ld32(colV, sk0);
+        tmem_ld32(colV + 32, sk1);
+        tmem_ld32(colV + 64, sk2);
+        tmem_ld32(colV + 96, sk3);
+        tmem_wait_ld();
+        // K[g] and V[g] are read out: the group's next tile may land in them
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(&sm.tm_free[g]);
+        auto finish = [&](const float (&sk)[32], uint4 w, int c) {
           uint32_t sgw = 0;
           sigma32<kMerged, FK>(sk, w, sgw);
           if (cur.blk && !failed) {
             store_chunk<KB, kMerged>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, w);
             if (!kMerged) *reinterpret_cast<uint32_t*>(cur.blk + L.ks + (size_t)cur.slot * 16 + 4 * c) = sgw;
           }
-        }
+        };
+        finish(sk0, kw0, 0);
+        finish(sk1, kw1, 1);
+        finish(sk2, kw2, 2);
+        finish(sk3, kw3, 3);
       } else {
         tc_fence_before();
         __syncwarp();
