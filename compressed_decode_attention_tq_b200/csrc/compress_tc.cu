@@ -467,6 +467,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   };
 
   // ---------------- set-up ----------------
+  // Launched as a programmatic dependent: the next kernel on the stream may be scheduled as
+  // SMs free up, and this one touches no global memory before its predecessor has finished.
+  asm volatile("griddepcontrol.launch_dependents;");
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s_u32(&sm.tmem_base)),
                  "r"(kTmemCols));
@@ -490,6 +493,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // tile 0 streams in while the rotation operands are built (stage 1 is set-up scratch)
   if (warp == kLoaderWarp && lane == 0 && my_tiles > 0) issue_load(0);
   __syncwarp();
@@ -928,8 +932,17 @@ cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtens
   const int tiles = a.cache.batch * a.cache.kv_heads * ((a.max_len + TT - 1) / TT);
   const int grid = tiles < sms ? tiles : sms;
   if (grid == 0) return cudaSuccess;
-  k<<<grid, kThreadsTC, kSmemTC, stream>>>(a, mk, mv);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreadsTC);
+  cfg.dynamicSmemBytes = kSmemTC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, a, mk, mv);
 }
 
 }  // namespace

@@ -45,7 +45,10 @@ __device__ __forceinline__ float block_max128(float v, float* red) {
 }
 
 __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_rows) {
-  // allow the dependent split kernel to start streaming pages right away
+  // Launched as a programmatic dependent of whatever precedes it on the stream: everything
+  // before it has finished once this wait returns.  Then the split kernel may start (its
+  // set-up reads only inputs no kernel of this call writes).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   __shared__ float qs[D], ys[D];
   __shared__ float red[2][4];
@@ -447,13 +450,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (fast_decode_supported(a)) {
     // query transforms (and zeroed merge counters), then the split kernel, whose last
     // split per (sequence, kv head) merges the partials: two launches
-    prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(prologue_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
     if (e != cudaSuccess) return e;
     return launch_fast_split(a, stream);
   }
-  prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prologue_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
   if (e != cudaSuccess) return e;
   e = launch_split(a, stream, false);
   if (e != cudaSuccess) return e;
@@ -464,8 +465,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream) {
   const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
-  prologue_kernel<<<total_rows, 128, 0, stream>>>(a, total_rows);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prologue_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
   if (e != cudaSuccess) return e;
   return launch_split(a, stream, true);
 }

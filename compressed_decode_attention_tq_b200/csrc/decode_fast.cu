@@ -181,6 +181,9 @@ __device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int
 
 template <int KP, int VP>
 __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
+  // the next kernel on the stream may be scheduled now; a programmatic dependent waits for
+  // this grid to finish before it touches what it writes
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SmemFast& sm = *reinterpret_cast<SmemFast*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
