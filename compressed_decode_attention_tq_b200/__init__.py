@@ -31,7 +31,8 @@ TQ_F32 = 1
 # Every function include/tq.h declares.
 EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_validate_config", "tq_page_bytes",
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
-           "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc")
+           "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc", "tq_operand_bytes",
+           "tq_prepare_operands")
 
 
 class tq_config(ctypes.Structure):
@@ -44,7 +45,8 @@ class tq_config(ctypes.Structure):
 class tq_params(ctypes.Structure):
     _fields_ = [("signs", ctypes.c_void_p), ("pi", ctypes.c_void_p), ("s", ctypes.c_void_p),
                 ("k_centroids", ctypes.c_void_p), ("k_boundaries", ctypes.c_void_p),
-                ("v_centroids", ctypes.c_void_p), ("v_boundaries", ctypes.c_void_p)]
+                ("v_centroids", ctypes.c_void_p), ("v_boundaries", ctypes.c_void_p),
+                ("operands", ctypes.c_void_p)]
 
 
 class tq_cache(ctypes.Structure):
@@ -79,6 +81,8 @@ def _load() -> ctypes.CDLL:
         "tq_decode_scores": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, SZ, P, P, P]),
         "tq_decompress": (I32, [cfgp, parp, cachep, I32, P, I32, P, P, P, P]),
         "tq_attend_decode_noalloc": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, P, P]),
+        "tq_operand_bytes": (SZ, [cfgp]),
+        "tq_prepare_operands": (I32, [cfgp, parp, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -137,10 +141,21 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_params(signs=None, pi=None, s=None, k_centroids=None, k_boundaries=None, v_centroids=None,
-                v_boundaries=None) -> tq_params:
-    """Device fp32 tensors -> tq_params (the tensors must outlive every call using it)."""
+                v_boundaries=None, operands=None) -> tq_params:
+    """Device fp32 tensors -> tq_params (the tensors must outlive every call using it);
+    operands: None or a device buffer filled by prepare_operands."""
     return tq_params(_ptr(signs), _ptr(pi), _ptr(s), _ptr(k_centroids), _ptr(k_boundaries),
-                     _ptr(v_centroids), _ptr(v_boundaries))
+                     _ptr(v_centroids), _ptr(v_boundaries), _ptr(operands))
+
+
+def operand_bytes(cfg: tq_config) -> int:
+    return lib.tq_operand_bytes(ctypes.byref(cfg))
+
+
+def prepare_operands(cfg, params, operands, stream=None):
+    """Fill operands (device uint8 tensor of operand_bytes(cfg) bytes) for params' signs/s."""
+    _check(lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), _ptr(operands),
+                                   _stream(stream)), "tq_prepare_operands")
 
 
 def make_cache(pages, block_table, num_pages, max_pages, batch, kv_heads, num_layers=1) -> tq_cache:

@@ -72,7 +72,9 @@ struct SmemTC {
   // chunk c written (y'_V read before the first), sketch done, tensor-memory columns
   // released, error drain
   unsigned long long bar_load[2], stage_free[2], fwd_done[2], a_chunk[2][4], sig_done[2], tm_free[2], bar_drain[2];
-  unsigned long long bar_setup, setup_read;  // S D H MMA done / read out into bshi, bslo
+  // set-up: B = H D built, S staged as an fp16 A operand, S D H MMA done, S D H read out
+  unsigned long long hd_ready, s_ready, bar_setup, setup_read;
+  unsigned long long ops_ready;  // prepared operands copied in
   uint32_t tmem_base;
   int bad_s;
   float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
@@ -144,6 +146,14 @@ __device__ __forceinline__ void tma_load_tile(void* dst, const CUtensorMap* map,
       "[%5];" ::"r"(s_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row0), "r"(0), "r"(s_u32(bar))
       : "memory");
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   s_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(s_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
@@ -485,6 +495,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bar_init(&sm.tm_free[g], kGroupWarps);
       bar_init(&sm.bar_drain[g], 1);
     }
+    bar_init(&sm.ops_ready, 1);
+    bar_init(&sm.hd_ready, kComputeWarps);
+    bar_init(&sm.s_ready, kComputeWarps);
     bar_init(&sm.bar_setup, 1);
     bar_init(&sm.setup_read, kGroupWarps);
     sm.bad_s = 0;
@@ -494,32 +507,58 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // tile 0 streams in while the rotation operands are built (stage 1 is set-up scratch)
-  if (warp == kLoaderWarp && lane == 0 && my_tiles > 0) issue_load(0);
+  // With prepared operands B = H D and S D H hi / lo are copied in (one 96 KB bulk copy);
+  // otherwise each CTA builds them (stage 1 is then set-up scratch for S).  Tile 0 streams
+  // in meanwhile.  (The copy thread issues tile 1 right after; group 1 starts its first tile
+  // that much later, and the two groups stay out of phase, which their ping-pong relies on.)
+  const bool prep = a.operands != nullptr;
+  if (warp == kLoaderWarp && lane == 0) {
+    if (prep) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(&sm.ops_ready)),
+                   "r"(3 * kTileBytes)
+                   : "memory");
+      const unsigned char* ops = static_cast<const unsigned char*>(a.operands);
+      bulk_load(sm.bhd, ops, kTileBytes, &sm.ops_ready);
+      bulk_load(sm.bshi, ops + kTileBytes, kTileBytes, &sm.ops_ready);
+      bulk_load(sm.bslo, ops + 2 * kTileBytes, kTileBytes, &sm.ops_ready);
+    }
+    if (my_tiles > 0) issue_load(0);
+  }
   __syncwarp();
   if (!producer) {
-    // S (fp16-exact by contract) is requested first: lanes read consecutive 16-byte pieces
-    // of a row (coalesced); it is converted and stored once the small tables are in
+    // The small tables (the rotation's D, the codebooks) are requested first, then S (fp16-
+    // exact by contract): lanes read consecutive 16-byte pieces of a row (coalesced), and
+    // each CTA starts at a different row, so that the CTAs' requests for the same 64 KB
+    // spread over the L2.  Nothing waits for S but the S D H operands: the forward MMAs of
+    // group 0's first tile need only B = H D (hd_ready).
+    const float sgn = !prep && tid < D ? a.signs[tid] : 0.f;
+    float tkc = 0.f, tkb = 0.f, tvc = 0.f, tvb = 0.f;
+    if (tid < 16) {
+      tkc = tid < 2 * HK ? a.k_centroids[tid] : 0.f;
+      tkb = tid < 2 * HK - 1 ? a.k_boundaries[tid] : 0.f;
+      tvc = tid < 2 * HV ? a.v_centroids[tid] : 0.f;
+      tvb = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
+    }
     constexpr int kSIter = QM * 16 / kComputeThreads;
     float4 sraw[KQ ? 2 * kSIter : 1];
-    if (KQ) {
+    auto s_row = [&](int c) { return ((c >> 4) + 8 * (int)blockIdx.x) & (QM - 1); };
+    if (KQ && !prep) {
 #pragma unroll
       for (int it = 0; it < kSIter; ++it) {
         const int c = tid + it * kComputeThreads;
-        const float4* src = reinterpret_cast<const float4*>(a.s + (size_t)(c >> 4) * D + 8 * (c & 15));
+        const float4* src = reinterpret_cast<const float4*>(a.s + (size_t)s_row(c) * D + 8 * (c & 15));
         sraw[2 * it] = src[0];
         sraw[2 * it + 1] = src[1];
       }
     }
-    // small inputs once into shared memory, one load per thread
     // D of the rotation, for the set-up only (in the space of the S D H operand, filled later)
     float* signs = reinterpret_cast<float*>(sm.bshi);
-    if (tid < D) signs[tid] = a.signs[tid];
+    if (!prep && tid < D) signs[tid] = sgn;
     if (tid < 16) {
-      sm.kc[tid] = tid < 2 * HK ? a.k_centroids[tid] : 0.f;
-      sm.kb[tid] = tid < 2 * HK - 1 ? a.k_boundaries[tid] : 0.f;
-      sm.vc[tid] = tid < 2 * HV ? a.v_centroids[tid] : 0.f;
-      sm.vb[tid] = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
+      sm.kc[tid] = tkc;
+      sm.kb[tid] = tkb;
+      sm.vc[tid] = tvc;
+      sm.vb[tid] = tvb;
     }
     asm volatile("bar.sync 5, %0;" ::"n"(kComputeThreads) : "memory");
     if (tid < 8) sm.kmag[tid] = tid < HK ? sm.kc[HK + tid] : 0.f;
@@ -535,6 +574,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // B = H D: row i, column k = (-1)^popcount(i & k) D_k
 #pragma unroll
     for (int it = 0; it < D * 16 / kComputeThreads; ++it) {
+      if (prep) break;
       const int c = tid + it * kComputeThreads;
       const int i = c & 127, ch = c >> 7;
       uint32_t w[4];
@@ -549,15 +589,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       *reinterpret_cast<uint4*>(sm.bhd + canon(i, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    if (KQ) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) bar_arrive(&sm.hd_ready);
+    if (KQ && !prep) {
       // S as an fp16 A operand in stage 1; S D H = S (H D)^T is then one MMA against the
-      // B = H D operand above
+      // B = H D operand above.  The D values in bshi are no longer read once every warp has
+      // passed hd_ready's arrival (the S D H readout, which overwrites them, waits for the MMA).
       unsigned char* sa = sm.x[1][0];
       int bad = 0;
 #pragma unroll
       for (int it = 0; it < kSIter; ++it) {
         const int c = tid + it * kComputeThreads;
-        const int m = c >> 4, ch = c & 15;
+        const int m = s_row(c), ch = c & 15;
         const float4 q0 = sraw[2 * it], q1 = sraw[2 * it + 1];
         const float e[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         uint32_t w[4];
@@ -571,11 +615,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         *reinterpret_cast<uint4*>(sa + canon(m, 8 * ch)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       if (bad) sm.bad_s = 1;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) bar_arrive(&sm.s_ready);
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  __syncthreads();
-  if (tid == 0 && sm.bad_s) report(a.status, TQ_ERR_INVALID_ARG);
   const uint32_t tmem = sm.tmem_base;
 
   if (producer) {
@@ -591,8 +635,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if ((warp == kIssuerWarp0 || warp == kIssuerWarp1) && lane == 0) {
       const int g = warp == kIssuerWarp0 ? 0 : 1;
       const uint32_t colK = tmem + kColGroup * g, colV = colK + kColV;
-      bool ok = true;
-      if (KQ && g == 1) {
+      // B = H D in shared memory (and for the S D H MMA, S as an A operand), or the
+      // prepared operands copied in
+      bool ok = bar_wait(prep ? &sm.ops_ready : &sm.hd_ready, 0);
+      if (ok && KQ && g == 1 && !prep) ok = bar_wait(&sm.s_ready, 0);
+      if (ok && KQ && g == 1 && !prep) {
         // S D H into K[1] (free until tile 1): read out by group 1 before its first tile
         tc_fence_after();
 #pragma unroll
@@ -600,7 +647,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         mma_commit(&sm.bar_setup);
       }
       // S D H read out of K[1]: group 1's first tile may land there
-      if (KQ && g == 1 && my_tiles > 1) ok = bar_wait(&sm.setup_read, 0);
+      if (ok && KQ && g == 1 && my_tiles > 1 && !prep) ok = bar_wait(&sm.setup_read, 0);
       // MMA issue is not on any critical path: the loops stay rolled to keep the producer's
       // registers few
       auto fwd = [&](int kv, uint32_t dcol) {
@@ -627,7 +674,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           // The sketch goes into V[g] (y'_V is read before the first key chunk is released),
           // chunk by chunk as the group writes A into K[g]; its B operands (S D H hi / lo) are
           // in shared memory once group 1 has read them out
-          if (g == 0 && n == 0 && !(ok = bar_wait(&sm.setup_read, 0))) break;
+          if (g == 0 && n == 0 && !prep && !(ok = bar_wait(&sm.setup_read, 0))) break;
 #pragma unroll 1
           for (int c = 0; c < 4 && ok; ++c) {
             if (!(ok = bar_wait(&sm.a_chunk[g][c], n & 1))) break;
@@ -663,8 +710,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     } else if (warp == kLoaderWarp && lane == 0 && my_tiles > 0) {
       int issued = 1;  // tile 0 went out before the set-up
       bool ok = true;
-      // stage 1 holds S until the S D H MMA has read it
-      if (KQ && !(ok = bar_wait(&sm.bar_setup, 0))) report(a.status, TQ_ERR_TIMEOUT);
+      // stage 1 holds S until the S D H MMA has read it (operands built in the CTA)
+      if (KQ && !prep && !(ok = bar_wait(&sm.bar_setup, 0))) report(a.status, TQ_ERR_TIMEOUT);
       if (ok && my_tiles > 1) {
         issue_load(1);
         issued = 2;
@@ -679,6 +726,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // the last copy into each stage is that stage's final phase: wait (bounded) for both to
       // land so that no copy is still in flight when the shared memory goes away
       for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) bar_wait(&sm.bar_load[i & 1], (i >> 1) & 1);
+      if (prep) bar_wait(&sm.ops_ready, 0);
     }
     __syncwarp();
   } else {
@@ -716,9 +764,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       return r;
     };
     bool failed = false;
-    if (KQ && g == 1) {
+    if (KQ && g == 1 && !prep) {
       // S D H (fp32 in K[1], row = sketch index) split into the fp16 hi / lo B operands
-      if (!bar_wait(&sm.bar_setup, 0)) failed = true;
+      if (!bar_wait(&sm.bar_setup, 0) || !bar_wait(&sm.s_ready, 0)) failed = true;
+      if (tid == kGroupWarps * 32 && sm.bad_s) report(a.status, TQ_ERR_INVALID_ARG);
       __syncwarp();
       tc_fence_after();
 #pragma unroll 1
@@ -880,6 +929,48 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 }
 
 // ---------------------------------------------------------------------------
+// prepared operands: B = H D, then S D H split into fp16 hi and lo, each a canonical tile
+// ---------------------------------------------------------------------------
+// The last CTA builds B = H D.  With QJL, CTA m < QM forms row m of S D H = (S D) H by a
+// Walsh-Hadamard transform of S_m . D (fp32, H symmetric and unnormalised) and splits it
+// into fp16 hi + lo (the same operands the compress kernel otherwise forms in every CTA).
+__global__ void __launch_bounds__(128) prepare_operands_kernel(const float* signs, const float* s,
+                                                               unsigned char* ops) {
+  const int t = threadIdx.x;
+  if ((int)blockIdx.x == (int)gridDim.x - 1) {
+    for (int c = t; c < D * 16; c += 128) {
+      const int i = c & 127, ch = c >> 7;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k0 = ch * 8 + 2 * e;
+        const float s0 = signs[k0], s1 = signs[k0 + 1];
+        const __half2 h = __floats2half2_rn((__popc(i & k0) & 1) ? -s0 : s0, (__popc(i & (k0 + 1)) & 1) ? -s1 : s1);
+        w[e] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(ops + canon(i, ch * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return;
+  }
+  __shared__ float v[D];
+  const int m = blockIdx.x;
+  v[t] = s[(size_t)m * D + t] * signs[t];
+  __syncthreads();
+#pragma unroll
+  for (int h = 1; h < D; h <<= 1) {
+    const float x = v[t], y = v[t ^ h];
+    __syncthreads();
+    v[t] = (t & h) ? y - x : x + y;
+    __syncthreads();
+  }
+  const float x = v[t];
+  const __half hi = __float2half_rn(x);
+  const __half lo = __float2half_rn(x - __half2float(hi));
+  *reinterpret_cast<__half*>(ops + kTileBytes + canon(m, t)) = hi;
+  *reinterpret_cast<__half*>(ops + 2 * kTileBytes + canon(m, t)) = lo;
+}
+
+// ---------------------------------------------------------------------------
 // host: tensor maps
 // ---------------------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -955,7 +1046,15 @@ bool compress_tc_supported(const CompressArgs& a) {
   if (!L.qjl && !(L.kbits >= 2 && L.kbits <= 4)) return false;
   if (!(L.vbits >= 2 && L.vbits <= 4)) return false;
   if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.v) & 15)) return false;
+  if (reinterpret_cast<uintptr_t>(a.operands) & 15) return false;
   return encode_fn() != nullptr;
+}
+
+size_t operand_bytes() { return 3 * (size_t)kTileBytes; }
+
+cudaError_t launch_prepare_operands(const float* signs, const float* s, int qjl, void* ops, cudaStream_t stream) {
+  prepare_operands_kernel<<<qjl ? QM + 1 : 1, 128, 0, stream>>>(signs, s, static_cast<unsigned char*>(ops));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {

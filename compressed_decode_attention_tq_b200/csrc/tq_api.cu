@@ -132,9 +132,32 @@ tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq
   a.k_boundaries = params->k_boundaries;
   a.v_centroids = params->v_centroids;
   a.v_boundaries = params->v_boundaries;
+  a.operands = cfg->rotation == TQ_ROT_HADAMARD ? params->operands : nullptr;
+  if (a.operands && (reinterpret_cast<uintptr_t>(a.operands) & 15))
+    return fail(TQ_ERR_INVALID_ARG, "params->operands must be 16-byte aligned");
   a.status = dev_status;
   cudaError_t e = tqk::launch_compress(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_compress_kv launch");
+  return TQ_OK;
+}
+
+size_t tq_operand_bytes(const tq_config* cfg) {
+  if (check_config(cfg) != TQ_OK || cfg->rotation != TQ_ROT_HADAMARD) return 0;
+  return tqk::operand_bytes();
+}
+
+tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, void* operands, tq_stream_t stream) {
+  clear_error();
+  tq_status st;
+  if ((st = check_config(cfg)) != TQ_OK) return st;
+  if (cfg->rotation != TQ_ROT_HADAMARD) return fail(TQ_ERR_UNSUPPORTED, "operands exist for TQ_ROT_HADAMARD only");
+  if (!params || !params->signs) return fail(TQ_ERR_INVALID_ARG, "params or params->signs is NULL");
+  if (cfg->key_qjl && !params->s) return fail(TQ_ERR_INVALID_ARG, "params->s is NULL");
+  if (!operands || (reinterpret_cast<uintptr_t>(operands) & 15))
+    return fail(TQ_ERR_INVALID_ARG, "operands must be a 16-byte aligned device pointer");
+  cudaError_t e = tqk::launch_prepare_operands(params->signs, params->s, cfg->key_qjl, operands,
+                                               reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_prepare_operands launch");
   return TQ_OK;
 }
 

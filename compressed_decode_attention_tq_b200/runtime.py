@@ -11,7 +11,7 @@ import torch
 
 from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, attend_decode, codebook, compress_kv,
                decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
-               page_bytes, status_str)
+               operand_bytes, page_bytes, prepare_operands, status_str)
 
 
 def _f32(x, device):
@@ -33,7 +33,7 @@ class PagedKV:
     def __init__(self, *, batch: int, kv_heads: int, num_pages: int, block_table, key_bits: int,
                  key_qjl: bool, value_bits: int, rotation: int = TQ_ROT_HADAMARD,
                  num_layers: int = 1, signs=None, pi=None, s=None, codebooks=None,
-                 device: str = "cuda"):
+                 device: str = "cuda", prepared_operands: bool = True):
         self.device = torch.device(device)
         self.cfg = make_config(key_bits=key_bits, key_qjl=key_qjl, value_bits=value_bits,
                                rotation=rotation)
@@ -57,7 +57,14 @@ class PagedKV:
             "vc": _f32(vc, self.device), "vb": _f32(vb, self.device),
         }
         t = self.tensors
-        self.params = make_params(t["signs"], t["pi"], t["s"], t["kc"], t["kb"], t["vc"], t["vb"])
+        # the compress kernel's tensor-core operands (H D, S D H), formed once for the cache
+        # instead of in every thread block of every call
+        t["ops"] = None
+        nops = operand_bytes(self.cfg)
+        if prepared_operands and nops and t["signs"] is not None and (not key_qjl or t["s"] is not None):
+            t["ops"] = torch.empty(nops, dtype=torch.uint8, device=self.device)
+            prepare_operands(self.cfg, make_params(t["signs"], s=t["s"]), t["ops"])
+        self.params = make_params(t["signs"], t["pi"], t["s"], t["kc"], t["kb"], t["vc"], t["vb"], t["ops"])
         self.cache = make_cache(self.pages, self.block_table, num_pages, self.max_pages, batch, kv_heads,
                                 num_layers)
         self._ws = {}

@@ -119,13 +119,20 @@ typedef struct tq_config {
 typedef struct tq_params {
   const float* signs;         /* [d] +-1 diagonal of D (TQ_ROT_HADAMARD), else unused     */
   const float* pi;            /* [d*d] Pi, row-major, y = Pi u (TQ_ROT_DENSE), else unused */
-  const float* s;             /* [m*d] S, row-major; every entry must be exactly
-                                 representable in fp16 (checked on the device,
-                                 TQ_ERR_INVALID_ARG); unused unless key_qjl            */
+  const float* s;             /* [m*d] S, row-major; unused unless key_qjl.  When
+                                 tq_compress_kv forms its operands itself (operands
+                                 NULL), every entry must be exactly representable in
+                                 fp16 (checked on the device, TQ_ERR_INVALID_ARG)      */
   const float* k_centroids;   /* [2^key_bits] sorted, symmetric (c_i = -c_{n-1-i})      */
   const float* k_boundaries;  /* [2^key_bits - 1] sorted, symmetric, middle one 0        */
   const float* v_centroids;   /* [2^value_bits]                                          */
   const float* v_boundaries;  /* [2^value_bits - 1]                                      */
+  const void* operands;       /* NULL, or device memory of tq_operand_bytes() bytes (16-byte
+                                 aligned) that tq_prepare_operands filled for these signs
+                                 and s: tq_compress_kv then copies its tensor-core operands
+                                 from it instead of forming them in every thread block.
+                                 Read only by tq_compress_kv, and only with
+                                 TQ_ROT_HADAMARD.                                      */
 } tq_params;
 
 /* A paged cache ([LIMITS] vLLM-style packed paged cache). */
@@ -186,6 +193,26 @@ TQ_API tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, c
                          int32_t layer, const void* k, const void* v, int32_t in_dtype,
                          int32_t max_len, const int32_t* seq_lens, int32_t* dev_status,
                          tq_stream_t stream);
+
+/* Bytes of the prepared tensor-core operands of tq_compress_kv for cfg (96 KiB for a
+ * TQ_ROT_HADAMARD configuration; 0 if cfg is invalid or uses TQ_ROT_DENSE). */
+TQ_API size_t tq_operand_bytes(const tq_config* cfg);
+
+/* Prepare the operands tq_compress_kv uses on the tensor cores for the rotation
+ * R = H D / sqrt(d) ([MOBILINT] "How JL Matrices Evolved") and, with key_qjl, the QJL
+ * sketch taken in the rotated domain ([MOBILINT] "QJL: Inner Product Recovery from a
+ * Single Sign Bit": S r = (S D H) (H D r) / d): three 128 x 128 fp16 tiles in the
+ * tensor cores' canonical K-major layout, B = H D (entries +-1, exact), then S D H
+ * (formed in fp32) as a high fp16 part and the fp16 rounding of the remainder.
+ *   params    signs (and s with key_qjl) as for tq_compress_kv; S need not be
+ *             fp16-exact on this path
+ *   operands  device, tq_operand_bytes(cfg) bytes, 16-byte aligned; written
+ *             asynchronously on stream; owned by the caller, who passes it in
+ *             tq_params.operands while signs and s stay unchanged
+ * Errors: TQ_ERR_UNSUPPORTED for TQ_ROT_DENSE, TQ_ERR_INVALID_ARG for NULL or
+ * misaligned pointers. */
+TQ_API tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, void* operands,
+                                     tq_stream_t stream);
 
 /* Workspace bytes tq_attend_decode and tq_decode_scores need for these sizes. */
 TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int32_t q_heads,

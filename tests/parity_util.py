@@ -50,7 +50,7 @@ class Run:
     V: dict = None
 
 
-def setup(w: wl.Workload, layers=(0,)):
+def setup(w: wl.Workload, layers=(0,), prepared_operands=True):
     """Builds the library cache for w and compresses `layers` on the GPU (inputs from workloads)."""
     from compressed_decode_attention_tq_b200.runtime import PagedKV
     lens = wl.seq_lens(w)
@@ -65,7 +65,7 @@ def setup(w: wl.Workload, layers=(0,)):
     run.kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
                      key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits,
                      rotation=w.rotation, num_layers=max(layers) + 1, signs=rin["signs"],
-                     pi=rin["pi"], s=rin["s"])
+                     pi=rin["pi"], s=rin["s"], prepared_operands=prepared_operands)
     run.K, run.V = {}, {}
     dt = torch.float16 if w.in_dtype == "f16" else torch.float32
     seq = torch.as_tensor(lens, dtype=torch.int32, device="cuda")

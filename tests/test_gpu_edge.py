@@ -74,15 +74,18 @@ def test_norm_overflow_reported():
 
 
 def test_non_fp16_sketch_matrix_rejected():
+    # compress forming S D H in every thread block takes S as an fp16 MMA operand, so S must
+    # be fp16-exact there; prepared operands are formed in fp32 and accept any S
     from compressed_decode_attention_tq_b200.runtime import PagedKV
     rin = wl.rotation_inputs(wl.config2())
     s = rin["s"].copy()
     s[3, 5] = 0.1  # not representable in fp16
-    kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[0]]), key_bits=3, key_qjl=True,
-                 value_bits=3, signs=rin["signs"], s=s)
     k = torch.randn((1, 1, 4, 128), device="cuda").half()
-    kv.compress(0, k, k, torch.tensor([4], dtype=torch.int32, device="cuda"))
-    assert kv.check() == 1
+    for prepared, expect in ((False, 1), (True, 0)):
+        kv = PagedKV(batch=1, kv_heads=1, num_pages=1, block_table=np.array([[0]]), key_bits=3, key_qjl=True,
+                     value_bits=3, signs=rin["signs"], s=s, prepared_operands=prepared)
+        kv.compress(0, k, k, torch.tensor([4], dtype=torch.int32, device="cuda"))
+        assert kv.check() == expect
 
 
 def test_zero_vector_compresses_to_zero_norm():

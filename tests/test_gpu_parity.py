@@ -27,11 +27,21 @@ SMALL = {
 }
 
 
-@pytest.fixture(scope="module", params=sorted(SMALL))
+# the same kernels with the tensor-core operands (H D, S D H) formed inside every thread
+# block instead of prepared once per cache
+IN_BLOCK = {
+    "c2_in_block_operands": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4,
+                                               name="c2_in_block_operands"),
+    "c4_in_block_operands": lambda: wl.config4(batch=2, kv_heads=2, q_heads=8, max_len=2000, n_splits=8,
+                                               name="c4_in_block_operands"),
+}
+
+
+@pytest.fixture(scope="module", params=sorted(SMALL) + sorted(IN_BLOCK))
 def run(request):
-    w = SMALL[request.param]()
+    w = (SMALL.get(request.param) or IN_BLOCK[request.param])()
     layers = tuple(range(w.num_layers))
-    r = setup(w, layers)
+    r = setup(w, layers, prepared_operands=request.param not in IN_BLOCK)
     r.kv.raise_on_error("compress")
     r.pages = r.kv.pages_numpy()
     return r
