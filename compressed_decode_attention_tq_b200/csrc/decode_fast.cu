@@ -670,34 +670,44 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   if (!sm.last) return;
   const int ns = a.n_splits;
   if (tid < 32 * R) {
-    // thread (row r, float4 c4) of the output: online log-sum-exp over the splits'
-    // (m, l, acc), sixteen splits' loads in flight at a time
+    // thread (row r, float4 c4) of the output: the row's maximum over the splits, then every
+    // split's weight exp(m - M) is independent of the others; the partials are loaded in
+    // batches of kMB (registers), the first batch before the maximum is formed, so that about
+    // two round trips to L2 cover 37 splits
+    constexpr int kMB = 20;
     const int r = tid >> 5, c4 = tid & 31;
     const size_t rowq = row0 + r;
     const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * ns * 2);
     const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    // every partial this thread needs, requested into L1 at once (no registers held)
-    for (int sp = 0; sp < ns; ++sp) {
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(pa4 + (size_t)sp * (D / 4)));
-      if (c4 == 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(ml2 + sp));
-    }
-#pragma unroll 16
-    for (int sp = 0; sp < ns; ++sp) {
-      const float2 m2 = ml2[sp];
-      const float4 v = pa4[(size_t)sp * (D / 4)];
-      // branch-free update (the loads of later splits do not wait on it)
-      const float Mn = fmaxf(M, m2.x);
-      const bool live = Mn != -CUDART_INF_F;
-      const float f = live ? __expf(M - Mn) : 1.f;
-      const float wgt = live ? __expf(m2.x - Mn) : 0.f;
-      l = fmaf(wgt, m2.y, l * f);
-      o.x = fmaf(wgt, v.x, o.x * f);
-      o.y = fmaf(wgt, v.y, o.y * f);
-      o.z = fmaf(wgt, v.z, o.z * f);
-      o.w = fmaf(wgt, v.w, o.w * f);
-      M = Mn;
+    for (int s0 = 0; s0 < ns; s0 += kMB) {
+      float4 v[kMB];
+      float2 m2[kMB];
+#pragma unroll
+      for (int k = 0; k < kMB; ++k) {
+        if (s0 + k < ns) {
+          v[k] = pa4[(size_t)(s0 + k) * (D / 4)];
+          m2[k] = ml2[s0 + k];
+        }
+      }
+      if (s0 == 0) {
+        for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
+#pragma unroll
+        for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
+      }
+      const bool live = M != -CUDART_INF_F;
+#pragma unroll
+      for (int k = 0; k < kMB; ++k) {
+        if (s0 + k < ns) {
+          const float wgt = live ? __expf(m2[k].x - M) : 0.f;
+          l = fmaf(wgt, m2[k].y, l);
+          o.x = fmaf(wgt, v[k].x, o.x);
+          o.y = fmaf(wgt, v[k].y, o.y);
+          o.z = fmaf(wgt, v[k].z, o.z);
+          o.w = fmaf(wgt, v[k].w, o.w);
+        }
+      }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
     // out = D H (o / l) / sqrt(d): H over coordinates 4 c4 + e, spans 1 and 2 in the
