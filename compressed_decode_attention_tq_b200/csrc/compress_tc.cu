@@ -827,17 +827,29 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // chunk is released to the sketch MMAs while the next chunk's load is in flight ----
       const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
       const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float z[32];
-        tmem_ld32(colV + 32 * c, z);
-        tmem_wait_ld();
+      // Value chunks are quantised from one register buffer while the next chunk's load into
+      // the other is in flight (two chunks per iteration, the buffers alternating).
+      auto quant_v = [&](const float (&z)[32], int c) {
         constexpr uint32_t vw0 = FV::init(0, 0), vw1 = FV::init(1, 0), vw2 = FV::init(2, 0), vw3 = FV::init(3, 0);
         uint32_t vw[4] = {vw0, vw1, vw2, vw3}, dh[16], dl[16];
         f2_t drr = 0;
         quantise32<HV - 1, FV, false>(z, qv, sm.kmag, vw, dh, dl, drr);
         if (cur.blk && !failed)
           store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
+      };
+      {
+        float za[32], zb[32];
+        tmem_ld32(colV, za);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          tmem_ld32(colV + 32 * (c + 1), zb);
+          quant_v(za, c);
+          tmem_wait_ld();
+          if (c + 2 < 4) tmem_ld32(colV + 32 * (c + 2), za);
+          quant_v(zb, c + 1);
+          if (c + 2 < 4) tmem_wait_ld();
+        }
       }
       f2_t rr2 = 0;
       // key words of the four chunks (completed by the signs)
