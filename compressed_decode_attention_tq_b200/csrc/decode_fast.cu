@@ -94,6 +94,30 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t pari
   return false;
 }
 
+// The same wait for a thread that can afford to react late (the copy producer, three stages
+// ahead): between polls it sleeps, so that it takes few issue slots from the consumer warps
+// of its SM sub-partition; gives up after about 1 s.
+__device__ __forceinline__ bool mbar_wait_sleepy(unsigned long long* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  unsigned long long t0 = 0;
+  for (long long it = 0; it < kWaitLimit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (it == 0) t0 = t;
+    else if (t - t0 > 1000000000ull) break;
+    __nanosleep(128);
+  }
+  return false;
+}
+
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -222,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     if (lane == 0) {
       for (int i = 0; i < nunits; ++i) {
         const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&sm.empty[s], ((i / kStages) - 1) & 1)) {
+        if (i >= kStages && !mbar_wait_sleepy(&sm.empty[s], ((i / kStages) - 1) & 1)) {
           report(a.status, TQ_ERR_TIMEOUT);
           break;
         }
