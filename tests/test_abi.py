@@ -117,3 +117,28 @@ def test_host_argument_errors_do_not_launch(tq):
     bad = tq.make_config(head_dim=96)
     st = tq.lib.tq_decompress(by(bad), by(params), by(cache), 0, None, 0, None, None, None, None)
     assert st == tq.TQ_ERR_UNSUPPORTED
+
+
+def test_operand_bytes_and_prepare_validation(tq):
+    # host-side checks of the operand preparation entry points (no device work)
+    import ctypes
+    ops = 3 * 128 * 128 * 2
+    cfg = tq.make_config()
+    assert tq.lib.tq_operand_bytes(ctypes.byref(cfg)) == ops
+    dense = tq.make_config(rotation=tq.TQ_ROT_DENSE)
+    assert tq.lib.tq_operand_bytes(ctypes.byref(dense)) == 0
+    bad = tq.make_config(head_dim=64)
+    assert tq.lib.tq_operand_bytes(ctypes.byref(bad)) == 0
+    params = tq.tq_params()
+    buf = ctypes.create_string_buffer(ops + 16)
+    aligned = (ctypes.addressof(buf) + 15) & ~15
+    st = tq.lib.tq_prepare_operands(ctypes.byref(dense), ctypes.byref(params), aligned, None)
+    assert st == tq.TQ_ERR_UNSUPPORTED
+    st = tq.lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), aligned, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "signs" in tq.last_error()
+    params.signs = aligned  # any non-null pointer: the call is rejected before it is read
+    st = tq.lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), aligned, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "params->s" in tq.last_error()
+    params.s = aligned
+    st = tq.lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), aligned + 4, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "aligned" in tq.last_error()
