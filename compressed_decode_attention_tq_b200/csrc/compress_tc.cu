@@ -135,6 +135,27 @@ __device__ __forceinline__ bool bar_wait(unsigned long long* b, uint32_t parity)
   return false;
 }
 
+// The same wait for a thread that can afford to react late (the copy thread, a tile ahead):
+// plain polls with a sleep between them, so that it takes few issue slots from the compute
+// warps of its SM sub-partition; false after kWaitNs.
+__device__ __forceinline__ bool bar_wait_sleepy(unsigned long long* b, uint32_t parity) {
+  const uint32_t addr = s_u32(b);
+  const unsigned long long t0 = global_ns();
+  for (int it = 0; it < (1 << 24); ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (global_ns() - t0 > kWaitNs) break;
+    __nanosleep(256);
+  }
+  return false;
+}
+
 __device__ __forceinline__ void bar_arrive(unsigned long long* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s_u32(b)) : "memory");
 }
@@ -718,7 +739,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       for (int i = 0; ok && i + 2 < my_tiles; ++i) {
         // phase i >> 1 of stage_free[i & 1]: the forward MMAs of tile i are done with it
-        if (!(ok = bar_wait(&sm.stage_free[i & 1], (i >> 1) & 1))) break;
+        if (!(ok = bar_wait_sleepy(&sm.stage_free[i & 1], (i >> 1) & 1))) break;
         issue_load(i + 2);
         issued = i + 3;
       }
