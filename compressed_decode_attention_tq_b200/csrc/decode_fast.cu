@@ -49,11 +49,21 @@ constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
 enum KPol { K3Q = 0, K2Q = 1 };
 enum VPol { V3 = 0, V2 = 1 };
 
+// the merging CTA copies the partials of up to kMergeSplits splits into shared memory at once
+constexpr int kMergeSplits = 40;
 struct SmemFast {
-  unsigned char stage[kStages][kStageBytes];
+  union {
+    struct {
+      unsigned char stage[kStages][kStageBytes];
+      float wacc[kConsumerWarps][4][D];
+    } ring;
+    // at the end: the partial accumulators of every split of the (sequence, kv head) being
+    // merged (the ring and the warp partials are no longer used then)
+    float merge[4][kMergeSplits][D];
+  };
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
-  float wacc[kConsumerWarps][4][D];
+  unsigned long long mbar;  // the merge copies landed
   float wm[kConsumerWarps][4], wl[kConsumerWarps][4], wf[kConsumerWarps][4];
   int last;
 };
@@ -237,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
+    mbar_init(&sm.mbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -257,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
           phys = 0;
         }
         const unsigned char* blk = a.cache.block(phys, gh);
-        unsigned char* st = sm.stage[s];
+        unsigned char* st = sm.ring.stage[s];
         const uint32_t hb2 = half * kUnit * 2, hb16 = half * kUnit * 16;
         mbar_expect_tx(&sm.full[s], unit_bytes);
         bulk_g2s(st, blk + L.kn + hb2, kUnit * 2, &sm.full[s]);
@@ -464,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         if (lane == 0) report(a.status, TQ_ERR_TIMEOUT);
         break;
       }
-      const unsigned char* st = sm.stage[s];
+      const unsigned char* st = sm.ring.stage[s];
       const unsigned char* kc = st + kNormBytes;
       const unsigned char* vc = kc + kMaxKChunks * kChunkStride;
       const int tok0 = (u_begin + i) * kUnit;
@@ -647,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         const int row = 2 * t4 + (e & 1);
         const int cb = 2 * mt + (e >> 1);
         const int coord = 32 * (g >> 1) + pair_base(cb) + 4 * (g & 1);
-        if (row < R) sm.wacc[warp][row][coord] = acc[mt][e];
+        if (row < R) sm.ring.wacc[warp][row][coord] = acc[mt][e];
       }
     }
   }
@@ -675,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     const int r = idx / D, j = idx % D;
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm.wf[w][r], sm.wacc[w][r][j], o);
+    for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm.wf[w][r], sm.ring.wacc[w][r][j], o);
     a.part_acc[((row0 + r) * a.n_splits + split) * D + j] = o;
   }
   // ---- the last split of this (sequence, kv head) to finish merges all of them ----
@@ -694,42 +705,70 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   if (!sm.last) return;
   const int ns = a.n_splits;
   if (tid < 32 * R) {
-    // thread (row r, float4 c4) of the output: the row's maximum over the splits, then every
-    // split's weight exp(m - M) is independent of the others; the partials are loaded in
-    // batches of kMB (registers), the first batch before the maximum is formed, so that about
-    // two round trips to L2 cover 37 splits
-    constexpr int kMB = 20;
     const int r = tid >> 5, c4 = tid & 31;
     const size_t rowq = row0 + r;
     const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * ns * 2);
-    const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < ns; s0 += kMB) {
-      float4 v[kMB];
-      float2 m2[kMB];
-#pragma unroll
-      for (int k = 0; k < kMB; ++k) {
-        if (s0 + k < ns) {
-          v[k] = pa4[(size_t)(s0 + k) * (D / 4)];
-          m2[k] = ml2[s0 + k];
-        }
+    if (ns <= kMergeSplits) {
+      // every split's accumulators of every row in one round trip: a bulk copy per row (the
+      // rows' partials are contiguous), while the maxima are formed from the (m, l) pairs
+      if (tid == 0) {
+        // the other splits' partials were made visible to this thread by the acquire above;
+        // order them before this thread's async-proxy reads
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        mbar_expect_tx(&sm.mbar, (uint32_t)(R * ns * D * sizeof(float)));
+        for (int rr = 0; rr < R; ++rr)
+          bulk_g2s(&sm.merge[rr][0][0], a.part_acc + (row0 + rr) * ns * D, (uint32_t)(ns * D * sizeof(float)), &sm.mbar);
       }
-      if (s0 == 0) {
-        for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
+      for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
 #pragma unroll
-        for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
-      }
+      for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
       const bool live = M != -CUDART_INF_F;
+      if (!mbar_wait(&sm.mbar, 0)) report(a.status, TQ_ERR_TIMEOUT);
+      const float4* pa4 = reinterpret_cast<const float4*>(&sm.merge[r][0][0]) + c4;
+#pragma unroll 8
+      for (int sp = 0; sp < ns; ++sp) {
+        const float2 m2 = ml2[sp];
+        const float4 v = pa4[sp * (D / 4)];
+        const float wgt = live ? __expf(m2.x - M) : 0.f;
+        l = fmaf(wgt, m2.y, l);
+        o.x = fmaf(wgt, v.x, o.x);
+        o.y = fmaf(wgt, v.y, o.y);
+        o.z = fmaf(wgt, v.z, o.z);
+        o.w = fmaf(wgt, v.w, o.w);
+      }
+    } else {
+      // many splits: thread (row r, float4 c4) loads the partials in register batches of kMB,
+      // the first batch before the maximum is formed (about ns / kMB round trips to L2)
+      constexpr int kMB = 20;
+      const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
+      for (int s0 = 0; s0 < ns; s0 += kMB) {
+        float4 v[kMB];
+        float2 m2[kMB];
 #pragma unroll
-      for (int k = 0; k < kMB; ++k) {
-        if (s0 + k < ns) {
-          const float wgt = live ? __expf(m2[k].x - M) : 0.f;
-          l = fmaf(wgt, m2[k].y, l);
-          o.x = fmaf(wgt, v[k].x, o.x);
-          o.y = fmaf(wgt, v[k].y, o.y);
-          o.z = fmaf(wgt, v[k].z, o.z);
-          o.w = fmaf(wgt, v[k].w, o.w);
+        for (int k = 0; k < kMB; ++k) {
+          if (s0 + k < ns) {
+            v[k] = pa4[(size_t)(s0 + k) * (D / 4)];
+            m2[k] = ml2[s0 + k];
+          }
+        }
+        if (s0 == 0) {
+          for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
+#pragma unroll
+          for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
+        }
+        const bool live = M != -CUDART_INF_F;
+#pragma unroll
+        for (int k = 0; k < kMB; ++k) {
+          if (s0 + k < ns) {
+            const float wgt = live ? __expf(m2[k].x - M) : 0.f;
+            l = fmaf(wgt, m2[k].y, l);
+            o.x = fmaf(wgt, v[k].x, o.x);
+            o.y = fmaf(wgt, v[k].y, o.y);
+            o.z = fmaf(wgt, v[k].z, o.z);
+            o.w = fmaf(wgt, v[k].w, o.w);
+          }
         }
       }
     }
