@@ -233,6 +233,23 @@ def config_dict(w, layers):
 # our arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own and receives the maximum
+    (one process per GPU; with one rank the time itself)."""
+    if world == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units all ranks processed in one step (each rank the same
+    amount: weak scaling) per second of the slowest rank's step."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -295,16 +312,12 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
     kv.raise_on_error("timed steps")
     ms_step = ms / args.steps
     comp_ms = sum(e[0].elapsed_time(e[1]) for e in phase_ev) / args.steps
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in phase_ev) / args.steps
-    value = world * units / (ms_step / 1e3)
+    value = job_value(units, world, ms_step)
 
     hbm, peak_kind = peaks()
     comp_bytes_launch = tok_heads_layer * (2 * 128 * 2 + kv.block_bytes / 256)
@@ -391,13 +404,9 @@ def run_e2e(args, kv, w, L, Ks, Vs, Qs, Outs, seq, stream, dev, units, world):
         step()
     e.record(stream)
     torch.cuda.synchronize(dev)
-    ms = s.elapsed_time(e)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e), world, dev)
     kv.raise_on_error("e2e")
-    return {"value": world * units / (ms / args.e2e_steps / 1e3), "unit": UNIT,
+    return {"value": job_value(units, world, ms / args.e2e_steps), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
 
