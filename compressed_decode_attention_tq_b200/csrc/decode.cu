@@ -35,15 +35,6 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 //   qrot = R q (fp32), q8 = int8 rounding of qrot * 127 / max|qrot| (with its scale),
 //   sq = S q (fp32), sq_int = S q in 16-bit fixed point with a power-of-two scale, sum.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float block_max128(float v, float* red) {
-  v = warp_max(v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  const float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  return m;
-}
-
 __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_rows) {
   // Launched as a programmatic dependent of whatever precedes it on the stream: everything
   // before it has finished once this wait returns.  Then the split kernel may start (its
@@ -325,16 +316,17 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     }
     __syncthreads();
   }
-  if (kScoresOnly) return;
-  // ---- partials
+  // ---- partials (the score-only variant stops with the scores)
+  if constexpr (!kScoresOnly) {
 #pragma unroll
-  for (int r = 0; r < kRowsMax; ++r) {
-    if (r < R) {
-      const size_t pr = (row0 + r) * a.n_splits + split;
-      a.part_acc[pr * D + tid] = acc[r];
-      if (tid == 0) {
-        a.part_ml[pr * 2] = sm.m[r];
-        a.part_ml[pr * 2 + 1] = sm.l[r];
+    for (int r = 0; r < kRowsMax; ++r) {
+      if (r < R) {
+        const size_t pr = (row0 + r) * a.n_splits + split;
+        a.part_acc[pr * D + tid] = acc[r];
+        if (tid == 0) {
+          a.part_ml[pr * 2] = sm.m[r];
+          a.part_ml[pr * 2 + 1] = sm.l[r];
+        }
       }
     }
   }
