@@ -10,14 +10,17 @@
 //    +-1 entries (exact), fp32 accumulation in tensor memory.  y = y' / ||y'||.
 //  * QJL sketch in the rotated domain: with R = H D / sqrt(d) orthogonal,
 //      S r = S R^T R r = (S D H) r_rot' / d,   r_rot' = y' - sqrt(d) fp16(||x||) c[idx],
-//    so sign(S r) = sign((S D H) a r_rot') for any a > 0.  S D H is formed once per CTA
-//    and held as an fp16 hi + lo pair; a r_rot' (scaled to O(1)) is split hi + lo as
-//    well; three MMAs (hi.hi, hi.lo, lo.hi) give the projections to ~2^-22 relative.
+//    so sign(S r) = sign((S D H) a r_rot') for any a > 0.  S D H is held as an fp16 hi + lo
+//    pair, prepared once per cache (prepare_operands_kernel, passed in as operands) or
+//    formed by one MMA in every CTA; a r_rot' (scaled to O(1)) is split hi + lo as well;
+//    three MMAs (hi.hi, hi.lo, lo.hi) give the projections to ~2^-22 relative.  They are
+//    issued chunk by chunk as the keys' residual is written.
 //
 // Quantisation works on y' directly: |y| > beta  <=>  |y'| > beta ||y'||, so each token
-// scales its boundaries once instead of normalising every coordinate; the rank is a sum
-// of saturated unit steps (the boundaries are sorted), and the residual's centroid is read
-// from a table by the code field just formed.
+// scales its boundaries once instead of normalising every coordinate; the rank is formed
+// from saturated unit steps (a binary search for three positive boundaries), sign bits are
+// placed in the packed words by sign-replicating byte permutes, and the residual's centroid
+// is read from a table at the offset the rank's code bits hold.
 //
 // One persistent CTA per SM: two compute groups of four warps and a producer warpgroup.
 // Group g takes the CTA's tiles g, g + 2, ... (ping-pong), so that one group's waits for
