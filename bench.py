@@ -70,12 +70,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and whitespace: what the compiler sees of it (string
+    literals in these sources hold no comment markers)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def kernel_hash(kernel: str) -> str:
     h = hashlib.sha256()
     src = os.path.join(ROOT, "compressed_decode_attention_tq_b200", "csrc")
     for name in KERNEL_SOURCES.get(kernel, tuple(sorted(os.listdir(src)))):
-        with open(os.path.join(src, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(src, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
