@@ -255,12 +255,14 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
     if (lane == 0) {
+      int issued = 0;
       for (int i = 0; i < nunits; ++i) {
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait_sleepy(&sm.empty[s], ((i / kStages) - 1) & 1)) {
           report(a.status, TQ_ERR_TIMEOUT);
           break;
         }
+        issued = i + 1;
         const int u = u_begin + i, half = u % kUnitsPerPage;
         int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + u / kUnitsPerPage];
         if (phys < 0 || phys >= a.cache.num_pages) {
@@ -283,6 +285,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         for (int c = 0; c < kVChunks; ++c)
           bulk_g2s(vc + c * kChunkStride, blk + L.vc + c * PT * 16 + hb16, kUnit * 16, &sm.full[s]);
       }
+      // the last copy into each stage has landed (consumers that gave up early did not wait
+      // for it) before the ring's space is reused or released; bounded
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait(&sm.full[i % kStages], (i / kStages) & 1);
     }
   } else {
     // ---------------- consumers ----------------
@@ -725,7 +731,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
       for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
       const bool live = M != -CUDART_INF_F;
-      if (!mbar_wait(&sm.mbar, 0)) report(a.status, TQ_ERR_TIMEOUT);
+      if (!mbar_wait(&sm.mbar, 0)) {
+        report(a.status, TQ_ERR_TIMEOUT);
+        mbar_wait(&sm.mbar, 0);  // the copies in flight land before the CTA ends (bounded)
+      }
       const float4* pa4 = reinterpret_cast<const float4*>(&sm.merge[r][0][0]) + c4;
 #pragma unroll 8
       for (int sp = 0; sp < ns; ++sp) {
