@@ -47,8 +47,9 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   const int row = blockIdx.x;
   if (row >= total_rows) return;
-  // the merge counters of the fused split kernel start every call at zero
-  if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads) a.counter[row] = 0u;
+  // the merge counters of the fused split kernel (one per sequence, kv head and run of up to
+  // four query rows) start every call at zero
+  if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads * ((a.rows + 3) / 4)) a.counter[row] = 0u;
   // the rows of S this warp needs, requested before the query (they do not depend on it)
   float4 p[32];
   if (a.qjl) {
@@ -395,8 +396,8 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   w.sq_sum = off; off = align256(off + rows * sizeof(int));
   w.q8 = off; off = align256(off + rows * D);
   w.q8_scale = off; off = align256(off + rows * sizeof(float));
-  // one counter per (sequence, kv head); kv_heads divides q_heads, so batch * q_heads bounds it
-  w.counter = off; off = align256(off + (size_t)batch * q_heads * sizeof(unsigned int));
+  // one counter per (sequence, kv head, run of up to four query rows): at most one per query row
+  w.counter = off; off = align256(off + rows * sizeof(unsigned int));
   w.total = off;
   return w;
 }

@@ -221,10 +221,13 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SmemFast& sm = *reinterpret_cast<SmemFast*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x, gh = blockIdx.y, b = blockIdx.z;
+  // The query rows of one (sequence, kv head) (its G heads times seq_q positions, consecutive)
+  // are taken in runs of up to four, one run per CTA along the grid's z with the sequence.
+  const int nchunk = (a.rows + 3) / 4;
+  const int split = blockIdx.x, gh = blockIdx.y, b = blockIdx.z / nchunk, chunk = blockIdx.z % nchunk;
   const Layout& L = a.cache.L;
-  const int R = a.rows;
-  const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q;
+  const int R = min(4, a.rows - 4 * chunk);
+  const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q + 4 * chunk;
 
   const int len = a.seq_lens[b];
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
@@ -703,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     unsigned int done;
     asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;"
                  : "=r"(done)
-                 : "l"(&a.counter[(size_t)b * a.cache.kv_heads + gh])
+                 : "l"(&a.counter[((size_t)b * a.cache.kv_heads + gh) * nchunk + chunk])
                  : "memory");
     sm.last = done == (unsigned int)a.n_splits - 1;
   }
@@ -809,7 +812,6 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 
 bool fast_decode_supported(const DecodeArgs& a) {
   const Layout& L = a.cache.L;
-  if (a.rows > 4) return false;
   const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl);
   const bool vok = L.vbits == 3 || L.vbits == 2;
   return kok && vok;
@@ -820,7 +822,7 @@ size_t fast_decode_smem_bytes() { return sizeof(SmemFast); }
 cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
   const Layout& L = a.cache.L;
   const size_t smem = sizeof(SmemFast);
-  dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch);
+  dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch * ((a.rows + 3) / 4));
   void (*k)(DecodeArgs) = nullptr;
   if (L.kbits == 3 && L.vbits == 3) k = fast_split_kernel<K3Q, V3>;
   if (L.kbits == 3 && L.vbits == 2) k = fast_split_kernel<K3Q, V2>;

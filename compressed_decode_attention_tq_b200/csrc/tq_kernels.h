@@ -34,7 +34,8 @@ struct DecodeArgs {
   int* sq_sum;      // [B*Hq*seq_q] workspace: sum_i sq_int
   int8_t* q8;       // [B*Hq*seq_q][D] workspace: R q in int8 (scaled by q8_scale)
   float* q8_scale;  // [B*Hq*seq_q] workspace
-  unsigned int* counter;  // [B*Hkv] workspace (sized B*Hq): finished splits per (sequence, kv head)
+  unsigned int* counter;  // workspace (sized B*Hq*seq_q): finished splits per (sequence, kv head,
+                          // run of up to four query rows)
   float* out;       // [B*Hq*seq_q][D]
   float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
   int max_len;
