@@ -32,7 +32,7 @@ TQ_F32 = 1
 EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_validate_config", "tq_page_bytes",
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
            "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc", "tq_operand_bytes",
-           "tq_prepare_operands")
+           "tq_prepare_operands", "tq_append_kv", "tq_append_attend_decode")
 
 
 class tq_config(ctypes.Structure):
@@ -83,6 +83,9 @@ def _load() -> ctypes.CDLL:
         "tq_attend_decode_noalloc": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, P, P]),
         "tq_operand_bytes": (SZ, [cfgp]),
         "tq_prepare_operands": (I32, [cfgp, parp, P, P]),
+        "tq_append_kv": (I32, [cfgp, parp, cachep, I32, P, P, I32, I32, P, P, P]),
+        "tq_append_attend_decode": (I32, [cfgp, parp, cachep, I32, P, P, I32, I32, P, I32, I32, I32, P, I32,
+                                          P, SZ, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -200,6 +203,29 @@ def attend_decode_noalloc(cfg, params, cache, layer, q, seq_lens, n_splits, out,
                                         layer, _ptr(q), dtype_code(q), q.shape[1], q.shape[2],
                                         _ptr(seq_lens), n_splits, _ptr(out), _ptr(status),
                                         _stream(stream)), "tq_attend_decode_noalloc")
+
+
+def append_kv(cfg, params, cache, layer, k_new, v_new, seq_lens, status, stream=None):
+    """k_new, v_new: device [batch][kv_heads][n_new][d]; seq_lens: device int32 [batch], the
+    lengths after the append (new token n goes to position seq_lens[b] - n_new + n)."""
+    if v_new.shape != k_new.shape or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    _check(lib.tq_append_kv(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
+                            _ptr(k_new), _ptr(v_new), dtype_code(k_new), k_new.shape[2], _ptr(seq_lens),
+                            _ptr(status), _stream(stream)), "tq_append_kv")
+
+
+def append_attend_decode(cfg, params, cache, layer, k_new, v_new, q, seq_lens, n_splits, workspace,
+                         out, status, stream=None):
+    """append_kv then attend_decode in one call; seq_lens are the lengths after the append."""
+    if v_new.shape != k_new.shape or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    _check(lib.tq_append_attend_decode(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
+                                       _ptr(k_new), _ptr(v_new), dtype_code(k_new), k_new.shape[2],
+                                       _ptr(q), dtype_code(q), q.shape[1], q.shape[2], _ptr(seq_lens),
+                                       n_splits, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(out),
+                                       _ptr(status), _stream(stream)), "tq_append_attend_decode")
 
 
 def decode_scores(cfg, params, cache, layer, q, seq_lens, workspace, scores, status, stream=None):

@@ -31,6 +31,223 @@ constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------------------------
+// append: one CTA of 128 threads per new token of one (sequence, kv head); thread i owns
+// coordinate i, warp w the coordinates 32w..32w+31.  The same encoding as the compress
+// kernels ("TurboQuant explained", section "Two-Stage Approach: MSE Approximation + QJL
+// Correction"; "tq-kv" crate documentation, incremental cache: a new token is compressed
+// and appended to its page without touching the tokens already stored).
+// ---------------------------------------------------------------------------
+constexpr int kMergedNibble = 0;  // pack_code's `bits` for a merged key nibble, passed whole in r
+
+struct __align__(16) AppendShared {
+  float xs[D];          // the vector being transformed
+  float tab[4][16];     // k centroids, k boundaries, v centroids, v boundaries
+  float red[4];
+  uint32_t kw[16], ksw[4], vw[16];
+};
+
+__device__ __forceinline__ float block_sum128(float v, float* red, int lane, int warp) {
+  v = warp_sum(v);
+  __syncthreads();  // red may still be read by an earlier sum
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  return (red[0] + red[1]) + (red[2] + red[3]);
+}
+
+// y = R x / n for thread i's coordinate (x_i in x): H D through the warp-level transform
+// in warp 0, or a row of Pi.
+__device__ __forceinline__ float rotate_coord(const DecodeArgs& a, AppendShared& sh, float x, float inv,
+                                              int i, int lane, int warp) {
+  float y;
+  if (!a.dense) {
+    sh.xs[i] = x * a.signs[i];
+    __syncthreads();
+    if (warp == 0) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = sh.xs[lane + 32 * e];
+      fwht128_warp(v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sh.xs[lane + 32 * e] = v[e];
+    }
+    __syncthreads();
+    y = sh.xs[i] * (inv * kInvSqrtD);
+  } else {
+    sh.xs[i] = x * inv;
+    __syncthreads();
+    const float4* prow = reinterpret_cast<const float4*>(a.pi + (size_t)i * D);
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D / 4; ++k) {
+      const float4 p = prow[k];
+      acc = fmaf(p.x, sh.xs[4 * k], acc);
+      acc = fmaf(p.y, sh.xs[4 * k + 1], acc);
+      acc = fmaf(p.z, sh.xs[4 * k + 2], acc);
+      acc = fmaf(p.w, sh.xs[4 * k + 3], acc);
+    }
+    y = acc;
+  }
+  __syncthreads();  // xs is free again
+  return y;
+}
+
+// Code words of one token for `bits` from this thread's (s, r); warp w writes the words
+// that hold coordinates 32w..32w+31 (the stored layout of the cache format).
+__device__ __forceinline__ void pack_code(int s, int r, int bits, int lane, int warp, uint32_t* w) {
+  const int e = warp;
+  if (bits == 1) {
+    const uint32_t b = __ballot_sync(FULL, s);
+    if (lane == 0) w[e] = b;
+  } else if (bits == 2 || bits == 3) {
+    const uint32_t f = bits == 2 ? (uint32_t)(r | (s << 1)) : (uint32_t)r;
+    const uint32_t sh = f << (2 * (lane & 15));
+    const uint32_t lo = __reduce_or_sync(FULL, lane < 16 ? sh : 0u);
+    const uint32_t hi = __reduce_or_sync(FULL, lane < 16 ? 0u : sh);
+    const uint32_t sp = bits == 3 ? __reduce_or_sync(FULL, (uint32_t)s << (sign_plane_pos(lane) & 31)) : 0u;
+    if (lane == 0) {
+      w[2 * e] = lo;
+      w[2 * e + 1] = hi;
+      if (bits == 3) w[8 + e] = sp;
+    }
+  } else {
+    // 4-bit fields (r in bits 0..2, s in bit 3), or a merged key nibble (r0, r1, s, sigma)
+    const uint32_t f = bits == kMergedNibble ? (uint32_t)r : (uint32_t)(r | (s << 3));
+    const uint32_t sh = f << (4 * (lane & 7));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t v = __reduce_or_sync(FULL, (lane >> 3) == q ? sh : 0u);
+      if (lane == 0) w[4 * e + q] = v;
+    }
+  }
+}
+
+// Encodes thread i's coordinate of one vector: stored norm, index, (s, r); returns y.
+__device__ __forceinline__ float encode_coord(const DecodeArgs& a, AppendShared& sh, float x, const float* bnd,
+                                              int bits, int i, int lane, int warp, __half& nh, int& idx,
+                                              int& s, int& r) {
+  const float n = sqrtf(block_sum128(x * x, sh.red, lane, warp));
+  nh = __float2half_rn(n);
+  if (__hisinf(nh) && i == 0) report(a.status, TQ_ERR_OVERFLOW);
+  const float y = rotate_coord(a, sh, x, n > 0.f ? 1.0f / n : 0.0f, i, lane, warp);
+  const int nb = (1 << bits) - 1, h = 1 << (bits - 1);
+  idx = 0;
+  for (int k = 0; k < nb; ++k) idx += (y > bnd[k]) ? 1 : 0;
+  s = idx >= h;
+  r = s ? idx - h : h - 1 - idx;
+  return y;
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_new(const void* p, size_t i) {
+  return (float)reinterpret_cast<const T*>(p)[i];
+}
+
+// Token job = ((b * kv_heads + h) * n_new + n) goes to position seq_lens[b] - n_new + n.
+__device__ void append_token(const DecodeArgs& a, int job) {
+  __shared__ AppendShared sh;
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int n = job % a.n_new, h = (job / a.n_new) % a.cache.kv_heads, b = job / (a.n_new * a.cache.kv_heads);
+  const Layout& L = a.cache.L;
+  const int nk = 1 << L.kbits, nv = 1 << L.vbits;
+  if (i < nk) sh.tab[0][i] = a.k_centroids[i];
+  if (i < nk - 1) sh.tab[1][i] = a.k_boundaries[i];
+  if (i < nv) sh.tab[2][i] = a.v_centroids[i];
+  if (i < nv - 1) sh.tab[3][i] = a.v_boundaries[i];
+  const int len = a.seq_lens[b];
+  const int pos = len - a.n_new + n;
+  if (len < a.n_new || len > a.cache.max_pages * PT) {
+    if (i == 0) report(a.status, TQ_ERR_BOUNDS);
+    return;
+  }
+  const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + pos / PT];
+  if (phys < 0 || phys >= a.cache.num_pages) {
+    if (i == 0) report(a.status, TQ_ERR_BOUNDS);
+    return;
+  }
+  uint8_t* blk = a.cache.block(phys, h);
+  const int slot = pos % PT;
+  const size_t src = (size_t)job * D + i;
+  __syncthreads();
+
+  // ---- key: norm, rotation, quantisation
+  const float x = a.new_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.k_new)[src])
+                                        : ld_new<float>(a.k_new, src);
+  __half nh;
+  int idx, s, r;
+  encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r);
+  if (!L.kmerged) pack_code(s, r, L.kbits, lane, warp, sh.kw);
+  if (a.qjl) {
+    // residual in the original space r = k - fp16(n) R^T c[idx], its norm, and the signs
+    // of S r (sign(0) stored as +1)
+    float z;
+    if (!a.dense) {
+      sh.xs[i] = sh.tab[0][idx];
+      __syncthreads();
+      if (warp == 0) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = sh.xs[lane + 32 * e];
+        fwht128_warp(v, lane);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sh.xs[lane + 32 * e] = v[e];
+      }
+      __syncthreads();
+      z = sh.xs[i] * kInvSqrtD * a.signs[i];
+    } else {
+      sh.xs[i] = sh.tab[0][idx];
+      __syncthreads();
+      float acc = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) acc = fmaf(a.pi[(size_t)k * D + i], sh.xs[k], acc);  // (Pi^T z)_i
+      z = acc;
+    }
+    __syncthreads();
+    const float res = x - __half2float(nh) * z;
+    const __half rho = __float2half_rn(sqrtf(block_sum128(res * res, sh.red, lane, warp)));
+    sh.xs[i] = res;
+    __syncthreads();
+    // (S r)_o for the 32 rows o of this warp: lanes read 4 consecutive entries of row o
+    const float4 r4 = reinterpret_cast<const float4*>(sh.xs)[lane];
+    float sr = 0.f;
+#pragma unroll 8
+    for (int u = 0; u < 32; ++u) {
+      const float4 p = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
+      float t = p.x * r4.x;
+      t = fmaf(p.y, r4.y, t);
+      t = fmaf(p.z, r4.z, t);
+      t = fmaf(p.w, r4.w, t);
+      t = warp_sum(t);
+      if (lane == u) sr = t;
+    }
+    const int sigma = sr >= 0.f;
+    if (L.kmerged) {
+      pack_code(s, r | (s << 2) | (sigma << 3), kMergedNibble, lane, warp, sh.kw);
+    } else {
+      const uint32_t bw = __ballot_sync(FULL, sigma);
+      if (lane == 0) sh.ksw[warp] = bw;
+    }
+    if (i == 0) reinterpret_cast<__half*>(blk + L.kr)[slot] = rho;
+  }
+  __syncthreads();
+  if (i < L.kchunks)
+    reinterpret_cast<uint4*>(blk + L.kc)[i * PT + slot] = reinterpret_cast<const uint4*>(sh.kw)[i];
+  if (a.qjl && !L.kmerged && i == 0)
+    reinterpret_cast<uint4*>(blk + L.ks)[slot] = reinterpret_cast<const uint4*>(sh.ksw)[0];
+  if (i == 0) reinterpret_cast<__half*>(blk + L.kn)[slot] = nh;
+
+  // ---- value
+  const float xv = a.new_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.v_new)[src])
+                                         : ld_new<float>(a.v_new, src);
+  __half nv16;
+  encode_coord(a, sh, xv, sh.tab[3], L.vbits, i, lane, warp, nv16, idx, s, r);
+  pack_code(s, r, L.vbits, lane, warp, sh.vw);
+  __syncthreads();
+  if (i < L.vbits)
+    reinterpret_cast<uint4*>(blk + L.vc)[i * PT + slot] = reinterpret_cast<const uint4*>(sh.vw)[i];
+  if (i == 0) reinterpret_cast<__half*>(blk + L.vn)[slot] = nv16;
+}
+
+// ---------------------------------------------------------------------------
 // prologue: one CTA of 128 threads per query row.  Thread i owns coordinate i.
 //   qrot = R q (fp32), q8 = int8 rounding of qrot * 127 / max|qrot| (with its scale),
 //   sq = S q (fp32), sq_int = S q in 16-bit fixed point with a power-of-two scale, sum.
@@ -41,12 +258,17 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
   // set-up reads only inputs no kernel of this call writes).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
-  __shared__ float qs[D], ys[D];
+  const int row = blockIdx.x;
+  if (row >= total_rows) {
+    // thread blocks past the query rows append the new tokens (none unless a.n_new > 0)
+    if (a.n_new > 0 && row - total_rows < a.cache.batch * a.cache.kv_heads * a.n_new) append_token(a, row - total_rows);
+    return;
+  }
+  __shared__ __align__(16) float qs[D];
+  __shared__ float ys[D];
   __shared__ float red[2][4];
   __shared__ int ired[4];
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
-  const int row = blockIdx.x;
-  if (row >= total_rows) return;
   // the merge counters of the fused split kernel (one per sequence, kv head and run of up to
   // four query rows) start every call at zero
   if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads * ((a.rows + 3) / 4)) a.counter[row] = 0u;
@@ -440,20 +662,30 @@ static cudaError_t launch_pdl(void (*k)(Args...), dim3 grid, dim3 block, size_t 
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int total_rows = a.cache.batch * a.q_heads * a.seq_q;
+  // the prologue's grid: one thread block per query row, then one per appended token
+  const int blocks = total_rows + (a.n_new > 0 ? a.cache.batch * a.cache.kv_heads * a.n_new : 0);
   if (fast_decode_supported(a)) {
     // query transforms (and zeroed merge counters), then the split kernel, whose last
     // split per (sequence, kv head) merges the partials: two launches
-    cudaError_t e = launch_pdl(prologue_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
+    cudaError_t e = launch_pdl(prologue_kernel, dim3(blocks), dim3(128), 0, stream, a, total_rows);
     if (e != cudaSuccess) return e;
     return launch_fast_split(a, stream);
   }
-  cudaError_t e = launch_pdl(prologue_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
+  // the split kernel is an ordinary launch: it starts once the prologue (and any append)
+  // has finished
+  cudaError_t e = launch_pdl(prologue_kernel, dim3(blocks), dim3(128), 0, stream, a, total_rows);
   if (e != cudaSuccess) return e;
   e = launch_split(a, stream, false);
   if (e != cudaSuccess) return e;
   e = launch_pdl(combine_kernel, dim3(total_rows), dim3(128), 0, stream, a, total_rows);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_append(const DecodeArgs& a, cudaStream_t stream) {
+  const int blocks = a.cache.batch * a.cache.kv_heads * a.n_new;
+  if (blocks == 0) return cudaSuccess;
+  return launch_pdl(prologue_kernel, dim3(blocks), dim3(128), 0, stream, a, 0);
 }
 
 cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream) {

@@ -19,8 +19,11 @@
 //    (sequence, kv head) to finish (a counter the prologue zeroes) merges all partials
 //    and applies R^T.
 //
-// Supported here: query rows per KV head R = G * seq_q <= 4, keys 3-bit + QJL (merged
-// nibbles) or 2-bit + QJL, values 3-bit or 2-bit.  Everything else uses decode.cu.
+// The R = G * seq_q query rows of a KV head are taken four at a time: one run of up to four
+// rows per CTA along the grid's z, each run with its own merge counter.
+//
+// Supported here: keys 3-bit + QJL (merged nibbles) or 2-bit + QJL, values 3-bit or 2-bit,
+// any R.  Everything else uses decode.cu.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -258,6 +261,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
     if (lane == 0) {
+      // tokens from t_new on are appended by the prologue of this call: a unit that holds
+      // one is copied only after the prologue has finished
+      const int t_new = n_eff - a.n_new;
+      bool prologue_done = false;
       int issued = 0;
       for (int i = 0; i < nunits; ++i) {
         const int s = i % kStages;
@@ -267,6 +274,11 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         }
         issued = i + 1;
         const int u = u_begin + i, half = u % kUnitsPerPage;
+        if (a.n_new > 0 && !prologue_done && (u + 1) * kUnit > t_new) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          prologue_done = true;
+        }
         int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + u / kUnitsPerPage];
         if (phys < 0 || phys >= a.cache.num_pages) {
           report(a.status, TQ_ERR_BOUNDS);

@@ -217,6 +217,28 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.out = nullptr;
   a.scores = nullptr;
   a.max_len = 0;
+  a.k_new = nullptr;
+  a.v_new = nullptr;
+  a.new_dtype = TQ_F16;
+  a.n_new = 0;
+  a.k_boundaries = params->k_boundaries;
+  a.v_boundaries = params->v_boundaries;
+  return TQ_OK;
+}
+
+// Checks of the appended tokens' arguments shared by tq_append_kv and tq_append_attend_decode.
+static tq_status check_append(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                              const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new) {
+  if (!params->k_boundaries || !params->v_boundaries) return fail(TQ_ERR_INVALID_ARG, "boundary pointer is NULL");
+  if (!k_new || !v_new) return fail(TQ_ERR_INVALID_ARG, "k_new or v_new is NULL");
+  if (in_dtype != TQ_F16 && in_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "in_dtype must be TQ_F16 or TQ_F32");
+  if (n_new < 1) return fail(TQ_ERR_INVALID_ARG, "n_new must be >= 1");
+  if ((int64_t)cache->batch * cache->kv_heads * n_new > (int64_t)1 << 30)
+    return fail(TQ_ERR_INVALID_ARG, "batch * kv_heads * n_new too large");
+  if (cfg->key_qjl && (reinterpret_cast<uintptr_t>(params->s) & 15))
+    return fail(TQ_ERR_INVALID_ARG, "params->s must be 16-byte aligned");
+  if (cfg->rotation == TQ_ROT_DENSE && (reinterpret_cast<uintptr_t>(params->pi) & 15))
+    return fail(TQ_ERR_INVALID_ARG, "params->pi must be 16-byte aligned");
   return TQ_OK;
 }
 
@@ -234,6 +256,64 @@ tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const 
   a.status = dev_status;
   cudaError_t e = tqk::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_attend_decode launch");
+  return TQ_OK;
+}
+
+tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                  int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
+                                  int32_t n_new, const void* q, int32_t q_dtype, int32_t q_heads,
+                                  int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
+                                  size_t workspace_bytes, float* out, int32_t* dev_status,
+                                  tq_stream_t stream) {
+  clear_error();
+  tqk::DecodeArgs a;
+  tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, n_splits,
+                               workspace, workspace_bytes, a);
+  if (st != TQ_OK) return st;
+  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new)) != TQ_OK) return st;
+  if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
+  if ((int64_t)cache->batch * q_heads * seq_q + (int64_t)cache->batch * cache->kv_heads * n_new > (int64_t)1 << 30)
+    return fail(TQ_ERR_INVALID_ARG, "too many query rows and appended tokens");
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.new_dtype = in_dtype;
+  a.n_new = n_new;
+  a.out = out;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_append_attend_decode launch");
+  return TQ_OK;
+}
+
+tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
+                       const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new,
+                       const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  tq_status st;
+  if ((st = check_config(cfg)) != TQ_OK) return st;
+  if ((st = check_params(cfg, params, true)) != TQ_OK) return st;
+  if ((st = check_cache(cache, layer)) != TQ_OK) return st;
+  if (!seq_lens) return fail(TQ_ERR_INVALID_ARG, "seq_lens is NULL");
+  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new)) != TQ_OK) return st;
+  tqk::DecodeArgs a = {};
+  a.cache = cache_ref(cfg, cache, layer);
+  a.qjl = cfg->key_qjl;
+  a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.seq_lens = seq_lens;
+  a.signs = params->signs;
+  a.pi = params->pi;
+  a.s = params->s;
+  a.k_centroids = params->k_centroids;
+  a.v_centroids = params->v_centroids;
+  a.k_boundaries = params->k_boundaries;
+  a.v_boundaries = params->v_boundaries;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.new_dtype = in_dtype;
+  a.n_new = n_new;
+  a.status = dev_status;
+  cudaError_t e = tqk::launch_append(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "tq_append_kv launch");
   return TQ_OK;
 }
 

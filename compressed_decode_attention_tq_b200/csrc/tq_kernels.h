@@ -39,6 +39,12 @@ struct DecodeArgs {
   float* out;       // [B*Hq*seq_q][D]
   float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
   int max_len;
+  // tokens appended before attending (n_new = 0: none): k_new, v_new [B][Hkv][n_new][D] of
+  // element type new_dtype go to positions seq_lens[b] - n_new .. seq_lens[b] - 1
+  const void* k_new;
+  const void* v_new;
+  int new_dtype, n_new;
+  const float *k_boundaries, *v_boundaries;
   int32_t* status;
 };
 
@@ -71,6 +77,8 @@ bool fast_decode_supported(const DecodeArgs& a);
 size_t fast_decode_smem_bytes();
 cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_scores(const DecodeArgs& a, cudaStream_t stream);
+// the append alone: a.n_new tokens per (sequence, kv head), no query
+cudaError_t launch_append(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_decompress(const DecompressArgs& a, cudaStream_t stream);
 
 }  // namespace tqk

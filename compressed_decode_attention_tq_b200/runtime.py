@@ -9,7 +9,8 @@ from typing import Optional
 
 import torch
 
-from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, attend_decode, codebook, compress_kv,
+from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, append_attend_decode, append_kv, attend_decode,
+               codebook, compress_kv,
                decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
                operand_bytes, page_bytes, prepare_operands, status_str)
 
@@ -73,6 +74,12 @@ class PagedKV:
     def compress(self, layer: int, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, stream=None):
         compress_kv(self.cfg, self.params, self.cache, layer, k, v, seq_lens, self.status, stream)
 
+    def append(self, layer: int, k_new: torch.Tensor, v_new: torch.Tensor, seq_lens: torch.Tensor,
+               stream=None):
+        """Compresses k_new, v_new [batch][kv_heads][n_new][d] into positions
+        seq_lens[b] - n_new .. seq_lens[b] - 1 (seq_lens: the lengths after the append)."""
+        append_kv(self.cfg, self.params, self.cache, layer, k_new, v_new, seq_lens, self.status, stream)
+
     def workspace(self, q_heads: int, seq_q: int, n_splits: int) -> torch.Tensor:
         key = (q_heads, seq_q, n_splits)
         if key not in self._ws:
@@ -81,12 +88,19 @@ class PagedKV:
         return self._ws[key]
 
     def decode(self, layer: int, q: torch.Tensor, seq_lens: torch.Tensor, n_splits: int,
-               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+               out: Optional[torch.Tensor] = None, stream=None, k_new: Optional[torch.Tensor] = None,
+               v_new: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Attention of q over the first seq_lens[b] tokens.  With k_new and v_new the step's
+        new tokens are appended first, in the same call (seq_lens count them)."""
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
         ws = self.workspace(q.shape[1], q.shape[2], n_splits)
-        attend_decode(self.cfg, self.params, self.cache, layer, q, seq_lens, n_splits, ws, out,
-                      self.status, stream)
+        if k_new is not None:
+            append_attend_decode(self.cfg, self.params, self.cache, layer, k_new, v_new, q, seq_lens,
+                                 n_splits, ws, out, self.status, stream)
+        else:
+            attend_decode(self.cfg, self.params, self.cache, layer, q, seq_lens, n_splits, ws, out,
+                          self.status, stream)
         return out
 
     def scores(self, layer: int, q: torch.Tensor, seq_lens: torch.Tensor, max_len: int, stream=None):

@@ -241,6 +241,40 @@ TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params,
                            void* workspace, size_t workspace_bytes, float* out,
                            int32_t* dev_status, tq_stream_t stream);
 
+/* Incremental append ([TQKV] incremental cache: CompressedKeys::append_raw and
+ * compress_single_key_with_signs; [LIMITS] packed page update): compresses n_new new
+ * tokens of every (sequence, kv head) exactly as tq_compress_kv would and writes them to
+ * their slots, leaving every other slot of the cache untouched (a token's bytes are
+ * independent of its neighbours' in the packed format above).
+ *   k_new, v_new  device [batch][kv_heads][n_new][d], element type in_dtype
+ *   n_new         >= 1 (batch * kv_heads * n_new <= 2^30)
+ *   seq_lens      device int32 [batch]: the lengths AFTER the append; new token n of
+ *                 sequence b goes to position seq_lens[b] - n_new + n (logical page
+ *                 pos / P, slot pos % P of the block table)
+ *   dev_status    TQ_ERR_BOUNDS when seq_lens[b] < n_new, seq_lens[b] exceeds the
+ *                 block-table row or a page id is out of range (that token is skipped);
+ *                 TQ_ERR_OVERFLOW as for tq_compress_kv
+ * params.s (with key_qjl) and params.pi (TQ_ROT_DENSE) must be 16-byte aligned; S is
+ * used in fp32 as given (no fp16 requirement).  One thread block per new token. */
+TQ_API tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                              int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
+                              int32_t n_new, const int32_t* seq_lens, int32_t* dev_status,
+                              tq_stream_t stream);
+
+/* One decode step with its append fused in: the effect of tq_append_kv(k_new, v_new,
+ * n_new, seq_lens) followed by tq_attend_decode(q, seq_lens), so the new tokens are
+ * attended to by the query rows of the same step (seq_lens are the lengths after the
+ * append).  The new tokens are encoded by extra thread blocks of the decode's query
+ * prologue; the attention kernels copy a page range holding a new token only after the
+ * prologue has finished.  Arguments, errors and workspace as for the two calls. */
+TQ_API tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params,
+                                         const tq_cache* cache, int32_t layer, const void* k_new,
+                                         const void* v_new, int32_t in_dtype, int32_t n_new,
+                                         const void* q, int32_t q_dtype, int32_t q_heads,
+                                         int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,
+                                         void* workspace, size_t workspace_bytes, float* out,
+                                         int32_t* dev_status, tq_stream_t stream);
+
 /* Decode attention for callers that cannot allocate device memory (no counterpart on
  * the source pages; it exists for users of this library).  Same computation, arguments
  * and results as tq_attend_decode, minus the workspace: a plugin inside a runtime that

@@ -50,8 +50,10 @@ class Run:
     V: dict = None
 
 
-def setup(w: wl.Workload, layers=(0,), prepared_operands=True):
-    """Builds the library cache for w and compresses `layers` on the GPU (inputs from workloads)."""
+def setup(w: wl.Workload, layers=(0,), prepared_operands=True, compress_lens=None):
+    """Builds the library cache for w and compresses `layers` on the GPU (inputs from workloads).
+    compress_lens: optional per-sequence token counts to compress instead of the full
+    lengths (the cache's block table still covers the full lengths)."""
     from compressed_decode_attention_tq_b200.runtime import PagedKV
     lens = wl.seq_lens(w)
     bt, npages = wl.block_table(w, lens)
@@ -68,7 +70,7 @@ def setup(w: wl.Workload, layers=(0,), prepared_operands=True):
                      pi=rin["pi"], s=rin["s"], prepared_operands=prepared_operands)
     run.K, run.V = {}, {}
     dt = torch.float16 if w.in_dtype == "f16" else torch.float32
-    seq = torch.as_tensor(lens, dtype=torch.int32, device="cuda")
+    seq = torch.as_tensor(lens if compress_lens is None else compress_lens, dtype=torch.int32, device="cuda")
     for layer in layers:
         K, V = wl.make_kv(w, layer)
         run.K[layer], run.V[layer] = K, V

@@ -142,3 +142,40 @@ def test_operand_bytes_and_prepare_validation(tq):
     params.s = aligned
     st = tq.lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), aligned + 4, None)
     assert st == tq.TQ_ERR_INVALID_ARG and "aligned" in tq.last_error()
+
+
+def test_append_argument_errors_do_not_launch(tq):
+    # host-side checks of tq_append_kv and tq_append_attend_decode (no device work)
+    by = ctypes.byref
+    cfg = tq.make_config()
+    params = tq.tq_params()
+    cache = tq.tq_cache()
+    st = tq.lib.tq_append_kv(by(cfg), None, by(cache), 0, None, None, 0, 1, None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "params" in tq.last_error()
+    buf = ctypes.create_string_buffer(4096)
+    p = (ctypes.addressof(buf) + 255) & ~255  # any non-null pointer: nothing is dereferenced
+    params = tq.tq_params(p, None, p, p, p, p, p, None)
+    cache = tq.tq_cache(p, p, 4, 4, 1, 1, 1)
+    st = tq.lib.tq_append_kv(by(cfg), by(params), by(cache), 0, p, p, 0, 0, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "n_new" in tq.last_error()
+    st = tq.lib.tq_append_kv(by(cfg), by(params), by(cache), 0, None, p, 0, 1, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "k_new" in tq.last_error()
+    st = tq.lib.tq_append_kv(by(cfg), by(params), by(cache), 0, p, p, 7, 1, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "in_dtype" in tq.last_error()
+    st = tq.lib.tq_append_kv(by(cfg), by(params), by(cache), 0, p, p, 0, 1, None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "seq_lens" in tq.last_error()
+    st = tq.lib.tq_append_kv(by(cfg), by(params), by(cache), 1, p, p, 0, 1, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "layer" in tq.last_error()
+    misaligned = tq.tq_params(p, None, p + 4, p, p, p, p, None)
+    st = tq.lib.tq_append_kv(by(cfg), by(misaligned), by(cache), 0, p, p, 0, 1, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "aligned" in tq.last_error()
+    nb = tq.decode_workspace_bytes(cfg, 1, 4, 1, 2)
+    st = tq.lib.tq_append_attend_decode(by(cfg), by(params), by(cache), 0, p, p, 0, 0, p, 0, 4, 1, p, 2,
+                                        p, nb, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "n_new" in tq.last_error()
+    st = tq.lib.tq_append_attend_decode(by(cfg), by(params), by(cache), 0, p, None, 0, 1, p, 0, 4, 1, p, 2,
+                                        p, nb, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "v_new" in tq.last_error()
+    st = tq.lib.tq_append_attend_decode(by(cfg), by(params), by(cache), 0, p, p, 0, 1, p, 0, 4, 1, p, 2,
+                                        p, nb, None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "out" in tq.last_error()
