@@ -10,6 +10,9 @@ Sources:
       - section "Two-Stage Approach: MSE Approximation + QJL Correction" and
         "Unbiasedness Proof": the key is x_mse + x_qjl, so
         <q, k>^ = <q, k_mse> + ||r|| sqrt(pi/2)/m <S q, sign(S r)>;
+      - the same section, on the value cache: a vector is reconstructed as
+        x_mse + sqrt(pi/2)/d ||r|| S^T sign(S r), unbiased, so TurboQuant_prod serves the
+        value cache as well (values with QJL);
       - section "How is this different from PolarQuant's reconstruction?": the
         identity <q, R^T c> = <R q, c>, which the device path uses; this oracle
         computes <q, k_mse> directly in the original space instead.
@@ -82,9 +85,12 @@ def attend_scores(scores, Vhat) -> np.ndarray:
 
 
 def decode_sequence(q, unpacked: lay.Unpacked, R, ck, cv, S=None, return_scores=False):
-    """Decode attention of q [nq, d] over one (sequence, kv head) read from packed pages."""
+    """Decode attention of q [nq, d] over one (sequence, kv head) read from packed pages.
+    Values with QJL are reconstructed as v_mse + x_qjl (S is then required)."""
     k_mse = qt.reconstruct_mse(unpacked.k_idx, unpacked.k_norm, R, ck)
     v_hat = qt.reconstruct_mse(unpacked.v_idx, unpacked.v_norm, R, cv)
+    if unpacked.v_sigma is not None:
+        v_hat = v_hat + qt.qjl_reconstruct(unpacked.v_sigma, unpacked.v_rnorm, S)
     sc = scores_compressed(q, k_mse, unpacked.k_rnorm, unpacked.k_sigma, S)
     out = attend_scores(sc, v_hat)
     return (out, sc) if return_scores else out

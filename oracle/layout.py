@@ -19,6 +19,8 @@ page, kv head); the cache is [layer][physical page][kv head][block]):
   KC      key codes, b_k*d/8 bytes per token     b_k*16*P  (merged keys: 4*16*P)
   KS      QJL sign bits, m/8 bytes per token     16*P   (keys with QJL, not merged)
   VC      value codes, b_v*d/8 bytes per token   b_v*16*P
+  VS      QJL sign bits of the value residual    16*P   (values with QJL)
+  VR      stored ||r_v|| as fp16                 2P     (values with QJL)
 
 Each code region is a sequence of 16-byte chunks per token, stored chunk-major:
 chunk c of token t sits at byte (c*P + t)*16 of the region.  Token t's chunks,
@@ -38,6 +40,12 @@ c[idx] = (+1 if s else -1) * c[h + r].  Fields of coordinate j in the bit string
 Keys with b_k = 3 and QJL ("merged keys") store one 4-bit field per coordinate,
 bits 4j..4j+3 = r0, r1, s, sigma_j, and have no KS region; other keys with QJL keep
 the sign bits in KS, bit i = sigma_i.
+
+Values with QJL (TurboQuant_prod applied to the value cache: "TurboQuant explained",
+section "Two-Stage Approach: MSE Approximation + QJL Correction", which reconstructs a
+vector as x_mse + sqrt(pi/2)/d ||r|| S^T sign(S r) and notes that this serves the value
+cache too) store the residual's signs in VS (bit i = sigma_i, as KS) and its norm in VR;
+the two regions come last, so every other offset is the same with or without them.
 """
 from __future__ import annotations
 
@@ -54,6 +62,7 @@ class Format:
     qjl_m: int = 128
     value_bits: int = 3
     page_tokens: int = 256
+    value_qjl: bool = False
 
     @property
     def merged_keys(self) -> bool:
@@ -69,7 +78,9 @@ class Format:
         ks = m // 8 * P if (self.key_qjl and not self.merged_keys) else 0
         sizes = [("KN", 2 * P), ("KR", 2 * P if self.key_qjl else 0), ("VN", 2 * P),
                  ("KC", self.key_bytes * P), ("KS", ks),
-                 ("VC", self.value_bits * d // 8 * P)]
+                 ("VC", self.value_bits * d // 8 * P),
+                 ("VS", m // 8 * P if self.value_qjl else 0),
+                 ("VR", 2 * P if self.value_qjl else 0)]
         out, off = {}, 0
         for name, sz in sizes:
             out[name] = (off, sz)
@@ -214,6 +225,7 @@ def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_
         kbytes = bits_to_bytes(code_bits(kcomp.idx, fmt.key_bits))
         sbytes = bits_to_bytes(kcomp.sigma.astype(np.uint8)) if fmt.key_qjl else None
     vbytes = bits_to_bytes(code_bits(vcomp.idx, fmt.value_bits))
+    vsbytes = bits_to_bytes(vcomp.sigma.astype(np.uint8)) if fmt.value_qjl else None
     for lp in range((n + P - 1) // P):
         t0, t1 = lp * P, min(n, (lp + 1) * P)
         blk = cache[layer, pages_of_seq[lp], head]
@@ -230,6 +242,9 @@ def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_
             _put_chunked(region("KS"), sbytes[t0:t1], 0, P)
         _put_chunked(region("KC"), kbytes[t0:t1], 0, P)
         _put_chunked(region("VC"), vbytes[t0:t1], 0, P)
+        if fmt.value_qjl:
+            region("VR")[0:2 * (t1 - t0)] = fp16_bytes(vcomp.rnorm[t0:t1])
+            _put_chunked(region("VS"), vsbytes[t0:t1], 0, P)
 
 
 @dataclasses.dataclass
@@ -240,6 +255,8 @@ class Unpacked:
     v_norm: np.ndarray
     k_rnorm: np.ndarray = None
     k_sigma: np.ndarray = None
+    v_rnorm: np.ndarray = None
+    v_sigma: np.ndarray = None
 
 
 def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_of_seq,
@@ -248,7 +265,7 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
     P, d, m = fmt.page_tokens, fmt.head_dim, fmt.qjl_m
     reg = fmt.regions()
     kb, vb = fmt.key_bytes, fmt.value_bits * d // 8
-    parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc")}
+    parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc", "vr", "vs")}
     for lp in range((n + P - 1) // P):
         cnt = min(n, (lp + 1) * P) - lp * P
         blk = cache[layer, pages_of_seq[lp], head]
@@ -265,6 +282,9 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
             parts["kr"].append(region("KR")[:2 * cnt].view(np.float16).astype(np.float64))
         if fmt.key_qjl and not fmt.merged_keys:
             parts["ks"].append(_get_chunked(region("KS"), cnt, m // 8, P))
+        if fmt.value_qjl:
+            parts["vr"].append(region("VR")[:2 * cnt].view(np.float16).astype(np.float64))
+            parts["vs"].append(_get_chunked(region("VS"), cnt, m // 8, P))
     cat = lambda k, w: np.concatenate(parts[k]) if parts[k] else np.zeros((0,) + w)
     kc = cat("kc", (kb,))
     vc = cat("vc", (vb,))
@@ -278,4 +298,7 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
     if fmt.key_qjl:
         out.k_rnorm = cat("kr", ())
         out.k_sigma = k_sigma if fmt.merged_keys else bytes_to_bits(cat("ks", (m // 8,))).astype(bool)
+    if fmt.value_qjl:
+        out.v_rnorm = cat("vr", ())
+        out.v_sigma = bytes_to_bits(cat("vs", (m // 8,))).astype(bool)
     return out

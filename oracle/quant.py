@@ -89,7 +89,8 @@ def reconstruct_mse(idx, norm, R, centroids) -> np.ndarray:
 
 
 def compress_prod(x, R, centroids, boundaries, S) -> Compressed:
-    """TurboQuant_prod for keys: MSE stage, residual r = x - x_mse, sigma = [S r >= 0], ||r||."""
+    """TurboQuant_prod (keys, and values with QJL): MSE stage, residual r = x - x_mse,
+    sigma = [S r >= 0], ||r||."""
     x = np.asarray(x, dtype=np.float64)
     comp = compress_mse(x, R, centroids, boundaries)
     x_mse = reconstruct_mse(comp.idx, comp.norm, R, centroids)

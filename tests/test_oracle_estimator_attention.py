@@ -236,3 +236,58 @@ def test_more_bits_lower_score_error():
         err = np.mean((est - q @ K.T / math.sqrt(128)) ** 2)
         assert err < prev
         prev = err
+
+
+def test_value_qjl_decode_is_unbiased_where_mse_only_is_not():
+    # Values with QJL ("TurboQuant explained", section "Two-Stage Approach": x_mse + x_qjl is
+    # an unbiased reconstruction, so TurboQuant_prod serves the value cache too).  With all
+    # keys equal the softmax weights are uniform, so the decode output is the mean of the
+    # reconstructed values: over fresh S its average must reach mean_t v_t, while the
+    # MSE-only decode keeps the 1-bit quantiser's shrinkage.  A wrong sign, scale or
+    # orientation of the value QJL term in the decode fails this.
+    rng = np.random.default_rng(31)
+    d, T, trials = 64, 6, 3000
+    R = rot.hd_matrix(hadamard_signs(d, 4))
+    ck, kb = cb.codebook_f32(2, d)
+    cv, vb = cb.codebook_f32(1, d)
+    V = rng.standard_normal((T, d)) * 3.0
+    K = np.tile(rng.standard_normal(d), (T, 1))
+    q = rng.standard_normal((1, d))
+    kc = qt.compress_mse(K, R, ck, kb)
+    target = V.mean(axis=0)
+    acc_q = np.zeros(d)
+    acc_m = np.zeros(d)
+    for _ in range(trials):
+        S = rng.standard_normal((d, d))
+        vc = qt.compress_prod(V, R, cv, vb, S)
+        u = lay.Unpacked(k_idx=kc.idx, k_norm=kc.norm, v_idx=vc.idx, v_norm=vc.norm,
+                         v_rnorm=vc.rnorm, v_sigma=vc.sigma)
+        acc_q += att.decode_sequence(q, u, R, ck, cv, S)[0]
+        u.v_rnorm = u.v_sigma = None
+        acc_m += att.decode_sequence(q, u, R, ck, cv, S)[0]
+    err_q = np.linalg.norm(acc_q / trials - target)
+    err_m = np.linalg.norm(acc_m / trials - target)
+    assert err_m > 0.15 * np.linalg.norm(target)       # the MSE-only output is biased
+    assert err_q < 0.25 * err_m                        # the QJL term removes the bias
+    assert err_q < 0.05 * np.linalg.norm(target)
+
+
+def test_value_qjl_single_token_output_is_the_prod_reconstruction():
+    # one cached token: softmax weight 1, so decode returns that token's v_mse + x_qjl
+    rng = np.random.default_rng(32)
+    d = 128
+    R = rot.hd_matrix(hadamard_signs(d, 0))
+    S = qjl_matrix(128, d, 1)
+    ck, kb = cb.codebook_f32(3, d)
+    cv, vb = cb.codebook_f32(2, d)
+    k = rng.standard_normal((1, d))
+    v = rng.standard_normal((1, d))
+    kc = qt.compress_prod(k, R, ck, kb, S)
+    vc = qt.compress_prod(v, R, cv, vb, S)
+    u = lay.Unpacked(k_idx=kc.idx, k_norm=kc.norm, v_idx=vc.idx, v_norm=vc.norm, k_rnorm=kc.rnorm,
+                     k_sigma=kc.sigma, v_rnorm=vc.rnorm, v_sigma=vc.sigma)
+    out = att.decode_sequence(rng.standard_normal((2, d)), u, R, ck, cv, S)
+    r = v[0] - qt.reconstruct_mse(vc.idx, vc.norm, R, cv)[0]
+    expect = qt.reconstruct_mse(vc.idx, vc.norm, R, cv)[0] + \
+        math.sqrt(math.pi / 2) / 128 * vc.rnorm[0] * (S.T @ np.where(S @ r >= 0, 1.0, -1.0))
+    np.testing.assert_allclose(out, np.tile(expect, (2, 1)), rtol=1e-12, atol=1e-12)

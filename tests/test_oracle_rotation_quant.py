@@ -168,8 +168,9 @@ def test_sign_plane_permutation_is_a_bijection():
     assert np.all(pos // 32 == np.arange(128) // 32)
 
 
-def test_region_offsets_match_hand_derivation(packing_golden):
-    g = packing_golden["c2_regions"]
+@pytest.mark.parametrize("name", ["c2_regions", "c2_value_qjl_regions"])
+def test_region_offsets_match_hand_derivation(packing_golden, name):
+    g = packing_golden[name]
     fmt = lay.Format(**g["format"])
     reg = fmt.regions()
     for k, v in g["offsets"].items():
@@ -212,3 +213,30 @@ def test_page_round_trip_with_partial_last_page():
     blk = cache[0, 0, 1]
     assert blk[o + (256 + 44) * 16: o + (256 + 44) * 16 + 16].tobytes() == tok_bytes[16:32].tobytes()
     assert not cache[0, :, 0].any()
+
+
+def test_value_qjl_page_round_trip_and_hand_placed_bytes():
+    # values with QJL: the residual's sign bits go to VS (bit i = sigma_i, 16-byte chunk per
+    # token) and its fp16 norm to VR, both after VC (offsets 30208 and 34304 for this format)
+    fmt = lay.Format(key_bits=3, key_qjl=True, value_bits=3, page_tokens=256, value_qjl=True)
+    n = 300
+    rng = np.random.default_rng(2)
+    K = qt.Compressed(idx=rng.integers(0, 8, (n, 128)), norm=rng.uniform(0, 50, n).astype(np.float16).astype(float),
+                      y=None, rnorm=rng.uniform(0, 5, n).astype(np.float16).astype(float),
+                      sigma=rng.integers(0, 2, (n, 128)).astype(bool))
+    vs = np.zeros((n, 128), dtype=bool)
+    vs[5, 0] = vs[5, 9] = vs[5, 127] = True  # token 5: bits 0, 9 and 127 of its chunk
+    V = qt.Compressed(idx=rng.integers(0, 8, (n, 128)), norm=rng.uniform(0, 50, n).astype(np.float16).astype(float),
+                      y=None, rnorm=np.full(n, 1.5), sigma=vs)
+    cache = lay.empty_cache(fmt, num_pages=3, kv_heads=1)
+    lay.write_sequence(cache, fmt, 0, 0, [2, 0], K, V)
+    u = lay.read_sequence(cache, fmt, 0, 0, [2, 0], n)
+    np.testing.assert_array_equal(u.v_sigma, vs)
+    np.testing.assert_array_equal(u.v_rnorm, V.rnorm)
+    np.testing.assert_array_equal(u.v_idx, V.idx)
+    np.testing.assert_array_equal(u.k_sigma, K.sigma)
+    blk = cache[0, 2, 0]
+    assert blk[30208 + 5 * 16: 30208 + 6 * 16].tobytes().hex() == "0102" + "00" * 13 + "80"
+    assert blk[34304 + 10: 34304 + 12].tobytes() == np.float16(1.5).tobytes()
+    # token 256 is slot 0 of the second page (physical 0)
+    assert cache[0, 0, 0][34304: 34306].tobytes() == np.float16(1.5).tobytes()
