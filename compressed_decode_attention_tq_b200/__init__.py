@@ -39,7 +39,7 @@ class tq_config(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32),
                 ("key_qjl", ctypes.c_int32), ("qjl_m", ctypes.c_int32),
                 ("value_bits", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
-                ("rotation", ctypes.c_int32)]
+                ("rotation", ctypes.c_int32), ("value_qjl", ctypes.c_int32)]
 
 
 class tq_params(ctypes.Structure):
@@ -111,8 +111,9 @@ def _check(st: int, where: str):
 
 
 def make_config(head_dim=128, key_bits=3, key_qjl=True, qjl_m=128, value_bits=3, page_tokens=256,
-                rotation=TQ_ROT_HADAMARD) -> tq_config:
-    return tq_config(head_dim, key_bits, int(bool(key_qjl)), qjl_m, value_bits, page_tokens, rotation)
+                rotation=TQ_ROT_HADAMARD, value_qjl=False) -> tq_config:
+    return tq_config(head_dim, key_bits, int(bool(key_qjl)), qjl_m, value_bits, page_tokens, rotation,
+                     int(bool(value_qjl)))
 
 
 def validate_config(cfg: tq_config) -> int:

@@ -150,6 +150,56 @@ __device__ __forceinline__ void encode_vector(const float (&x)[4], int bits, con
   (void)cent;
 }
 
+// QJL sketch of the residual in the original space, r = x - fp16(n) R^T c[idx] ("TurboQuant
+// explained", section "Two-Stage Approach"): returns fp16(||r||) and the signs
+// sg[e] = [(S r)_j >= 0] of the lane's rows j = lane + 32 e (sign(0) stored as +1).
+__device__ __forceinline__ __half qjl_residual_signs(const float (&x)[4], const int (&idx)[4], __half norm,
+                                                     const float* cent, const float* signs,
+                                                     const float* pi_s, const float* s_s, float* stage,
+                                                     int lane, int (&sg)[4]) {
+  float z[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) z[e] = cent[idx[e]];
+  if (pi_s == nullptr) {
+    fwht128_warp(z, lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) z[e] *= 0.08838834764831845f * signs[lane + 32 * e];
+  } else {
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) stage[lane + 32 * e] = z[e];
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float acc = 0.f;
+      for (int i = 0; i < D; ++i) acc = fmaf(pi_s[i * kPad + lane + 32 * e], stage[i], acc);
+      z[e] = acc;
+    }
+  }
+  const float nh = __half2float(norm);
+  float rr[4], r2 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    rr[e] = x[e] - nh * z[e];
+    r2 = fmaf(rr[e], rr[e], r2);
+  }
+  r2 = warp_sum(r2);
+  const __half rho = __float2half_rn(sqrtf(r2));
+  __syncwarp();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) stage[lane + 32 * e] = rr[e];
+  __syncwarp();
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float* srow = s_s + (lane + 32 * e) * kPad;
+    float acc = 0.f;
+    for (int k = 0; k < D; ++k) acc = fmaf(srow[k], stage[k], acc);
+    sg[e] = acc >= 0.f;
+  }
+  __syncwarp();
+  return rho;
+}
+
 template <typename T>
 __device__ __forceinline__ float ld_in(const T* p) { return (float)p[0]; }
 template <>
@@ -160,7 +210,8 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SmemCompress& sm = *reinterpret_cast<SmemCompress*>(smem_raw);
   float* s_s = reinterpret_cast<float*>(smem_raw + sizeof(SmemCompress));  // [QM][kPad] if qjl
-  float* pi_s = s_s + (a.qjl ? QM * kPad : 0);                             // [D][kPad] if dense
+  const bool sketch = a.qjl || a.cache.L.vqjl;                               // S is used
+  float* pi_s = s_s + (sketch ? QM * kPad : 0);                              // [D][kPad] if dense
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = blockIdx.z, h = blockIdx.y;
   const Layout& L = a.cache.L;
@@ -171,7 +222,7 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
   if (tid < nv - 1) sm.vb[tid] = a.v_boundaries[tid];
   if (!a.dense)
     for (int i = tid; i < D; i += blockDim.x) sm.signs[i] = a.signs[i];
-  if (a.qjl) {
+  if (sketch) {
     for (int i = tid; i < QM * D; i += blockDim.x) {
       const float v = a.s[i];
       if (__half2float(__float2half_rn(v)) != v) report(a.status, TQ_ERR_INVALID_ARG);
@@ -221,59 +272,21 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
       reinterpret_cast<uint4*>(blk + L.kc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
     if (lane == 0) reinterpret_cast<__half*>(blk + L.kn)[slot] = ko.norm;
     if (a.qjl) {
-      // residual in the original space: r = k - fp16(n) R^T c[idx]
-      float z[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) z[e] = sm.kc[ko.idx[e]];
-      if (!a.dense) {
-        fwht128_warp(z, lane);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) z[e] *= 0.08838834764831845f * sm.signs[lane + 32 * e];
-      } else {
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) stage[lane + 32 * e] = z[e];
-        __syncwarp();
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float acc = 0.f;
-          for (int i = 0; i < D; ++i) acc = fmaf(pi_s[i * kPad + lane + 32 * e], stage[i], acc);
-          z[e] = acc;
-        }
-      }
-      const float nh = __half2float(ko.norm);
-      float rr[4], r2 = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        rr[e] = x[e] - nh * z[e];
-        r2 = fmaf(rr[e], rr[e], r2);
-      }
-      r2 = warp_sum(r2);
-      const __half rho = __float2half_rn(sqrtf(r2));
-      __syncwarp();
-#pragma unroll
-      for (int e = 0; e < 4; ++e) stage[lane + 32 * e] = rr[e];
-      __syncwarp();
       int sg[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float* srow = s_s + (lane + 32 * e) * kPad;
-        float acc = 0.f;
-        for (int k = 0; k < D; ++k) acc = fmaf(srow[k], stage[k], acc);
-        sg[e] = acc >= 0.f;
-        if (!L.kmerged) {
-          const uint32_t w = __ballot_sync(FULL, sg[e]);
-          if (lane == 0) wbuf[e] = w;
-        }
-      }
-      __syncwarp();
+      const __half rho = qjl_residual_signs(x, ko.idx, ko.norm, sm.kc, sm.signs, pis, s_s, stage, lane, sg);
       if (L.kmerged) {
         pack_merged(ko.s, ko.r, sg, lane, wbuf);
         __syncwarp();
         if (lane < 4)
           reinterpret_cast<uint4*>(blk + L.kc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
-      } else if (lane == 0) {
-        reinterpret_cast<uint4*>(blk + L.ks)[slot] = reinterpret_cast<const uint4*>(wbuf)[0];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t w = __ballot_sync(FULL, sg[e]);
+          if (lane == 0) wbuf[e] = w;
+        }
+        __syncwarp();
+        if (lane == 0) reinterpret_cast<uint4*>(blk + L.ks)[slot] = reinterpret_cast<const uint4*>(wbuf)[0];
       }
       if (lane == 0) reinterpret_cast<__half*>(blk + L.kr)[slot] = rho;
       __syncwarp();
@@ -289,6 +302,22 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
       reinterpret_cast<uint4*>(blk + L.vc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
     if (lane == 0) reinterpret_cast<__half*>(blk + L.vn)[slot] = vo.norm;
     __syncwarp();
+    if (L.vqjl) {
+      // values with QJL: the same sketch of the value residual, signs in VS, norm in VR
+      int sg[4];
+      const __half rho = qjl_residual_signs(x, vo.idx, vo.norm, sm.vc, sm.signs, pis, s_s, stage, lane, sg);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t w = __ballot_sync(FULL, sg[e]);
+        if (lane == 0) wbuf[e] = w;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        reinterpret_cast<uint4*>(blk + L.vs)[slot] = reinterpret_cast<const uint4*>(wbuf)[0];
+        reinterpret_cast<__half*>(blk + L.vr)[slot] = rho;
+      }
+      __syncwarp();
+    }
   }
 }
 
@@ -304,7 +333,7 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
     const cudaError_t e = launch_compress_tc(a, stream);
     if (e != cudaErrorInvalidValue) return e;  // otherwise fall through to the CUDA-core kernel
   }
-  const size_t smem = compress_smem_bytes(a.qjl, a.dense);
+  const size_t smem = compress_smem_bytes(a.qjl || a.cache.L.vqjl, a.dense);
   dim3 grid((a.max_len + kTokPerBlock - 1) / kTokPerBlock, a.cache.kv_heads, a.cache.batch);
   if (grid.x == 0) return cudaSuccess;
   if (a.in_dtype == TQ_F16) {

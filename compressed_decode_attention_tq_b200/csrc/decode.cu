@@ -43,7 +43,7 @@ struct __align__(16) AppendShared {
   float xs[D];          // the vector being transformed
   float tab[4][16];     // k centroids, k boundaries, v centroids, v boundaries
   float red[4];
-  uint32_t kw[16], ksw[4], vw[16];
+  uint32_t kw[16], ksw[4], vw[16], vsw[4];
 };
 
 __device__ __forceinline__ float block_sum128(float v, float* red, int lane, int warp) {
@@ -137,6 +137,54 @@ __device__ __forceinline__ float encode_coord(const DecodeArgs& a, AppendShared&
   return y;
 }
 
+// Residual of thread i's coordinate in the original space, r = x - fp16(n) R^T c[idx] (c_i:
+// the centroid of its index), its stored norm fp16(||r||) (returned), and the sign
+// sigma = [(S r)_i >= 0] of row i of S (sign(0) stored as +1).
+__device__ __forceinline__ __half append_qjl(const DecodeArgs& a, AppendShared& sh, float x, __half nh, float c_i,
+                                             int i, int lane, int warp, int& sigma) {
+  float z;
+  sh.xs[i] = c_i;
+  __syncthreads();
+  if (!a.dense) {
+    if (warp == 0) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = sh.xs[lane + 32 * e];
+      fwht128_warp(v, lane);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sh.xs[lane + 32 * e] = v[e];
+    }
+    __syncthreads();
+    z = sh.xs[i] * kInvSqrtD * a.signs[i];
+  } else {
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D; ++k) acc = fmaf(a.pi[(size_t)k * D + i], sh.xs[k], acc);  // (Pi^T z)_i
+    z = acc;
+  }
+  __syncthreads();
+  const float res = x - __half2float(nh) * z;
+  const __half rho = __float2half_rn(sqrtf(block_sum128(res * res, sh.red, lane, warp)));
+  sh.xs[i] = res;
+  __syncthreads();
+  // (S r)_o for the 32 rows o of this warp: lanes read 4 consecutive entries of row o
+  const float4 r4 = reinterpret_cast<const float4*>(sh.xs)[lane];
+  float sr = 0.f;
+#pragma unroll 8
+  for (int u = 0; u < 32; ++u) {
+    const float4 p = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
+    float t = p.x * r4.x;
+    t = fmaf(p.y, r4.y, t);
+    t = fmaf(p.z, r4.z, t);
+    t = fmaf(p.w, r4.w, t);
+    t = warp_sum(t);
+    if (lane == u) sr = t;
+  }
+  sigma = sr >= 0.f;
+  __syncthreads();  // xs is free again
+  return rho;
+}
+
 template <typename T>
 __device__ __forceinline__ float ld_new(const void* p, size_t i) {
   return (float)reinterpret_cast<const T*>(p)[i];
@@ -177,49 +225,8 @@ __device__ void append_token(const DecodeArgs& a, int job) {
   encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r);
   if (!L.kmerged) pack_code(s, r, L.kbits, lane, warp, sh.kw);
   if (a.qjl) {
-    // residual in the original space r = k - fp16(n) R^T c[idx], its norm, and the signs
-    // of S r (sign(0) stored as +1)
-    float z;
-    if (!a.dense) {
-      sh.xs[i] = sh.tab[0][idx];
-      __syncthreads();
-      if (warp == 0) {
-        float v[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = sh.xs[lane + 32 * e];
-        fwht128_warp(v, lane);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sh.xs[lane + 32 * e] = v[e];
-      }
-      __syncthreads();
-      z = sh.xs[i] * kInvSqrtD * a.signs[i];
-    } else {
-      sh.xs[i] = sh.tab[0][idx];
-      __syncthreads();
-      float acc = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) acc = fmaf(a.pi[(size_t)k * D + i], sh.xs[k], acc);  // (Pi^T z)_i
-      z = acc;
-    }
-    __syncthreads();
-    const float res = x - __half2float(nh) * z;
-    const __half rho = __float2half_rn(sqrtf(block_sum128(res * res, sh.red, lane, warp)));
-    sh.xs[i] = res;
-    __syncthreads();
-    // (S r)_o for the 32 rows o of this warp: lanes read 4 consecutive entries of row o
-    const float4 r4 = reinterpret_cast<const float4*>(sh.xs)[lane];
-    float sr = 0.f;
-#pragma unroll 8
-    for (int u = 0; u < 32; ++u) {
-      const float4 p = reinterpret_cast<const float4*>(a.s + (size_t)(32 * warp + u) * D)[lane];
-      float t = p.x * r4.x;
-      t = fmaf(p.y, r4.y, t);
-      t = fmaf(p.z, r4.z, t);
-      t = fmaf(p.w, r4.w, t);
-      t = warp_sum(t);
-      if (lane == u) sr = t;
-    }
-    const int sigma = sr >= 0.f;
+    int sigma;
+    const __half rho = append_qjl(a, sh, x, nh, sh.tab[0][idx], i, lane, warp, sigma);
     if (L.kmerged) {
       pack_code(s, r | (s << 2) | (sigma << 3), kMergedNibble, lane, warp, sh.kw);
     } else {
@@ -241,9 +248,19 @@ __device__ void append_token(const DecodeArgs& a, int job) {
   __half nv16;
   encode_coord(a, sh, xv, sh.tab[3], L.vbits, i, lane, warp, nv16, idx, s, r);
   pack_code(s, r, L.vbits, lane, warp, sh.vw);
+  if (L.vqjl) {
+    // values with QJL: the same sketch of the value residual, signs in VS, norm in VR
+    int sigma;
+    const __half rho = append_qjl(a, sh, xv, nv16, sh.tab[2][idx], i, lane, warp, sigma);
+    const uint32_t bw = __ballot_sync(FULL, sigma);
+    if (lane == 0) sh.vsw[warp] = bw;
+    if (i == 0) reinterpret_cast<__half*>(blk + L.vr)[slot] = rho;
+  }
   __syncthreads();
   if (i < L.vbits)
     reinterpret_cast<uint4*>(blk + L.vc)[i * PT + slot] = reinterpret_cast<const uint4*>(sh.vw)[i];
+  if (L.vqjl && i == 0)
+    reinterpret_cast<uint4*>(blk + L.vs)[slot] = reinterpret_cast<const uint4*>(sh.vsw)[0];
   if (i == 0) reinterpret_cast<__half*>(blk + L.vn)[slot] = nv16;
 }
 
@@ -372,6 +389,8 @@ struct SmemSplit {
   float p[kRowsMax][kTile];
   uint32_t vcode[kTile][17];  // up to 16 words per token (+1 pad)
   float vnorm[kTile];
+  uint32_t vsig[kTile][4];    // values with QJL: the residual's sign bits
+  float vrho[kTile];          // and its stored norm
   float kmag[8], vmag[8];
   float sqsum[kRowsMax];
   float m[kRowsMax], l[kRowsMax], alpha[kRowsMax];
@@ -413,6 +432,11 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
   float acc[kRowsMax];
 #pragma unroll
   for (int r = 0; r < kRowsMax; ++r) acc[r] = 0.f;
+  // values with QJL: thread i also sums p_t ||r_v||_t (2 sigma_t,i - 1) over the tokens, the
+  // sign-space half of the value reconstruction (S^T is applied once, after the merge)
+  float accs[kRowsMax];
+#pragma unroll
+  for (int r = 0; r < kRowsMax; ++r) accs[r] = 0.f;
   __syncthreads();
 
   for (int tile0 = t_begin; tile0 < t_end; tile0 += kTile) {
@@ -489,12 +513,18 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
           sm.vcode[tid][4 * c + 2] = v4.z; sm.vcode[tid][4 * c + 3] = v4.w;
         }
         vn = __half2float(reinterpret_cast<const __half*>(blk + L.vn)[slot]);
+        if (L.vqjl) {
+          const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.vs)[slot];
+          sm.vsig[tid][0] = s4.x; sm.vsig[tid][1] = s4.y; sm.vsig[tid][2] = s4.z; sm.vsig[tid][3] = s4.w;
+          sm.vrho[tid] = __half2float(reinterpret_cast<const __half*>(blk + L.vr)[slot]);
+        }
       }
     } else if (!kScoresOnly) {
       for (int r = 0; r < R; ++r) sm.p[r][tid] = -CUDART_INF_F;
     }
     if (kScoresOnly) continue;
     sm.vnorm[tid] = valid ? vn : 0.f;
+    if (L.vqjl && !valid) sm.vrho[tid] = 0.f;
     __syncthreads();
     // ---- phase B: online softmax bookkeeping, warp per row
     for (int r = warp; r < R; r += 4) {
@@ -537,6 +567,18 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       for (int r = 0; r < kRowsMax; ++r)
         if (r < R) acc[r] = fmaf(sm.p[r][tt], val, acc[r]);
     }
+    if (L.vqjl) {
+      // thread j holds sign index i = j (m = d = blockDim)
+#pragma unroll
+      for (int r = 0; r < kRowsMax; ++r)
+        if (r < R) accs[r] *= sm.alpha[r];
+      for (int tt = 0; tt < nt; ++tt) {
+        const float sv = ((sm.vsig[tt][j >> 5] >> (j & 31)) & 1u) ? sm.vrho[tt] : -sm.vrho[tt];
+#pragma unroll
+        for (int r = 0; r < kRowsMax; ++r)
+          if (r < R) accs[r] = fmaf(sm.p[r][tt], sv, accs[r]);
+      }
+    }
     __syncthreads();
   }
   // ---- partials (the score-only variant stops with the scores)
@@ -546,6 +588,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       if (r < R) {
         const size_t pr = (row0 + r) * a.n_splits + split;
         a.part_acc[pr * D + tid] = acc[r];
+        if (L.vqjl) a.part_sig[pr * QM + tid] = accs[r];
         if (tid == 0) {
           a.part_ml[pr * 2] = sm.m[r];
           a.part_ml[pr * 2 + 1] = sm.l[r];
@@ -561,15 +604,17 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
 __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int total_rows) {
   // wait for the split kernel (launched as our programmatic predecessor) to finish
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ float os[D];
+  __shared__ float os[D], ss[QM];
   const int j = threadIdx.x;
   const int row = blockIdx.x;
   if (row >= total_rows) return;
+  const bool vqjl = a.cache.L.vqjl != 0;
   const float* ml = a.part_ml + (size_t)row * a.n_splits * 2;
   const float* pa = a.part_acc + (size_t)row * a.n_splits * D;
+  const float* ps = vqjl ? a.part_sig + (size_t)row * a.n_splits * QM : nullptr;
   float M = -CUDART_INF_F;
   for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, ml[2 * s]);
-  float l = 0.f, o = 0.f;
+  float l = 0.f, o = 0.f, osig = 0.f;
   if (M != -CUDART_INF_F) {
     for (int s = 0; s < a.n_splits; ++s) {
       const float ms = ml[2 * s];
@@ -577,9 +622,11 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int total_ro
       const float wgt = __expf(ms - M);
       l = fmaf(wgt, ml[2 * s + 1], l);
       o = fmaf(wgt, pa[(size_t)s * D + j], o);
+      if (vqjl) osig = fmaf(wgt, ps[(size_t)s * QM + j], osig);
     }
   }
   o = l > 0.f ? o / l : 0.f;
+  osig = l > 0.f ? osig / l : 0.f;
   float y;
   if (!a.dense) {
     // R^T = D H: butterflies in shared memory, then the sign flips
@@ -600,12 +647,20 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int total_ro
     for (int i = 0; i < D; ++i) acc = fmaf(a.pi[(size_t)i * D + j], os[i], acc);
     y = acc;
   }
+  if (vqjl) {
+    // values with QJL: + sqrt(pi/2)/m S^T (sum_t p_t ||r_v||_t (2 sigma_t - 1)) / l
+    ss[j] = osig;
+    __syncthreads();
+    float acc = 0.f;
+    for (int i = 0; i < QM; ++i) acc = fmaf(a.s[(size_t)i * D + j], ss[i], acc);
+    y = fmaf(kQjlScale, acc, y);
+  }
   a.out[(size_t)row * D + j] = y;
 }
 
 }  // namespace
 
-DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits) {
+DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits, int vqjl) {
   const size_t rows = (size_t)batch * q_heads * seq_q;
   DecodeWorkspace w;
   size_t off = 0;
@@ -613,6 +668,7 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   w.sq = off; off = align256(off + rows * QM * sizeof(float));
   w.part_acc = off; off = align256(off + rows * (size_t)n_splits * D * sizeof(float));
   w.part_ml = off; off = align256(off + rows * (size_t)n_splits * 2 * sizeof(float));
+  w.part_sig = off; off = align256(off + (vqjl ? rows * (size_t)n_splits * QM * sizeof(float) : 0));
   w.sq_int = off; off = align256(off + rows * QM * sizeof(int16_t));
   w.sq_scale = off; off = align256(off + rows * sizeof(float));
   w.sq_sum = off; off = align256(off + rows * sizeof(int));

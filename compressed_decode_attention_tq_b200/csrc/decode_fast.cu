@@ -825,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 bool fast_decode_supported(const DecodeArgs& a) {
   const Layout& L = a.cache.L;
   const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl);
-  const bool vok = L.vbits == 3 || L.vbits == 2;
+  const bool vok = (L.vbits == 3 || L.vbits == 2) && !L.vqjl;
   return kok && vok;
 }
 

@@ -34,6 +34,7 @@ static tq_status check_config(const tq_config* cfg) {
   if (cfg->value_bits < 1 || cfg->value_bits > 4)
     return fail(TQ_ERR_UNSUPPORTED, "value_bits must be in 1..4");
   if (cfg->key_qjl != 0 && cfg->key_qjl != 1) return fail(TQ_ERR_INVALID_ARG, "key_qjl must be 0 or 1");
+  if (cfg->value_qjl != 0 && cfg->value_qjl != 1) return fail(TQ_ERR_INVALID_ARG, "value_qjl must be 0 or 1");
   if (cfg->rotation != TQ_ROT_HADAMARD && cfg->rotation != TQ_ROT_DENSE)
     return fail(TQ_ERR_INVALID_ARG, "unknown rotation kind");
   return TQ_OK;
@@ -43,7 +44,7 @@ static tq_status check_params(const tq_config* cfg, const tq_params* p, bool nee
   if (!p) return fail(TQ_ERR_INVALID_ARG, "params is NULL");
   if (cfg->rotation == TQ_ROT_HADAMARD && !p->signs) return fail(TQ_ERR_INVALID_ARG, "params.signs is NULL");
   if (cfg->rotation == TQ_ROT_DENSE && !p->pi) return fail(TQ_ERR_INVALID_ARG, "params.pi is NULL");
-  if (need_s && cfg->key_qjl && !p->s) return fail(TQ_ERR_INVALID_ARG, "params.s is NULL");
+  if (need_s && (cfg->key_qjl || cfg->value_qjl) && !p->s) return fail(TQ_ERR_INVALID_ARG, "params.s is NULL");
   if (!p->k_centroids || !p->v_centroids) return fail(TQ_ERR_INVALID_ARG, "centroid pointer is NULL");
   return TQ_OK;
 }
@@ -67,7 +68,7 @@ static tqk::CacheRef cache_ref(const tq_config* cfg, const tq_cache* c, int32_t 
   r.batch = c->batch;
   r.kv_heads = c->kv_heads;
   r.layer = layer;
-  r.L = tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits);
+  r.L = tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl);
   return r;
 }
 
@@ -77,7 +78,7 @@ using namespace tqi;
 
 extern "C" {
 
-int32_t tq_version(void) { return 100; }
+int32_t tq_version(void) { return 101; }
 
 const char* tq_status_str(tq_status st) {
   switch (st) {
@@ -101,7 +102,7 @@ tq_status tq_validate_config(const tq_config* cfg) {
 
 size_t tq_page_bytes(const tq_config* cfg) {
   if (check_config(cfg) != TQ_OK) return 0;
-  return (size_t)tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits).bytes;
+  return (size_t)tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl).bytes;
 }
 
 tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
@@ -164,7 +165,7 @@ tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, voi
 size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int32_t q_heads, int32_t seq_q,
                                  int32_t n_splits) {
   if (check_config(cfg) != TQ_OK || batch < 1 || q_heads < 1 || seq_q < 1 || n_splits < 1) return 0;
-  return tqk::decode_workspace(batch, q_heads, seq_q, n_splits).total;
+  return tqk::decode_workspace(batch, q_heads, seq_q, n_splits, cfg->value_qjl).total;
 }
 
 static tq_status decode_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
@@ -185,7 +186,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   if (n_splits < 1 || n_splits > 1024) return fail(TQ_ERR_INVALID_ARG, "n_splits must be in 1..1024");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
     return fail(TQ_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const tqk::DecodeWorkspace w = tqk::decode_workspace(cache->batch, q_heads, seq_q, n_splits);
+  const tqk::DecodeWorkspace w = tqk::decode_workspace(cache->batch, q_heads, seq_q, n_splits, cfg->value_qjl);
   if (workspace_bytes < w.total) return fail(TQ_ERR_INVALID_ARG, "workspace too small");
   char* ws = static_cast<char*>(workspace);
   a.cache = cache_ref(cfg, cache, layer);
@@ -208,6 +209,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.sq = reinterpret_cast<float*>(ws + w.sq);
   a.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
   a.part_ml = reinterpret_cast<float*>(ws + w.part_ml);
+  a.part_sig = cfg->value_qjl ? reinterpret_cast<float*>(ws + w.part_sig) : nullptr;
   a.sq_int = reinterpret_cast<int16_t*>(ws + w.sq_int);
   a.sq_scale = reinterpret_cast<float*>(ws + w.sq_scale);
   a.sq_sum = reinterpret_cast<int*>(ws + w.sq_sum);
@@ -235,7 +237,7 @@ static tq_status check_append(const tq_config* cfg, const tq_params* params, con
   if (n_new < 1) return fail(TQ_ERR_INVALID_ARG, "n_new must be >= 1");
   if ((int64_t)cache->batch * cache->kv_heads * n_new > (int64_t)1 << 30)
     return fail(TQ_ERR_INVALID_ARG, "batch * kv_heads * n_new too large");
-  if (cfg->key_qjl && (reinterpret_cast<uintptr_t>(params->s) & 15))
+  if ((cfg->key_qjl || cfg->value_qjl) && (reinterpret_cast<uintptr_t>(params->s) & 15))
     return fail(TQ_ERR_INVALID_ARG, "params->s must be 16-byte aligned");
   if (cfg->rotation == TQ_ROT_DENSE && (reinterpret_cast<uintptr_t>(params->pi) & 15))
     return fail(TQ_ERR_INVALID_ARG, "params->pi must be 16-byte aligned");

@@ -20,13 +20,16 @@ struct Layout {
   int kbits, vbits, qjl;
   int kmerged;  // 3-bit keys with QJL: one 4-bit field (r0, r1, s, sigma) per coordinate
   int kchunks;  // 16-byte chunks of one token's key bit string
+  int vqjl;     // values carry the QJL signs of their residual (VS) and its norm (VR)
+  int vs, vr;
 };
 
-__host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits) {
+__host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits, int vqjl = 0) {
   Layout L;
   L.kbits = kbits;
   L.vbits = vbits;
   L.qjl = qjl;
+  L.vqjl = vqjl;
   L.kmerged = (qjl && kbits == 3) ? 1 : 0;
   L.kchunks = L.kmerged ? 4 : kbits;
   int off = 0;
@@ -36,6 +39,8 @@ __host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits) {
   L.kc = off; off += L.kchunks * 16 * PT;
   L.ks = off; off += (qjl && !L.kmerged) ? (QM / 8) * PT : 0;
   L.vc = off; off += vbits * (D / 8) * PT;
+  L.vs = off; off += vqjl ? (QM / 8) * PT : 0;
+  L.vr = off; off += vqjl ? 2 * PT : 0;
   L.bytes = off;
   return L;
 }

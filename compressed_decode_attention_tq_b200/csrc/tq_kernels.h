@@ -29,6 +29,7 @@ struct DecodeArgs {
   float* sq;        // [B*Hq*seq_q][QM] workspace
   float* part_acc;  // [B*Hq*seq_q][n_splits][D] workspace
   float* part_ml;   // [B*Hq*seq_q][n_splits][2] workspace
+  float* part_sig;  // [B*Hq*seq_q][n_splits][QM] workspace (values with QJL): sum_t p_t ||r_v|| (2 sigma - 1)
   int16_t* sq_int;  // [B*Hq*seq_q][QM] workspace: S q in 16-bit fixed point
   float* sq_scale;  // [B*Hq*seq_q] workspace: S q ~= sq_int * sq_scale (a power of two)
   int* sq_sum;      // [B*Hq*seq_q] workspace: sum_i sq_int
@@ -68,9 +69,9 @@ cudaError_t launch_prepare_operands(const float* signs, const float* s, int qjl,
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {
-  size_t qrot, sq, part_acc, part_ml, sq_int, sq_scale, sq_sum, q8, q8_scale, counter, total;
+  size_t qrot, sq, part_acc, part_ml, part_sig, sq_int, sq_scale, sq_sum, q8, q8_scale, counter, total;
 };
-DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits);
+DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits, int vqjl);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 bool fast_decode_supported(const DecodeArgs& a);

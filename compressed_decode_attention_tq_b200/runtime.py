@@ -34,10 +34,10 @@ class PagedKV:
     def __init__(self, *, batch: int, kv_heads: int, num_pages: int, block_table, key_bits: int,
                  key_qjl: bool, value_bits: int, rotation: int = TQ_ROT_HADAMARD,
                  num_layers: int = 1, signs=None, pi=None, s=None, codebooks=None,
-                 device: str = "cuda", prepared_operands: bool = True):
+                 device: str = "cuda", prepared_operands: bool = True, value_qjl: bool = False):
         self.device = torch.device(device)
         self.cfg = make_config(key_bits=key_bits, key_qjl=key_qjl, value_bits=value_bits,
-                               rotation=rotation)
+                               rotation=rotation, value_qjl=value_qjl)
         self.block_bytes = page_bytes(self.cfg)
         if self.block_bytes == 0:
             raise TQError(2, "PagedKV", "unsupported configuration")

@@ -49,6 +49,8 @@
  *   KC      key codes, key_bits*d/8 bytes per token    key_bits*16*P  (merged keys: 64*P)
  *   KS      QJL sign bits, m/8 bytes per token          16*P   (QJL keys, not merged)
  *   VC      value codes                               value_bits*16*P
+ *   VS      QJL sign bits of the value residual        16*P   (value_qjl)
+ *   VR      stored ||r_v|| (fp16) per token            2P     (value_qjl)
  *
  *   A code region stores each token's bytes as 16-byte chunks, chunk-major:
  *   chunk c of slot t is at region byte (c*P + t)*16.  A token's chunks,
@@ -65,6 +67,7 @@
  *   Merged keys (key_bits = 3 with QJL): bits 4j..4j+3 = r0, r1, s, sigma_j, where
  *   sigma_i = [(S r)_i >= 0] (sign(0) is stored as +1); there is no KS region.
  *   Other QJL keys: bit i of the KS chunk = sigma_i.
+ *   Values with QJL: bit i of the VS chunk = [(S r_v)_i >= 0], r_v = v - v_mse.
  *   Slots past a sequence's length are never read and their bytes unspecified.
  */
 #ifndef TQ_H_
@@ -101,7 +104,8 @@ typedef enum tq_density { TQ_DENSITY_BETA = 0, TQ_DENSITY_GAUSS = 1 } tq_density
 typedef enum tq_rotation_kind { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rotation_kind;
 typedef enum tq_dtype { TQ_F16 = 0, TQ_F32 = 1 } tq_dtype;
 
-/* Configuration of one cache ([TQKV] TurboQuantConfig: bits, rotation, QJL mode). */
+/* Configuration of one cache ([TQKV] TurboQuantConfig: bits, rotation, QJL mode).
+ * Callers set every field (value_qjl = 0 for the format of version 1.00). */
 typedef struct tq_config {
   int32_t head_dim;     /* d, must be 128                                             */
   int32_t key_bits;     /* b_k: bits of the key MSE stage, 1..4                        */
@@ -110,6 +114,11 @@ typedef struct tq_config {
   int32_t value_bits;   /* b_v: bits of the value MSE stage, 1..4                      */
   int32_t page_tokens;  /* P: tokens per page, must be 256                             */
   int32_t rotation;     /* tq_rotation_kind                                            */
+  int32_t value_qjl;    /* 1: values carry the 1-bit QJL sketch of their residual and
+                           ||r_v|| (TurboQuant_prod on the value cache, [MOBILINT]
+                           "Two-Stage Approach": the value is reconstructed as
+                           v_mse + sqrt(pi/2)/m ||r_v|| S^T (2 sigma_v - 1)); served by
+                           the general (CUDA-core) kernels                             */
 } tq_config;
 
 /* Random inputs of the method and the codebooks, all device memory, fp32.
@@ -119,7 +128,7 @@ typedef struct tq_config {
 typedef struct tq_params {
   const float* signs;         /* [d] +-1 diagonal of D (TQ_ROT_HADAMARD), else unused     */
   const float* pi;            /* [d*d] Pi, row-major, y = Pi u (TQ_ROT_DENSE), else unused */
-  const float* s;             /* [m*d] S, row-major; unused unless key_qjl.  When
+  const float* s;             /* [m*d] S, row-major; unused unless key_qjl or value_qjl.  When
                                  tq_compress_kv forms its operands itself (operands
                                  NULL), every entry must be exactly representable in
                                  fp16 (checked on the device, TQ_ERR_INVALID_ARG)      */
@@ -226,6 +235,7 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int
  *   score_t = ( ||k||_t <R q, c_k[idx_t]>
  *               + [QJL] ||r||_t sqrt(pi/2)/m <S q, 2 sigma_t - 1> ) / sqrt(d)
  *   out     = R^T sum_t softmax(score)_t ||v||_t c_v[idx_v,t]
+ *             [+ with value_qjl: sqrt(pi/2)/m S^T sum_t softmax(score)_t ||r_v||_t (2 sigma_v,t - 1)]
  * over t < seq_lens[b] (no causal mask between the seq_q rows; an empty sequence
  * gives 0).  The sequence is cut into n_splits contiguous ranges processed in
  * parallel and merged by their log-sum-exp.
@@ -310,7 +320,8 @@ TQ_API tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params,
 
 /* Decompress ([CUTILE] "indices -> centroids -> un-rotate -> rescale"):
  * k_hat = ||k|| R^T c_k[idx] (the MSE part k_mse for QJL keys) and
- * v_hat = ||v|| R^T c_v[idx_v], for tokens t < seq_lens[b]; rows past the
+ * v_hat = ||v|| R^T c_v[idx_v] (the MSE part for values with QJL), for tokens
+ * t < seq_lens[b]; rows past the
  * length are left untouched.
  *   k_hat, v_hat  device float [batch][kv_heads][max_len][d] (either may be NULL) */
 TQ_API tq_status tq_decompress(const tq_config* cfg, const tq_params* params, const tq_cache* cache,

@@ -60,12 +60,13 @@ def setup(w: wl.Workload, layers=(0,), prepared_operands=True, compress_lens=Non
     rin = wl.rotation_inputs(w)
     run = Run(w=w, lens=lens, bt=bt, npages=npages, rin=rin,
               R=orot.rotation_matrix(w.rotation, rin["signs"], rin["pi"]),
-              fmt=olay.Format(key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits),
+              fmt=olay.Format(key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits,
+                              value_qjl=w.value_qjl),
               ck=None, kb=None, cv=None, vb=None)
     run.ck, run.kb = ocb.codebook_f32(w.key_bits, 128)
     run.cv, run.vb = ocb.codebook_f32(w.value_bits, 128)
     run.kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
-                     key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits,
+                     key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits, value_qjl=w.value_qjl,
                      rotation=w.rotation, num_layers=max(layers) + 1, signs=rin["signs"],
                      pi=rin["pi"], s=rin["s"], prepared_operands=prepared_operands)
     run.K, run.V = {}, {}
@@ -100,25 +101,37 @@ class CompressReport:
     norm_fail: int = 0
 
 
-def compare_compress_rows(fmt, u, K, V, R, ck, kb, cv, vb, S, rep: CompressReport):
-    """Compares unpacked GPU codes u (tokens in the order of the rows) with the oracle's
-    compression of the same float64 rows K, V [n][d]."""
-    kc = (oq.compress_prod(K, R, ck, kb, S) if fmt.key_qjl else oq.compress_mse(K, R, ck, kb))
-    vc = oq.compress_mse(V, R, cv, vb)
+def _check_qjl(gpu_sigma, gpu_rnorm, comp, mis, rep):
+    """Residual norms and sign bits of the tokens whose indices all agree (a token whose
+    index differs inside the band has a different residual, so its signs are skipped)."""
+    ok_tok = ~mis
+    rep.sign_tokens_skipped += int(np.sum(mis))
+    rep.norm_fail += int(np.sum(~close(gpu_rnorm[ok_tok], comp.rnorm[ok_tok])))
+    diff = (gpu_sigma != comp.sigma) & ok_tok[:, None]
+    band = np.abs(comp.sr) <= SIGN_BAND * comp.sr_scale
+    rep.sign_mismatch_in_band += int(np.sum(diff & band))
+    rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
+
+
+def _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep):
+    kc = oq.compress_prod(K, R, ck, kb, S) if fmt.key_qjl else oq.compress_mse(K, R, ck, kb)
+    vc = oq.compress_prod(V, R, cv, vb, S) if fmt.value_qjl else oq.compress_mse(V, R, cv, vb)
     rep.tokens += K.shape[0]
     kmis = _check_idx(u.k_idx, kc, kb, rep)
-    _check_idx(u.v_idx, vc, vb, rep)
+    vmis = _check_idx(u.v_idx, vc, vb, rep)
     rep.norm_fail += int(np.sum(~close(u.k_norm, kc.norm)))
     rep.norm_fail += int(np.sum(~close(u.v_norm, vc.norm)))
     if fmt.key_qjl:
-        ok_tok = ~kmis
-        rep.sign_tokens_skipped += int(np.sum(kmis))
-        rep.norm_fail += int(np.sum(~close(u.k_rnorm[ok_tok], kc.rnorm[ok_tok])))
-        diff = (u.k_sigma != kc.sigma) & ok_tok[:, None]
-        band = np.abs(kc.sr) <= SIGN_BAND * kc.sr_scale
-        rep.sign_mismatch_in_band += int(np.sum(diff & band))
-        rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
+        _check_qjl(u.k_sigma, u.k_rnorm, kc, kmis, rep)
+    if fmt.value_qjl:
+        _check_qjl(u.v_sigma, u.v_rnorm, vc, vmis, rep)
     return rep
+
+
+def compare_compress_rows(fmt, u, K, V, R, ck, kb, cv, vb, S, rep: CompressReport):
+    """Compares unpacked GPU codes u (tokens in the order of the rows) with the oracle's
+    compression of the same float64 rows K, V [n][d]."""
+    return _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep)
 
 
 def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport = None):
@@ -128,26 +141,12 @@ def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport =
     n = int(run.lens[b])
     u = olay.read_sequence(pages, run.fmt, layer, h, run.bt[b], n)
     sel = np.arange(n) if tokens is None else np.asarray(tokens)
-    K = run.K[layer][b, h][sel]
-    V = run.V[layer][b, h][sel]
-    S = run.rin["s"]
-    kc = (oq.compress_prod(K, run.R, run.ck, run.kb, S) if run.w.key_qjl
-          else oq.compress_mse(K, run.R, run.ck, run.kb))
-    vc = oq.compress_mse(V, run.R, run.cv, run.vb)
-    rep.tokens += len(sel)
-    kmis = _check_idx(u.k_idx[sel], kc, run.kb, rep)
-    _check_idx(u.v_idx[sel], vc, run.vb, rep)
-    rep.norm_fail += int(np.sum(~close(u.k_norm[sel], kc.norm)))
-    rep.norm_fail += int(np.sum(~close(u.v_norm[sel], vc.norm)))
-    if run.w.key_qjl:
-        ok_tok = ~kmis
-        rep.sign_tokens_skipped += int(np.sum(kmis))
-        rep.norm_fail += int(np.sum(~close(u.k_rnorm[sel][ok_tok], kc.rnorm[ok_tok])))
-        diff = (u.k_sigma[sel] != kc.sigma) & ok_tok[:, None]
-        band = np.abs(kc.sr) <= SIGN_BAND * kc.sr_scale
-        rep.sign_mismatch_in_band += int(np.sum(diff & band))
-        rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
-    return rep
+    sub = olay.Unpacked(k_idx=u.k_idx[sel], k_norm=u.k_norm[sel], v_idx=u.v_idx[sel], v_norm=u.v_norm[sel])
+    for f in ("k_rnorm", "k_sigma", "v_rnorm", "v_sigma"):
+        if getattr(u, f) is not None:
+            setattr(sub, f, getattr(u, f)[sel])
+    return _compare_unpacked(run.fmt, sub, run.K[layer][b, h][sel], run.V[layer][b, h][sel], run.R,
+                             run.ck, run.kb, run.cv, run.vb, run.rin["s"], rep)
 
 
 def _check_idx(gpu_idx, comp, boundaries, rep):
@@ -161,7 +160,7 @@ def _check_idx(gpu_idx, comp, boundaries, rep):
 
 def oracle_decode(run, pages, layer, q, heads=None):
     return oatt.decode(pages, run.fmt, layer, q, run.bt, run.lens, run.R, run.ck, run.cv,
-                       run.rin["s"] if run.w.key_qjl else None, heads=heads)
+                       run.rin["s"] if (run.w.key_qjl or run.w.value_qjl) else None, heads=heads)
 
 
 def oracle_scores(run, pages, layer, q, b, h):

@@ -77,14 +77,17 @@ def test_page_bytes_match_format(tq, packing_golden):
     for kb in range(1, 5):
         for vb in range(1, 5):
             for qjl in (False, True):
-                cfg = tq.make_config(key_bits=kb, key_qjl=qjl, value_bits=vb)
-                fmt = olay.Format(key_bits=kb, key_qjl=qjl, value_bits=vb)
-                assert tq.page_bytes(cfg) == fmt.block_bytes
+                for vqjl in (False, True):
+                    cfg = tq.make_config(key_bits=kb, key_qjl=qjl, value_bits=vb, value_qjl=vqjl)
+                    fmt = olay.Format(key_bits=kb, key_qjl=qjl, value_bits=vb, value_qjl=vqjl)
+                    assert tq.page_bytes(cfg) == fmt.block_bytes
+    g = packing_golden["c2_value_qjl_regions"]
+    assert tq.page_bytes(tq.make_config(key_bits=3, key_qjl=True, value_bits=3, value_qjl=True)) == g["total"]
 
 
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 64, 2), ("qjl_m", 64, 2), ("page_tokens", 128, 2), ("key_bits", 5, 2),
-    ("value_bits", 0, 2), ("key_qjl", 2, 1), ("rotation", 7, 1)])
+    ("value_bits", 0, 2), ("key_qjl", 2, 1), ("rotation", 7, 1), ("value_qjl", 3, 1)])
 def test_validate_config_rejects(tq, field, value, code):
     cfg = tq.make_config()
     assert tq.validate_config(cfg) == 0
@@ -100,6 +103,9 @@ def test_workspace_bytes(tq):
     assert nb >= rows * (128 + 128 + 16 * 130) * 4
     assert nb % 256 == 0
     assert tq.decode_workspace_bytes(cfg, 1, 32, 1, 0) == 0
+    # values with QJL add the sign-space partials: m floats per query row and split
+    vq = tq.make_config(value_qjl=True)
+    assert tq.decode_workspace_bytes(vq, 1, 32, 1, 16) >= nb + rows * 16 * 128 * 4
 
 
 def test_host_argument_errors_do_not_launch(tq):

@@ -40,6 +40,11 @@ CASES = {
     "k4qjl_v1_dense": (lambda: wl.config2(kv_heads=1, q_heads=3, max_len=300, key_bits=4,
                                           value_bits=1, rotation=wl.ROT_DENSE, rot_seed=9,
                                           n_splits=1, name="k4qjl_v1_dense"), (3,)),
+    # values with QJL
+    "c2_vqjl": (lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1283, n_splits=4, value_qjl=True,
+                                   name="c2_vqjl"), (1, 3)),
+    "c3_vqjl_dense": (lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=2, value_qjl=True,
+                                         name="c3_vqjl_dense"), (2,)),
 }
 
 
@@ -85,7 +90,7 @@ def _check_old_tokens_unchanged(run, before, after, start):
             n = int(start[b])
             u0 = olay.read_sequence(before, run.fmt, 0, h, run.bt[b], n)
             u1 = olay.read_sequence(after, run.fmt, 0, h, run.bt[b], n)
-            for f in ("k_idx", "v_idx", "k_norm", "v_norm", "k_rnorm", "k_sigma"):
+            for f in ("k_idx", "v_idx", "k_norm", "v_norm", "k_rnorm", "k_sigma", "v_rnorm", "v_sigma"):
                 a0, a1 = getattr(u0, f), getattr(u1, f)
                 if a0 is not None:
                     np.testing.assert_array_equal(a0, a1, err_msg=f"{f} of b={b} h={h} changed")

@@ -24,6 +24,12 @@ SMALL = {
     "k4qjl_v1_dense": lambda: wl.config2(kv_heads=1, q_heads=3, max_len=300, key_bits=4,
                                          value_bits=1, rotation=wl.ROT_DENSE, rot_seed=9,
                                          n_splits=1, name="k4qjl_v1_dense"),
+    # values with QJL (TurboQuant_prod on the value cache): with merged QJL keys under HD,
+    # and with MSE-only keys under a dense rotation (the value sketch alone)
+    "c2_vqjl": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4, value_qjl=True,
+                                  name="c2_vqjl"),
+    "c3_vqjl_dense": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3, value_qjl=True,
+                                        name="c3_vqjl_dense"),
 }
 
 

@@ -95,6 +95,7 @@ class Workload:
     outlier_scale: float = 1.0
     outlier_seed: int = 3
     min_len: int = 0
+    value_qjl: bool = False        # values carry the QJL sketch of their residual too
 
     @property
     def group(self) -> int:
