@@ -27,15 +27,22 @@ def build(verbose: bool = False, extra: list[str] | None = None) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"),
-               "-I", os.path.join(PKG, "csrc"), "-c", src, "-o", obj]
+        cmds.append([nvcc, *NVCC_FLAGS, *(extra or []), "-I", os.path.join(ROOT, "include"),
+                     "-I", os.path.join(PKG, "csrc"), "-c", src, "-o", obj])
+        objs.append(obj)
+    # the translation units are independent: compile them side by side
+    from concurrent.futures import ThreadPoolExecutor
+
+    def compile_one(cmd):
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-        objs.append(obj)
+
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        list(ex.map(compile_one, cmds))
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs,
            "-Xcompiler", "-fvisibility=hidden"]
     if verbose:

@@ -396,8 +396,13 @@ struct SmemSplit {
   float m[kRowsMax], l[kRowsMax], alpha[kRowsMax];
 };
 
-template <bool kScoresOnly>
+// Key formats of the split kernel's template: b-bit codes (1..4) or the merged 3-bit + QJL
+// nibbles; RB: the smallest of 4, 8, 32 at least R (the per-row loops run to RB).
+constexpr int kKeyMerged = 5;
+
+template <bool kScoresOnly, int KF, int RB>
 __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
+  static_assert(QM == D, "the QJL sum shares the coordinate loop");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SmemSplit& sm = *reinterpret_cast<SmemSplit*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -429,14 +434,14 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
   const int cp = (npages + a.n_splits - 1) / a.n_splits;
   const int t_begin = min(n_eff, split * cp * PT);
   const int t_end = min(n_eff, (split + 1) * cp * PT);
-  float acc[kRowsMax];
+  float acc[RB];
 #pragma unroll
-  for (int r = 0; r < kRowsMax; ++r) acc[r] = 0.f;
+  for (int r = 0; r < RB; ++r) acc[r] = 0.f;
   // values with QJL: thread i also sums p_t ||r_v||_t (2 sigma_t,i - 1) over the tokens, the
   // sign-space half of the value reconstruction (S^T is applied once, after the merge)
-  float accs[kRowsMax];
+  float accs[RB];
 #pragma unroll
-  for (int r = 0; r < kRowsMax; ++r) accs[r] = 0.f;
+  for (int r = 0; r < RB; ++r) accs[r] = 0.f;
   __syncthreads();
 
   for (int tile0 = t_begin; tile0 < t_end; tile0 += kTile) {
@@ -457,45 +462,73 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       }
     }
     if (valid) {
-      uint32_t kw[16];
-      for (int c = 0; c < L.kchunks; ++c) {
-        const uint4 v4 = reinterpret_cast<const uint4*>(blk + L.kc)[c * PT + slot];
-        kw[4 * c] = v4.x; kw[4 * c + 1] = v4.y; kw[4 * c + 2] = v4.z; kw[4 * c + 3] = v4.w;
+      // the token's key, 32 coordinates at a time: the words holding coordinates
+      // 32q..32q+31 sit in registers and every field below has a constant position
+      float dot[RB], qj[RB];
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        dot[r] = 0.f;
+        qj[r] = 0.f;
       }
-      float dot[kRowsMax];
-#pragma unroll
-      for (int r = 0; r < kRowsMax; ++r) dot[r] = 0.f;
-      uint32_t sw[4] = {0u, 0u, 0u, 0u};
-      for (int j = 0; j < D; ++j) {
-        int s, rk, sig;
-        key_fields(kw, L, j, s, rk, sig);
-        sw[j >> 5] |= (uint32_t)sig << (j & 31);
-        const float val = s ? sm.kmag[rk] : -sm.kmag[rk];
-#pragma unroll
-        for (int r = 0; r < kRowsMax; ++r)
-          if (r < R) dot[r] = fmaf(sm.qrot[r][j], val, dot[r]);
-      }
-      const float kn = __half2float(reinterpret_cast<const __half*>(blk + L.kn)[slot]);
-      float qj[kRowsMax];
-#pragma unroll
-      for (int r = 0; r < kRowsMax; ++r) qj[r] = 0.f;
-      float rho = 0.f;
-      if (L.qjl) {
-        if (!L.kmerged) {
-          const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.ks)[slot];
-          sw[0] = s4.x; sw[1] = s4.y; sw[2] = s4.z; sw[3] = s4.w;
+      const uint8_t* kcb = blk + L.kc + (size_t)slot * 16;
+      const bool qjl = L.qjl != 0;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t g[4] = {0u, 0u, 0u, 0u}, sp = 0u, sgw = 0u;
+        if constexpr (KF == 1) {
+          g[0] = *reinterpret_cast<const uint32_t*>(kcb + 4 * q);
+        } else if constexpr (KF == 2 || KF == 3) {
+          const uint2 v2 = *reinterpret_cast<const uint2*>(kcb + (q >> 1) * PT * 16 + (q & 1) * 8);
+          g[0] = v2.x;
+          g[1] = v2.y;
+          if constexpr (KF == 3) sp = *reinterpret_cast<const uint32_t*>(kcb + 2 * PT * 16 + 4 * q);
+        } else {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(kcb + q * PT * 16);
+          g[0] = v4.x; g[1] = v4.y; g[2] = v4.z; g[3] = v4.w;
         }
-        rho = __half2float(reinterpret_cast<const __half*>(blk + L.kr)[slot]);
-        for (int i = 0; i < QM; ++i) {
-          if ((sw[i >> 5] >> (i & 31)) & 1u) {
+        if (KF != kKeyMerged && qjl) sgw = *reinterpret_cast<const uint32_t*>(blk + L.ks + (size_t)slot * 16 + 4 * q);
 #pragma unroll
-            for (int r = 0; r < kRowsMax; ++r)
-              if (r < R) qj[r] += sm.sq[r][i];
+        for (int jj = 0; jj < 32; ++jj) {
+          int s, rk, sig;
+          if constexpr (KF == 1) {
+            s = (g[0] >> jj) & 1;
+            rk = 0;
+          } else if constexpr (KF == 2) {
+            const uint32_t f = (g[jj >> 4] >> ((jj & 15) * 2)) & 3u;
+            rk = f & 1;
+            s = f >> 1;
+          } else if constexpr (KF == 3) {
+            rk = (g[jj >> 4] >> ((jj & 15) * 2)) & 3u;
+            s = (sp >> (sign_plane_pos(jj) & 31)) & 1;
+          } else if constexpr (KF == 4) {
+            const uint32_t f = (g[jj >> 3] >> ((jj & 7) * 4)) & 15u;
+            rk = f & 7;
+            s = f >> 3;
+          } else {
+            const uint32_t f = (g[jj >> 3] >> ((jj & 7) * 4)) & 15u;
+            rk = f & 3;
+            s = (f >> 2) & 1;
+          }
+          if constexpr (KF == kKeyMerged)
+            sig = (g[jj >> 3] >> ((jj & 7) * 4 + 3)) & 1;
+          else
+            sig = (sgw >> jj) & 1;
+          const int j = 32 * q + jj;
+          const float val = s ? sm.kmag[rk] : -sm.kmag[rk];
+#pragma unroll
+          for (int r = 0; r < RB; ++r)
+            if (r < R) dot[r] = fmaf(sm.qrot[r][j], val, dot[r]);
+          if (qjl && sig) {
+#pragma unroll
+            for (int r = 0; r < RB; ++r)
+              if (r < R) qj[r] += sm.sq[r][j];
           }
         }
       }
+      const float kn = __half2float(reinterpret_cast<const __half*>(blk + L.kn)[slot]);
+      const float rho = qjl ? __half2float(reinterpret_cast<const __half*>(blk + L.kr)[slot]) : 0.f;
 #pragma unroll
-      for (int r = 0; r < kRowsMax; ++r) {
+      for (int r = 0; r < RB; ++r) {
         if (r < R) {
           float sc = kn * dot[r];
           if (L.qjl) sc = fmaf(rho * kQjlScale, 2.f * qj[r] - sm.sqsum[r], sc);
@@ -556,7 +589,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     // ---- phase C: thread = coordinate j, V accumulation in rotated space
     const int j = tid;
 #pragma unroll
-    for (int r = 0; r < kRowsMax; ++r)
+    for (int r = 0; r < RB; ++r)
       if (r < R) acc[r] *= sm.alpha[r];
     const int nt = min(kTile, t_end - tile0);
     for (int tt = 0; tt < nt; ++tt) {
@@ -564,18 +597,18 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       code_fields(sm.vcode[tt], L.vbits, j, s, rk);
       const float val = (s ? sm.vmag[rk] : -sm.vmag[rk]) * sm.vnorm[tt];
 #pragma unroll
-      for (int r = 0; r < kRowsMax; ++r)
+      for (int r = 0; r < RB; ++r)
         if (r < R) acc[r] = fmaf(sm.p[r][tt], val, acc[r]);
     }
     if (L.vqjl) {
       // thread j holds sign index i = j (m = d = blockDim)
 #pragma unroll
-      for (int r = 0; r < kRowsMax; ++r)
+      for (int r = 0; r < RB; ++r)
         if (r < R) accs[r] *= sm.alpha[r];
       for (int tt = 0; tt < nt; ++tt) {
         const float sv = ((sm.vsig[tt][j >> 5] >> (j & 31)) & 1u) ? sm.vrho[tt] : -sm.vrho[tt];
 #pragma unroll
-        for (int r = 0; r < kRowsMax; ++r)
+        for (int r = 0; r < RB; ++r)
           if (r < R) accs[r] = fmaf(sm.p[r][tt], sv, accs[r]);
       }
     }
@@ -584,7 +617,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
   // ---- partials (the score-only variant stops with the scores)
   if constexpr (!kScoresOnly) {
 #pragma unroll
-    for (int r = 0; r < kRowsMax; ++r) {
+    for (int r = 0; r < RB; ++r) {
       if (r < R) {
         const size_t pr = (row0 + r) * a.n_splits + split;
         a.part_acc[pr * D + tid] = acc[r];
@@ -680,20 +713,31 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   return w;
 }
 
+template <bool kScoresOnly, int KF>
+static void (*split_for_rows(int rows))(DecodeArgs) {
+  if (rows <= 4) return split_kernel<kScoresOnly, KF, 4>;
+  if (rows <= 8) return split_kernel<kScoresOnly, KF, 8>;
+  return split_kernel<kScoresOnly, KF, kRowsMax>;
+}
+
+template <bool kScoresOnly>
+static void (*split_for(const Layout& L, int rows))(DecodeArgs) {
+  if (L.kmerged) return split_for_rows<kScoresOnly, kKeyMerged>(rows);
+  switch (L.kbits) {
+    case 1: return split_for_rows<kScoresOnly, 1>(rows);
+    case 2: return split_for_rows<kScoresOnly, 2>(rows);
+    case 3: return split_for_rows<kScoresOnly, 3>(rows);
+    default: return split_for_rows<kScoresOnly, 4>(rows);
+  }
+}
+
 static cudaError_t launch_split(const DecodeArgs& a, cudaStream_t stream, bool scores_only) {
   const size_t smem = sizeof(SmemSplit);
   dim3 grid(scores_only ? 1 : a.n_splits, a.cache.kv_heads, a.cache.batch);
-  if (scores_only) {
-    auto k = split_kernel<true>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 128, smem, stream>>>(a);
-  } else {
-    auto k = split_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, 128, smem, stream>>>(a);
-  }
+  void (*k)(DecodeArgs) = scores_only ? split_for<true>(a.cache.L, a.rows) : split_for<false>(a.cache.L, a.rows);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, 128, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
