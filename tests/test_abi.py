@@ -185,3 +185,17 @@ def test_append_argument_errors_do_not_launch(tq):
     st = tq.lib.tq_append_attend_decode(by(cfg), by(params), by(cache), 0, p, p, 0, 1, p, 0, 4, 1, p, 2,
                                         p, nb, None, None, None)
     assert st == tq.TQ_ERR_INVALID_ARG and "out" in tq.last_error()
+
+
+def test_plain_c_caller_links_and_runs(tq, tmp_path):
+    # the boundary is a C ABI: a C program that includes only tq.h and links libtq.so
+    # compiles with gcc and passes its host-side checks
+    exe = tmp_path / "c_abi_host"
+    libdir = os.path.dirname(tq.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c_abi_host.c"), "-o", str(exe), "-L", libdir, "-ltq",
+           "-Wl,-rpath," + libdir, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert "FAIL" not in out.stdout and out.stdout.count("ok ") >= 12
