@@ -20,7 +20,7 @@ Sources:
     term2 (QJL correction)"; "Full pipeline: scores -> softmax -> weighted V
     sum"; "Scores should be scaled by 1/sqrt(d)"; the decode case seq_q = 1.
 
-Readings (also in DESIGN.md):
+Readings taken where the pages are open:
   * grouped-query attention: query head h reads kv head floor(h / G), G = q_heads / kv_heads;
   * every query position of a block sees the whole cached sequence (no causal mask);
   * an empty sequence gives an all-zero output;

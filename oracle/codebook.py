@@ -17,7 +17,7 @@ Source: "TurboQuant explained" (Mobilint blog)
     float32 tensors, centroids (2^b,) and boundaries (2^b - 1,).
   * "tq-kv" crate documentation, module codebook: a Gaussian-fitted variant.
 
-Readings taken where the pages are open (listed in the design doc as well):
+Readings taken where the pages are open:
   * the integrals are computed with closed forms: the cell mass is a difference
     of the regularized incomplete Beta function, and the first moment of
     f_X has the antiderivative -K (1 - t^2)^((d-1)/2) / (d - 1);

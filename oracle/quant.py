@@ -16,7 +16,7 @@ Sources:
       - section "QJL: Inner Product Recovery from a Single Sign Bit": per token
         the sketch stores m sign bits plus a 16-bit norm.
 
-Readings (also in DESIGN.md):
+Readings taken where the pages are open:
   * index = number of boundaries strictly below the value, so a value equal to a
     boundary goes to the lower cell;
   * norms (||x|| and ||r||) are stored as IEEE fp16, round to nearest even; a
