@@ -92,7 +92,7 @@ typedef struct CUstream_st* tq_stream_t;
 typedef enum tq_status {
   TQ_OK = 0,
   TQ_ERR_INVALID_ARG = 1,  /* null pointer, inconsistent sizes, bad parameter values   */
-  TQ_ERR_UNSUPPORTED = 2,  /* a size or mode outside what this build supports          */
+  TQ_ERR_UNSUPPORTED = 2,  /* a size or mode outside what this library supports        */
   TQ_ERR_CUDA = 3,         /* a CUDA runtime call or a kernel launch failed            */
   TQ_ERR_OVERFLOW = 4,     /* a norm does not fit in fp16 (device)                     */
   TQ_ERR_TIMEOUT = 5,      /* a bounded wait inside a kernel gave up (device)          */
@@ -166,7 +166,7 @@ TQ_API const char* tq_status_str(tq_status st);
  * buffer, empty string if none). */
 TQ_API const char* tq_last_error(void);
 
-/* Checks a configuration; TQ_OK if this build supports it. */
+/* Checks a configuration; TQ_OK if this library supports it. */
 TQ_API tq_status tq_validate_config(const tq_config* cfg);
 
 /* Bytes of one (layer, page, kv head) block for cfg; 0 if cfg is invalid. */
