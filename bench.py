@@ -44,13 +44,32 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--n-splits", type=int, default=0, help="override the split count")
+    p.add_argument("--no-configs", action="store_true", help="skip the per-workload one-layer timings")
     return p.parse_args()
 
 
-def workload():
+B200_SMS = 148  # SM count of the target GPU, used where no GPU can be queried
+
+
+def sm_count(device_index: int = 0) -> int:
+    try:
+        import torch
+        if torch.cuda.is_available():
+            return torch.cuda.get_device_properties(device_index).multi_processor_count
+    except Exception:
+        pass
+    return B200_SMS
+
+
+def workload(n_splits: int = 0, device_index: int = 0):
+    """The benchmark layer (configuration 2) with the decode split count both arms report:
+    the override if given, else the library's default for this GPU (B200's 148 SMs when
+    there is none)."""
     import workloads as wl
-    # 32 splits x 8 KV heads = 256 CTAs: every SM busy (2 resident per SM), 4 pages each
-    return wl.config2(n_splits=32)
+    from compressed_decode_attention_tq_b200.runtime import splits_for
+    w = wl.config2()
+    w.n_splits = n_splits or splits_for(w.batch, w.kv_heads, sm_count(device_index))
+    return w
 
 
 def peaks():
@@ -165,10 +184,24 @@ class ClockSampler:
 # oracle timing (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(tokens: int, heads: int):
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def oracle_sample(tokens: int, heads: int, single_thread: bool = False):
     """Times the oracle on `heads` KV heads of layer 0, `tokens` tokens each: compress K (3-bit
     + QJL) and V (3-bit), pack, decode the G query heads of each KV head.  Returns
-    (token*kv-heads processed, seconds, threads)."""
+    (token*kv-heads processed, seconds, threads).  single_thread: the BLAS thread pool limited
+    to one thread."""
+    if single_thread:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            u, dt, _ = oracle_sample(tokens, heads)
+        return u, dt, 1
     import numpy as np
     import workloads as wl
     from oracle import attention as oatt, codebook as ocb, layout as olay, quant as oq, rotation as orot
@@ -192,18 +225,13 @@ def oracle_sample(tokens: int, heads: int):
         olay.write_sequence(cache, fmt, 0, h, bt[0], kc, vc)
     oatt.decode(cache, fmt, 0, q, bt, lens, R, ck, cv, rin["s"])
     dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = 1
-    return tokens * heads, dt, threads
+    return tokens * heads, dt, blas_threads()
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload()
+    w = workload(args.n_splits)
     tokens, heads = w.max_len, 1
     for _ in range(args.warmup):
         oracle_sample(tokens, heads)
@@ -219,8 +247,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(w, args.layers),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count() or 1, "threads": threads,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -235,6 +263,10 @@ def config_dict(w, layers):
             "head_dim": 128, "key_bits": w.key_bits, "key_qjl": w.key_qjl, "value_bits": w.value_bits,
             "page_tokens": 256, "n_splits": w.n_splits, "rotation": "hadamard",
             "l2": "inputs larger than L2 (4.3 GB K/V read + 0.99 GB packed cache per step); no flush",
+            "value_is": "token x kv-head positions compressed and then decoded per second of the whole "
+                        "step (compress of 32 layers, then decode of 32 layers); the metric's separate "
+                        "figures are in phases: decode kv_tokens_per_s, compress keys_per_s, each with "
+                        "its HBM GB/s and roofline fraction",
             "parallelism": "replicas"}
 
 
@@ -267,12 +299,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = workload()
-    if args.n_splits:
-        w.n_splits = args.n_splits
-    else:
-        from compressed_decode_attention_tq_b200.runtime import default_splits
-        w.n_splits = default_splits(w.batch, w.kv_heads, local_rank)
+    w = workload(args.n_splits, local_rank)
     L = args.layers
     rin = wl.rotation_inputs(w)
     lens = wl.seq_lens(w)
@@ -359,9 +386,18 @@ def run_ours(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         u, s, threads = oracle_sample(w.max_len, 1)
-        cpu = {"value": u / s, "unit": UNIT, "cores": threads, "kind": "oracle",
+        u1, s1, _ = oracle_sample(w.max_len // 4, 1, single_thread=True)
+        cpu = {"value": u / s, "unit": UNIT, "cores": os.cpu_count() or 1, "threads": threads,
+               "kind": "oracle",
                "sample": f"layer 0, 1 of 8 KV heads, {w.max_len} tokens: compress K/V + pack + "
-                         f"decode 4 query heads ({s:.1f} s)"}
+                         f"decode 4 query heads ({s:.1f} s, BLAS pool of {threads} threads on "
+                         f"{os.cpu_count()} host cores)",
+               "single_thread": {"value": u1 / s1, "unit": UNIT,
+                                 "sample": f"the same on {w.max_len // 4} tokens with one thread ({s1:.1f} s)"}}
+
+    configs = None
+    if rank == 0 and not args.no_configs:
+        configs = config_timings(dev)
 
     if rank == 0:
         line = {
@@ -369,12 +405,82 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(w, L), "phases": phases, "roofline": roofline,
-            "cpu_baseline": cpu, "e2e": e2e,
+            "cpu_baseline": cpu, "e2e": e2e, "configs": configs,
             # per layer: compress_tc_kernel, then prologue_kernel + fast_split_kernel
             "gpu_launches": args.steps * L * 3,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
+
+
+def config_timings(dev, reps: int = 10):
+    """One layer of every workload at full size: compress and decode each timed alone with CUDA
+    events around the launch, L2 flushed (a 256 MB write) before every timed launch.  Returns
+    {config: {...}} with the microseconds per call, the kernel path taken and the HBM GB/s of
+    the algorithmic bytes (compress: inputs read + packed bytes written; decode: packed bytes
+    read + q in and out)."""
+    import torch
+    import workloads as wl
+    from compressed_decode_attention_tq_b200.runtime import PagedKV, default_splits
+    hbm, _ = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for c in (1, 2, 3, 4, 5):
+        w = wl.CONFIGS[c]()
+        lens = wl.seq_lens(w)
+        bt, npages = wl.block_table(w, lens)
+        rin = wl.rotation_inputs(w)
+        kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
+                     key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits, rotation=w.rotation,
+                     num_layers=1, signs=rin["signs"], pi=rin["pi"], s=rin["s"], device=str(dev))
+        if c == 1:
+            Kh, Vh = wl.make_kv(w, 0)
+            K = torch.as_tensor(Kh, dtype=torch.float32, device=dev)
+            V = torch.as_tensor(Vh, dtype=torch.float32, device=dev)
+            q = torch.as_tensor(wl.make_q(w, 0), dtype=torch.float32, device=dev)
+        else:
+            K, V = wl.make_kv_device(w, 0, dev)
+            q = wl.make_q_device(w, 0, dev)
+        seq = torch.as_tensor(lens, dtype=torch.int32, device=dev)
+        ns = default_splits(w.batch, w.kv_heads, dev.index or 0) if c == 2 else w.n_splits
+        out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+
+        def timed(fn):
+            fn()
+            tot = 0.0
+            for _ in range(reps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                b.synchronize()
+                tot += a.elapsed_time(b)
+            return 1e3 * tot / reps
+
+        comp_us = timed(lambda: kv.compress(0, K, V, seq, stream))
+        dec_us = timed(lambda: kv.decode(0, q, seq, ns, out=out, stream=stream))
+        kv.raise_on_error(f"config {c}")
+        tokh = int(lens.sum()) * w.kv_heads
+        in_b = 2 if w.in_dtype == "f16" else 4
+        per_tok = kv.block_bytes / 256
+        comp_bytes = tokh * (2 * 128 * in_b + per_tok)
+        dec_bytes = tokh * per_tok + w.batch * w.q_heads * w.seq_q * 128 * (in_b + 4)
+        res[str(c)] = {
+            "workload": w.name, "n_splits": ns, "seq_q": w.seq_q,
+            "compress_us": comp_us, "compress_gbs": comp_bytes / comp_us / 1e3,
+            "compress_frac": comp_bytes / comp_us / 1e3 / hbm,
+            "keys_per_s": tokh / (comp_us * 1e-6),
+            "decode_us": dec_us, "decode_gbs": dec_bytes / dec_us / 1e3,
+            "decode_frac": dec_bytes / dec_us / 1e3 / hbm,
+            "kv_tokens_per_s": tokh / (dec_us * 1e-6),
+            "bytes_per_token_kv_head": per_tok,
+            "l2": "flushed (256 MB write) before every timed launch",
+        }
+        del kv, K, V, q, out
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(args, kv, w, L, Ks, Vs, Qs, Outs, seq, stream, dev, units, world):

@@ -29,7 +29,7 @@ TQ_F16 = 0
 TQ_F32 = 1
 
 # Every function include/tq.h declares.
-EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_validate_config", "tq_page_bytes",
+EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_check", "tq_validate_config", "tq_page_bytes",
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
            "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc", "tq_operand_bytes",
            "tq_prepare_operands", "tq_append_kv", "tq_append_attend_decode")
@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "tq_version": (I32, []),
         "tq_status_str": (ctypes.c_char_p, [I32]),
         "tq_last_error": (ctypes.c_char_p, []),
+        "tq_check": (I32, [ctypes.POINTER(ctypes.c_int32)]),
         "tq_validate_config": (I32, [cfgp]),
         "tq_page_bytes": (SZ, [cfgp]),
         "tq_codebook": (I32, [I32, I32, I32, P, P]),
@@ -103,6 +104,12 @@ def status_str(st: int) -> str:
 
 def last_error() -> str:
     return lib.tq_last_error().decode()
+
+
+def check_status(dev_status_value: int) -> int:
+    """tq_check on a host copy of a dev_status word: the recorded status code."""
+    v = ctypes.c_int32(int(dev_status_value))
+    return lib.tq_check(ctypes.byref(v))
 
 
 def _check(st: int, where: str):
@@ -176,7 +183,11 @@ def dtype_code(t) -> int:
 
 
 def compress_kv(cfg, params, cache, layer, k, v, seq_lens, status, stream=None):
-    """k, v: device [batch][kv_heads][max_len][d]; seq_lens: device int32 [batch]."""
+    """k, v: device [batch][kv_heads][max_len][d] of one dtype; seq_lens: device int32 [batch]."""
+    if v.shape != k.shape or v.dtype != k.dtype:
+        raise ValueError("k and v must have the same shape and dtype")
+    if k.dim() != 4:
+        raise ValueError("k and v must be [batch][kv_heads][max_len][d]")
     max_len = k.shape[2]
     _check(lib.tq_compress_kv(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
                               _ptr(k), _ptr(v), dtype_code(k), max_len, _ptr(seq_lens), _ptr(status),

@@ -95,6 +95,27 @@ const char* tq_status_str(tq_status st) {
 
 const char* tq_last_error(void) { return g_last_error; }
 
+tq_status tq_check(const int32_t* dev_status_host_copy) {
+  clear_error();
+  if (!dev_status_host_copy) return fail(TQ_ERR_INVALID_ARG, "tq_check: dev_status_host_copy is NULL");
+  const int32_t v = *dev_status_host_copy;
+  if (v < TQ_OK || v > TQ_ERR_BOUNDS) {
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "tq_check: %d is not a status code", (int)v);
+    return fail(TQ_ERR_INVALID_ARG, buf);
+  }
+  const tq_status st = static_cast<tq_status>(v);
+  switch (st) {
+    case TQ_OK: break;
+    case TQ_ERR_OVERFLOW: fail(st, "device: a norm does not fit in fp16"); break;
+    case TQ_ERR_TIMEOUT: fail(st, "device: a bounded wait inside a kernel gave up"); break;
+    case TQ_ERR_BOUNDS: fail(st, "device: a sequence length or page id is outside the cache"); break;
+    case TQ_ERR_INVALID_ARG: fail(st, "device: a parameter failed a device-side check"); break;
+    default: fail(st, "device: error recorded"); break;
+  }
+  return st;
+}
+
 tq_status tq_validate_config(const tq_config* cfg) {
   clear_error();
   return check_config(cfg);

@@ -10,9 +10,9 @@ from typing import Optional
 import torch
 
 from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, append_attend_decode, append_kv, attend_decode,
-               codebook, compress_kv,
+               check_status, codebook, compress_kv, last_error,
                decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
-               operand_bytes, page_bytes, prepare_operands, status_str)
+               operand_bytes, page_bytes, prepare_operands)
 
 
 def _f32(x, device):
@@ -21,11 +21,16 @@ def _f32(x, device):
     return torch.as_tensor(x, dtype=torch.float32).to(device).contiguous()
 
 
-def default_splits(batch: int, kv_heads: int, device=None) -> int:
-    """Split count that fills the GPU once: the fast decode kernel keeps two CTAs per SM,
-    one CTA per (split, kv head, sequence)."""
-    sms = torch.cuda.get_device_properties(device if device is not None else 0).multi_processor_count
+def splits_for(batch: int, kv_heads: int, sms: int) -> int:
+    """Split count that fills a GPU of `sms` SMs once: the fast decode kernel keeps two CTAs
+    per SM, one CTA per (split, kv head, sequence)."""
     return max(1, min(1024, (2 * sms) // max(1, batch * kv_heads)))
+
+
+def default_splits(batch: int, kv_heads: int, device=None) -> int:
+    """splits_for on the current (or given) GPU."""
+    sms = torch.cuda.get_device_properties(device if device is not None else 0).multi_processor_count
+    return splits_for(batch, kv_heads, sms)
 
 
 class PagedKV:
@@ -117,16 +122,17 @@ class PagedKV:
         return kh, vh
 
     def check(self) -> int:
-        """Synchronise and return the device status word (0 = ok); resets it."""
+        """Synchronise, read the device status word through tq_check and reset it; returns
+        the recorded status (0 = ok)."""
         torch.cuda.synchronize(self.device)
-        st = int(self.status.item())
+        st = check_status(int(self.status.item()))
         self.status.zero_()
         return st
 
     def raise_on_error(self, where: str = "device"):
         st = self.check()
         if st:
-            raise TQError(st, where, status_str(st))
+            raise TQError(st, where, last_error())
 
     def pages_numpy(self):
         """Host copy of the cache as [num_layers][num_pages][kv_heads][block_bytes] uint8."""

@@ -162,6 +162,15 @@ TQ_API int32_t tq_version(void);
 /* Human-readable name of a status code (static string). */
 TQ_API const char* tq_status_str(tq_status st);
 
+/* Status of the device work of earlier calls, from the caller's host copy of their
+ * dev_status word (copy it back after synchronising the stream the calls ran on).
+ *   dev_status_host_copy  host pointer to that int32 value
+ * Returns the recorded code (TQ_OK when the word is 0) and describes it in
+ * tq_last_error(); TQ_ERR_INVALID_ARG for a NULL pointer or a value that is no
+ * status code.  The word itself is not changed: the caller resets it to 0 before the
+ * next calls that should be checked on their own. */
+TQ_API tq_status tq_check(const int32_t* dev_status_host_copy);
+
 /* Detail of the last host-side error on the calling thread (static per-thread
  * buffer, empty string if none). */
 TQ_API const char* tq_last_error(void);
@@ -290,12 +299,17 @@ TQ_API tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* 
  * and results as tq_attend_decode, minus the workspace: a plugin inside a runtime that
  * owns all device memory, or a serving loop that must not call cudaMalloc mid-step, can
  * call this instead.  The scratch lives in a built-in 8 MiB array in device global
- * memory that every GPU loading the library holds until the process exits.
+ * memory, held until the CUDA context ends.
  *   - Sizes whose tq_decode_workspace_bytes(...) exceeds 8 MiB return
  *     TQ_ERR_UNSUPPORTED with an explanation in tq_last_error(); nothing is enqueued.
- *   - The first call on each device looks up the array's device address on the host
- *     (with that device current); make that first call before any stream capture
- *     begins on the device.
+ *   - Under lazy module loading (the CUDA default) the array's 8 MiB are reserved on a
+ *     device by the first call there, not when the library is loaded: make that first
+ *     call at start-up, before the caller's runtime claims the device memory pool.
+ *   - Every call made outside stream capture looks up the array's device address in the
+ *     current context (so a context that was reset gets its own address); a call made
+ *     while its stream is being captured reuses the address its context found before and
+ *     returns TQ_ERR_INVALID_ARG if there is none: make the first call in each context
+ *     before any stream capture begins.
  *   - All calls on a device share the one array: calls whose kernels can overlap in
  *     time race and give undefined results.  Order them on a single stream.
  *   - Nothing in the array needs clearing between calls (every byte read is first

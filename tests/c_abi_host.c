@@ -20,6 +20,15 @@ int main(void) {
   CHECK(tq_version() >= 100, "version");
   CHECK(strcmp(tq_status_str(TQ_ERR_BOUNDS), "TQ_ERR_BOUNDS") == 0, "status string");
 
+  /* the host copy of a dev_status word, decoded */
+  int32_t word = 0;
+  CHECK(tq_check(&word) == TQ_OK, "tq_check of a clear word");
+  word = TQ_ERR_TIMEOUT;
+  CHECK(tq_check(&word) == TQ_ERR_TIMEOUT && strlen(tq_last_error()) > 0, "tq_check of a timeout");
+  word = 99;
+  CHECK(tq_check(&word) == TQ_ERR_INVALID_ARG, "tq_check of a value that is no status");
+  CHECK(tq_check(NULL) == TQ_ERR_INVALID_ARG, "tq_check of NULL");
+
   tq_config cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.head_dim = 128;

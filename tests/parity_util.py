@@ -101,6 +101,17 @@ class CompressReport:
     norm_fail: int = 0
 
 
+# Every compress comparison and decode check of the session, printed at the end of the run by
+# tests/conftest.py (pytest_terminal_summary), so that the counts the tolerances allow are
+# visible in the run's output even under -q.
+REPORTS: list = []
+
+
+def record(name: str, rep) -> None:
+    """Keeps a CompressReport (or a one-line decode summary string) for the session summary."""
+    REPORTS.append((name, rep))
+
+
 def _check_qjl(gpu_sigma, gpu_rnorm, comp, mis, rep):
     """Residual norms and sign bits of the tokens whose indices all agree (a token whose
     index differs inside the band has a different residual, so its signs are skipped)."""

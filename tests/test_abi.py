@@ -199,3 +199,26 @@ def test_plain_c_caller_links_and_runs(tq, tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stdout + out.stderr
     assert "FAIL" not in out.stdout and out.stdout.count("ok ") >= 12
+
+
+def test_tq_check_decodes_the_status_word(tq):
+    # the host copy of a dev_status word goes through tq_check: every code comes back as
+    # itself, with a description of the device errors; anything else is an argument error
+    for code in range(0, 7):
+        assert tq.check_status(code) == code
+        if code in (tq.TQ_ERR_OVERFLOW, tq.TQ_ERR_TIMEOUT, tq.TQ_ERR_BOUNDS):
+            assert tq.last_error().startswith("device:")
+    assert tq.check_status(0) == tq.TQ_OK and tq.last_error() == ""
+    assert tq.check_status(7) == tq.TQ_ERR_INVALID_ARG and "not a status code" in tq.last_error()
+    assert tq.check_status(-1) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_check(None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_compress_binding_rejects_mismatched_k_and_v(tq):
+    # the kernel reads v with k's geometry, so the binding refuses a v that differs
+    import torch
+    cfg, params, cache = tq.make_config(), tq.tq_params(), tq.tq_cache()
+    k = torch.zeros((1, 2, 8, 128), dtype=torch.float16)
+    for v in (torch.zeros((1, 2, 9, 128), dtype=torch.float16), torch.zeros((1, 2, 8, 128), dtype=torch.float32)):
+        with pytest.raises(ValueError, match="same shape and dtype"):
+            tq.compress_kv(cfg, params, cache, 0, k, v, None, None, stream=0)

@@ -11,7 +11,7 @@ import workloads as wl
 pytestmark = pytest.mark.gpu
 
 from parity_util import (CompressReport, close, compare_compress, oracle_decode, oracle_scores,
-                         q_dev, seq_dev, setup)
+                         q_dev, record, seq_dev, setup)
 
 SMALL = {
     "c1": lambda: wl.config1(max_len=1000, n_splits=3),
@@ -60,6 +60,7 @@ def test_compress_bit_exact(run):
             for h in range(run.w.kv_heads):
                 compare_compress(run, run.pages, layer, b, h, rep=rep)
     print(f"\n{run.w.name}: {rep}")
+    record(f"compress {run.w.name}", rep)
     assert rep.idx_mismatch_out_of_band == 0
     assert rep.sign_mismatch_out_of_band == 0
     assert rep.norm_fail == 0
