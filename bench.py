@@ -415,7 +415,8 @@ def run_ours(args, rank, world, local_rank):
 
 def config_timings(dev, reps: int = 10):
     """One layer of every workload at full size: compress and decode each timed alone with CUDA
-    events around the launch, L2 flushed (a 256 MB write) before every timed launch.  Returns
+    events around the launch, L2 flushed before every timed launch (a 256 MB buffer written and
+    read back, so that no dirty lines are left to write back during the timed launch).  Returns
     {config: {...}} with the microseconds per call, the kernel path taken and the HBM GB/s of
     the algorithmic bytes (compress: inputs read + packed bytes written; decode: packed bytes
     read + q in and out)."""
@@ -450,7 +451,10 @@ def config_timings(dev, reps: int = 10):
             fn()
             tot = 0.0
             for _ in range(reps):
+                # writing the buffer evicts the cache's lines; reading it back evicts the written
+                # ones, so that the timed launch meets no write-back traffic
                 flush.zero_()
+                flush.sum()
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 fn()
@@ -476,7 +480,7 @@ def config_timings(dev, reps: int = 10):
             "decode_frac": dec_bytes / dec_us / 1e3 / hbm,
             "kv_tokens_per_s": tokh / (dec_us * 1e-6),
             "bytes_per_token_kv_head": per_tok,
-            "l2": "flushed (256 MB write) before every timed launch",
+            "l2": "flushed before every timed launch (a 256 MB buffer written, then read back)",
         }
         del kv, K, V, q, out
         torch.cuda.empty_cache()

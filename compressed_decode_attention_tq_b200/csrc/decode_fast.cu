@@ -44,7 +44,7 @@ constexpr int kNormBytes = 3 * kUnit * 2;      // KN | KR | VN of the unit
 constexpr int kMaxKChunks = 4;
 constexpr int kMaxVChunks = 3;
 constexpr int kStageBytes = kNormBytes + (kMaxKChunks + kMaxVChunks) * kChunkStride;
-constexpr long long kWaitLimit = 1ll << 26;  // bounded mbarrier waits
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // every mbarrier wait gives up after 1 s
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
@@ -67,6 +67,7 @@ struct SmemFast {
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   unsigned long long mbar;  // the merge copies landed
+  unsigned long long never;  // completed by nothing: the target of the bounded-wait test
   float wm[kConsumerWarps][4], wl[kConsumerWarps][4], wf[kConsumerWarps][4];
   int last;
 };
@@ -91,44 +92,50 @@ __device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait on the given phase parity; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity) {
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Wait on the given phase parity for at most limit_ns nanoseconds of the global timer
+// (read once every 256 polls, so that a wait that succeeds soon costs no timer reads);
+// false if it gave up.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
-  for (long long it = 0; it < kWaitLimit; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
+  if (mbar_try(addr, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    for (int it = 0; it < 256; ++it)
+      if (mbar_try(addr, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
   }
-  return false;
 }
 
 // The same wait for a thread that can afford to react late (the copy producer, three stages
 // ahead): between polls it sleeps, so that it takes few issue slots from the consumer warps
-// of its SM sub-partition; gives up after about 1 s.
+// of its SM sub-partition.
 __device__ __forceinline__ bool mbar_wait_sleepy(unsigned long long* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
-  unsigned long long t0 = 0;
-  for (long long it = 0; it < kWaitLimit; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    if (it == 0) t0 = t;
-    else if (t - t0 > 1000000000ull) break;
+  if (mbar_try(addr, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
     __nanosleep(128);
+    if (mbar_try(addr, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
   }
-  return false;
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
@@ -254,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       mbar_init(&sm.empty[s], kConsumerWarps);
     }
     mbar_init(&sm.mbar, 1);
+    mbar_init(&sm.never, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -482,6 +490,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       const float lam = a.q8_scale[row0 + t4];
       corr_down = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
     }
+
+    if (a.debug_wait_ns > 0 && warp == 0 && split == 0 && gh == 0 && blockIdx.z == 0 &&
+        !mbar_wait(&sm.never, 0, (unsigned long long)a.debug_wait_ns) && lane == 0)
+      report(a.status, TQ_ERR_TIMEOUT);
 
     float m_run = -CUDART_INF_F, l_run = 0.f;
     float acc[8][4];

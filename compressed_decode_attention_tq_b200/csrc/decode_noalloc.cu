@@ -18,7 +18,8 @@
 // kernels overlap in time (different streams, or different host threads without
 // ordering) race on it and their results are undefined; order them on one stream.  The
 // decode kernels write every scratch byte they later read (rotated queries, S-projected
-// queries and every (row, split) partial), so nothing has to be cleared between calls.
+// queries, the merge counters and every (row, split) partial), so nothing has to be
+// cleared between calls.
 #include <cuda_runtime.h>
 
 #include <cstdio>

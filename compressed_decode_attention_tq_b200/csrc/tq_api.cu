@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "tq.h"
@@ -189,6 +190,18 @@ size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int32_t q_
   return tqk::decode_workspace(batch, q_heads, seq_q, n_splits, cfg->value_qjl).total;
 }
 
+// A test of the device's bounded waits: TQ_DEBUG_BOUNDED_WAIT_US=<n> (1..1000000) makes one
+// consumer warp of the tensor-core split kernel wait n microseconds on a barrier nothing
+// arrives on and report TQ_ERR_TIMEOUT; the call's results are unaffected.  Read on every
+// call.
+static int debug_wait_ns() {
+  const char* v = std::getenv("TQ_DEBUG_BOUNDED_WAIT_US");
+  if (!v || !*v) return 0;
+  const long us = std::strtol(v, nullptr, 10);
+  if (us <= 0 || us > 1000000) return 0;
+  return (int)(us * 1000);
+}
+
 static tq_status decode_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                                int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
                                int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
@@ -246,6 +259,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.n_new = 0;
   a.k_boundaries = params->k_boundaries;
   a.v_boundaries = params->v_boundaries;
+  a.debug_wait_ns = debug_wait_ns();
   return TQ_OK;
 }
 

@@ -46,6 +46,10 @@ struct DecodeArgs {
   const void* v_new;
   int new_dtype, n_new;
   const float *k_boundaries, *v_boundaries;
+  // > 0: a test of the bounded waits (one consumer warp of the first thread block of the
+  // fast split kernel waits this many nanoseconds on a barrier nothing arrives on and
+  // reports TQ_ERR_TIMEOUT; the results are computed as usual)
+  int debug_wait_ns;
   int32_t* status;
 };
 

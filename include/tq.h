@@ -253,7 +253,12 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int
  *   n_splits   1..1024
  *   workspace  device, >= tq_decode_workspace_bytes(...) bytes, 256-byte aligned;
  *              scratch only, contents on return unspecified
- *   out        device float [batch][q_heads][seq_q][d] */
+ *   out        device float [batch][q_heads][seq_q][d]
+ * A test of the device's bounded waits: with the environment variable
+ * TQ_DEBUG_BOUNDED_WAIT_US set to n (1..1000000) when the call is made, one warp of the
+ * tensor-core split kernel (keys 2- or 3-bit with QJL, values 2- or 3-bit, Hadamard
+ * rotation) waits n microseconds on a barrier that nothing completes and writes
+ * TQ_ERR_TIMEOUT to dev_status; the results are computed as usual. */
 TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                            int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
                            int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,

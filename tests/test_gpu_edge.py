@@ -102,3 +102,22 @@ def test_zero_vector_compresses_to_zero_norm():
     assert np.all(u.k_norm == 0) and np.all(u.v_norm == 0) and np.all(u.k_rnorm == 0)
     # y = 0 lies on the middle boundary: index h - 1 (tie to the lower cell); sign(0) -> +1
     assert np.all(u.k_idx == 3) and np.all(u.v_idx == 1) and np.all(u.k_sigma)
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable(monkeypatch):
+    # a device wait that runs out: with TQ_DEBUG_BOUNDED_WAIT_US one warp of the tensor-core
+    # split kernel waits 2 ms on a barrier nothing completes; the kernel reports
+    # TQ_ERR_TIMEOUT through dev_status and returns, and the next call on the same context
+    # (without the knob) matches the oracle
+    w = wl.config2(kv_heads=2, q_heads=8, max_len=700, n_splits=3)
+    r = _run(w)
+    r.kv.raise_on_error("compress")
+    seq = torch.as_tensor(r.lens, dtype=torch.int32, device="cuda")
+    q, qd = q_dev(r)
+    monkeypatch.setenv("TQ_DEBUG_BOUNDED_WAIT_US", "2000")
+    r.kv.decode(0, qd, seq, w.n_splits)
+    assert r.kv.check() == 5  # TQ_ERR_TIMEOUT
+    monkeypatch.delenv("TQ_DEBUG_BOUNDED_WAIT_US")
+    out = r.kv.decode(0, qd, seq, w.n_splits).cpu().numpy()
+    assert r.kv.check() == 0
+    assert close(out, oracle_decode(r, r.pages, 0, q)).all()
