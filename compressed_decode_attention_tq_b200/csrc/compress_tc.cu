@@ -1,4 +1,5 @@
-// Compression on the tensor cores (tcgen05 + TMEM + TMA), randomized-Hadamard rotation.
+// Compression on the tensor cores (tcgen05 + TMEM + TMA), randomized-Hadamard or dense
+// Haar rotation.
 //
 // What is computed is the same as compress.cu ("TurboQuant explained", sections "How JL
 // Matrices Evolved", "Coordinates Become Predictable After Rotation" and "Two-Stage
@@ -8,6 +9,11 @@
 //
 //  * y' = (H D) x for a tile of 128 tokens: A = the fp16 input tile (exact), B = H D with
 //    +-1 entries (exact), fp32 accumulation in tensor memory.  y = y' / ||y'||.
+//  * With the dense rotation Pi ("turboquant_cutile" function list: Haar matrix from the QR
+//    of a Gaussian) y' = (sqrt(d) Pi) x, the same scale as (H D) x: B = sqrt(d) Pi is held
+//    as an fp16 hi + lo pair (prepared once per cache by prepare_dense_kernel), and two
+//    MMAs per K step (x . hi, x . lo) accumulate y' to ~2^-22 relative.  Keys without QJL
+//    only: the sketch's two more operand tiles would not fit beside the input stages.
 //  * QJL sketch in the rotated domain: with R = H D / sqrt(d) orthogonal,
 //      S r = S R^T R r = (S D H) r_rot' / d,   r_rot' = y' - sqrt(d) fp16(||x||) c[idx],
 //    so sign(S r) = sign((S D H) a r_rot') for any a > 0.  S D H is held as an fp16 hi + lo
@@ -68,8 +74,8 @@ constexpr float kSqrtD = 11.313708498984761f;
 
 struct SmemTC {
   unsigned char x[2][2][kTileBytes];  // [stage][K, V] input tiles (canonical layout); S at set-up
-  unsigned char bhd[kTileBytes];      // B = H D
-  unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part
+  unsigned char bhd[kTileBytes];      // B = H D (dense rotation: sqrt(d) Pi, fp16 hi part)
+  unsigned char bshi[kTileBytes];     // B = S D H, fp16 hi part (dense rotation: sqrt(d) Pi, lo part)
   unsigned char bslo[kTileBytes];     // fp16 lo part
   // [stage]: tile landed / read by its forward MMAs; [group]: forward MMAs done, A of key
   // chunk c written (y'_V read before the first), sketch done, tensor-memory columns
@@ -535,16 +541,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // otherwise each CTA builds them (stage 1 is then set-up scratch for S).  Tile 0 streams
   // in meanwhile.  (The copy thread issues tile 1 right after; group 1 starts its first tile
   // that much later, and the two groups stay out of phase, which their ping-pong relies on.)
+  // (The dense rotation always comes prepared: sqrt(d) Pi hi / lo, two tiles.)
   const bool prep = a.operands != nullptr;
+  const bool dense = a.dense != 0;
   if (warp == kLoaderWarp && lane == 0) {
     if (prep) {
+      const uint32_t nops = dense ? 2 : 3;
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(&sm.ops_ready)),
-                   "r"(3 * kTileBytes)
+                   "r"(nops * kTileBytes)
                    : "memory");
       const unsigned char* ops = static_cast<const unsigned char*>(a.operands);
       bulk_load(sm.bhd, ops, kTileBytes, &sm.ops_ready);
       bulk_load(sm.bshi, ops + kTileBytes, kTileBytes, &sm.ops_ready);
-      bulk_load(sm.bslo, ops + 2 * kTileBytes, kTileBytes, &sm.ops_ready);
+      if (!dense) bulk_load(sm.bslo, ops + 2 * kTileBytes, kTileBytes, &sm.ops_ready);
     }
     if (my_tiles > 0) issue_load(0);
   }
@@ -677,6 +686,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       auto fwd = [&](int kv, uint32_t dcol) {
 #pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) mma_ss(dcol, smem_desc(sm.x[g][kv], ks), smem_desc(sm.bhd, ks), ks > 0);
+        if (dense) {
+#pragma unroll 1
+          for (int ks = 0; ks < 8; ++ks) mma_ss(dcol, smem_desc(sm.x[g][kv], ks), smem_desc(sm.bshi, ks), 1);
+        }
       };
       bool k_issued = false;  // y'_K of the group's next tile already requested
       for (int n = 0, j = g; ok && j < my_tiles; ++n, j += 2) {
@@ -1006,6 +1019,17 @@ __global__ void __launch_bounds__(128) prepare_operands_kernel(const float* sign
   *reinterpret_cast<__half*>(ops + 2 * kTileBytes + canon(m, t)) = lo;
 }
 
+// Dense rotation: B = sqrt(d) Pi (row i = output coordinate, column k = input coordinate,
+// y = Pi u) as an fp16 hi tile and the fp16 rounding of the fp32 remainder; one CTA per row.
+__global__ void __launch_bounds__(128) prepare_dense_kernel(const float* pi, unsigned char* ops) {
+  const int i = blockIdx.x, k = threadIdx.x;
+  const float x = pi[(size_t)i * D + k] * kSqrtD;
+  const __half hi = __float2half_rn(x);
+  const __half lo = __float2half_rn(x - __half2float(hi));
+  *reinterpret_cast<__half*>(ops + canon(i, k)) = hi;
+  *reinterpret_cast<__half*>(ops + kTileBytes + canon(i, k)) = lo;
+}
+
 // ---------------------------------------------------------------------------
 // host: tensor maps
 // ---------------------------------------------------------------------------
@@ -1076,7 +1100,8 @@ cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtens
 
 bool compress_tc_supported(const CompressArgs& a) {
   const Layout& L = a.cache.L;
-  if (a.dense || a.in_dtype != TQ_F16 || L.vqjl) return false;
+  if (a.in_dtype != TQ_F16 || L.vqjl) return false;
+  if (a.dense && (L.qjl || a.operands == nullptr)) return false;
   if ((size_t)a.cache.batch * a.cache.kv_heads * a.max_len >= (1ull << 31)) return false;
   if (L.qjl && !(L.kbits == 2 || L.kbits == 3)) return false;
   if (!L.qjl && !(L.kbits >= 2 && L.kbits <= 4)) return false;
@@ -1086,10 +1111,15 @@ bool compress_tc_supported(const CompressArgs& a) {
   return encode_fn() != nullptr;
 }
 
-size_t operand_bytes() { return 3 * (size_t)kTileBytes; }
+size_t operand_bytes(bool dense) { return (dense ? 2 : 3) * (size_t)kTileBytes; }
 
 cudaError_t launch_prepare_operands(const float* signs, const float* s, int qjl, void* ops, cudaStream_t stream) {
   prepare_operands_kernel<<<qjl ? QM + 1 : 1, 128, 0, stream>>>(signs, s, static_cast<unsigned char*>(ops));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prepare_dense(const float* pi, void* ops, cudaStream_t stream) {
+  prepare_dense_kernel<<<D, D, 0, stream>>>(pi, static_cast<unsigned char*>(ops));
   return cudaGetLastError();
 }
 

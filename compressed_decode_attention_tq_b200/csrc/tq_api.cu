@@ -155,7 +155,7 @@ tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq
   a.k_boundaries = params->k_boundaries;
   a.v_centroids = params->v_centroids;
   a.v_boundaries = params->v_boundaries;
-  a.operands = cfg->rotation == TQ_ROT_HADAMARD ? params->operands : nullptr;
+  a.operands = params->operands;
   if (a.operands && (reinterpret_cast<uintptr_t>(a.operands) & 15))
     return fail(TQ_ERR_INVALID_ARG, "params->operands must be 16-byte aligned");
   a.status = dev_status;
@@ -165,21 +165,26 @@ tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq
 }
 
 size_t tq_operand_bytes(const tq_config* cfg) {
-  if (check_config(cfg) != TQ_OK || cfg->rotation != TQ_ROT_HADAMARD) return 0;
-  return tqk::operand_bytes();
+  if (check_config(cfg) != TQ_OK) return 0;
+  return tqk::operand_bytes(cfg->rotation == TQ_ROT_DENSE);
 }
 
 tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, void* operands, tq_stream_t stream) {
   clear_error();
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
-  if (cfg->rotation != TQ_ROT_HADAMARD) return fail(TQ_ERR_UNSUPPORTED, "operands exist for TQ_ROT_HADAMARD only");
-  if (!params || !params->signs) return fail(TQ_ERR_INVALID_ARG, "params or params->signs is NULL");
-  if (cfg->key_qjl && !params->s) return fail(TQ_ERR_INVALID_ARG, "params->s is NULL");
   if (!operands || (reinterpret_cast<uintptr_t>(operands) & 15))
     return fail(TQ_ERR_INVALID_ARG, "operands must be a 16-byte aligned device pointer");
-  cudaError_t e = tqk::launch_prepare_operands(params->signs, params->s, cfg->key_qjl, operands,
-                                               reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (cfg->rotation == TQ_ROT_DENSE) {
+    if (!params || !params->pi) return fail(TQ_ERR_INVALID_ARG, "params or params->pi is NULL");
+    e = tqk::launch_prepare_dense(params->pi, operands, reinterpret_cast<cudaStream_t>(stream));
+  } else {
+    if (!params || !params->signs) return fail(TQ_ERR_INVALID_ARG, "params or params->signs is NULL");
+    if (cfg->key_qjl && !params->s) return fail(TQ_ERR_INVALID_ARG, "params->s is NULL");
+    e = tqk::launch_prepare_operands(params->signs, params->s, cfg->key_qjl, operands,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) return cuda_fail(e, "tq_prepare_operands launch");
   return TQ_OK;
 }

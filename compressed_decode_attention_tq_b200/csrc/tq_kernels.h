@@ -15,7 +15,7 @@ struct CompressArgs {
   int in_dtype, max_len, qjl, dense;
   const int32_t* seq_lens;
   const float *signs, *pi, *s, *k_centroids, *k_boundaries, *v_centroids, *v_boundaries;
-  const void* operands;  // prepared tensor-core operands (B = H D, S D H hi / lo) or null
+  const void* operands;  // prepared tensor-core operands (B = H D, S D H hi / lo; or sqrt(d) Pi hi / lo) or null
   int32_t* status;
 };
 
@@ -68,8 +68,9 @@ bool compress_tc_supported(const CompressArgs& a);
 cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream);
 // Tensor-core operands of the compress kernel for a Hadamard rotation (and with QJL the
 // sketch): three canonical 128 x 128 fp16 tiles, B = H D, then S D H as hi and lo parts.
-size_t operand_bytes();
+size_t operand_bytes(bool dense);
 cudaError_t launch_prepare_operands(const float* signs, const float* s, int qjl, void* ops, cudaStream_t stream);
+cudaError_t launch_prepare_dense(const float* pi, void* ops, cudaStream_t stream);
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {

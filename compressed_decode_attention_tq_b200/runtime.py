@@ -63,13 +63,17 @@ class PagedKV:
             "vc": _f32(vc, self.device), "vb": _f32(vb, self.device),
         }
         t = self.tensors
-        # the compress kernel's tensor-core operands (H D, S D H), formed once for the cache
-        # instead of in every thread block of every call
+        # the compress kernel's tensor-core operands (H D, S D H; or sqrt(d) Pi), formed once
+        # for the cache instead of in every thread block of every call
         t["ops"] = None
         nops = operand_bytes(self.cfg)
-        if prepared_operands and nops and t["signs"] is not None and (not key_qjl or t["s"] is not None):
+        if rotation == TQ_ROT_DENSE:
+            have = t["pi"] is not None
+        else:
+            have = t["signs"] is not None and (not key_qjl or t["s"] is not None)
+        if prepared_operands and nops and have:
             t["ops"] = torch.empty(nops, dtype=torch.uint8, device=self.device)
-            prepare_operands(self.cfg, make_params(t["signs"], s=t["s"]), t["ops"])
+            prepare_operands(self.cfg, make_params(t["signs"], t["pi"], s=t["s"]), t["ops"])
         self.params = make_params(t["signs"], t["pi"], t["s"], t["kc"], t["kb"], t["vc"], t["vb"], t["ops"])
         self.cache = make_cache(self.pages, self.block_table, num_pages, self.max_pages, batch, kv_heads,
                                 num_layers)

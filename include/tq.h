@@ -138,10 +138,12 @@ typedef struct tq_params {
   const float* v_boundaries;  /* [2^value_bits - 1]                                      */
   const void* operands;       /* NULL, or device memory of tq_operand_bytes() bytes (16-byte
                                  aligned) that tq_prepare_operands filled for these signs
-                                 and s: tq_compress_kv then copies its tensor-core operands
-                                 from it instead of forming them in every thread block.
-                                 Read only by tq_compress_kv, and only with
-                                 TQ_ROT_HADAMARD.                                      */
+                                 and s (or this pi): tq_compress_kv then copies its
+                                 tensor-core operands from it instead of forming them in
+                                 every thread block.  Read only by tq_compress_kv.  With
+                                 TQ_ROT_DENSE, compression runs on the tensor cores only
+                                 when these operands are given (and keys and values carry
+                                 no QJL sketch); otherwise on the CUDA cores.          */
 } tq_params;
 
 /* A paged cache ([LIMITS] vLLM-style packed paged cache). */
@@ -213,7 +215,7 @@ TQ_API tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, c
                          tq_stream_t stream);
 
 /* Bytes of the prepared tensor-core operands of tq_compress_kv for cfg (96 KiB for a
- * TQ_ROT_HADAMARD configuration; 0 if cfg is invalid or uses TQ_ROT_DENSE). */
+ * TQ_ROT_HADAMARD configuration, 64 KiB for TQ_ROT_DENSE; 0 if cfg is invalid). */
 TQ_API size_t tq_operand_bytes(const tq_config* cfg);
 
 /* Prepare the operands tq_compress_kv uses on the tensor cores for the rotation
@@ -221,14 +223,15 @@ TQ_API size_t tq_operand_bytes(const tq_config* cfg);
  * sketch taken in the rotated domain ([MOBILINT] "QJL: Inner Product Recovery from a
  * Single Sign Bit": S r = (S D H) (H D r) / d): three 128 x 128 fp16 tiles in the
  * tensor cores' canonical K-major layout, B = H D (entries +-1, exact), then S D H
- * (formed in fp32) as a high fp16 part and the fp16 rounding of the remainder.
- *   params    signs (and s with key_qjl) as for tq_compress_kv; S need not be
- *             fp16-exact on this path
+ * (formed in fp32) as a high fp16 part and the fp16 rounding of the remainder.  For
+ * TQ_ROT_DENSE ([CUTILE]: Haar Pi), two tiles: sqrt(d) Pi (row i, column k = Pi_ik,
+ * formed in fp32) as a high fp16 part and the fp16 rounding of the remainder.
+ *   params    signs (and s with key_qjl) as for tq_compress_kv, or pi for TQ_ROT_DENSE;
+ *             S need not be fp16-exact on this path
  *   operands  device, tq_operand_bytes(cfg) bytes, 16-byte aligned; written
  *             asynchronously on stream; owned by the caller, who passes it in
  *             tq_params.operands while signs and s stay unchanged
- * Errors: TQ_ERR_UNSUPPORTED for TQ_ROT_DENSE, TQ_ERR_INVALID_ARG for NULL or
- * misaligned pointers. */
+ * Errors: TQ_ERR_INVALID_ARG for NULL or misaligned pointers. */
 TQ_API tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, void* operands,
                                      tq_stream_t stream);
 

@@ -132,14 +132,14 @@ def test_operand_bytes_and_prepare_validation(tq):
     cfg = tq.make_config()
     assert tq.lib.tq_operand_bytes(ctypes.byref(cfg)) == ops
     dense = tq.make_config(rotation=tq.TQ_ROT_DENSE)
-    assert tq.lib.tq_operand_bytes(ctypes.byref(dense)) == 0
+    assert tq.lib.tq_operand_bytes(ctypes.byref(dense)) == 2 * 128 * 128 * 2
     bad = tq.make_config(head_dim=64)
     assert tq.lib.tq_operand_bytes(ctypes.byref(bad)) == 0
     params = tq.tq_params()
     buf = ctypes.create_string_buffer(ops + 16)
     aligned = (ctypes.addressof(buf) + 15) & ~15
     st = tq.lib.tq_prepare_operands(ctypes.byref(dense), ctypes.byref(params), aligned, None)
-    assert st == tq.TQ_ERR_UNSUPPORTED
+    assert st == tq.TQ_ERR_INVALID_ARG and "pi" in tq.last_error()
     st = tq.lib.tq_prepare_operands(ctypes.byref(cfg), ctypes.byref(params), aligned, None)
     assert st == tq.TQ_ERR_INVALID_ARG and "signs" in tq.last_error()
     params.signs = aligned  # any non-null pointer: the call is rejected before it is read

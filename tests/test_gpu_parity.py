@@ -34,8 +34,11 @@ SMALL = {
 
 
 # the same kernels with the tensor-core operands (H D, S D H) formed inside every thread
-# block instead of prepared once per cache
+# block instead of prepared once per cache; the dense rotation without prepared operands
+# compresses on the CUDA cores
 IN_BLOCK = {
+    "c3_unprepared_dense": lambda: wl.config3(batch=3, max_len=900, min_len=300, n_splits=2,
+                                              name="c3_unprepared_dense"),
     "c2_in_block_operands": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4,
                                                name="c2_in_block_operands"),
     "c4_in_block_operands": lambda: wl.config4(batch=2, kv_heads=2, q_heads=8, max_len=2000, n_splits=8,
