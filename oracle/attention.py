@@ -86,9 +86,10 @@ def attend_scores(scores, Vhat) -> np.ndarray:
 
 def decode_sequence(q, unpacked: lay.Unpacked, R, ck, cv, S=None, return_scores=False):
     """Decode attention of q [nq, d] over one (sequence, kv head) read from packed pages.
-    Values with QJL are reconstructed as v_mse + x_qjl (S is then required)."""
-    k_mse = qt.reconstruct_mse(unpacked.k_idx, unpacked.k_norm, R, ck)
-    v_hat = qt.reconstruct_mse(unpacked.v_idx, unpacked.v_norm, R, cv)
+    Values with QJL are reconstructed as v_mse + x_qjl (S is then required); dithered
+    vectors add their stored offset back before un-rotating."""
+    k_mse = qt.reconstruct_mse(unpacked.k_idx, unpacked.k_norm, R, ck, unpacked.k_offset)
+    v_hat = qt.reconstruct_mse(unpacked.v_idx, unpacked.v_norm, R, cv, unpacked.v_offset)
     if unpacked.v_sigma is not None:
         v_hat = v_hat + qt.qjl_reconstruct(unpacked.v_sigma, unpacked.v_rnorm, S)
     sc = scores_compressed(q, k_mse, unpacked.k_rnorm, unpacked.k_sigma, S)

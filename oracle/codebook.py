@@ -17,6 +17,24 @@ Source: "TurboQuant explained" (Mobilint blog)
     float32 tensors, centroids (2^b,) and boundaries (2^b - 1,).
   * "tq-kv" crate documentation, module codebook: a Gaussian-fitted variant.
 
+Dithered quantization ("Minimum Distortion Quantization with Specified Output
+Distribution" page, third abstract: one randomized Hadamard transform, then a random
+scalar offset subtracted before a scalar quantizer; unbiased, MSE near
+(pi sqrt(3)/2) 4^-b):
+  * reading: the scalar quantizer is a uniform grid of n = 2^b levels with step
+    delta, c_j = (j - (n-1)/2) delta, boundaries at the midpoints, and the offset xi
+    is uniform on [-delta/2, delta/2), one per vector; a coordinate y is coded as
+    idx = Quant(y - xi) and reconstructed as c[idx] + xi (subtractive dither, which
+    is what makes the reconstruction unbiased inside the grid's range);
+  * for a coordinate y the expected squared error over xi is exactly
+        delta^2/12 + max(|y| - A, 0)^2,   A = (n-1) delta / 2
+    (inside the outer levels the error is uniform on one cell; beyond them the
+    outer level is taken for every xi), so the per-coordinate MSE on f_X is
+        D(delta) = delta^2/12 + 2 [P2(A) - 2 A P1(A) + A^2 P0(A)],
+    P_k(A) = int_A^inf t^k f_X(t) dt;
+  * reading: delta is the minimiser of D; dD/d delta = delta/6 - 2(n-1)[P1(A) - A P0(A)]
+    is increasing in delta, so the minimiser is its unique root (found by bisection).
+
 Readings taken where the pages are open:
   * the integrals are computed with closed forms: the cell mass is a difference
     of the regularized incomplete Beta function, and the first moment of
@@ -148,3 +166,75 @@ def distortion(centroids, d: int, density: str = "beta") -> float:
                                 epsabs=1e-15, epsrel=1e-12, limit=200)
         total += val
     return total
+
+
+# ---------------------------------------------------------------------------
+# dithered quantization: uniform grid, MSE-optimal step
+# ---------------------------------------------------------------------------
+
+def tail_moments(A: float, d: int, density: str = "beta") -> tuple[float, float, float]:
+    """(P0, P1, P2): int_A^inf t^k f_X(t) dt for k = 0, 1, 2 and A >= 0.
+
+    beta:  P0 = 1 - F(A); P1 from the first-moment antiderivative; with u = t^2,
+           P2 = (1 / (2d)) (1 - I_{A^2}(3/2, (d-1)/2))  (B(3/2, a) / B(1/2, a) = 1/d, a = (d-1)/2).
+    gauss: with s = 1/sqrt(d), z = A/s: P0 = Q(z), P1 = s phi(z), P2 = s^2 (z phi(z) + Q(z))."""
+    if A < 0:
+        raise ValueError("A must be >= 0")
+    if density == "beta":
+        if A >= 1.0:
+            return 0.0, 0.0, 0.0
+        P0 = float(1.0 - beta_cdf(A, d))
+        P1 = float(beta_first_moment(A, 1.0, d))
+        P2 = float((1.0 - special.betainc(1.5, (d - 1) / 2.0, A * A)) / (2.0 * d))
+        return P0, P1, P2
+    s = 1.0 / math.sqrt(d)
+    z = A / s
+    phi = math.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+    Q = float(special.ndtr(-z))
+    return Q, s * phi, s * s * (z * phi + Q)
+
+
+def dither_mse(step: float, bits: int, d: int, density: str = "beta") -> float:
+    """D(delta): expected squared error of one coordinate under the dithered uniform grid."""
+    n = 2 ** bits
+    A = (n - 1) * step / 2.0
+    P0, P1, P2 = tail_moments(A, d, density)
+    return step * step / 12.0 + 2.0 * (P2 - 2.0 * A * P1 + A * A * P0)
+
+
+def dither_step(bits: int, d: int, density: str = "beta") -> float:
+    """The minimiser of D: root of delta/6 - 2(n-1)[P1(A) - A P0(A)] by bisection."""
+    if bits < 1:
+        raise ValueError("bits must be >= 1")
+    n = 2 ** bits
+
+    def slope(step):
+        A = (n - 1) * step / 2.0
+        P0, P1, _ = tail_moments(A, d, density)
+        return step / 6.0 - 2.0 * (n - 1) * (P1 - A * P0)
+
+    lo = 0.0
+    hi = 2.0 / (n - 1) if density == "beta" else 2.0 * 40.0 / math.sqrt(d) / (n - 1)
+    while slope(hi) <= 0.0:
+        hi *= 2.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if mid == lo or mid == hi:
+            break
+        if slope(mid) > 0.0:
+            hi = mid
+        else:
+            lo = mid
+    return 0.5 * (lo + hi)
+
+
+def dither_codebook_f32(bits: int, d: int, density: str = "beta") -> tuple[np.ndarray, np.ndarray]:
+    """(centroids, boundaries) of the dithered quantizer as sorted float32 arrays:
+    c_j = (j - (n-1)/2) delta, boundaries (j + 1 - n/2) delta (the middle one exactly 0),
+    each rounded to fp32 from double."""
+    n = 2 ** bits
+    step = dither_step(bits, d, density)
+    j = np.arange(n, dtype=np.float64)
+    c = (j - (n - 1) / 2.0) * step
+    b = (np.arange(n - 1, dtype=np.float64) + 1.0 - n / 2.0) * step
+    return c.astype(np.float32), b.astype(np.float32)

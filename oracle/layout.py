@@ -21,6 +21,8 @@ page, kv head); the cache is [layer][physical page][kv head][block]):
   VC      value codes, b_v*d/8 bytes per token   b_v*16*P
   VS      QJL sign bits of the value residual    16*P   (values with QJL)
   VR      stored ||r_v|| as fp16                 2P     (values with QJL)
+  KD      key dither offset xi as fp16           2P     (dithered configurations)
+  VD      value dither offset xi as fp16         2P     (dithered configurations)
 
 Each code region is a sequence of 16-byte chunks per token, stored chunk-major:
 chunk c of token t sits at byte (c*P + t)*16 of the region.  Token t's chunks,
@@ -46,6 +48,10 @@ section "Two-Stage Approach: MSE Approximation + QJL Correction", which reconstr
 vector as x_mse + sqrt(pi/2)/d ||r|| S^T sign(S r) and notes that this serves the value
 cache too) store the residual's signs in VS (bit i = sigma_i, as KS) and its norm in VR;
 the two regions come last, so every other offset is the same with or without them.
+
+Dithered configurations (the "Minimum Distortion Quantization with Specified Output
+Distribution" page, third abstract: a random scalar offset per vector) keep each vector's
+offset, which the reconstruction adds back, in KD and VD after everything else.
 """
 from __future__ import annotations
 
@@ -63,6 +69,7 @@ class Format:
     value_bits: int = 3
     page_tokens: int = 256
     value_qjl: bool = False
+    dither: bool = False
 
     @property
     def merged_keys(self) -> bool:
@@ -80,7 +87,9 @@ class Format:
                  ("KC", self.key_bytes * P), ("KS", ks),
                  ("VC", self.value_bits * d // 8 * P),
                  ("VS", m // 8 * P if self.value_qjl else 0),
-                 ("VR", 2 * P if self.value_qjl else 0)]
+                 ("VR", 2 * P if self.value_qjl else 0),
+                 ("KD", 2 * P if self.dither else 0),
+                 ("VD", 2 * P if self.dither else 0)]
         out, off = {}, 0
         for name, sz in sizes:
             out[name] = (off, sz)
@@ -245,6 +254,9 @@ def write_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_
         if fmt.value_qjl:
             region("VR")[0:2 * (t1 - t0)] = fp16_bytes(vcomp.rnorm[t0:t1])
             _put_chunked(region("VS"), vsbytes[t0:t1], 0, P)
+        if fmt.dither:
+            region("KD")[0:2 * (t1 - t0)] = fp16_bytes(kcomp.offset[t0:t1])
+            region("VD")[0:2 * (t1 - t0)] = fp16_bytes(vcomp.offset[t0:t1])
 
 
 @dataclasses.dataclass
@@ -257,6 +269,8 @@ class Unpacked:
     k_sigma: np.ndarray = None
     v_rnorm: np.ndarray = None
     v_sigma: np.ndarray = None
+    k_offset: np.ndarray = None
+    v_offset: np.ndarray = None
 
 
 def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_of_seq,
@@ -265,7 +279,7 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
     P, d, m = fmt.page_tokens, fmt.head_dim, fmt.qjl_m
     reg = fmt.regions()
     kb, vb = fmt.key_bytes, fmt.value_bits * d // 8
-    parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc", "vr", "vs")}
+    parts = {k: [] for k in ("kn", "vn", "kr", "kc", "ks", "vc", "vr", "vs", "kd", "vd")}
     for lp in range((n + P - 1) // P):
         cnt = min(n, (lp + 1) * P) - lp * P
         blk = cache[layer, pages_of_seq[lp], head]
@@ -285,6 +299,9 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
         if fmt.value_qjl:
             parts["vr"].append(region("VR")[:2 * cnt].view(np.float16).astype(np.float64))
             parts["vs"].append(_get_chunked(region("VS"), cnt, m // 8, P))
+        if fmt.dither:
+            parts["kd"].append(region("KD")[:2 * cnt].view(np.float16).astype(np.float64))
+            parts["vd"].append(region("VD")[:2 * cnt].view(np.float16).astype(np.float64))
     cat = lambda k, w: np.concatenate(parts[k]) if parts[k] else np.zeros((0,) + w)
     kc = cat("kc", (kb,))
     vc = cat("vc", (vb,))
@@ -301,4 +318,7 @@ def read_sequence(cache: np.ndarray, fmt: Format, layer: int, head: int, pages_o
     if fmt.value_qjl:
         out.v_rnorm = cat("vr", ())
         out.v_sigma = bytes_to_bits(cat("vs", (m // 8,))).astype(bool)
+    if fmt.dither:
+        out.k_offset = cat("kd", ())
+        out.v_offset = cat("vd", ())
     return out
