@@ -427,14 +427,26 @@ def config_timings(dev, reps: int = 10):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     res = {}
-    for c in (1, 2, 3, 4, 5):
-        w = wl.CONFIGS[c]()
+    # the five workloads, then the config-2 layer in the other formats of the library: values
+    # with QJL, dithered HD, corrected key norms
+    cases = [(str(c), c, wl.CONFIGS[c]) for c in (1, 2, 3, 4, 5)]
+    cases += [("2_value_qjl", 2, lambda: wl.config2(value_qjl=True, name="c2_value_qjl")),
+              ("2_dither", 2, lambda: wl.config2(dither=True, name="c2_dither")),
+              ("2_corrected_norm", 2, lambda: wl.config2(key_corrected_norm=True, name="c2_corrected_norm"))]
+    for key, c, make in cases:
+        w = make()
         lens = wl.seq_lens(w)
         bt, npages = wl.block_table(w, lens)
         rin = wl.rotation_inputs(w)
         kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
                      key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits, rotation=w.rotation,
-                     num_layers=1, signs=rin["signs"], pi=rin["pi"], s=rin["s"], device=str(dev))
+                     num_layers=1, signs=rin["signs"], pi=rin["pi"], s=rin["s"], device=str(dev),
+                     value_qjl=w.value_qjl, dither=w.dither, key_corrected_norm=w.key_corrected_norm)
+        offs = {}
+        if w.dither:
+            t = kv.tensors
+            offs = dict(zip(("k_offsets", "v_offsets"), wl.dither_offsets_device(
+                w, 0, 0.5 * float(t["kc"][1] - t["kc"][0]), 0.5 * float(t["vc"][1] - t["vc"][0]), dev)))
         if c == 1:
             Kh, Vh = wl.make_kv(w, 0)
             K = torch.as_tensor(Kh, dtype=torch.float32, device=dev)
@@ -463,15 +475,15 @@ def config_timings(dev, reps: int = 10):
                 tot += a.elapsed_time(b)
             return 1e3 * tot / reps
 
-        comp_us = timed(lambda: kv.compress(0, K, V, seq, stream))
+        comp_us = timed(lambda: kv.compress(0, K, V, seq, stream, **offs))
         dec_us = timed(lambda: kv.decode(0, q, seq, ns, out=out, stream=stream))
-        kv.raise_on_error(f"config {c}")
+        kv.raise_on_error(f"config {key}")
         tokh = int(lens.sum()) * w.kv_heads
         in_b = 2 if w.in_dtype == "f16" else 4
         per_tok = kv.block_bytes / 256
         comp_bytes = tokh * (2 * 128 * in_b + per_tok)
         dec_bytes = tokh * per_tok + w.batch * w.q_heads * w.seq_q * 128 * (in_b + 4)
-        res[str(c)] = {
+        res[key] = {
             "workload": w.name, "n_splits": ns, "seq_q": w.seq_q,
             "compress_us": comp_us, "compress_gbs": comp_bytes / comp_us / 1e3,
             "compress_frac": comp_bytes / comp_us / 1e3 / hbm,
@@ -482,7 +494,7 @@ def config_timings(dev, reps: int = 10):
             "bytes_per_token_kv_head": per_tok,
             "l2": "flushed before every timed launch (a 256 MB buffer written, then read back)",
         }
-        del kv, K, V, q, out
+        del kv, K, V, q, out, offs
         torch.cuda.empty_cache()
     return res
 

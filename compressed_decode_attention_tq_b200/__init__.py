@@ -32,14 +32,16 @@ TQ_F32 = 1
 EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_check", "tq_validate_config", "tq_page_bytes",
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
            "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc", "tq_operand_bytes",
-           "tq_prepare_operands", "tq_append_kv", "tq_append_attend_decode")
+           "tq_prepare_operands", "tq_append_kv", "tq_append_attend_decode", "tq_dither_codebook",
+           "tq_compress_kv_dithered")
 
 
 class tq_config(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int32), ("key_bits", ctypes.c_int32),
                 ("key_qjl", ctypes.c_int32), ("qjl_m", ctypes.c_int32),
                 ("value_bits", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
-                ("rotation", ctypes.c_int32), ("value_qjl", ctypes.c_int32)]
+                ("rotation", ctypes.c_int32), ("value_qjl", ctypes.c_int32),
+                ("dither", ctypes.c_int32), ("key_corrected_norm", ctypes.c_int32)]
 
 
 class tq_params(ctypes.Structure):
@@ -76,7 +78,9 @@ def _load() -> ctypes.CDLL:
         "tq_validate_config": (I32, [cfgp]),
         "tq_page_bytes": (SZ, [cfgp]),
         "tq_codebook": (I32, [I32, I32, I32, P, P]),
+        "tq_dither_codebook": (I32, [I32, I32, I32, P, P]),
         "tq_compress_kv": (I32, [cfgp, parp, cachep, I32, P, P, I32, I32, P, P, P]),
+        "tq_compress_kv_dithered": (I32, [cfgp, parp, cachep, I32, P, P, P, P, I32, I32, P, P, P]),
         "tq_decode_workspace_bytes": (SZ, [cfgp, I32, I32, I32, I32]),
         "tq_attend_decode": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, SZ, P, P, P]),
         "tq_decode_scores": (I32, [cfgp, parp, cachep, I32, P, I32, I32, I32, P, I32, P, SZ, P, P, P]),
@@ -118,9 +122,9 @@ def _check(st: int, where: str):
 
 
 def make_config(head_dim=128, key_bits=3, key_qjl=True, qjl_m=128, value_bits=3, page_tokens=256,
-                rotation=TQ_ROT_HADAMARD, value_qjl=False) -> tq_config:
+                rotation=TQ_ROT_HADAMARD, value_qjl=False, dither=False, key_corrected_norm=False) -> tq_config:
     return tq_config(head_dim, key_bits, int(bool(key_qjl)), qjl_m, value_bits, page_tokens, rotation,
-                     int(bool(value_qjl)))
+                     int(bool(value_qjl)), int(bool(dither)), int(bool(key_corrected_norm)))
 
 
 def validate_config(cfg: tq_config) -> int:
@@ -137,6 +141,15 @@ def codebook(bits: int, head_dim: int = 128, density: int = TQ_DENSITY_BETA):
     c = np.zeros(1 << bits, dtype=np.float32)
     b = np.zeros((1 << bits) - 1, dtype=np.float32)
     _check(lib.tq_codebook(bits, head_dim, density, c.ctypes.data, b.ctypes.data), "tq_codebook")
+    return c, b
+
+
+def dither_codebook(bits: int, head_dim: int = 128, density: int = TQ_DENSITY_BETA):
+    """Uniform grid of the dithered quantizer -> (centroids, boundaries), numpy float32."""
+    import numpy as np
+    c = np.zeros(1 << bits, dtype=np.float32)
+    b = np.zeros((1 << bits) - 1, dtype=np.float32)
+    _check(lib.tq_dither_codebook(bits, head_dim, density, c.ctypes.data, b.ctypes.data), "tq_dither_codebook")
     return c, b
 
 
@@ -192,6 +205,23 @@ def compress_kv(cfg, params, cache, layer, k, v, seq_lens, status, stream=None):
     _check(lib.tq_compress_kv(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
                               _ptr(k), _ptr(v), dtype_code(k), max_len, _ptr(seq_lens), _ptr(status),
                               _stream(stream)), "tq_compress_kv")
+
+
+def compress_kv_dithered(cfg, params, cache, layer, k, v, k_offsets, v_offsets, seq_lens, status, stream=None):
+    """compress_kv for a dithered configuration; k_offsets, v_offsets: device float32
+    [batch][kv_heads][max_len], the offset of each vector."""
+    if v.shape != k.shape or v.dtype != k.dtype:
+        raise ValueError("k and v must have the same shape and dtype")
+    if k.dim() != 4:
+        raise ValueError("k and v must be [batch][kv_heads][max_len][d]")
+    import torch
+    for o in (k_offsets, v_offsets):
+        if tuple(o.shape) != tuple(k.shape[:3]) or o.dtype != torch.float32 or not o.is_contiguous():
+            raise ValueError("offsets must be contiguous float32 [batch][kv_heads][max_len]")
+    _check(lib.tq_compress_kv_dithered(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
+                                       _ptr(k), _ptr(v), _ptr(k_offsets), _ptr(v_offsets), dtype_code(k),
+                                       k.shape[2], _ptr(seq_lens), _ptr(status), _stream(stream)),
+           "tq_compress_kv_dithered")
 
 
 def decode_workspace_bytes(cfg, batch, q_heads, seq_q, n_splits) -> int:

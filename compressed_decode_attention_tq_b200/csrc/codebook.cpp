@@ -134,3 +134,51 @@ extern "C" tq_status tq_codebook(int32_t bits, int32_t head_dim, int32_t density
   for (int i = 0; i + 1 < n; ++i) boundaries[i] = (i == n / 2 - 1) ? 0.0f : (float)(0.5 * (c[i] + c[i + 1]));
   return TQ_OK;
 }
+
+// Uniform grid of the dithered quantizer ("Minimum Distortion Quantization with Specified
+// Output Distribution" page, third abstract).  With subtractive dither the expected squared
+// error of a coordinate y is delta^2/12 inside the outer levels and delta^2/12 + (|y| - A)^2
+// beyond them (A = (n-1) delta / 2), so D(delta) = delta^2/12 + 2 int_A^inf (t - A)^2 f(t) dt
+// and dD/d delta = delta/6 - 2 (n-1) [P1(A) - A P0(A)], P_k(A) = int_A^inf t^k f(t) dt.  The
+// derivative grows with delta (its own derivative is 1/6 + (n-1)^2 P0 > 0); its root is
+// found by bisection.
+extern "C" tq_status tq_dither_codebook(int32_t bits, int32_t head_dim, int32_t density, float* centroids,
+                                        float* boundaries) {
+  if (bits < 1 || bits > 8) return tqi::fail(TQ_ERR_INVALID_ARG, "tq_dither_codebook: bits must be in 1..8");
+  if (head_dim < 3) return tqi::fail(TQ_ERR_INVALID_ARG, "tq_dither_codebook: head_dim must be >= 3");
+  if (density != TQ_DENSITY_BETA && density != TQ_DENSITY_GAUSS)
+    return tqi::fail(TQ_ERR_INVALID_ARG, "tq_dither_codebook: unknown density");
+  if (!centroids || !boundaries)
+    return tqi::fail(TQ_ERR_INVALID_ARG, "tq_dither_codebook: null output pointer");
+  const int n = 1 << bits;
+  const Density f{head_dim, density == TQ_DENSITY_GAUSS};
+  const double hi_end = f.gauss ? INFINITY : 1.0;
+  auto slope = [&](double step) {
+    const double A = (n - 1) * step / 2.0;
+    if (!f.gauss && A >= 1.0) return step / 6.0;
+    double p0;
+    if (f.gauss) {
+      p0 = 0.5 * std::erfc(A * std::sqrt(f.d / 2.0));
+    } else {
+      const double a = (f.d - 1) / 2.0;
+      p0 = inc_beta(a, a, (1.0 - A) / 2.0);  // 1 - F(A), by the density's symmetry
+    }
+    const double p1 = f.first_moment(A, hi_end);
+    return step / 6.0 - 2.0 * (n - 1) * (p1 - A * p0);
+  };
+  double lo = 0.0;
+  double hi = f.gauss ? 80.0 / std::sqrt((double)head_dim) / (n - 1) : 2.0 / (n - 1);
+  while (slope(hi) <= 0.0) hi *= 2.0;
+  for (int it = 0; it < 200; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (mid == lo || mid == hi) break;
+    if (slope(mid) > 0.0)
+      hi = mid;
+    else
+      lo = mid;
+  }
+  const double step = 0.5 * (lo + hi);
+  for (int j = 0; j < n; ++j) centroids[j] = (float)((j - (n - 1) / 2.0) * step);
+  for (int j = 0; j + 1 < n; ++j) boundaries[j] = (float)((j + 1.0 - n / 2.0) * step);
+  return TQ_OK;
+}

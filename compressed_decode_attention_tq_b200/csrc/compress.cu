@@ -99,18 +99,19 @@ struct VecOut {
   int s[4], r[4];
 };
 
-// norm, rotation, quantization, packing of one vector (x already loaded).
+// norm, rotation, quantization, packing of one vector (x already loaded).  xi: the
+// vector's dither offset (0 when not dithered): idx = Quant(y - xi).  corr: store the
+// corrected norm n / ||c[idx] + xi|| ("tq-kv" documentation: corrected_norm) instead of n.
 __device__ __forceinline__ void encode_vector(const float (&x)[4], int bits, const float* cent,
                                               const float* bnd, const float* signs, const float* pi_s,
                                               float* stage, int lane, uint32_t* wbuf, VecOut& out,
-                                              int32_t* status, bool defer_pack = false) {
+                                              int32_t* status, bool defer_pack = false, float xi = 0.f,
+                                              bool corr = false) {
   float ss = 0.f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) ss = fmaf(x[e], x[e], ss);
   ss = warp_sum(ss);
   const float n = sqrtf(ss);
-  out.norm = __float2half_rn(n);
-  if (__hisinf(out.norm) && lane == 0) report(status, TQ_ERR_OVERFLOW);
   const float inv = n > 0.f ? 1.0f / n : 0.0f;
   float y[4];
   if (pi_s == nullptr) {
@@ -136,30 +137,40 @@ __device__ __forceinline__ void encode_vector(const float (&x)[4], int bits, con
   const int nb = (1 << bits) - 1;
   const int h = 1 << (bits - 1);
   int s[4], r[4];
+  float yy = 0.f;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
+    const float yq = y[e] - xi;
     int idx = 0;
-    for (int i = 0; i < nb; ++i) idx += (y[e] > bnd[i]) ? 1 : 0;
+    for (int i = 0; i < nb; ++i) idx += (yq > bnd[i]) ? 1 : 0;
     out.idx[e] = idx;
     s[e] = idx >= h;
     r[e] = s[e] ? idx - h : h - 1 - idx;
     out.s[e] = s[e];
     out.r[e] = r[e];
+    const float yh = cent[idx] + xi;
+    yy = fmaf(yh, yh, yy);
   }
+  float stored = n;
+  if (corr) {
+    const float yn = sqrtf(warp_sum(yy));
+    stored = yn > 0.f ? n / yn : 0.f;
+  }
+  out.norm = __float2half_rn(stored);
+  if (__hisinf(out.norm) && lane == 0) report(status, TQ_ERR_OVERFLOW);
   if (!defer_pack) pack_words(s, r, bits, lane, wbuf);
-  (void)cent;
 }
 
-// QJL sketch of the residual in the original space, r = x - fp16(n) R^T c[idx] ("TurboQuant
-// explained", section "Two-Stage Approach"): returns fp16(||r||) and the signs
+// QJL sketch of the residual in the original space, r = x - fp16(n) R^T (c[idx] + xi)
+// ("TurboQuant explained", section "Two-Stage Approach"): returns fp16(||r||) and the signs
 // sg[e] = [(S r)_j >= 0] of the lane's rows j = lane + 32 e (sign(0) stored as +1).
 __device__ __forceinline__ __half qjl_residual_signs(const float (&x)[4], const int (&idx)[4], __half norm,
                                                      const float* cent, const float* signs,
                                                      const float* pi_s, const float* s_s, float* stage,
-                                                     int lane, int (&sg)[4]) {
+                                                     int lane, int (&sg)[4], float xi = 0.f) {
   float z[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) z[e] = cent[idx[e]];
+  for (int e = 0; e < 4; ++e) z[e] = cent[idx[e]] + xi;
   if (pi_s == nullptr) {
     fwht128_warp(z, lane);
 #pragma unroll
@@ -260,20 +271,31 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
     uint8_t* blk = a.cache.block(phys, h);
     const int slot = t % PT;
     const size_t row = (head_off + t) * D;
+    // dithered: the vectors' offsets, used and stored as fp16
+    __half kxi = __float2half_rn(0.f), vxi = kxi;
+    if (L.dither) {
+      kxi = __float2half_rn(a.k_off[head_off + t]);
+      vxi = __float2half_rn(a.v_off[head_off + t]);
+      if (lane == 0) {
+        reinterpret_cast<__half*>(blk + L.kd)[slot] = kxi;
+        reinterpret_cast<__half*>(blk + L.vd)[slot] = vxi;
+      }
+    }
     // ---- key
     float x[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) x[e] = ld_in<T>(kin + row + lane + 32 * e);
     VecOut ko;
     encode_vector(x, L.kbits, sm.kc, sm.kb, sm.signs, pis, stage, lane, wbuf, ko, a.status,
-                  L.kmerged != 0);
+                  L.kmerged != 0, __half2float(kxi), a.key_corr != 0);
     __syncwarp();
     if (!L.kmerged && lane < L.kbits)
       reinterpret_cast<uint4*>(blk + L.kc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
     if (lane == 0) reinterpret_cast<__half*>(blk + L.kn)[slot] = ko.norm;
     if (a.qjl) {
       int sg[4];
-      const __half rho = qjl_residual_signs(x, ko.idx, ko.norm, sm.kc, sm.signs, pis, s_s, stage, lane, sg);
+      const __half rho =
+          qjl_residual_signs(x, ko.idx, ko.norm, sm.kc, sm.signs, pis, s_s, stage, lane, sg, __half2float(kxi));
       if (L.kmerged) {
         pack_merged(ko.s, ko.r, sg, lane, wbuf);
         __syncwarp();
@@ -296,7 +318,8 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
     for (int e = 0; e < 4; ++e) x[e] = ld_in<T>(vin + row + lane + 32 * e);
     VecOut vo;
     __syncwarp();
-    encode_vector(x, L.vbits, sm.vc, sm.vb, sm.signs, pis, stage, lane, wbuf, vo, a.status);
+    encode_vector(x, L.vbits, sm.vc, sm.vb, sm.signs, pis, stage, lane, wbuf, vo, a.status, false,
+                  __half2float(vxi));
     __syncwarp();
     if (lane < L.vbits)
       reinterpret_cast<uint4*>(blk + L.vc)[lane * PT + slot] = reinterpret_cast<const uint4*>(wbuf)[lane];
@@ -305,7 +328,8 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
     if (L.vqjl) {
       // values with QJL: the same sketch of the value residual, signs in VS, norm in VR
       int sg[4];
-      const __half rho = qjl_residual_signs(x, vo.idx, vo.norm, sm.vc, sm.signs, pis, s_s, stage, lane, sg);
+      const __half rho =
+          qjl_residual_signs(x, vo.idx, vo.norm, sm.vc, sm.signs, pis, s_s, stage, lane, sg, __half2float(vxi));
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t w = __ballot_sync(FULL, sg[e]);

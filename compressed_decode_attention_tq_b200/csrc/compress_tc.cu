@@ -1100,7 +1100,7 @@ cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtens
 
 bool compress_tc_supported(const CompressArgs& a) {
   const Layout& L = a.cache.L;
-  if (a.in_dtype != TQ_F16 || L.vqjl) return false;
+  if (a.in_dtype != TQ_F16 || L.vqjl || L.dither || a.key_corr) return false;
   if (a.dense && (L.qjl || a.operands == nullptr)) return false;
   if ((size_t)a.cache.batch * a.cache.kv_heads * a.max_len >= (1ull << 31)) return false;
   if (L.qjl && !(L.kbits == 2 || L.kbits == 3)) return false;

@@ -122,18 +122,26 @@ __device__ __forceinline__ void pack_code(int s, int r, int bits, int lane, int 
 }
 
 // Encodes thread i's coordinate of one vector: stored norm, index, (s, r); returns y.
+// cent non-null: store the corrected norm n / ||c[idx]|| ("tq-kv" documentation:
+// corrected_norm) instead of n.
 __device__ __forceinline__ float encode_coord(const DecodeArgs& a, AppendShared& sh, float x, const float* bnd,
                                               int bits, int i, int lane, int warp, __half& nh, int& idx,
-                                              int& s, int& r) {
+                                              int& s, int& r, const float* cent = nullptr) {
   const float n = sqrtf(block_sum128(x * x, sh.red, lane, warp));
-  nh = __float2half_rn(n);
-  if (__hisinf(nh) && i == 0) report(a.status, TQ_ERR_OVERFLOW);
   const float y = rotate_coord(a, sh, x, n > 0.f ? 1.0f / n : 0.0f, i, lane, warp);
   const int nb = (1 << bits) - 1, h = 1 << (bits - 1);
   idx = 0;
   for (int k = 0; k < nb; ++k) idx += (y > bnd[k]) ? 1 : 0;
   s = idx >= h;
   r = s ? idx - h : h - 1 - idx;
+  float stored = n;
+  if (cent) {
+    const float c = cent[idx];
+    const float yn = sqrtf(block_sum128(c * c, sh.red, lane, warp));
+    stored = yn > 0.f ? n / yn : 0.f;
+  }
+  nh = __float2half_rn(stored);
+  if (__hisinf(nh) && i == 0) report(a.status, TQ_ERR_OVERFLOW);
   return y;
 }
 
@@ -222,7 +230,7 @@ __device__ void append_token(const DecodeArgs& a, int job) {
                                         : ld_new<float>(a.k_new, src);
   __half nh;
   int idx, s, r;
-  encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r);
+  encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r, a.key_corr ? sh.tab[0] : nullptr);
   if (!L.kmerged) pack_code(s, r, L.kbits, lane, warp, sh.kw);
   if (a.qjl) {
     int sigma;
@@ -389,10 +397,12 @@ struct SmemSplit {
   float p[kRowsMax][kTile];
   uint32_t vcode[kTile][17];  // up to 16 words per token (+1 pad)
   float vnorm[kTile];
+  float vxi[kTile];           // dithered values: the offset of each token
   uint32_t vsig[kTile][4];    // values with QJL: the residual's sign bits
   float vrho[kTile];          // and its stored norm
   float kmag[8], vmag[8];
   float sqsum[kRowsMax];
+  float qsum[kRowsMax];  // dithered keys: sum_i (R q)_i, the weight of a key's offset
   float m[kRowsMax], l[kRowsMax], alpha[kRowsMax];
 };
 
@@ -425,6 +435,12 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     float t = 0.f;
     for (int i = 0; i < QM; ++i) t += sm.sq[tid][i];
     sm.sqsum[tid] = t;
+  }
+  if (L.dither && tid < R) {
+    // <R q, c[idx] + xi 1> = <R q, c[idx]> + xi sum_i (R q)_i
+    float t = 0.f;
+    for (int i = 0; i < D; ++i) t += sm.qrot[tid][i];
+    sm.qsum[tid] = t;
   }
   const int len = a.seq_lens[b];
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT || (kScoresOnly && len > a.max_len);
@@ -527,10 +543,11 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
       }
       const float kn = __half2float(reinterpret_cast<const __half*>(blk + L.kn)[slot]);
       const float rho = qjl ? __half2float(reinterpret_cast<const __half*>(blk + L.kr)[slot]) : 0.f;
+      const float kxi = L.dither ? __half2float(reinterpret_cast<const __half*>(blk + L.kd)[slot]) : 0.f;
 #pragma unroll
       for (int r = 0; r < RB; ++r) {
         if (r < R) {
-          float sc = kn * dot[r];
+          float sc = kn * (L.dither ? fmaf(kxi, sm.qsum[r], dot[r]) : dot[r]);
           if (L.qjl) sc = fmaf(rho * kQjlScale, 2.f * qj[r] - sm.sqsum[r], sc);
           sc *= kInvSqrtD;
           if (kScoresOnly)
@@ -546,6 +563,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
           sm.vcode[tid][4 * c + 2] = v4.z; sm.vcode[tid][4 * c + 3] = v4.w;
         }
         vn = __half2float(reinterpret_cast<const __half*>(blk + L.vn)[slot]);
+        if (L.dither) sm.vxi[tid] = __half2float(reinterpret_cast<const __half*>(blk + L.vd)[slot]);
         if (L.vqjl) {
           const uint4 s4 = reinterpret_cast<const uint4*>(blk + L.vs)[slot];
           sm.vsig[tid][0] = s4.x; sm.vsig[tid][1] = s4.y; sm.vsig[tid][2] = s4.z; sm.vsig[tid][3] = s4.w;
@@ -557,6 +575,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     }
     if (kScoresOnly) continue;
     sm.vnorm[tid] = valid ? vn : 0.f;
+    if (L.dither && !valid) sm.vxi[tid] = 0.f;
     if (L.vqjl && !valid) sm.vrho[tid] = 0.f;
     __syncthreads();
     // ---- phase B: online softmax bookkeeping, warp per row
@@ -595,7 +614,9 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
     for (int tt = 0; tt < nt; ++tt) {
       int s, rk;
       code_fields(sm.vcode[tt], L.vbits, j, s, rk);
-      const float val = (s ? sm.vmag[rk] : -sm.vmag[rk]) * sm.vnorm[tt];
+      float c = s ? sm.vmag[rk] : -sm.vmag[rk];
+      if (L.dither) c += sm.vxi[tt];
+      const float val = c * sm.vnorm[tt];
 #pragma unroll
       for (int r = 0; r < RB; ++r)
         if (r < R) acc[r] = fmaf(sm.p[r][tt], val, acc[r]);

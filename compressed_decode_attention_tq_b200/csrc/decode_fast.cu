@@ -836,6 +836,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 
 bool fast_decode_supported(const DecodeArgs& a) {
   const Layout& L = a.cache.L;
+  // the merge un-rotates with H D; dithered codes need their offsets (general kernels)
+  if (a.dense || L.dither) return false;
   const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl);
   const bool vok = (L.vbits == 3 || L.vbits == 2) && !L.vqjl;
   return kok && vok;

@@ -1,7 +1,8 @@
 // Decompression of the packed cache to dense fp32 K_hat / V_hat.
 //
 // "turboquant_cutile" function list: "indices -> centroids -> un-rotate -> rescale"
-// (4-level and 8-level decompress kernels).  For keys with QJL this returns the MSE
+// (4-level and 8-level decompress kernels); dithered codes add their stored offset to the
+// centroids before un-rotating.  For keys with QJL this returns the MSE
 // part k_mse = ||k|| R^T c[idx] ("k_mse should be a reasonable approximation of K").
 // One warp per (token, kv head), lane l holds coordinates l + 32 e.
 #include <cuda_fp16.h>
@@ -15,9 +16,9 @@ namespace {
 
 constexpr float kInvSqrtD = 0.08838834764831845f;
 
-__device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, int bits, int merged,
-                              int slot, const float* cent, const float* signs, const float* pi,
-                              float* stage, int lane, float* dst) {
+__device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, int off_off, int bits,
+                              int merged, int slot, const float* cent, const float* signs,
+                              const float* pi, float* stage, int lane, float* dst) {
   uint32_t w[16];
   const int chunks = merged ? 4 : bits;
   for (int c = 0; c < chunks; ++c) {
@@ -38,6 +39,12 @@ __device__ void decode_vector(const uint8_t* blk, int code_off, int norm_off, in
       code_fields(w, bits, lane + 32 * e, s, r);
     }
     z[e] = s ? cent[h + r] : -cent[h + r];
+  }
+  if (off_off >= 0) {
+    // dithered: c[idx] + xi
+    const float xi = __half2float(reinterpret_cast<const __half*>(blk + off_off)[slot]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) z[e] += xi;
   }
   const float n = __half2float(reinterpret_cast<const __half*>(blk + norm_off)[slot]);
   if (pi == nullptr) {
@@ -80,11 +87,11 @@ __global__ void decompress_kernel(DecompressArgs a) {
   const Layout& L = a.cache.L;
   const float* pi = a.dense ? a.pi : nullptr;
   if (a.k_hat)
-    decode_vector(blk, L.kc, L.kn, L.kbits, L.kmerged, slot, a.k_centroids, a.signs, pi, stage[w], lane,
-                  a.k_hat + row);
+    decode_vector(blk, L.kc, L.kn, L.dither ? L.kd : -1, L.kbits, L.kmerged, slot, a.k_centroids, a.signs, pi,
+                  stage[w], lane, a.k_hat + row);
   if (a.v_hat)
-    decode_vector(blk, L.vc, L.vn, L.vbits, 0, slot, a.v_centroids, a.signs, pi, stage[w], lane,
-                  a.v_hat + row);
+    decode_vector(blk, L.vc, L.vn, L.dither ? L.vd : -1, L.vbits, 0, slot, a.v_centroids, a.signs, pi,
+                  stage[w], lane, a.v_hat + row);
 }
 
 }  // namespace

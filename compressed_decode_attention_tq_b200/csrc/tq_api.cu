@@ -38,6 +38,11 @@ static tq_status check_config(const tq_config* cfg) {
   if (cfg->value_qjl != 0 && cfg->value_qjl != 1) return fail(TQ_ERR_INVALID_ARG, "value_qjl must be 0 or 1");
   if (cfg->rotation != TQ_ROT_HADAMARD && cfg->rotation != TQ_ROT_DENSE)
     return fail(TQ_ERR_INVALID_ARG, "unknown rotation kind");
+  if (cfg->dither != 0 && cfg->dither != 1) return fail(TQ_ERR_INVALID_ARG, "dither must be 0 or 1");
+  if (cfg->dither && cfg->rotation != TQ_ROT_HADAMARD)
+    return fail(TQ_ERR_UNSUPPORTED, "dither needs TQ_ROT_HADAMARD");
+  if (cfg->key_corrected_norm != 0 && cfg->key_corrected_norm != 1)
+    return fail(TQ_ERR_INVALID_ARG, "key_corrected_norm must be 0 or 1");
   return TQ_OK;
 }
 
@@ -69,7 +74,7 @@ static tqk::CacheRef cache_ref(const tq_config* cfg, const tq_cache* c, int32_t 
   r.batch = c->batch;
   r.kv_heads = c->kv_heads;
   r.layer = layer;
-  r.L = tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl);
+  r.L = tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl, cfg->dither);
   return r;
 }
 
@@ -79,7 +84,7 @@ using namespace tqi;
 
 extern "C" {
 
-int32_t tq_version(void) { return 101; }
+int32_t tq_version(void) { return 102; }
 
 const char* tq_status_str(tq_status st) {
   switch (st) {
@@ -124,13 +129,14 @@ tq_status tq_validate_config(const tq_config* cfg) {
 
 size_t tq_page_bytes(const tq_config* cfg) {
   if (check_config(cfg) != TQ_OK) return 0;
-  return (size_t)tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl).bytes;
+  return (size_t)tqk::make_layout(cfg->key_bits, cfg->key_qjl, cfg->value_bits, cfg->value_qjl, cfg->dither)
+      .bytes;
 }
 
-tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
-                         int32_t layer, const void* k, const void* v, int32_t in_dtype, int32_t max_len,
-                         const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
-  clear_error();
+static tq_status compress_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                 int32_t layer, const void* k, const void* v, const float* k_offsets,
+                                 const float* v_offsets, int32_t in_dtype, int32_t max_len,
+                                 const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
   if ((st = check_params(cfg, params, true)) != TQ_OK) return st;
@@ -147,6 +153,9 @@ tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq
   a.max_len = max_len;
   a.qjl = cfg->key_qjl;
   a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.key_corr = cfg->key_corrected_norm;
+  a.k_off = k_offsets;
+  a.v_off = v_offsets;
   a.seq_lens = seq_lens;
   a.signs = params->signs;
   a.pi = params->pi;
@@ -162,6 +171,27 @@ tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq
   cudaError_t e = tqk::launch_compress(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_compress_kv launch");
   return TQ_OK;
+}
+
+tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                         int32_t layer, const void* k, const void* v, int32_t in_dtype, int32_t max_len,
+                         const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  if (cfg && cfg->dither)
+    return fail(TQ_ERR_INVALID_ARG, "a dithered configuration is compressed by tq_compress_kv_dithered");
+  return compress_common(cfg, params, cache, layer, k, v, nullptr, nullptr, in_dtype, max_len, seq_lens,
+                         dev_status, stream);
+}
+
+tq_status tq_compress_kv_dithered(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                  int32_t layer, const void* k, const void* v, const float* k_offsets,
+                                  const float* v_offsets, int32_t in_dtype, int32_t max_len,
+                                  const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  clear_error();
+  if (!cfg || !cfg->dither) return fail(TQ_ERR_INVALID_ARG, "tq_compress_kv_dithered needs cfg->dither = 1");
+  if (!k_offsets || !v_offsets) return fail(TQ_ERR_INVALID_ARG, "k_offsets or v_offsets is NULL");
+  return compress_common(cfg, params, cache, layer, k, v, k_offsets, v_offsets, in_dtype, max_len, seq_lens,
+                         dev_status, stream);
 }
 
 size_t tq_operand_bytes(const tq_config* cfg) {
@@ -238,6 +268,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.n_splits = n_splits;
   a.qjl = cfg->key_qjl;
   a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.key_corr = cfg->key_corrected_norm;
   a.seq_lens = seq_lens;
   a.signs = params->signs;
   a.pi = params->pi;
@@ -271,6 +302,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
 // Checks of the appended tokens' arguments shared by tq_append_kv and tq_append_attend_decode.
 static tq_status check_append(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                               const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new) {
+  if (cfg->dither) return fail(TQ_ERR_UNSUPPORTED, "appends take no dither offsets");
   if (!params->k_boundaries || !params->v_boundaries) return fail(TQ_ERR_INVALID_ARG, "boundary pointer is NULL");
   if (!k_new || !v_new) return fail(TQ_ERR_INVALID_ARG, "k_new or v_new is NULL");
   if (in_dtype != TQ_F16 && in_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "in_dtype must be TQ_F16 or TQ_F32");
@@ -341,6 +373,7 @@ tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_c
   a.cache = cache_ref(cfg, cache, layer);
   a.qjl = cfg->key_qjl;
   a.dense = cfg->rotation == TQ_ROT_DENSE;
+  a.key_corr = cfg->key_corrected_norm;
   a.seq_lens = seq_lens;
   a.signs = params->signs;
   a.pi = params->pi;

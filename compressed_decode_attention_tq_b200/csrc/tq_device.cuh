@@ -22,14 +22,17 @@ struct Layout {
   int kchunks;  // 16-byte chunks of one token's key bit string
   int vqjl;     // values carry the QJL signs of their residual (VS) and its norm (VR)
   int vs, vr;
+  int dither;   // dithered: each vector's offset xi (fp16) in KD (keys) and VD (values)
+  int kd, vd;
 };
 
-__host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits, int vqjl = 0) {
+__host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits, int vqjl = 0, int dither = 0) {
   Layout L;
   L.kbits = kbits;
   L.vbits = vbits;
   L.qjl = qjl;
   L.vqjl = vqjl;
+  L.dither = dither;
   L.kmerged = (qjl && kbits == 3) ? 1 : 0;
   L.kchunks = L.kmerged ? 4 : kbits;
   int off = 0;
@@ -41,6 +44,8 @@ __host__ __device__ inline Layout make_layout(int kbits, int qjl, int vbits, int
   L.vc = off; off += vbits * (D / 8) * PT;
   L.vs = off; off += vqjl ? (QM / 8) * PT : 0;
   L.vr = off; off += vqjl ? 2 * PT : 0;
+  L.kd = off; off += dither ? 2 * PT : 0;
+  L.vd = off; off += dither ? 2 * PT : 0;
   L.bytes = off;
   return L;
 }

@@ -13,6 +13,8 @@ struct CompressArgs {
   const void* k;
   const void* v;
   int in_dtype, max_len, qjl, dense;
+  int key_corr;                  // keys store the corrected norm ||k|| / ||y_hat||
+  const float *k_off, *v_off;    // dithered: the offsets [batch][kv_heads][max_len], else null
   const int32_t* seq_lens;
   const float *signs, *pi, *s, *k_centroids, *k_boundaries, *v_centroids, *v_boundaries;
   const void* operands;  // prepared tensor-core operands (B = H D, S D H hi / lo; or sqrt(d) Pi hi / lo) or null
@@ -23,6 +25,7 @@ struct DecodeArgs {
   CacheRef cache;
   const void* q;
   int q_dtype, q_heads, seq_q, group, rows, n_splits, qjl, dense;
+  int key_corr;  // appended keys store the corrected norm
   const int32_t* seq_lens;
   const float *signs, *pi, *s, *k_centroids, *v_centroids;
   float* qrot;      // [B*Hq*seq_q][D]  workspace

@@ -10,7 +10,7 @@ from typing import Optional
 import torch
 
 from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, append_attend_decode, append_kv, attend_decode,
-               check_status, codebook, compress_kv, last_error,
+               check_status, codebook, compress_kv, compress_kv_dithered, dither_codebook, last_error,
                decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
                operand_bytes, page_bytes, prepare_operands)
 
@@ -39,10 +39,13 @@ class PagedKV:
     def __init__(self, *, batch: int, kv_heads: int, num_pages: int, block_table, key_bits: int,
                  key_qjl: bool, value_bits: int, rotation: int = TQ_ROT_HADAMARD,
                  num_layers: int = 1, signs=None, pi=None, s=None, codebooks=None,
-                 device: str = "cuda", prepared_operands: bool = True, value_qjl: bool = False):
+                 device: str = "cuda", prepared_operands: bool = True, value_qjl: bool = False,
+                 dither: bool = False, key_corrected_norm: bool = False):
         self.device = torch.device(device)
         self.cfg = make_config(key_bits=key_bits, key_qjl=key_qjl, value_bits=value_bits,
-                               rotation=rotation, value_qjl=value_qjl)
+                               rotation=rotation, value_qjl=value_qjl, dither=dither,
+                               key_corrected_norm=key_corrected_norm)
+        self.dither = bool(dither)
         self.block_bytes = page_bytes(self.cfg)
         if self.block_bytes == 0:
             raise TQError(2, "PagedKV", "unsupported configuration")
@@ -53,8 +56,9 @@ class PagedKV:
         self.pages = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
         if codebooks is None:
-            kc, kb = codebook(key_bits)
-            vc, vb = codebook(value_bits)
+            book = dither_codebook if dither else codebook
+            kc, kb = book(key_bits)
+            vc, vb = book(value_bits)
         else:
             kc, kb, vc, vb = codebooks
         self.tensors = {
@@ -80,8 +84,16 @@ class PagedKV:
         self._ws = {}
 
     # ---- calls -----------------------------------------------------------------------------
-    def compress(self, layer: int, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, stream=None):
-        compress_kv(self.cfg, self.params, self.cache, layer, k, v, seq_lens, self.status, stream)
+    def compress(self, layer: int, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, stream=None,
+                 k_offsets: Optional[torch.Tensor] = None, v_offsets: Optional[torch.Tensor] = None):
+        """A dithered cache takes each vector's offset (device float32 [batch][kv_heads][max_len])."""
+        if self.dither:
+            if k_offsets is None or v_offsets is None:
+                raise ValueError("a dithered cache needs k_offsets and v_offsets")
+            compress_kv_dithered(self.cfg, self.params, self.cache, layer, k, v, k_offsets, v_offsets,
+                                 seq_lens, self.status, stream)
+        else:
+            compress_kv(self.cfg, self.params, self.cache, layer, k, v, seq_lens, self.status, stream)
 
     def append(self, layer: int, k_new: torch.Tensor, v_new: torch.Tensor, seq_lens: torch.Tensor,
                stream=None):

@@ -51,6 +51,8 @@
  *   VC      value codes                               value_bits*16*P
  *   VS      QJL sign bits of the value residual        16*P   (value_qjl)
  *   VR      stored ||r_v|| (fp16) per token            2P     (value_qjl)
+ *   KD      key dither offset xi (fp16) per token      2P     (dither)
+ *   VD      value dither offset xi (fp16) per token    2P     (dither)
  *
  *   A code region stores each token's bytes as 16-byte chunks, chunk-major:
  *   chunk c of slot t is at region byte (c*P + t)*16.  A token's chunks,
@@ -68,7 +70,15 @@
  *   sigma_i = [(S r)_i >= 0] (sign(0) is stored as +1); there is no KS region.
  *   Other QJL keys: bit i of the KS chunk = sigma_i.
  *   Values with QJL: bit i of the VS chunk = [(S r_v)_i >= 0], r_v = v - v_mse.
+ *   Dithered configurations: a vector is coded as idx = Quant(y - xi) and read back as
+ *   n R^T (c[idx] + xi), xi its stored offset.
  *   Slots past a sequence's length are never read and their bytes unspecified.
+ *
+ * [DITHER]  "Minimum Distortion Quantization with Specified Output Distribution"
+ *           (thelatestinai.com), third abstract: dithered TurboQuant, one randomized
+ *           Hadamard transform and a random scalar offset subtracted before the scalar
+ *           quantizer; unbiased, MSE (pi sqrt(3)/2 + o(1)) 4^-b.  This library reads the
+ *           quantizer as a uniform grid (tq_dither_codebook) with subtractive dither.
  */
 #ifndef TQ_H_
 #define TQ_H_
@@ -119,6 +129,16 @@ typedef struct tq_config {
                            "Two-Stage Approach": the value is reconstructed as
                            v_mse + sqrt(pi/2)/m ||r_v|| S^T (2 sigma_v - 1)); served by
                            the general (CUDA-core) kernels                             */
+  int32_t dither;       /* 1: dithered HD ([DITHER]): every key and value is coded as
+                           Quant(y - xi) with its own offset xi, stored in KD / VD and added
+                           back at reconstruction; needs TQ_ROT_HADAMARD and the uniform
+                           grids of tq_dither_codebook; compressed by
+                           tq_compress_kv_dithered; served by the general kernels     */
+  int32_t key_corrected_norm; /* 1: keys store the corrected norm ([TQKV]
+                           compress_single_key returns "corrected_norm"): ||k|| / ||y_hat||
+                           with y_hat = c[idx] (+ xi), so that the reconstruction has the
+                           key's norm (0 for y_hat = 0); the decoder is unchanged. With
+                           QJL the residual is taken against this reconstruction.      */
 } tq_config;
 
 /* Random inputs of the method and the codebooks, all device memory, fp32.
@@ -198,6 +218,16 @@ TQ_API size_t tq_page_bytes(const tq_config* cfg);
 TQ_API tq_status tq_codebook(int32_t bits, int32_t head_dim, int32_t density, float* centroids,
                       float* boundaries);
 
+/* Uniform codebook of the dithered quantizer ([DITHER]; HOST call, synchronous):
+ * centroids c_j = (j - (2^b - 1)/2) delta, boundaries at their midpoints (the middle one
+ * 0), each rounded to fp32 from double.  delta minimises the expected squared error of a
+ * coordinate with density f_X (as for tq_codebook) under subtractive dither, xi uniform
+ * on [-delta/2, delta/2):  D(delta) = delta^2/12 + 2 int_A^inf (t - A)^2 f_X(t) dt,
+ * A = (2^b - 1) delta / 2; it is the root of dD/d delta (increasing in delta), found by
+ * bisection on the closed-form tail moments.  Arguments as for tq_codebook. */
+TQ_API tq_status tq_dither_codebook(int32_t bits, int32_t head_dim, int32_t density, float* centroids,
+                                    float* boundaries);
+
 /* Compress K and V into the packed cache ([CUTILE] compress K (MSE + QJL) and
  * compress V (MSE only); [MOBILINT] "Two-Stage Approach": per vector n = ||x||,
  * u = x/n, y = R u, idx_j = #{i : beta_i < y_j}, stored fp16(n); for keys with
@@ -208,11 +238,26 @@ TQ_API tq_status tq_codebook(int32_t bits, int32_t head_dim, int32_t density, fl
  *   seq_lens   device int32 [batch]; tokens 0..seq_lens[b]-1 of each (b, head) are
  *              written to slots via the block table (logical page t/P, slot t%P)
  *   dev_status device int32; TQ_ERR_OVERFLOW, TQ_ERR_BOUNDS, TQ_ERR_INVALID_ARG
- * Pages not covered by a sequence are not touched. */
+ * Pages not covered by a sequence are not touched.  A dithered configuration returns
+ * TQ_ERR_INVALID_ARG (its offsets come through tq_compress_kv_dithered). */
 TQ_API tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                          int32_t layer, const void* k, const void* v, int32_t in_dtype,
                          int32_t max_len, const int32_t* seq_lens, int32_t* dev_status,
                          tq_stream_t stream);
+
+/* tq_compress_kv for a dithered configuration (cfg->dither = 1, [DITHER]): every vector
+ * x = k or v of token t is coded with its own offset xi = fp16(offsets[b][h][t]) (RNE):
+ * y = H D x / ||x||, idx = #{i : beta_i < y_j - xi}, xi stored in KD / VD.  The caller
+ * draws the offsets (uniform on [-delta/2, delta/2), delta = c[1] - c[0] of the
+ * tq_dither_codebook grid, makes the reconstruction unbiased inside the grid's range).
+ *   k_offsets, v_offsets  device float [batch][kv_heads][max_len]
+ * Everything else as for tq_compress_kv; TQ_ERR_INVALID_ARG for a configuration that is
+ * not dithered. */
+TQ_API tq_status tq_compress_kv_dithered(const tq_config* cfg, const tq_params* params,
+                                         const tq_cache* cache, int32_t layer, const void* k,
+                                         const void* v, const float* k_offsets, const float* v_offsets,
+                                         int32_t in_dtype, int32_t max_len, const int32_t* seq_lens,
+                                         int32_t* dev_status, tq_stream_t stream);
 
 /* Bytes of the prepared tensor-core operands of tq_compress_kv for cfg (96 KiB for a
  * TQ_ROT_HADAMARD configuration, 64 KiB for TQ_ROT_DENSE; 0 if cfg is invalid). */
@@ -282,7 +327,8 @@ TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params,
  *                 block-table row or a page id is out of range (that token is skipped);
  *                 TQ_ERR_OVERFLOW as for tq_compress_kv
  * params.s (with key_qjl) and params.pi (TQ_ROT_DENSE) must be 16-byte aligned; S is
- * used in fp32 as given (no fp16 requirement).  One thread block per new token. */
+ * used in fp32 as given (no fp16 requirement).  One thread block per new token.
+ * Dithered configurations return TQ_ERR_UNSUPPORTED (no offsets are taken here). */
 TQ_API tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                               int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
                               int32_t n_new, const int32_t* seq_lens, int32_t* dev_status,
@@ -342,7 +388,8 @@ TQ_API tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params,
 
 /* Decompress ([CUTILE] "indices -> centroids -> un-rotate -> rescale"):
  * k_hat = ||k|| R^T c_k[idx] (the MSE part k_mse for QJL keys) and
- * v_hat = ||v|| R^T c_v[idx_v] (the MSE part for values with QJL), for tokens
+ * v_hat = ||v|| R^T c_v[idx_v] (the MSE part for values with QJL), c[idx] + xi for
+ * dithered configurations, with the stored (possibly corrected) norms, for tokens
  * t < seq_lens[b]; rows past the
  * length are left untouched.
  *   k_hat, v_hat  device float [batch][kv_heads][max_len][d] (either may be NULL) */

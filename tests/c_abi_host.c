@@ -39,12 +39,17 @@ int main(void) {
   cfg.page_tokens = 256;
   cfg.rotation = TQ_ROT_HADAMARD;
   cfg.value_qjl = 0;
+  cfg.dither = 0;
+  cfg.key_corrected_norm = 0;
   CHECK(tq_validate_config(&cfg) == TQ_OK, "validate config");
   /* KN, KR, VN 512 B each, merged key nibbles 64 * 256 B, 3-bit values 48 * 256 B */
   CHECK(tq_page_bytes(&cfg) == 3 * 512 + 64 * 256 + 48 * 256, "page bytes");
   cfg.value_qjl = 1;
   CHECK(tq_page_bytes(&cfg) == 3 * 512 + 64 * 256 + 48 * 256 + 16 * 256 + 512, "page bytes, values with QJL");
   cfg.value_qjl = 0;
+  cfg.dither = 1;
+  CHECK(tq_page_bytes(&cfg) == 3 * 512 + 64 * 256 + 48 * 256 + 2 * 512, "page bytes, dithered");
+  cfg.dither = 0;
   CHECK(tq_operand_bytes(&cfg) == 3 * 128 * 128 * 2, "operand bytes");
   CHECK(tq_decode_workspace_bytes(&cfg, 1, 32, 1, 16) > 0, "workspace bytes");
 
@@ -53,6 +58,11 @@ int main(void) {
   CHECK(tq_codebook(1, 128, TQ_DENSITY_BETA, c, b) == TQ_OK, "codebook call");
   const double e_abs = exp(lgamma(64.0) - lgamma(64.5)) / sqrt(acos(-1.0));
   CHECK(fabs(c[1] - e_abs) < 1e-6 && c[0] == -c[1] && b[0] == 0.0f, "1-bit Beta centroids");
+
+  /* the dithered quantizer's grid: uniform, symmetric, middle boundary 0 */
+  float dc[8], db[7];
+  CHECK(tq_dither_codebook(3, 128, TQ_DENSITY_BETA, dc, db) == TQ_OK, "dither codebook call");
+  CHECK(dc[0] == -dc[7] && db[3] == 0.0f && fabs((dc[2] - dc[1]) - (dc[1] - dc[0])) < 1e-6, "dither grid");
 
   /* host-side argument errors are returned, nothing is enqueued, the detail is kept */
   CHECK(tq_compress_kv(&cfg, NULL, NULL, 0, NULL, NULL, TQ_F16, 16, NULL, NULL, NULL) == TQ_ERR_INVALID_ARG,

@@ -48,6 +48,8 @@ class Run:
     kv: object = None
     K: dict = None
     V: dict = None
+    KO: dict = None   # dithered: the key offsets of each layer [batch][kv_heads][max_len]
+    VO: dict = None
 
 
 def setup(w: wl.Workload, layers=(0,), prepared_operands=True, compress_lens=None):
@@ -61,22 +63,32 @@ def setup(w: wl.Workload, layers=(0,), prepared_operands=True, compress_lens=Non
     run = Run(w=w, lens=lens, bt=bt, npages=npages, rin=rin,
               R=orot.rotation_matrix(w.rotation, rin["signs"], rin["pi"]),
               fmt=olay.Format(key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits,
-                              value_qjl=w.value_qjl),
+                              value_qjl=w.value_qjl, dither=w.dither),
               ck=None, kb=None, cv=None, vb=None)
-    run.ck, run.kb = ocb.codebook_f32(w.key_bits, 128)
-    run.cv, run.vb = ocb.codebook_f32(w.value_bits, 128)
+    book = ocb.dither_codebook_f32 if w.dither else ocb.codebook_f32
+    run.ck, run.kb = book(w.key_bits, 128)
+    run.cv, run.vb = book(w.value_bits, 128)
     run.kv = PagedKV(batch=w.batch, kv_heads=w.kv_heads, num_pages=npages, block_table=bt,
                      key_bits=w.key_bits, key_qjl=w.key_qjl, value_bits=w.value_bits, value_qjl=w.value_qjl,
                      rotation=w.rotation, num_layers=max(layers) + 1, signs=rin["signs"],
-                     pi=rin["pi"], s=rin["s"], prepared_operands=prepared_operands)
-    run.K, run.V = {}, {}
+                     pi=rin["pi"], s=rin["s"], prepared_operands=prepared_operands, dither=w.dither,
+                     key_corrected_norm=w.key_corrected_norm)
+    run.K, run.V, run.KO, run.VO = {}, {}, {}, {}
     dt = torch.float16 if w.in_dtype == "f16" else torch.float32
     seq = torch.as_tensor(lens if compress_lens is None else compress_lens, dtype=torch.int32, device="cuda")
     for layer in layers:
         K, V = wl.make_kv(w, layer)
         run.K[layer], run.V[layer] = K, V
+        offs = {}
+        if w.dither:
+            # offsets uniform over one cell of each grid
+            KO, VO = wl.dither_offsets(w, layer, 0.5 * float(run.ck[1] - run.ck[0]),
+                                       0.5 * float(run.cv[1] - run.cv[0]))
+            run.KO[layer], run.VO[layer] = KO, VO
+            offs = dict(k_offsets=torch.as_tensor(KO, dtype=torch.float32, device="cuda"),
+                        v_offsets=torch.as_tensor(VO, dtype=torch.float32, device="cuda"))
         run.kv.compress(layer, torch.as_tensor(K, dtype=dt, device="cuda"),
-                        torch.as_tensor(V, dtype=dt, device="cuda"), seq)
+                        torch.as_tensor(V, dtype=dt, device="cuda"), seq, **offs)
     return run
 
 
@@ -124,10 +136,15 @@ def _check_qjl(gpu_sigma, gpu_rnorm, comp, mis, rep):
     rep.sign_mismatch_out_of_band += int(np.sum(diff & ~band))
 
 
-def _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep):
-    kc = oq.compress_prod(K, R, ck, kb, S) if fmt.key_qjl else oq.compress_mse(K, R, ck, kb)
-    vc = oq.compress_prod(V, R, cv, vb, S) if fmt.value_qjl else oq.compress_mse(V, R, cv, vb)
+def _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep, KO=None, VO=None, corrected=False):
+    kx = dict(offsets=KO, corrected_norm=corrected)
+    vx = dict(offsets=VO)
+    kc = oq.compress_prod(K, R, ck, kb, S, **kx) if fmt.key_qjl else oq.compress_mse(K, R, ck, kb, **kx)
+    vc = oq.compress_prod(V, R, cv, vb, S, **vx) if fmt.value_qjl else oq.compress_mse(V, R, cv, vb, **vx)
     rep.tokens += K.shape[0]
+    if fmt.dither:
+        # the stored offsets are the fp16 roundings of the given ones, exactly
+        rep.norm_fail += int(np.sum(u.k_offset != kc.offset)) + int(np.sum(u.v_offset != vc.offset))
     kmis = _check_idx(u.k_idx, kc, kb, rep)
     vmis = _check_idx(u.v_idx, vc, vb, rep)
     rep.norm_fail += int(np.sum(~close(u.k_norm, kc.norm)))
@@ -139,10 +156,10 @@ def _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep):
     return rep
 
 
-def compare_compress_rows(fmt, u, K, V, R, ck, kb, cv, vb, S, rep: CompressReport):
+def compare_compress_rows(fmt, u, K, V, R, ck, kb, cv, vb, S, rep: CompressReport, corrected=False):
     """Compares unpacked GPU codes u (tokens in the order of the rows) with the oracle's
     compression of the same float64 rows K, V [n][d]."""
-    return _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep)
+    return _compare_unpacked(fmt, u, K, V, R, ck, kb, cv, vb, S, rep, corrected=corrected)
 
 
 def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport = None):
@@ -153,11 +170,14 @@ def compare_compress(run, pages, layer, b, h, tokens=None, rep: CompressReport =
     u = olay.read_sequence(pages, run.fmt, layer, h, run.bt[b], n)
     sel = np.arange(n) if tokens is None else np.asarray(tokens)
     sub = olay.Unpacked(k_idx=u.k_idx[sel], k_norm=u.k_norm[sel], v_idx=u.v_idx[sel], v_norm=u.v_norm[sel])
-    for f in ("k_rnorm", "k_sigma", "v_rnorm", "v_sigma"):
+    for f in ("k_rnorm", "k_sigma", "v_rnorm", "v_sigma", "k_offset", "v_offset"):
         if getattr(u, f) is not None:
             setattr(sub, f, getattr(u, f)[sel])
+    KO = run.KO[layer][b, h][sel] if run.w.dither else None
+    VO = run.VO[layer][b, h][sel] if run.w.dither else None
     return _compare_unpacked(run.fmt, sub, run.K[layer][b, h][sel], run.V[layer][b, h][sel], run.R,
-                             run.ck, run.kb, run.cv, run.vb, run.rin["s"], rep)
+                             run.ck, run.kb, run.cv, run.vb, run.rin["s"], rep, KO, VO,
+                             run.w.key_corrected_norm)
 
 
 def _check_idx(gpu_idx, comp, boundaries, rep):
@@ -178,6 +198,6 @@ def oracle_scores(run, pages, layer, q, b, h):
     """Scores of query head h of sequence b over its cached tokens: [seq_q, n]."""
     G = run.w.group
     u = olay.read_sequence(pages, run.fmt, layer, h // G, run.bt[b], int(run.lens[b]))
-    k_mse = oq.reconstruct_mse(u.k_idx, u.k_norm, run.R, run.ck)
+    k_mse = oq.reconstruct_mse(u.k_idx, u.k_norm, run.R, run.ck, u.k_offset)
     return oatt.scores_compressed(q[b, h], k_mse, u.k_rnorm, u.k_sigma,
                                   run.rin["s"] if run.w.key_qjl else None)

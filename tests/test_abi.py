@@ -59,6 +59,69 @@ def test_library_codebook_other_d(tq, d):
     np.testing.assert_array_equal(b, ob)
 
 
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("density", [0, 1])
+def test_library_dither_codebook_equals_oracle(tq, bits, density):
+    from oracle import codebook as ocb
+    c, b = tq.dither_codebook(bits, 128, density)
+    oc, ob = ocb.dither_codebook_f32(bits, 128, "beta" if density == 0 else "gauss")
+    np.testing.assert_array_equal(c, oc)
+    np.testing.assert_array_equal(b, ob)
+
+
+def test_dither_codebook_argument_errors(tq):
+    c = np.zeros(4, np.float32)
+    b = np.zeros(3, np.float32)
+    assert tq.lib.tq_dither_codebook(0, 128, 0, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_dither_codebook(2, 2, 0, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_dither_codebook(2, 128, 9, c.ctypes.data, b.ctypes.data) == tq.TQ_ERR_INVALID_ARG
+    assert tq.lib.tq_dither_codebook(2, 128, 0, c.ctypes.data, None) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_dither_and_corrected_norm_config(tq):
+    from oracle import layout as olay
+    for kb, qjl, vb in ((3, True, 3), (2, False, 4), (1, True, 1)):
+        cfg = tq.make_config(key_bits=kb, key_qjl=qjl, value_bits=vb, dither=True)
+        assert tq.validate_config(cfg) == 0
+        fmt = olay.Format(key_bits=kb, key_qjl=qjl, value_bits=vb, dither=True)
+        assert tq.page_bytes(cfg) == fmt.block_bytes
+        assert tq.page_bytes(cfg) == tq.page_bytes(tq.make_config(key_bits=kb, key_qjl=qjl, value_bits=vb)) + 4 * 256
+    # dithered HD only; corrected norms change no byte of the format
+    assert tq.validate_config(tq.make_config(dither=True, rotation=tq.TQ_ROT_DENSE)) == tq.TQ_ERR_UNSUPPORTED
+    cn = tq.make_config(key_corrected_norm=True)
+    assert tq.validate_config(cn) == 0 and tq.page_bytes(cn) == tq.page_bytes(tq.make_config())
+    bad = tq.make_config()
+    bad.dither = 2
+    assert tq.validate_config(bad) == tq.TQ_ERR_INVALID_ARG
+    bad = tq.make_config()
+    bad.key_corrected_norm = -1
+    assert tq.validate_config(bad) == tq.TQ_ERR_INVALID_ARG
+
+
+def test_dithered_compress_entry_points_check_the_mode(tq):
+    by = ctypes.byref
+    params, cache = tq.tq_params(), tq.tq_cache()
+    dith = tq.make_config(dither=True)
+    st = tq.lib.tq_compress_kv(by(dith), by(params), by(cache), 0, None, None, 0, 16, None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "tq_compress_kv_dithered" in tq.last_error()
+    plain = tq.make_config()
+    st = tq.lib.tq_compress_kv_dithered(by(plain), by(params), by(cache), 0, None, None, None, None, 0, 16,
+                                        None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "dither" in tq.last_error()
+    st = tq.lib.tq_compress_kv_dithered(by(dith), by(params), by(cache), 0, None, None, None, None, 0, 16,
+                                        None, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "offsets" in tq.last_error()
+    # appends take no offsets
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.addressof(buf)
+    params = tq.make_params()
+    params.signs = params.k_centroids = params.v_centroids = params.k_boundaries = params.v_boundaries = p
+    params.s = (p + 15) & ~15
+    cache = tq.tq_cache(p, p, 1, 1, 1, 1, 1)
+    st = tq.lib.tq_append_kv(by(dith), by(params), by(cache), 0, p, p, 0, 1, p, None, None)
+    assert st == tq.TQ_ERR_UNSUPPORTED and "offsets" in tq.last_error()
+
+
 def test_codebook_argument_errors(tq):
     c = np.zeros(4, np.float32)
     b = np.zeros(3, np.float32)

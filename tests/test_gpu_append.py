@@ -45,6 +45,11 @@ CASES = {
                                    name="c2_vqjl"), (1, 3)),
     "c3_vqjl_dense": (lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=2, value_qjl=True,
                                          name="c3_vqjl_dense"), (2,)),
+    # corrected key norms: merged QJL keys (fused fast path) and 4-bit MSE-only keys (dense)
+    "c2_corrected_norm": (lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1283, n_splits=4,
+                                             key_corrected_norm=True, name="c2_corrected_norm"), (1, 3)),
+    "c3_corrected_norm": (lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=2,
+                                             key_corrected_norm=True, name="c3_corrected_norm"), (2,)),
 }
 
 

@@ -30,6 +30,19 @@ SMALL = {
                                   name="c2_vqjl"),
     "c3_vqjl_dense": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3, value_qjl=True,
                                         name="c3_vqjl_dense"),
+    # dithered HD: merged QJL keys and 3-bit values; MSE-only 2-bit keys and 4-bit values
+    "c2_dither": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4, dither=True,
+                                    name="c2_dither"),
+    "k2v4_dither": lambda: wl.config2(kv_heads=1, q_heads=4, max_len=600, key_bits=2, key_qjl=False,
+                                      value_bits=4, n_splits=2, dither=True, name="k2v4_dither"),
+    # corrected key norms: merged QJL keys (fast decode) and dense 4-bit keys without QJL
+    "c2_corrected_norm": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4,
+                                            key_corrected_norm=True, name="c2_corrected_norm"),
+    "c3_corrected_norm": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3,
+                                            key_corrected_norm=True, name="c3_corrected_norm"),
+    # the fast decode's key and value formats under a dense rotation (served by the general kernels)
+    "c2_dense": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=900, n_splits=3, rotation=wl.ROT_DENSE,
+                                   rot_seed=11, name="c2_dense"),
 }
 
 
@@ -116,8 +129,8 @@ def test_decompress_matches_oracle(run):
         n = int(run.lens[b])
         for h in range(run.w.kv_heads):
             u = olay.read_sequence(run.pages, run.fmt, 0, h, run.bt[b], n)
-            assert close(kh[b, h, :n], oq.reconstruct_mse(u.k_idx, u.k_norm, run.R, run.ck)).all()
-            assert close(vh[b, h, :n], oq.reconstruct_mse(u.v_idx, u.v_norm, run.R, run.cv)).all()
+            assert close(kh[b, h, :n], oq.reconstruct_mse(u.k_idx, u.k_norm, run.R, run.ck, u.k_offset)).all()
+            assert close(vh[b, h, :n], oq.reconstruct_mse(u.v_idx, u.v_norm, run.R, run.cv, u.v_offset)).all()
             assert np.all(kh[b, h, n:] == 0)
 
 

@@ -96,6 +96,8 @@ class Workload:
     outlier_seed: int = 3
     min_len: int = 0
     value_qjl: bool = False        # values carry the QJL sketch of their residual too
+    dither: bool = False           # dithered HD: one random offset per key and per value
+    key_corrected_norm: bool = False  # keys store the corrected norm
 
     @property
     def group(self) -> int:
@@ -251,6 +253,29 @@ def make_q(w: Workload, layer: int = 0) -> np.ndarray:
     q = rng.standard_normal((w.batch, w.q_heads, w.seq_q, HEAD_DIM))
     dt = np.float16 if w.in_dtype == "f16" else np.float32
     return q.astype(dt).astype(np.float64)
+
+
+def dither_offsets(w: Workload, layer: int, half_k: float, half_v: float) -> tuple[np.ndarray, np.ndarray]:
+    """The random offsets of a dithered workload ("Minimum Distortion Quantization with
+    Specified Output Distribution" page: a random scalar offset per vector): iid uniform on
+    [-half, half) for every (sequence, kv head, position), keys and values drawn apart,
+    rounded to fp32 (what the device receives), as float64 [batch][kv_heads][max_len]."""
+    rng = np.random.default_rng([w.data_seed, layer, 31])
+    shape = (w.batch, w.kv_heads, w.max_len)
+    k = rng.uniform(-half_k, half_k, shape)
+    v = rng.uniform(-half_v, half_v, shape)
+    return k.astype(np.float32).astype(np.float64), v.astype(np.float32).astype(np.float64)
+
+
+def dither_offsets_device(w: Workload, layer: int, half_k: float, half_v: float, device):
+    """dither_offsets drawn with torch on `device` (a different random stream), float32."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.data_seed) * 104729 + layer + 31)
+    shape = (w.batch, w.kv_heads, w.max_len)
+    k = (torch.rand(shape, generator=g, device=device) * 2.0 - 1.0) * half_k
+    v = (torch.rand(shape, generator=g, device=device) * 2.0 - 1.0) * half_v
+    return k, v
 
 
 def rotation_inputs(w: Workload) -> dict:
