@@ -22,8 +22,10 @@
 // The R = G * seq_q query rows of a KV head are taken four at a time: one run of up to four
 // rows per CTA along the grid's z, each run with its own merge counter.
 //
-// Supported here: keys 3-bit + QJL (merged nibbles) or 2-bit + QJL, values 3-bit or 2-bit,
-// any R.  Everything else uses decode.cu.
+// Supported here: keys 3-bit + QJL (merged nibbles), 2-bit + QJL, or 4-bit without QJL
+// (sign-magnitude nibbles, the signs applied by byte masks), values 3-bit or 2-bit, any R;
+// the randomized Hadamard rotation or a dense Pi (R^T applied in the merge).  Everything
+// else uses decode.cu.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -49,7 +51,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kInvSqrtD = 0.08838834764831845f;
 constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
 
-enum KPol { K3Q = 0, K2Q = 1 };
+enum KPol { K3Q = 0, K2Q = 1, K4 = 2 };
 enum VPol { V3 = 0, V2 = 1 };
 
 // the merging CTA copies the partials of up to kMergeSplits splits into shared memory at once
@@ -251,9 +253,11 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   const int nunits = u_end - u_begin;
   const int t_end = min(n_eff, u_end * kUnit);
 
-  constexpr int kKChunks = (KP == K3Q) ? 4 : 3;  // K2Q: 2 code chunks + the KS chunk
+  constexpr int kKChunks = (KP == K2Q) ? 3 : 4;  // K2Q: 2 code chunks + the KS chunk
   constexpr int kVChunks = (VP == V3) ? 3 : 2;
-  const uint32_t unit_bytes = kNormBytes + 16u * kUnit * (kKChunks + kVChunks);
+  constexpr bool kQjl = KP != K4;
+  // without QJL there is no KR region: its norm slots stay unused
+  const uint32_t unit_bytes = kNormBytes - (kQjl ? 0u : 2u * kUnit) + 16u * kUnit * (kKChunks + kVChunks);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -297,10 +301,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         const uint32_t hb2 = half * kUnit * 2, hb16 = half * kUnit * 16;
         mbar_expect_tx(&sm.full[s], unit_bytes);
         bulk_g2s(st, blk + L.kn + hb2, kUnit * 2, &sm.full[s]);
-        bulk_g2s(st + kUnit * 2, blk + L.kr + hb2, kUnit * 2, &sm.full[s]);
+        if (kQjl) bulk_g2s(st + kUnit * 2, blk + L.kr + hb2, kUnit * 2, &sm.full[s]);
         bulk_g2s(st + kUnit * 4, blk + L.vn + hb2, kUnit * 2, &sm.full[s]);
         unsigned char* kc = st + kNormBytes;
-        const int kcode_chunks = (KP == K3Q) ? 4 : 2;
+        const int kcode_chunks = (KP == K2Q) ? 2 : 4;
         for (int c = 0; c < kcode_chunks; ++c)
           bulk_g2s(kc + c * kChunkStride, blk + L.kc + c * PT * 16 + hb16, kUnit * 16, &sm.full[s]);
         if (KP == K2Q) bulk_g2s(kc + 2 * kChunkStride, blk + L.ks + hb16, kUnit * 16, &sm.full[s]);
@@ -329,6 +333,15 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         }
         table4(neg, kt_lo0, kt_hi0);
         table4(pos, kt_lo1, kt_hi1);
+      } else if (KP == K4) {
+        // stored code (r0, r1, r2, s) -> magnitude a[r] (the sign is applied by a byte mask)
+        float m0[4], m1[4];
+        for (int r = 0; r < 4; ++r) {
+          m0[r] = a.k_centroids[hk + r];
+          m1[r] = a.k_centroids[hk + 4 + r];
+        }
+        table4(m0, kt_lo0, kt_hi0);
+        table4(m1, kt_lo1, kt_hi1);
       } else {
         // stored code (r0, s) -> f = r0 + 2 s; value s ? +a[r0] : -a[r0]
         float t[4] = {-a.k_centroids[hk], -a.k_centroids[hk + 1], a.k_centroids[hk], a.k_centroids[hk + 1]};
@@ -354,6 +367,14 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       if (KP == K3Q) {
         for (int i = 0; i < 8; ++i) {
           const float c = (i >= 4) ? a.k_centroids[hk + (i & 3)] : -a.k_centroids[hk + (i & 3)];
+          e8[i] = c - __half2float(__float2half_rn(c));
+        }
+        n = 8;
+      } else if (KP == K4) {
+        // magnitudes; a negative centroid's residual is the negated code (its bitwise
+        // complement, -e - 1: one LSB of the scaled residual, 2^-7 of its largest entry)
+        for (int i = 0; i < 8; ++i) {
+          const float c = a.k_centroids[hk + i];
           e8[i] = c - __half2float(__float2half_rn(c));
         }
         n = 8;
@@ -405,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int4 v = frow ? sqp[k] : make_int4(0, 0, 0, 0);
+        const int4 v = (frow && kQjl) ? sqp[k] : make_int4(0, 0, 0, 0);
         const int w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -422,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         int c;  // quarter-local coordinate of B row (ks, e)
-        if (KP == K3Q) {
+        if (KP != K2Q) {
           c = 4 * ks + e;
         } else {
           const int n = 2 * ks + (e >> 1);  // half2 index: word n/8, pair n%8
@@ -445,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           int c;  // quarter-local coordinate of byte i of correction register (w, h)
-          if (KP == K3Q) {
+          if (KP != K2Q) {
             c = 8 * w + 4 * h + i;
           } else {
             // register (w, h) holds pairs n = 4w + 2h and 4w + 2h + 1: bytes (a1, a2, b1, b2)
@@ -459,9 +480,9 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       }
     }
     // B fragments of the QJL term: column g = (row g/2, digit g%2) of 16-bit (S q)
-    uint32_t bs[4][2];
+    uint32_t bs[4][2] = {};
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < 4 && kQjl; ++w) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t word = 0;
@@ -484,9 +505,9 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     int T_row = 0;
     float c_row_k = 0.f, c_row_q = 0.f, corr_down = 0.f;
     if (t4 < R) {
-      T_row = a.sq_sum[row0 + t4];
+      T_row = kQjl ? a.sq_sum[row0 + t4] : 0;
       c_row_k = kInvSqrtD * kLog2e;
-      c_row_q = kQjlScale * a.sq_scale[row0 + t4] * kInvSqrtD * kLog2e;
+      c_row_q = kQjl ? kQjlScale * a.sq_scale[row0 + t4] * kInvSqrtD * kLog2e : 0.f;
       const float lam = a.q8_scale[row0 + t4];
       corr_down = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
     }
@@ -549,6 +570,35 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
                   sg[2 * w + 1] = W & 0x80808080u;
                 }
               }
+            } else if (KP == K4) {
+              const uint4 wa = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + ta * 16);
+              const uint4 wb = *reinterpret_cast<const uint4*>(kc + t4 * kChunkStride + tb * 16);
+              const uint32_t A4[4] = {wa.x, wa.y, wa.z, wa.w}, B4[4] = {wb.x, wb.y, wb.z, wb.w};
+    #pragma unroll
+              for (int w = 0; w < 4; ++w) {
+    #pragma unroll
+                for (int side = 0; side < 2; ++side) {
+                  const uint32_t W = side ? B4[w] : A4[w];
+                  uint32_t* h = side ? hb : ha;
+                  uint32_t* ep = side ? eb : ea;
+                  const uint32_t s0 = W & 0x7777u;
+                  const uint32_t s1 = __umulhi(W, 1u << 16) & 0x7777u;
+                  // 0xFF in the byte of each coordinate whose s bit (nibble bit 3) is set:
+                  // the sign bits of nibbles 1, 3, ... are byte tops already, those of
+                  // nibbles 0, 2, ... become byte tops four bits up
+                  const uint32_t W4 = W << 4;
+                  const uint32_t m0 = prmt(W4, W, 0xD9C8u), m1 = prmt(W4, W, 0xFBEAu);
+                  ep[2 * w + 0] = prmt(et0, et1, s0) ^ ~m0;
+                  ep[2 * w + 1] = prmt(et0, et1, s1) ^ ~m1;
+                  const uint32_t l0 = prmt(kt_lo0, kt_lo1, s0), l1 = prmt(kt_lo0, kt_lo1, s1);
+                  const uint32_t h0 = prmt(kt_hi0, kt_hi1, s0) ^ (~m0 & 0x80808080u);
+                  const uint32_t h1 = prmt(kt_hi0, kt_hi1, s1) ^ (~m1 & 0x80808080u);
+                  h[4 * w + 0] = prmt(l0, h0, 0x5140);
+                  h[4 * w + 1] = prmt(l0, h0, 0x7362);
+                  h[4 * w + 2] = prmt(l1, h1, 0x5140);
+                  h[4 * w + 3] = prmt(l1, h1, 0x7362);
+                }
+              }
             } else {
               const unsigned char* kq = kc + (t4 >> 1) * kChunkStride + (t4 & 1) * 8;
               const uint2 ca = *reinterpret_cast<const uint2*>(kq + ta * 16);
@@ -583,8 +633,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
     #pragma unroll
             for (int w = 0; w < 4; w += 2) {
-              imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
-              imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
+              if (kQjl) {
+                imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
+                imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
+              }
               imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
               imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[w + 1][0], bc[w + 1][1]);
             }
@@ -596,7 +648,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             }
             // ---- scores of row t4 for tokens ta, tb (log2 domain)
             const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
-            const float rA = ld_h(st + 2 * kUnit + 2 * ta), rB = ld_h(st + 2 * kUnit + 2 * tb);
+            const float rA = kQjl ? ld_h(st + 2 * kUnit + 2 * ta) : 0.f;
+            const float rB = kQjl ? ld_h(st + 2 * kUnit + 2 * tb) : 0.f;
             const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
             const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
             const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
@@ -809,9 +862,31 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
+    float x[4] = {o.x * inv, o.y * inv, o.z * inv, o.w * inv};
+    if (a.dense) {
+      // out = Pi^T (o / l): the row's 128 values through shared memory (this CTA's rows
+      // are done with sm.merge once their weighted sums are in registers), then thread
+      // (r, c4) forms outputs 4 c4 .. 4 c4 + 3 from rows of Pi (coalesced across c4)
+      __syncwarp();
+      float* xs = &sm.merge[r][0][0];
+      *reinterpret_cast<float4*>(xs + 4 * c4) = make_float4(x[0], x[1], x[2], x[3]);
+      __syncwarp();
+      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4* pi4 = reinterpret_cast<const float4*>(a.pi) + c4;
+#pragma unroll 8
+      for (int i = 0; i < D; ++i) {
+        const float4 p = pi4[(size_t)i * (D / 4)];
+        const float xi = xs[i];
+        y.x = fmaf(p.x, xi, y.x);
+        y.y = fmaf(p.y, xi, y.y);
+        y.z = fmaf(p.z, xi, y.z);
+        y.w = fmaf(p.w, xi, y.w);
+      }
+      *reinterpret_cast<float4*>(a.out + rowq * D + 4 * c4) = y;
+      return;
+    }
     // out = D H (o / l) / sqrt(d): H over coordinates 4 c4 + e, spans 1 and 2 in the
     // thread, spans 4..64 across the row's 32 lanes
-    float x[4] = {o.x * inv, o.y * inv, o.z * inv, o.w * inv};
     {
       const float a0 = x[0] + x[1], a1 = x[0] - x[1], a2 = x[2] + x[3], a3 = x[2] - x[3];
       x[0] = a0 + a2;
@@ -836,9 +911,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 
 bool fast_decode_supported(const DecodeArgs& a) {
   const Layout& L = a.cache.L;
-  // the merge un-rotates with H D; dithered codes need their offsets (general kernels)
-  if (a.dense || L.dither) return false;
-  const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl);
+  // dithered codes need their offsets (general kernels); the merge reads Pi as float4
+  if (L.dither) return false;
+  if (a.dense && (reinterpret_cast<uintptr_t>(a.pi) & 15)) return false;
+  const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl) || (L.kbits == 4 && !L.qjl);
   const bool vok = (L.vbits == 3 || L.vbits == 2) && !L.vqjl;
   return kok && vok;
 }
@@ -854,6 +930,8 @@ cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
   if (L.kbits == 3 && L.vbits == 2) k = fast_split_kernel<K3Q, V2>;
   if (L.kbits == 2 && L.vbits == 3) k = fast_split_kernel<K2Q, V3>;
   if (L.kbits == 2 && L.vbits == 2) k = fast_split_kernel<K2Q, V2>;
+  if (L.kbits == 4 && L.vbits == 3) k = fast_split_kernel<K4, V3>;
+  if (L.kbits == 4 && L.vbits == 2) k = fast_split_kernel<K4, V2>;
   if (!k) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -18,12 +18,12 @@ import workloads as wl
 pytestmark = pytest.mark.gpu
 
 
-# the fused kernel's workload (3-bit keys with QJL, 3-bit values) and one that takes the
-# general kernels (dense rotation, 4-bit keys without QJL, G = 8): both use the scratch
-# array, for different partials
+# the tensor-core split kernel's workload (3-bit keys with QJL, 3-bit values) and one that
+# takes the general kernels (values with QJL: the sign-space partials; dense rotation, 4-bit
+# keys without QJL, G = 8): both use the scratch array, for different partials
 CASES = {
     "fused": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1500, n_splits=4),
-    "general": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3),
+    "general": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3, value_qjl=True),
 }
 
 
