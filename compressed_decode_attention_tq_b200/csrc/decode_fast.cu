@@ -19,8 +19,9 @@
 //    (sequence, kv head) to finish (a counter the prologue zeroes) merges all partials
 //    and applies R^T.
 //
-// The R = G * seq_q query rows of a KV head are taken four at a time: one run of up to four
-// rows per CTA along the grid's z, each run with its own merge counter.
+// The R = G * seq_q query rows of a KV head are taken four or eight at a time (eight when R
+// exceeds four): one run of rows per CTA along the grid's z, each run with its own merge
+// counter.
 //
 // Supported here: keys 3-bit + QJL (merged nibbles), 2-bit + QJL, or 4-bit without QJL
 // (sign-magnitude nibbles, the signs applied by byte masks), values 3-bit or 2-bit, any R;
@@ -54,23 +55,26 @@ constexpr float kQjlScale = 1.2533141373155003f / QM;  // sqrt(pi/2)/m
 enum KPol { K3Q = 0, K2Q = 1, K4 = 2 };
 enum VPol { V3 = 0, V2 = 1 };
 
-// the merging CTA copies the partials of up to kMergeSplits splits into shared memory at once
-constexpr int kMergeSplits = 40;
+// Query rows per CTA: 4 or 8 (the key and QJL products take one n-tile of the mma per four
+// rows; the value product's eight columns hold eight rows).
+constexpr int kMaxRows = 8;
+// the merging CTA copies the partials of up to 160 / rows splits into shared memory at once
+constexpr int kMergeFloats = 160 * D;
 struct SmemFast {
   union {
     struct {
       unsigned char stage[kStages][kStageBytes];
-      float wacc[kConsumerWarps][4][D];
+      float wacc[kConsumerWarps][kMaxRows][D];
     } ring;
     // at the end: the partial accumulators of every split of the (sequence, kv head) being
-    // merged (the ring and the warp partials are no longer used then)
-    float merge[4][kMergeSplits][D];
+    // merged, [row][split][D] (the ring and the warp partials are no longer used then)
+    float merge[kMergeFloats];
   };
   unsigned long long full[kStages];
   unsigned long long empty[kStages];
   unsigned long long mbar;  // the merge copies landed
   unsigned long long never;  // completed by nothing: the target of the bounded-wait test
-  float wm[kConsumerWarps][4], wl[kConsumerWarps][4], wf[kConsumerWarps][4];
+  float wm[kConsumerWarps][kMaxRows], wl[kConsumerWarps][kMaxRows], wf[kConsumerWarps][kMaxRows];
   int last;
 };
 
@@ -225,8 +229,10 @@ __device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int
   return (t1 & 0x3u) | ((t2 & 0x3u) << 4) | (t1 & 0x300u) | ((t2 & 0x300u) << 4);
 }
 
-template <int KP, int VP>
+template <int KP, int VP, int NR>
 __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
+  static_assert(NR == 4 || NR == 8, "four or eight rows per CTA");
+  constexpr int NT = NR / 4;  // n-tiles of the key and QJL products
   // the next kernel on the stream may be scheduled now; a programmatic dependent waits for
   // this grid to finish before it touches what it writes
   asm volatile("griddepcontrol.launch_dependents;");
@@ -234,12 +240,12 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   SmemFast& sm = *reinterpret_cast<SmemFast*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // The query rows of one (sequence, kv head) (its G heads times seq_q positions, consecutive)
-  // are taken in runs of up to four, one run per CTA along the grid's z with the sequence.
-  const int nchunk = (a.rows + 3) / 4;
+  // are taken in runs of up to NR, one run per CTA along the grid's z with the sequence.
+  const int nchunk = (a.rows + NR - 1) / NR;
   const int split = blockIdx.x, gh = blockIdx.y, b = blockIdx.z / nchunk, chunk = blockIdx.z % nchunk;
   const Layout& L = a.cache.L;
-  const int R = min(4, a.rows - 4 * chunk);
-  const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q + 4 * chunk;
+  const int R = min(NR, a.rows - NR * chunk);
+  const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q + NR * chunk;
 
   const int len = a.seq_lens[b];
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
@@ -400,123 +406,138 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     }
     // the prologue (our programmatic predecessor) must be done before its outputs are read
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    // this lane's 32-coordinate slices of row g/2: rotated query, its int8 copy, 16-bit S q
-    const int fr = g >> 1;
-    const bool frow = fr < R;
-    float qv[32];
-    int q8v[32], sqv[32];
-    {
-      const size_t rr = row0 + (frow ? fr : 0);
-      const float4* qp = reinterpret_cast<const float4*>(a.qrot + rr * D + 32 * t4);
-      const int4* q8p = reinterpret_cast<const int4*>(a.q8 + rr * D + 32 * t4);
-      const int4* sqp = reinterpret_cast<const int4*>(a.sq_int + rr * QM + 32 * t4);
+    // B fragments, one n-tile per four rows (tile nt: rows 4 nt .. 4 nt + 3)
+    uint32_t bq[NT][8][2], bc[NT][4][2], bs[NT][4][2];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 f = frow ? qp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
-        qv[4 * k] = f.x; qv[4 * k + 1] = f.y; qv[4 * k + 2] = f.z; qv[4 * k + 3] = f.w;
-      }
+    for (int nt = 0; nt < NT; ++nt) {
+      // this lane's 32-coordinate slices of row 4 nt + g/2: rotated query, its int8 copy,
+      // 16-bit S q
+      const int fr = 4 * nt + (g >> 1);
+      const bool frow = fr < R;
+      float qv[32];
+      int q8v[32], sqv[32];
+      {
+        const size_t rr = row0 + (frow ? fr : 0);
+        const float4* qp = reinterpret_cast<const float4*>(a.qrot + rr * D + 32 * t4);
+        const int4* q8p = reinterpret_cast<const int4*>(a.q8 + rr * D + 32 * t4);
+        const int4* sqp = reinterpret_cast<const int4*>(a.sq_int + rr * QM + 32 * t4);
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const int4 v = frow ? q8p[k] : make_int4(0, 0, 0, 0);
-        const int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int bb = 0; bb < 4; ++bb) q8v[16 * k + 4 * u + bb] = (int)(int8_t)((w4[u] >> (8 * bb)) & 255);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int4 v = (frow && kQjl) ? sqp[k] : make_int4(0, 0, 0, 0);
-        const int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          sqv[8 * k + 2 * u] = (int)(int16_t)(w4[u] & 0xffff);
-          sqv[8 * k + 2 * u + 1] = (int)(int16_t)((uint32_t)w4[u] >> 16);
+        for (int k = 0; k < 8; ++k) {
+          const float4 f = frow ? qp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+          qv[4 * k] = f.x; qv[4 * k + 1] = f.y; qv[4 * k + 2] = f.z; qv[4 * k + 3] = f.w;
         }
-      }
-    }
-    // B fragments of the key term: column g = (row g/2, hi or lo half)
-    uint32_t bq[8][2];
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      float v[4];
+        for (int k = 0; k < 2; ++k) {
+          const int4 v = frow ? q8p[k] : make_int4(0, 0, 0, 0);
+          const int w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        int c;  // quarter-local coordinate of B row (ks, e)
-        if (KP != K2Q) {
-          c = 4 * ks + e;
-        } else {
-          const int n = 2 * ks + (e >> 1);  // half2 index: word n/8, pair n%8
-          c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (e & 1);
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) q8v[16 * k + 4 * u + bb] = (int)(int8_t)((w4[u] >> (8 * bb)) & 255);
         }
-        const float x = qv[c];
-        const float hi = __half2float(__float2half_rn(x));
-        v[e] = (g & 1) ? (x - hi) : hi;
-      }
-      bq[ks][0] = pack_h2(v[0], v[1]);
-      bq[ks][1] = pack_h2(v[2], v[3]);
-    }
-    // B fragments of the centroid correction: int8 R q in column 2r (odd columns zero)
-    uint32_t bc[4][2];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+        for (int k = 0; k < 4; ++k) {
+          const int4 v = (frow && kQjl) ? sqp[k] : make_int4(0, 0, 0, 0);
+          const int w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int c;  // quarter-local coordinate of byte i of correction register (w, h)
-          if (KP != K2Q) {
-            c = 8 * w + 4 * h + i;
-          } else {
-            // register (w, h) holds pairs n = 4w + 2h and 4w + 2h + 1: bytes (a1, a2, b1, b2)
-            const int n = 4 * w + 2 * h + (i & 1);
-            c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (i >> 1);
+          for (int u = 0; u < 4; ++u) {
+            sqv[8 * k + 2 * u] = (int)(int16_t)(w4[u] & 0xffff);
+            sqv[8 * k + 2 * u + 1] = (int)(int16_t)((uint32_t)w4[u] >> 16);
           }
-          const int v = (g & 1) ? 0 : q8v[c];
-          word |= (uint32_t)(v & 255) << (8 * i);
         }
-        bc[w][h] = word;
+      }
+      // the key term: column g = (row 4 nt + g/2, hi or lo half)
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int c;  // quarter-local coordinate of B row (ks, e)
+          if (KP != K2Q) {
+            c = 4 * ks + e;
+          } else {
+            const int n = 2 * ks + (e >> 1);  // half2 index: word n/8, pair n%8
+            c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (e & 1);
+          }
+          const float x = qv[c];
+          const float hi = __half2float(__float2half_rn(x));
+          v[e] = (g & 1) ? (x - hi) : hi;
+        }
+        bq[nt][ks][0] = pack_h2(v[0], v[1]);
+        bq[nt][ks][1] = pack_h2(v[2], v[3]);
+      }
+      // the centroid correction: int8 R q in column 2r (odd columns zero)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            int c;  // quarter-local coordinate of byte i of correction register (w, h)
+            if (KP != K2Q) {
+              c = 8 * w + 4 * h + i;
+            } else {
+              // register (w, h) holds pairs n = 4w + 2h and 4w + 2h + 1: bytes (a1, a2, b1, b2)
+              const int n = 4 * w + 2 * h + (i & 1);
+              c = 16 * (n >> 3) + pair_base(n & 7) + 4 * (i >> 1);
+            }
+            const int v = (g & 1) ? 0 : q8v[c];
+            word |= (uint32_t)(v & 255) << (8 * i);
+          }
+          bc[nt][w][h] = word;
+        }
+      }
+      // the QJL term: column g = (row 4 nt + g/2, digit g%2) of 16-bit (S q)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int i = 0; i < 4 && kQjl; ++i) {
+            int c;  // quarter-local QJL index of byte i of register (w, h)
+            if (KP == K3Q)
+              c = 8 * w + 2 * i + h;
+            else
+              c = 8 * i + 7 - (2 * w + h);
+            const int v = sqv[c];
+            const int d0 = ((v + 128) & 255) - 128;
+            const int d1 = (v - d0) >> 8;
+            word |= (uint32_t)(((g & 1) ? d1 : d0) & 255) << (8 * i);
+          }
+          bs[nt][w][h] = word;
+        }
       }
     }
-    // B fragments of the QJL term: column g = (row g/2, digit g%2) of 16-bit (S q)
-    uint32_t bs[4][2] = {};
+    // per-row constants of the lane's own score rows t4 + 4 nt
+    int T_row[NT];
+    float c_row_q[NT], corr_down[NT];
+    const float c_row_k = kInvSqrtD * kLog2e;
 #pragma unroll
-    for (int w = 0; w < 4 && kQjl; ++w) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          int c;  // quarter-local QJL index of byte i of register (w, h)
-          if (KP == K3Q)
-            c = 8 * w + 2 * i + h;
-          else
-            c = 8 * i + 7 - (2 * w + h);
-          const int v = sqv[c];
-          const int d0 = ((v + 128) & 255) - 128;
-          const int d1 = (v - d0) >> 8;
-          word |= (uint32_t)(((g & 1) ? d1 : d0) & 255) << (8 * i);
-        }
-        bs[w][h] = word;
+    for (int nt = 0; nt < NT; ++nt) {
+      const int rr = t4 + 4 * nt;
+      T_row[nt] = 0;
+      c_row_q[nt] = 0.f;
+      corr_down[nt] = 0.f;
+      if (rr < R) {
+        T_row[nt] = kQjl ? a.sq_sum[row0 + rr] : 0;
+        c_row_q[nt] = kQjl ? kQjlScale * a.sq_scale[row0 + rr] * kInvSqrtD * kLog2e : 0.f;
+        const float lam = a.q8_scale[row0 + rr];
+        corr_down[nt] = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
       }
-    }
-    // per-row constants of the lane's own score row t4
-    int T_row = 0;
-    float c_row_k = 0.f, c_row_q = 0.f, corr_down = 0.f;
-    if (t4 < R) {
-      T_row = kQjl ? a.sq_sum[row0 + t4] : 0;
-      c_row_k = kInvSqrtD * kLog2e;
-      c_row_q = kQjl ? kQjlScale * a.sq_scale[row0 + t4] * kInvSqrtD * kLog2e : 0.f;
-      const float lam = a.q8_scale[row0 + t4];
-      corr_down = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
     }
 
     if (a.debug_wait_ns > 0 && warp == 0 && split == 0 && gh == 0 && blockIdx.z == 0 &&
         !mbar_wait(&sm.never, 0, (unsigned long long)a.debug_wait_ns) && lane == 0)
       report(a.status, TQ_ERR_TIMEOUT);
 
-    float m_run = -CUDART_INF_F, l_run = 0.f;
+    float m_run[NT], l_run[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m_run[nt] = -CUDART_INF_F;
+      l_run[nt] = 0.f;
+    }
     float acc[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt)
@@ -537,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       // two 16-token steps per iteration: their key and value work interleave, and one
       // joint running maximum (one rescale) serves both
       for (int pr = warp; pr * 32 < valid; pr += kConsumerWarps) {
-        float sc[2][2];
+        float sc[2][NT][2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int step = 2 * pr + u;
@@ -622,23 +643,28 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
                 sb[k] = (sB << k) & 0x80808080u;
               }
             }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
             // two accumulators per term halve the dependent mma chains
             float dk[4] = {0.f, 0.f, 0.f, 0.f}, dk2[4] = {0.f, 0.f, 0.f, 0.f};
     #pragma unroll
             for (int ks = 0; ks < 8; ks += 2) {
-              hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[ks][0], bq[ks][1]);
-              hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[ks + 1][0], bq[ks + 1][1]);
+              hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[nt][ks][0], bq[nt][ks][1]);
+              hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[nt][ks + 1][0],
+                   bq[nt][ks + 1][1]);
             }
             int dsum[4] = {0, 0, 0, 0}, dsum2[4] = {0, 0, 0, 0};
             int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
     #pragma unroll
             for (int w = 0; w < 4; w += 2) {
               if (kQjl) {
-                imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[w][0], bs[w][1]);
-                imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[w + 1][0], bs[w + 1][1]);
+                imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[nt][w][0], bs[nt][w][1]);
+                imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[nt][w + 1][0],
+                     bs[nt][w + 1][1]);
               }
-              imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[w][0], bc[w][1]);
-              imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[w + 1][0], bc[w + 1][1]);
+              imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[nt][w][0], bc[nt][w][1]);
+              imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[nt][w + 1][0],
+                   bc[nt][w + 1][1]);
             }
     #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -646,41 +672,62 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
               dsum[e] += dsum2[e];
               dcor[e] += dcor2[e];
             }
-            // ---- scores of row t4 for tokens ta, tb (log2 domain)
+            // ---- scores of row t4 + 4 nt for tokens ta, tb (log2 domain)
             const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
             const float rA = kQjl ? ld_h(st + 2 * kUnit + 2 * ta) : 0.f;
             const float rB = kQjl ? ld_h(st + 2 * kUnit + 2 * tb) : 0.f;
             const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
-            const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down;
-            const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down;
-            float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row) * c_row_q;
-            float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row) * c_row_q;
-            if (t4 >= R || ta >= valid) sca = -CUDART_INF_F;
-            if (t4 >= R || tb >= valid) scb = -CUDART_INF_F;
-          sc[u][0] = sca;
-          sc[u][1] = scb;
-        }
-        float mx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-        const float m_new = fmaxf(m_run, mx);
-        // the running sums are rescaled only when some row maximum grew
-        const bool grow = __any_sync(FULL, m_new > m_run);
-        float alpha = 1.f, p[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        if (m_new != -CUDART_INF_F) {
-          if (grow) alpha = exp2f(m_run - m_new);
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            p[u][0] = exp2f(sc[u][0] - m_new);
-            p[u][1] = exp2f(sc[u][1] - m_new);
+            const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down[nt];
+            const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down[nt];
+            float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row[nt]) * c_row_q[nt];
+            float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row[nt]) * c_row_q[nt];
+            if (t4 + 4 * nt >= R || ta >= valid) sca = -CUDART_INF_F;
+            if (t4 + 4 * nt >= R || tb >= valid) scb = -CUDART_INF_F;
+            sc[u][nt][0] = sca;
+            sc[u][nt][1] = scb;
           }
         }
-        l_run = l_run * alpha + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-        m_run = m_new;
+        float m_new[NT];
+        bool up = false;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float mx = fmaxf(fmaxf(sc[0][nt][0], sc[0][nt][1]), fmaxf(sc[1][nt][0], sc[1][nt][1]));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+          m_new[nt] = fmaxf(m_run[nt], mx);
+          up |= m_new[nt] > m_run[nt];
+        }
+        // the running sums are rescaled only when some row maximum grew
+        const bool grow = __any_sync(FULL, up);
+        float alpha[NT], p[2][NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          alpha[nt] = 1.f;
+          p[0][nt][0] = p[0][nt][1] = p[1][nt][0] = p[1][nt][1] = 0.f;
+          if (m_new[nt] != -CUDART_INF_F) {
+            if (grow) alpha[nt] = exp2f(m_run[nt] - m_new[nt]);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              p[u][nt][0] = exp2f(sc[u][nt][0] - m_new[nt]);
+              p[u][nt][1] = exp2f(sc[u][nt][1] - m_new[nt]);
+            }
+          }
+          l_run[nt] = l_run[nt] * alpha[nt] + (p[0][nt][0] + p[0][nt][1]) + (p[1][nt][0] + p[1][nt][1]);
+          m_run[nt] = m_new[nt];
+        }
         if (grow) {
-          const float al0 = __shfl_sync(FULL, alpha, (2 * t4) & 31);
-          const float al1 = __shfl_sync(FULL, alpha, (2 * t4 + 1) & 31);
+          // the accumulator columns are rows 2 t4 and 2 t4 + 1: their factors come from the
+          // lanes holding those rows' scores (row r: lane r % 4, tile r / 4)
+          const int r0 = 2 * t4, r1 = 2 * t4 + 1;
+          float al0 = __shfl_sync(FULL, alpha[0], r0 & 3);
+          float al1 = __shfl_sync(FULL, alpha[0], r1 & 3);
+          if (NT == 2) {
+            const float b0 = __shfl_sync(FULL, alpha[NT - 1], r0 & 3);
+            const float b1 = __shfl_sync(FULL, alpha[NT - 1], r1 & 3);
+            if (r0 >= 4) al0 = b0;
+            if (r1 >= 4) al1 = b1;
+          }
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             acc[mt][0] *= al0;
@@ -694,10 +741,22 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
           const int step = 2 * pr + u;
           const int ta = step * 16 + g, tb = ta + 8;
           const float vnA = ld_h(st + 4 * kUnit + 2 * ta), vnB = ld_h(st + 4 * kUnit + 2 * tb);
-          // slots past the end may hold stale bytes: force their weight to exactly 0
-          const uint32_t pk = pack_h2(ta < valid ? p[u][0] * vnA : 0.f, tb < valid ? p[u][1] * vnB : 0.f);
-          const uint32_t x1 = __shfl_sync(FULL, pk, 4 * (2 * t4) + g);
-          const uint32_t x2 = __shfl_sync(FULL, pk, 4 * (2 * t4 + 1) + g);
+          // B = weights: column g is row g, from the lane holding row g's scores for the
+          // tokens of B rows 2 t4 (+ 1, + 8, + 9); slots past the end may hold stale bytes:
+          // their weight is forced to exactly 0
+          const int src1 = 4 * (2 * t4) + (g & 3), src2 = 4 * (2 * t4 + 1) + (g & 3);
+          uint32_t pk = pack_h2(ta < valid ? p[u][0][0] * vnA : 0.f, tb < valid ? p[u][0][1] * vnB : 0.f);
+          uint32_t x1 = __shfl_sync(FULL, pk, src1);
+          uint32_t x2 = __shfl_sync(FULL, pk, src2);
+          if (NT == 2) {
+            pk = pack_h2(ta < valid ? p[u][NT - 1][0] * vnA : 0.f, tb < valid ? p[u][NT - 1][1] * vnB : 0.f);
+            const uint32_t y1 = __shfl_sync(FULL, pk, src1);
+            const uint32_t y2 = __shfl_sync(FULL, pk, src2);
+            if (g >= 4) {
+              x1 = y1;
+              x2 = y2;
+            }
+          }
           const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
             // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
             uint32_t va[16], vb[16];
@@ -730,12 +789,16 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       if (lane == 0) mbar_arrive(&sm.empty[s]);
     }
     // ---- warp partial: l summed over the 8 lanes of a row, acc scattered by coordinate
-    l_run += __shfl_xor_sync(FULL, l_run, 4);
-    l_run += __shfl_xor_sync(FULL, l_run, 8);
-    l_run += __shfl_xor_sync(FULL, l_run, 16);
-    if (g == 0 && t4 < R) {
-      sm.wm[warp][t4] = m_run;
-      sm.wl[warp][t4] = l_run;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float lr = l_run[nt];
+      lr += __shfl_xor_sync(FULL, lr, 4);
+      lr += __shfl_xor_sync(FULL, lr, 8);
+      lr += __shfl_xor_sync(FULL, lr, 16);
+      if (g == 0 && t4 + 4 * nt < R) {
+        sm.wm[warp][t4 + 4 * nt] = m_run[nt];
+        sm.wl[warp][t4 + 4 * nt] = lr;
+      }
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
@@ -790,23 +853,29 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   __syncthreads();
   if (!sm.last) return;
   const int ns = a.n_splits;
-  if (tid < 32 * R) {
-    const int r = tid >> 5, c4 = tid & 31;
+  // every split's accumulators of every row in one round trip when they fit: a bulk copy per
+  // row (the rows' partials are contiguous), landing while the maxima are formed from the
+  // (m, l) pairs; otherwise register batches from L2
+  constexpr int kCap = kMergeFloats / (NR * D);
+  const bool in_smem = ns <= kCap;
+  if (in_smem && tid == 0) {
+    // the other splits' partials were made visible to this thread by the acquire above;
+    // order them before this thread's async-proxy reads
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    mbar_expect_tx(&sm.mbar, (uint32_t)(R * ns * D * sizeof(float)));
+    for (int rr = 0; rr < R; ++rr)
+      bulk_g2s(&sm.merge[rr * kCap * D], a.part_acc + (row0 + rr) * ns * D, (uint32_t)(ns * D * sizeof(float)),
+               &sm.mbar);
+  }
+  // warp w merges rows w, w + 5, ...; lane c4 owns coordinates 4 c4 .. 4 c4 + 3
+  for (int r = warp; r < R; r += kThreads / 32) {
+    const int c4 = lane;
     const size_t rowq = row0 + r;
     const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * ns * 2);
+    float* rs = &sm.merge[r * kCap * D];  // row r's region (its partials when in_smem)
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (ns <= kMergeSplits) {
-      // every split's accumulators of every row in one round trip: a bulk copy per row (the
-      // rows' partials are contiguous), while the maxima are formed from the (m, l) pairs
-      if (tid == 0) {
-        // the other splits' partials were made visible to this thread by the acquire above;
-        // order them before this thread's async-proxy reads
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        mbar_expect_tx(&sm.mbar, (uint32_t)(R * ns * D * sizeof(float)));
-        for (int rr = 0; rr < R; ++rr)
-          bulk_g2s(&sm.merge[rr][0][0], a.part_acc + (row0 + rr) * ns * D, (uint32_t)(ns * D * sizeof(float)), &sm.mbar);
-      }
+    if (in_smem) {
       for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
 #pragma unroll
       for (int h = 16; h > 0; h >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, h));
@@ -815,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         report(a.status, TQ_ERR_TIMEOUT);
         mbar_wait(&sm.mbar, 0);  // the copies in flight land before the CTA ends (bounded)
       }
-      const float4* pa4 = reinterpret_cast<const float4*>(&sm.merge[r][0][0]) + c4;
+      const float4* pa4 = reinterpret_cast<const float4*>(rs) + c4;
 #pragma unroll 8
       for (int sp = 0; sp < ns; ++sp) {
         const float2 m2 = ml2[sp];
@@ -828,8 +897,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         o.w = fmaf(wgt, v.w, o.w);
       }
     } else {
-      // many splits: thread (row r, float4 c4) loads the partials in register batches of kMB,
-      // the first batch before the maximum is formed (about ns / kMB round trips to L2)
+      // many splits: the partials in register batches of kMB, the first batch before the
+      // maximum is formed (about ns / kMB round trips to L2)
       constexpr int kMB = 20;
       const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
       for (int s0 = 0; s0 < ns; s0 += kMB) {
@@ -864,26 +933,25 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     const float inv = l > 0.f ? 1.f / l : 0.f;
     float x[4] = {o.x * inv, o.y * inv, o.z * inv, o.w * inv};
     if (a.dense) {
-      // out = Pi^T (o / l): the row's 128 values through shared memory (this CTA's rows
-      // are done with sm.merge once their weighted sums are in registers), then thread
-      // (r, c4) forms outputs 4 c4 .. 4 c4 + 3 from rows of Pi (coalesced across c4)
+      // out = Pi^T (o / l): the row's 128 values through its own region of shared memory
+      // (every lane of this warp is past reading it), then lane c4 forms outputs
+      // 4 c4 .. 4 c4 + 3 from rows of Pi (coalesced across c4)
       __syncwarp();
-      float* xs = &sm.merge[r][0][0];
-      *reinterpret_cast<float4*>(xs + 4 * c4) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(rs + 4 * c4) = make_float4(x[0], x[1], x[2], x[3]);
       __syncwarp();
       float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
       const float4* pi4 = reinterpret_cast<const float4*>(a.pi) + c4;
 #pragma unroll 8
       for (int i = 0; i < D; ++i) {
         const float4 p = pi4[(size_t)i * (D / 4)];
-        const float xi = xs[i];
+        const float xi = rs[i];
         y.x = fmaf(p.x, xi, y.x);
         y.y = fmaf(p.y, xi, y.y);
         y.z = fmaf(p.z, xi, y.z);
         y.w = fmaf(p.w, xi, y.w);
       }
       *reinterpret_cast<float4*>(a.out + rowq * D + 4 * c4) = y;
-      return;
+      continue;
     }
     // out = D H (o / l) / sqrt(d): H over coordinates 4 c4 + e, spans 1 and 2 in the
     // thread, spans 4..64 across the row's 32 lanes
@@ -924,14 +992,20 @@ size_t fast_decode_smem_bytes() { return sizeof(SmemFast); }
 cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
   const Layout& L = a.cache.L;
   const size_t smem = sizeof(SmemFast);
-  dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch * ((a.rows + 3) / 4));
+  // eight rows per CTA when a KV head has more than four query rows
+  const int nr = a.rows > 4 ? 8 : 4;
+  dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch * ((a.rows + nr - 1) / nr));
   void (*k)(DecodeArgs) = nullptr;
-  if (L.kbits == 3 && L.vbits == 3) k = fast_split_kernel<K3Q, V3>;
-  if (L.kbits == 3 && L.vbits == 2) k = fast_split_kernel<K3Q, V2>;
-  if (L.kbits == 2 && L.vbits == 3) k = fast_split_kernel<K2Q, V3>;
-  if (L.kbits == 2 && L.vbits == 2) k = fast_split_kernel<K2Q, V2>;
-  if (L.kbits == 4 && L.vbits == 3) k = fast_split_kernel<K4, V3>;
-  if (L.kbits == 4 && L.vbits == 2) k = fast_split_kernel<K4, V2>;
+#define TQ_FAST(KB, KPOL, VB, VPOL)                                                             \
+  if (L.kbits == KB && L.vbits == VB)                                                            \
+    k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8> : fast_split_kernel<KPOL, VPOL, 4>;
+  TQ_FAST(3, K3Q, 3, V3)
+  TQ_FAST(3, K3Q, 2, V2)
+  TQ_FAST(2, K2Q, 3, V3)
+  TQ_FAST(2, K2Q, 2, V2)
+  TQ_FAST(4, K4, 3, V3)
+  TQ_FAST(4, K4, 2, V2)
+#undef TQ_FAST
   if (!k) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
