@@ -5,9 +5,22 @@
 #include <cstdlib>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tq.h"
 #include "tq_internal.h"
 #include "tq_kernels.h"
+
+namespace {
+// One NVTX range per device-side API call, named after the call (visible in Nsight Systems
+// and in ncu's NVTX filters; the calls cost next to nothing when no tool is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
+}  // namespace
 
 namespace tqi {
 
@@ -176,6 +189,7 @@ static tq_status compress_common(const tq_config* cfg, const tq_params* params, 
 tq_status tq_compress_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                          int32_t layer, const void* k, const void* v, int32_t in_dtype, int32_t max_len,
                          const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_compress_kv");
   clear_error();
   if (cfg && cfg->dither)
     return fail(TQ_ERR_INVALID_ARG, "a dithered configuration is compressed by tq_compress_kv_dithered");
@@ -187,6 +201,7 @@ tq_status tq_compress_kv_dithered(const tq_config* cfg, const tq_params* params,
                                   int32_t layer, const void* k, const void* v, const float* k_offsets,
                                   const float* v_offsets, int32_t in_dtype, int32_t max_len,
                                   const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_compress_kv_dithered");
   clear_error();
   if (!cfg || !cfg->dither) return fail(TQ_ERR_INVALID_ARG, "tq_compress_kv_dithered needs cfg->dither = 1");
   if (!k_offsets || !v_offsets) return fail(TQ_ERR_INVALID_ARG, "k_offsets or v_offsets is NULL");
@@ -200,6 +215,7 @@ size_t tq_operand_bytes(const tq_config* cfg) {
 }
 
 tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, void* operands, tq_stream_t stream) {
+  CallRange range("tq_prepare_operands");
   clear_error();
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
@@ -320,6 +336,7 @@ tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const 
                            int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads, int32_t seq_q,
                            const int32_t* seq_lens, int32_t n_splits, void* workspace,
                            size_t workspace_bytes, float* out, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_attend_decode");
   clear_error();
   tqk::DecodeArgs a;
   tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, n_splits,
@@ -339,6 +356,7 @@ tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params,
                                   int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
                                   size_t workspace_bytes, float* out, int32_t* dev_status,
                                   tq_stream_t stream) {
+  CallRange range("tq_append_attend_decode");
   clear_error();
   tqk::DecodeArgs a;
   tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, n_splits,
@@ -362,6 +380,7 @@ tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params,
 tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
                        const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new,
                        const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_append_kv");
   clear_error();
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
@@ -396,6 +415,7 @@ tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params, const 
                            int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads, int32_t seq_q,
                            const int32_t* seq_lens, int32_t max_len, void* workspace,
                            size_t workspace_bytes, float* scores, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_decode_scores");
   clear_error();
   tqk::DecodeArgs a;
   tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, 1,
@@ -414,6 +434,7 @@ tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params, const 
 tq_status tq_decompress(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
                         const int32_t* seq_lens, int32_t max_len, float* k_hat, float* v_hat,
                         int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_decompress");
   clear_error();
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
