@@ -389,16 +389,24 @@ struct QuantConst {
 // steps.  s = [y' > 0] is the sign bit of tiny - y' (exact at +-0).  With KQ also the scaled
 // residual a y' - a sqrt(d) fp16(||x||) c[idx] (|c| read from a table by the rank, signed
 // by s) split into fp16 hi / lo pairs for the sketch MMAs, and its sum of squares (into rr2).
+// SH (dithered or corrected formats): the quantiser's input is y' + shift (shift = -xi ||y'||
+// for an offset xi) and the residual a (y' - sqrt(d) n (c + xi)) is formed as
+// a (y' + shift) + delta - csa c with delta = a xi (||y'|| - sqrt(d) n).  CK: also the sums of
+// |c| squared and of the signed c over the chunk (into cs2, cs1), for the corrected norm.
 constexpr float kTiny = 1.40129846e-45f;  // 2^-149
-template <int NB, class F, bool KQ>
+template <int NB, class F, bool KQ, bool SH = false, bool CK = false>
 __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantConst<NB>& qc, const float* cmag,
-                                           uint32_t (&w)[4], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2) {
+                                           uint32_t (&w)[4], uint32_t (&hi)[16], uint32_t (&lo)[16], f2_t& rr2,
+                                           float shift = 0.f, float delta = 0.f, f2_t* cs1 = nullptr,
+                                           f2_t* cs2 = nullptr) {
+  static_assert(!(KQ && CK), "the centroid sums are taken in a pass of their own");
   constexpr int MS = KQ ? 2 : 0;
   const f2_t magic = f2s(KQ ? kMagic21 : kMagic23);
   float u[32];
 #pragma unroll
   for (int i = 0; i < 32; i += 2) {
-    const float y0 = y[i], y1 = y[i + 1];
+    float y0 = y[i], y1 = y[i + 1];
+    if constexpr (SH) uf2(add2(f2(y0, y1), f2s(shift)), y0, y1);
     f2_t sum;
     if constexpr (NB == 3) {
       const f2_t s2 = f2(fma_sat(fabsf(y0), qc.ts.bs, qc.tb[1]), fma_sat(fabsf(y1), qc.ts.bs, qc.tb[1]));
@@ -418,12 +426,22 @@ __device__ __forceinline__ void quantise32(const float (&y)[32], const QuantCons
     w[F::word(i)] += shl(code0, F::shift(i) - MS);
     w[F::word(i + 1)] += shl(code1, F::shift(i + 1) - MS);
     uf2(fma2(f2(y0, y1), f2s(-1.f), f2s(kTiny)), u[i], u[i + 1]);
+    if constexpr (CK) {
+      // the rank sits at mantissa bit 0: |c| at byte offset 4 rank of the table
+      const uint32_t m0 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + ((code0 & NB) << 2));
+      const uint32_t m1 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + ((code1 & NB) << 2));
+      const f2_t M = f2(__uint_as_float(m0), __uint_as_float(m1));
+      *cs2 = fma2(M, M, *cs2);
+      *cs1 = add2(*cs1, f2(__uint_as_float(m0 | (~__float_as_uint(u[i]) & 0x80000000u)),
+                           __uint_as_float(m1 | (~__float_as_uint(u[i + 1]) & 0x80000000u))));
+    }
     if constexpr (KQ) {
       const uint32_t m0 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + (code0 & 0xCu));
       const uint32_t m1 = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(cmag) + (code1 & 0xCu));
       const f2_t C = f2(__uint_as_float(m0 | (~__float_as_uint(u[i]) & 0x80000000u)),
                         __uint_as_float(m1 | (~__float_as_uint(u[i + 1]) & 0x80000000u)));
-      const f2_t R = fma2(C, f2s(-qc.csa), mul2(f2(y0, y1), f2s(qc.alpha)));
+      const f2_t ay = SH ? fma2(f2(y0, y1), f2s(qc.alpha), f2s(delta)) : mul2(f2(y0, y1), f2s(qc.alpha));
+      const f2_t R = fma2(C, f2s(-qc.csa), ay);
       rr2 = fma2(R, R, rr2);
       float r0, r1;
       uf2(R, r0, r1);
@@ -470,7 +488,9 @@ struct TokRef {
   int slot;
 };
 
-template <int KB, int KQ, int VB>
+// MODE 1: the dithered (offsets read per token, stored in KD / VD) and corrected-norm (keys:
+// a first pass over the key chunks collects |c| sums for the stored norm) formats.
+template <int KB, int KQ, int VB, int MODE>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     compress_tc_kernel(CompressArgs a, const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv) {
@@ -778,15 +798,27 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     // independent loads, issued one group tile ahead and checked when the tile starts.
     struct TokLoad {
       int len, phys, t0, h;
+      float ko, vo;  // dithered: the token's key and value offsets
     };
+    const bool dith = MODE != 0 && L.dither != 0;
     auto token_load = [&](int j) -> TokLoad {
       int b, h, t0;
       tile_coords(j, b, h, t0);
       const int page = (t0 + row) / PT;
-      return TokLoad{a.seq_lens[b],
-                     page < a.cache.max_pages ? a.cache.block_table[(size_t)b * a.cache.max_pages + page] : -1, t0, h};
+      TokLoad l{a.seq_lens[b],
+                page < a.cache.max_pages ? a.cache.block_table[(size_t)b * a.cache.max_pages + page] : -1, t0, h,
+                0.f, 0.f};
+      if (dith && t0 + row < a.max_len) {
+        const size_t o = ((size_t)b * a.cache.kv_heads + h) * a.max_len + t0 + row;
+        l.ko = a.k_off[o];
+        l.vo = a.v_off[o];
+      }
+      return l;
     };
+    float cur_ko = 0.f, cur_vo = 0.f;
     auto token_ref = [&](const TokLoad& l) -> TokRef {
+      cur_ko = l.ko;
+      cur_vo = l.vo;
       const int tok = l.t0 + row;
       const bool bad_len = l.len < 0 || l.len > a.max_len || l.len > a.cache.max_pages * PT;
       if (bad_len && row == 0 && l.t0 == 0) report(a.status, TQ_ERR_BOUNDS);
@@ -856,13 +888,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       const float nyk = sqrtf(ssk);  // ||y'_K|| = sqrt(d) ||k||
       const float nyv = sqrtf(ssv);
-      const __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
+      __half nk16 = __float2half_rn(nyk * (1.0f / kSqrtD));
       const __half nv16 = __float2half_rn(nyv * (1.0f / kSqrtD));
-      if (cur.blk && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
+      // dithered: the offsets as used and stored (fp16); the quantiser's input is
+      // y' - xi ||y'|| (y - xi in unit-vector coordinates)
+      const __half kxi16 = __float2half_rn(cur_ko), vxi16 = __float2half_rn(cur_vo);
+      const float kxi = dith ? __half2float(kxi16) : 0.f, vxi = dith ? __half2float(vxi16) : 0.f;
 
       // ---- values, then keys chunk by chunk; the keys' residual goes to TMEM in place and each
       // chunk is released to the sketch MMAs while the next chunk's load is in flight ----
-      const QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
+      QuantConst<HK - 1> qk(nyk, sm.kb + HK, __half2float(nk16));
       const QuantConst<HV - 1> qv(nyv, sm.vb + HV, 0.f);
       // Value chunks are quantised from one register buffer while the next chunk's load into
       // the other is in flight (two chunks per iteration, the buffers alternating).
@@ -870,7 +905,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         constexpr uint32_t vw0 = FV::init(0, 0), vw1 = FV::init(1, 0), vw2 = FV::init(2, 0), vw3 = FV::init(3, 0);
         uint32_t vw[4] = {vw0, vw1, vw2, vw3}, dh[16], dl[16];
         f2_t drr = 0;
-        quantise32<HV - 1, FV, false>(z, qv, sm.kmag, vw, dh, dl, drr);
+        quantise32<HV - 1, FV, false, MODE != 0>(z, qv, sm.kmag, vw, dh, dl, drr, -vxi * nyv);
         if (cur.blk && !failed)
           store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
       };
@@ -888,6 +923,38 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (c + 2 < 4) tmem_wait_ld();
         }
       }
+      // corrected norm: a first pass over the key chunks collects sum |c|^2 and sum c for
+      // ||y_hat||^2 = sum (c + xi)^2; without QJL its words are the stored ones
+      const bool corr = MODE != 0 && a.key_corr != 0;
+      if (corr) {
+        f2_t cs1 = 0, cs2 = 0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float y[32];
+          tmem_ld32(colK + 32 * c, y);
+          tmem_wait_ld();
+          constexpr uint32_t pw0 = FK::init(0, 0), pw1 = FK::init(1, 0), pw2 = FK::init(2, 0), pw3 = FK::init(3, 0);
+          uint32_t pw[4] = {pw0, pw1, pw2, pw3}, dh[16], dl[16];
+          f2_t drr = 0;
+          quantise32<HK - 1, FK, false, true, true>(y, qk, sm.kmag, pw, dh, dl, drr, -kxi * nyk, 0.f, &cs1, &cs2);
+          if (!KQ && cur.blk && !failed)
+            store_chunk<KB, false>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+        }
+        float p0, p1, q0, q1;
+        uf2(cs1, p0, p1);
+        uf2(cs2, q0, q1);
+        const float yy = (q0 + q1) + kxi * (2.f * (p0 + p1) + (float)D * kxi);
+        const float yn = sqrtf(fmaxf(yy, 0.f));
+        nk16 = __float2half_rn(yn > 0.f ? (nyk * (1.0f / kSqrtD)) / yn : 0.f);
+        qk.csa = qk.alpha * kSqrtD * __half2float(nk16);
+      }
+      if (cur.blk && (__hisinf(nk16) || __hisinf(nv16))) report(a.status, TQ_ERR_OVERFLOW);
+      // residual offset of the dithered keys: a xi (||y'|| - sqrt(d) n)
+      const float kdelta = qk.alpha * kxi * (nyk - kSqrtD * __half2float(nk16));
+      if (MODE != 0 && dith && cur.blk && !failed) {
+        reinterpret_cast<__half*>(cur.blk + L.kd)[cur.slot] = kxi16;
+        reinterpret_cast<__half*>(cur.blk + L.vd)[cur.slot] = vxi16;
+      }
       f2_t rr2 = 0;
       // key words of the four chunks (completed by the signs)
       uint4 kw0 = make_uint4(0, 0, 0, 0), kw1 = kw0, kw2 = kw0, kw3 = kw0;
@@ -898,7 +965,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (lane == 0) bar_arrive(&sm.a_chunk[g][c]);
       };
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 4 && !(corr && !KQ); ++c) {
         float y[32];
         tmem_ld32(colK + 32 * c, y);
         if (KQ && c > 0) release(c - 1);
@@ -907,7 +974,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         constexpr uint32_t kwi0 = FK::init(0, kMS), kwi1 = FK::init(1, kMS), kwi2 = FK::init(2, kMS),
                            kwi3 = FK::init(3, kMS);
         uint32_t kw[4] = {kwi0, kwi1, kwi2, kwi3}, hi[16], lo[16];
-        quantise32<HK - 1, FK, KQ != 0>(y, qk, sm.kmag, kw, hi, lo, rr2);
+        quantise32<HK - 1, FK, KQ != 0, MODE != 0>(y, qk, sm.kmag, kw, hi, lo, rr2, -kxi * nyk, kdelta);
         const uint4 kq = make_uint4(kw[0], kw[1], kw[2], kw[3]);
         if constexpr (KQ) {
           tmem_st16(colK + 32 * c, hi);
@@ -1069,7 +1136,7 @@ bool make_tile_map(CUtensorMap* m, const void* base, size_t rows) {
 
 template <int KB, int KQ, int VB>
 cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
-  auto k = compress_tc_kernel<KB, KQ, VB>;
+  auto k = (a.cache.L.dither || a.key_corr) ? compress_tc_kernel<KB, KQ, VB, 1> : compress_tc_kernel<KB, KQ, VB, 0>;
   // the register hand-over inside the kernel assumes the launch allocation it was built for
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != kRegsLaunch ||
@@ -1100,7 +1167,7 @@ cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtens
 
 bool compress_tc_supported(const CompressArgs& a) {
   const Layout& L = a.cache.L;
-  if (a.in_dtype != TQ_F16 || L.vqjl || L.dither || a.key_corr) return false;
+  if (a.in_dtype != TQ_F16 || L.vqjl) return false;
   if (a.dense && (L.qjl || a.operands == nullptr)) return false;
   if ((size_t)a.cache.batch * a.cache.kv_heads * a.max_len >= (1ull << 31)) return false;
   if (L.qjl && !(L.kbits == 2 || L.kbits == 3)) return false;
