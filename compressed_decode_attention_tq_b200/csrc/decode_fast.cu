@@ -25,8 +25,10 @@
 //
 // Supported here: keys 3-bit + QJL (merged nibbles), 2-bit + QJL, or 4-bit without QJL
 // (sign-magnitude nibbles, the signs applied by byte masks), values 3-bit or 2-bit, any R;
-// the randomized Hadamard rotation or a dense Pi (R^T applied in the merge).  Everything
-// else uses decode.cu.
+// the randomized Hadamard rotation or a dense Pi (R^T applied in the merge); dithered codes
+// (DT: a key's offset adds xi_k sum_i (R q)_i to its dot product, a value's adds xi_v to
+// every coordinate, carried as one running sum per row next to the accumulator).
+// Everything else uses decode.cu.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -43,7 +45,7 @@ constexpr int kStages = 3;
 constexpr int kUnit = PT / 2;                  // tokens per copy unit: half a page
 constexpr int kUnitsPerPage = PT / kUnit;
 constexpr int kChunkStride = kUnit * 16 + 32;  // padded so the 4 lanes of a token group hit distinct banks
-constexpr int kNormBytes = 3 * kUnit * 2;      // KN | KR | VN of the unit
+constexpr int kNormBytes = 5 * kUnit * 2;      // KN | KR | VN | KD | VD of the unit
 constexpr int kMaxKChunks = 4;
 constexpr int kMaxVChunks = 3;
 constexpr int kStageBytes = kNormBytes + (kMaxKChunks + kMaxVChunks) * kChunkStride;
@@ -75,6 +77,7 @@ struct SmemFast {
   unsigned long long mbar;  // the merge copies landed
   unsigned long long never;  // completed by nothing: the target of the bounded-wait test
   float wm[kConsumerWarps][kMaxRows], wl[kConsumerWarps][kMaxRows], wf[kConsumerWarps][kMaxRows];
+  float wx[kConsumerWarps][kMaxRows];  // dithered values: sum_t p_t ||v_t|| xi_t of each warp and row
   int last;
 };
 
@@ -229,7 +232,7 @@ __device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int
   return (t1 & 0x3u) | ((t2 & 0x3u) << 4) | (t1 & 0x300u) | ((t2 & 0x300u) << 4);
 }
 
-template <int KP, int VP, int NR>
+template <int KP, int VP, int NR, bool DT>
 __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   static_assert(NR == 4 || NR == 8, "four or eight rows per CTA");
   constexpr int NT = NR / 4;  // n-tiles of the key and QJL products
@@ -263,7 +266,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   constexpr int kVChunks = (VP == V3) ? 3 : 2;
   constexpr bool kQjl = KP != K4;
   // without QJL there is no KR region: its norm slots stay unused
-  const uint32_t unit_bytes = kNormBytes - (kQjl ? 0u : 2u * kUnit) + 16u * kUnit * (kKChunks + kVChunks);
+  const uint32_t unit_bytes =
+      2u * kUnit * (2 + (kQjl ? 1 : 0) + (DT ? 2 : 0)) + 16u * kUnit * (kKChunks + kVChunks);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -309,6 +313,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         bulk_g2s(st, blk + L.kn + hb2, kUnit * 2, &sm.full[s]);
         if (kQjl) bulk_g2s(st + kUnit * 2, blk + L.kr + hb2, kUnit * 2, &sm.full[s]);
         bulk_g2s(st + kUnit * 4, blk + L.vn + hb2, kUnit * 2, &sm.full[s]);
+        if (DT) {
+          bulk_g2s(st + kUnit * 6, blk + L.kd + hb2, kUnit * 2, &sm.full[s]);
+          bulk_g2s(st + kUnit * 8, blk + L.vd + hb2, kUnit * 2, &sm.full[s]);
+        }
         unsigned char* kc = st + kNormBytes;
         const int kcode_chunks = (KP == K2Q) ? 2 : 4;
         for (int c = 0; c < kcode_chunks; ++c)
@@ -528,15 +536,40 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       }
     }
 
+    // dithered keys: sum_i (R q)_i of the lane's score rows (the 8 lanes of a row add 16
+    // coordinates each)
+    float qs[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      qs[nt] = 0.f;
+      if (DT) {
+        const int rr = t4 + 4 * nt;
+        float t = 0.f;
+        if (rr < R) {
+          const float4* qp = reinterpret_cast<const float4*>(a.qrot + (row0 + rr) * D + 16 * g);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float4 f = qp[k];
+            t += (f.x + f.y) + (f.z + f.w);
+          }
+        }
+        t += __shfl_xor_sync(FULL, t, 4);
+        t += __shfl_xor_sync(FULL, t, 8);
+        t += __shfl_xor_sync(FULL, t, 16);
+        qs[nt] = t;
+      }
+    }
+
     if (a.debug_wait_ns > 0 && warp == 0 && split == 0 && gh == 0 && blockIdx.z == 0 &&
         !mbar_wait(&sm.never, 0, (unsigned long long)a.debug_wait_ns) && lane == 0)
       report(a.status, TQ_ERR_TIMEOUT);
 
-    float m_run[NT], l_run[NT];
+    float m_run[NT], l_run[NT], x_run[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       m_run[nt] = -CUDART_INF_F;
       l_run[nt] = 0.f;
+      x_run[nt] = 0.f;
     }
     float acc[8][4];
 #pragma unroll
@@ -677,8 +710,12 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             const float rA = kQjl ? ld_h(st + 2 * kUnit + 2 * ta) : 0.f;
             const float rB = kQjl ? ld_h(st + 2 * kUnit + 2 * tb) : 0.f;
             const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
-            const float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down[nt];
-            const float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down[nt];
+            float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down[nt];
+            float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down[nt];
+            if (DT) {
+              dotA = fmaf(ld_h(st + 6 * kUnit + 2 * ta), qs[nt], dotA);
+              dotB = fmaf(ld_h(st + 6 * kUnit + 2 * tb), qs[nt], dotB);
+            }
             float sca = nA * dotA * c_row_k + rA * (float)(2 * s1a - T_row[nt]) * c_row_q[nt];
             float scb = nB * dotB * c_row_k + rB * (float)(2 * s1b - T_row[nt]) * c_row_q[nt];
             if (t4 + 4 * nt >= R || ta >= valid) sca = -CUDART_INF_F;
@@ -714,6 +751,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             }
           }
           l_run[nt] = l_run[nt] * alpha[nt] + (p[0][nt][0] + p[0][nt][1]) + (p[1][nt][0] + p[1][nt][1]);
+          if (DT) x_run[nt] *= alpha[nt];
           m_run[nt] = m_new[nt];
         }
         if (grow) {
@@ -741,6 +779,13 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
           const int step = 2 * pr + u;
           const int ta = step * 16 + g, tb = ta + 8;
           const float vnA = ld_h(st + 4 * kUnit + 2 * ta), vnB = ld_h(st + 4 * kUnit + 2 * tb);
+          if (DT) {
+            // the values' offsets: xi_v to every coordinate, one running sum per row
+            const float xa = ta < valid ? vnA * ld_h(st + 8 * kUnit + 2 * ta) : 0.f;
+            const float xb = tb < valid ? vnB * ld_h(st + 8 * kUnit + 2 * tb) : 0.f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) x_run[nt] = fmaf(p[u][nt][0], xa, fmaf(p[u][nt][1], xb, x_run[nt]));
+          }
           // B = weights: column g is row g, from the lane holding row g's scores for the
           // tokens of B rows 2 t4 (+ 1, + 8, + 9); slots past the end may hold stale bytes:
           // their weight is forced to exactly 0
@@ -791,13 +836,19 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     // ---- warp partial: l summed over the 8 lanes of a row, acc scattered by coordinate
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      float lr = l_run[nt];
+      float lr = l_run[nt], xr = x_run[nt];
       lr += __shfl_xor_sync(FULL, lr, 4);
       lr += __shfl_xor_sync(FULL, lr, 8);
       lr += __shfl_xor_sync(FULL, lr, 16);
+      if (DT) {
+        xr += __shfl_xor_sync(FULL, xr, 4);
+        xr += __shfl_xor_sync(FULL, xr, 8);
+        xr += __shfl_xor_sync(FULL, xr, 16);
+      }
       if (g == 0 && t4 + 4 * nt < R) {
         sm.wm[warp][t4 + 4 * nt] = m_run[nt];
         sm.wl[warp][t4 + 4 * nt] = lr;
+        sm.wx[warp][t4 + 4 * nt] = xr;
       }
     }
 #pragma unroll
@@ -835,7 +886,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     const int r = idx / D, j = idx % D;
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) o = fmaf(sm.wf[w][r], sm.ring.wacc[w][r][j], o);
+    for (int w = 0; w < kConsumerWarps; ++w)
+      o = fmaf(sm.wf[w][r], DT ? sm.ring.wacc[w][r][j] + sm.wx[w][r] : sm.ring.wacc[w][r][j], o);
     a.part_acc[((row0 + r) * a.n_splits + split) * D + j] = o;
   }
   // ---- the last split of this (sequence, kv head) to finish merges all of them ----
@@ -979,8 +1031,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 
 bool fast_decode_supported(const DecodeArgs& a) {
   const Layout& L = a.cache.L;
-  // dithered codes need their offsets (general kernels); the merge reads Pi as float4
-  if (L.dither) return false;
+  // the merge reads Pi as float4
   if (a.dense && (reinterpret_cast<uintptr_t>(a.pi) & 15)) return false;
   const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl) || (L.kbits == 4 && !L.qjl);
   const bool vok = (L.vbits == 3 || L.vbits == 2) && !L.vqjl;
@@ -996,9 +1047,13 @@ cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
   const int nr = a.rows > 4 ? 8 : 4;
   dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch * ((a.rows + nr - 1) / nr));
   void (*k)(DecodeArgs) = nullptr;
-#define TQ_FAST(KB, KPOL, VB, VPOL)                                                             \
-  if (L.kbits == KB && L.vbits == VB)                                                            \
-    k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8> : fast_split_kernel<KPOL, VPOL, 4>;
+#define TQ_FAST(KB, KPOL, VB, VPOL)                                                         \
+  if (L.kbits == KB && L.vbits == VB) {                                                      \
+    if (L.dither)                                                                            \
+      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, true> : fast_split_kernel<KPOL, VPOL, 4, true>;   \
+    else                                                                                     \
+      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, false> : fast_split_kernel<KPOL, VPOL, 4, false>; \
+  }
   TQ_FAST(3, K3Q, 3, V3)
   TQ_FAST(3, K3Q, 2, V2)
   TQ_FAST(2, K2Q, 3, V3)

@@ -35,6 +35,11 @@ SMALL = {
                                     name="c2_dither"),
     "k2v4_dither": lambda: wl.config2(kv_heads=1, q_heads=4, max_len=600, key_bits=2, key_qjl=False,
                                       value_bits=4, n_splits=2, dither=True, name="k2v4_dither"),
+    # dithered on the tensor-core split decode: 2-bit QJL keys and values; 32 rows per KV head
+    "c4_dither": lambda: wl.config4(batch=2, kv_heads=2, q_heads=8, max_len=1100, n_splits=5, dither=True,
+                                    name="c4_dither"),
+    "c5_dither": lambda: wl.config5(kv_heads=2, q_heads=8, max_len=700, num_layers=1, n_splits=3, dither=True,
+                                    name="c5_dither"),
     # corrected key norms: merged QJL keys (fast decode) and dense 4-bit keys without QJL
     "c2_corrected_norm": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4,
                                             key_corrected_norm=True, name="c2_corrected_norm"),
