@@ -88,8 +88,14 @@ struct SmemTC {
   int bad_s;
   float kc[16], kb[16], vc[16], vb[16];  // codebooks: centroids, boundaries
   float kmag[8];                         // |c| of a key's magnitude rank r: c[h + r]
+  // the tiles that hold tokens: sequence b's are tprefix[b] .. tprefix[b + 1] - 1 (batches of
+  // at most kMaxCompact sequences; larger ones walk every tile of max_len)
+  int tprefix[257];
+  int ntiles;
 };
+constexpr int kMaxCompact = 256;
 constexpr size_t kSmemTC = sizeof(SmemTC) + 128;  // + base alignment slack
+static_assert(kSmemTC <= 232448, "shared memory of one thread block");
 
 // Canonical no-swizzle K-major offset of element (row, k) of a 128 x 128 fp16 tile:
 // 16-byte core-matrix rows, 8-row groups 128 B apart, 8-element K chunks 2048 B apart.
@@ -488,9 +494,11 @@ struct TokRef {
   int slot;
 };
 
-// MODE 1: the dithered (offsets read per token, stored in KD / VD) and corrected-norm (keys:
-// a first pass over the key chunks collects |c| sums for the stored norm) formats.
-template <int KB, int KQ, int VB, int MODE>
+// MODE bit 0: the dithered (offsets read per token, stored in KD / VD) and corrected-norm
+// (keys: a first pass over the key chunks collects |c| sums for the stored norm) formats.
+// MODE bit 1: a batch of several sequences, whose tiles past each sequence's length are
+// skipped (the tile list is built from the lengths at the start).
+template <int KB, int KQ, int VB, int MODE_>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     compress_tc_kernel(CompressArgs a, const __grid_constant__ CUtensorMap tmk,
                        const __grid_constant__ CUtensorMap tmv) {
@@ -506,18 +514,37 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   constexpr bool kMerged = KQ && KB == 3;
   constexpr int kComputeThreads = kComputeWarps * 32;
 
+  // Tiles: for a batch of 2 .. kMaxCompact sequences only those that hold tokens (a ragged
+  // batch skips the tails of its shorter sequences; the list costs a read of the lengths
+  // before the first copy); otherwise every tile of max_len.  The CTAs take the tiles round
+  // robin.
+  constexpr int MODE = MODE_ & 1;
+  constexpr bool compact = (MODE_ & 2) != 0;
   const int tiles_per_head = (a.max_len + TT - 1) / TT;
-  const int total = a.cache.batch * a.cache.kv_heads * tiles_per_head;
-  const int my_tiles = (int)blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-  auto tile_coords = [&](int j, int& b, int& h, int& t0) {
+  const int all_tiles = a.cache.batch * a.cache.kv_heads * tiles_per_head;
+  int my_tiles = compact ? 0 : ((int)blockIdx.x < all_tiles ? (all_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0);
+  // cursor: the caller's sequence index from its previous tile (its tiles only move forward)
+  auto tile_coords = [&](int j, int& b, int& h, int& t0, int& cursor) {
     const int t = blockIdx.x + j * gridDim.x;
-    t0 = (t % tiles_per_head) * TT;
-    h = (t / tiles_per_head) % a.cache.kv_heads;
-    b = t / (tiles_per_head * a.cache.kv_heads);
+    if (compact) {
+      // the sequence: tprefix[b] <= t < tprefix[b + 1] (a sequence without tiles has
+      // tprefix[b] == tprefix[b + 1] and is stepped over)
+      while (sm.tprefix[cursor + 1] <= t) ++cursor;
+      b = cursor;
+      const int nt = (sm.tprefix[b + 1] - sm.tprefix[b]) / a.cache.kv_heads;
+      const int local = t - sm.tprefix[b];
+      h = local / nt;
+      t0 = (local - h * nt) * TT;
+    } else {
+      t0 = (t % tiles_per_head) * TT;
+      h = (t / tiles_per_head) % a.cache.kv_heads;
+      b = t / (tiles_per_head * a.cache.kv_heads);
+    }
   };
+  int load_cursor = 0;
   auto issue_load = [&](int j) {
     int b, h, t0;
-    tile_coords(j, b, h, t0);
+    tile_coords(j, b, h, t0, load_cursor);
     const int row0 = (int)(((size_t)b * a.cache.kv_heads + h) * a.max_len + t0);
     unsigned long long* bar = &sm.bar_load[j & 1];
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(bar)), "r"(2 * kTileBytes)
@@ -564,8 +591,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   // (The dense rotation always comes prepared: sqrt(d) Pi hi / lo, two tiles.)
   const bool prep = a.operands != nullptr;
   const bool dense = a.dense != 0;
-  if (warp == kLoaderWarp && lane == 0) {
-    if (prep) {
+  if (warp == kLoaderWarp) {
+    if (prep && lane == 0) {
       const uint32_t nops = dense ? 2 : 3;
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(&sm.ops_ready)),
                    "r"(nops * kTileBytes)
@@ -575,7 +602,35 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       bulk_load(sm.bshi, ops + kTileBytes, kTileBytes, &sm.ops_ready);
       if (!dense) bulk_load(sm.bslo, ops + 2 * kTileBytes, kTileBytes, &sm.ops_ready);
     }
-    if (my_tiles > 0) issue_load(0);
+    // the tile list: H ceil(len / TT) tiles per sequence (one per head for a length out of
+    // range, whose first tile reports it), by a warp-wide scan
+    if (compact) {
+      int carry = 0;
+      for (int b0 = 0; b0 < a.cache.batch; b0 += 32) {
+        const int b = b0 + lane;
+        int n = 0;
+        if (b < a.cache.batch) {
+          const int len = a.seq_lens[b];
+          const bool bad = len < 0 || len > a.max_len || len > a.cache.max_pages * PT;
+          n = a.cache.kv_heads * (bad ? 1 : (len + TT - 1) / TT);
+        }
+        int x = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (b < a.cache.batch) sm.tprefix[b + 1] = carry + x;
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+      if (lane == 0) {
+        sm.tprefix[0] = 0;
+        sm.ntiles = carry;
+      }
+      __syncwarp();
+      my_tiles = (int)blockIdx.x < sm.ntiles ? (sm.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    }
+    if (lane == 0 && my_tiles > 0) issue_load(0);
   }
   __syncwarp();
   if (!producer) {
@@ -672,6 +727,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       __syncwarp();
       if (lane == 0) bar_arrive(&sm.s_ready);
     }
+  }
+  if (compact) {
+    // the tile list is in shared memory for every role (compact is the same in every thread)
+    asm volatile("bar.sync 6, %0;" ::"n"(kThreadsTC) : "memory");
+    my_tiles = (int)blockIdx.x < sm.ntiles ? (sm.ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   }
   const uint32_t tmem = sm.tmem_base;
 
@@ -801,9 +861,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       float ko, vo;  // dithered: the token's key and value offsets
     };
     const bool dith = MODE != 0 && L.dither != 0;
+    int tok_cursor = 0;
     auto token_load = [&](int j) -> TokLoad {
       int b, h, t0;
-      tile_coords(j, b, h, t0);
+      tile_coords(j, b, h, t0, tok_cursor);
       const int page = (t0 + row) / PT;
       TokLoad l{a.seq_lens[b],
                 page < a.cache.max_pages ? a.cache.block_table[(size_t)b * a.cache.max_pages + page] : -1, t0, h,
@@ -1136,7 +1197,12 @@ bool make_tile_map(CUtensorMap* m, const void* base, size_t rows) {
 
 template <int KB, int KQ, int VB>
 cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
-  auto k = (a.cache.L.dither || a.key_corr) ? compress_tc_kernel<KB, KQ, VB, 1> : compress_tc_kernel<KB, KQ, VB, 0>;
+  const int mode = ((a.cache.L.dither || a.key_corr) ? 1 : 0) |
+                   ((a.cache.batch > 1 && a.cache.batch <= kMaxCompact) ? 2 : 0);
+  auto k = mode == 0 ? compress_tc_kernel<KB, KQ, VB, 0>
+           : mode == 1 ? compress_tc_kernel<KB, KQ, VB, 1>
+           : mode == 2 ? compress_tc_kernel<KB, KQ, VB, 2>
+                       : compress_tc_kernel<KB, KQ, VB, 3>;
   // the register hand-over inside the kernel assumes the launch allocation it was built for
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != kRegsLaunch ||
