@@ -498,6 +498,10 @@ struct TokRef {
 // (keys: a first pass over the key chunks collects |c| sums for the stored norm) formats.
 // MODE bit 1: a batch of several sequences, whose tiles past each sequence's length are
 // skipped (the tile list is built from the lengths at the start).
+// MODE bit 2: the value sketch of values with QJL, a second launch after the first one has
+// stored every code: the value tiles go through the key path (KB = VB, KQ = 1, the value
+// codebook in the key tables), which recomputes their codes, forms the residual against the
+// stored norm and sketches it; only the signs (VS) and the residual norm (VR) are stored.
 template <int KB, int KQ, int VB, int MODE_>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     compress_tc_kernel(CompressArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -510,16 +514,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int qd = warp & 3;           // tensor-memory lane quadrant
   const int row = 32 * qd + lane;    // token within the tile
   const Layout& L = a.cache.L;
+  constexpr int MODE = MODE_ & 1;
+  constexpr bool compact = (MODE_ & 2) != 0;
+  constexpr bool VSP = (MODE_ & 4) != 0;
+  static_assert(!VSP || (KB == VB && KQ && MODE == 0), "the value-sketch pass runs the key path");
   constexpr int HK = 1 << (KB - 1), HV = 1 << (VB - 1);
-  constexpr bool kMerged = KQ && KB == 3;
+  constexpr bool kMerged = KQ && KB == 3 && !VSP;
   constexpr int kComputeThreads = kComputeWarps * 32;
 
   // Tiles: for a batch of 2 .. kMaxCompact sequences only those that hold tokens (a ragged
   // batch skips the tails of its shorter sequences; the list costs a read of the lengths
   // before the first copy); otherwise every tile of max_len.  The CTAs take the tiles round
   // robin.
-  constexpr int MODE = MODE_ & 1;
-  constexpr bool compact = (MODE_ & 2) != 0;
   const int tiles_per_head = (a.max_len + TT - 1) / TT;
   const int all_tiles = a.cache.batch * a.cache.kv_heads * tiles_per_head;
   int my_tiles = compact ? 0 : ((int)blockIdx.x < all_tiles ? (all_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0);
@@ -547,10 +553,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     tile_coords(j, b, h, t0, load_cursor);
     const int row0 = (int)(((size_t)b * a.cache.kv_heads + h) * a.max_len + t0);
     unsigned long long* bar = &sm.bar_load[j & 1];
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(bar)), "r"(2 * kTileBytes)
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s_u32(bar)),
+                 "r"((VSP ? 1 : 2) * kTileBytes)
                  : "memory");
     tma_load_tile(sm.x[j & 1][0], &tmk, row0, bar);
-    tma_load_tile(sm.x[j & 1][1], &tmv, row0, bar);
+    if (!VSP) tma_load_tile(sm.x[j & 1][1], &tmv, row0, bar);
   };
 
   // ---------------- set-up ----------------
@@ -642,8 +649,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const float sgn = !prep && tid < D ? a.signs[tid] : 0.f;
     float tkc = 0.f, tkb = 0.f, tvc = 0.f, tvb = 0.f;
     if (tid < 16) {
-      tkc = tid < 2 * HK ? a.k_centroids[tid] : 0.f;
-      tkb = tid < 2 * HK - 1 ? a.k_boundaries[tid] : 0.f;
+      tkc = tid < 2 * HK ? (VSP ? a.v_centroids : a.k_centroids)[tid] : 0.f;
+      tkb = tid < 2 * HK - 1 ? (VSP ? a.v_boundaries : a.k_boundaries)[tid] : 0.f;
       tvc = tid < 2 * HV ? a.v_centroids[tid] : 0.f;
       tvb = tid < 2 * HV - 1 ? a.v_boundaries[tid] : 0.f;
     }
@@ -783,7 +790,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           if (!(ok = bar_wait(&sm.tm_free[g], (n - 1) & 1))) break;
           tc_fence_after();
         }
-        fwd(1, colV);
+        if (!VSP) fwd(1, colV);
         mma_commit(&sm.fwd_done[g]);
         mma_commit(&sm.stage_free[g]);  // both forward MMAs of tile j have read stage g
         k_issued = false;
@@ -942,10 +949,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       for (int c = 0; c < 4; ++c) {
         float y[32], z[32];
         tmem_ld32(colK + 32 * c, y);
-        tmem_ld32(colV + 32 * c, z);
+        if (!VSP) tmem_ld32(colV + 32 * c, z);
         tmem_wait_ld();
         ssk += sumsq32(y);
-        ssv += sumsq32(z);
+        if (!VSP) ssv += sumsq32(z);
       }
       const float nyk = sqrtf(ssk);  // ||y'_K|| = sqrt(d) ||k||
       const float nyv = sqrtf(ssv);
@@ -970,7 +977,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         if (cur.blk && !failed)
           store_chunk<VB, false>(cur.blk + L.vc, c >> 1, c & 1, cur.slot, make_uint4(vw[0], vw[1], vw[2], vw[3]));
       };
-      {
+      if (!VSP) {
         float za[32], zb[32];
         tmem_ld32(colV, za);
         tmem_wait_ld();
@@ -1044,7 +1051,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           kw1 = c == 1 ? kq : kw1;
           kw2 = c == 2 ? kq : kw2;
           kw3 = c == 3 ? kq : kw3;
-        } else if (cur.blk && !failed) {
+        } else if (cur.blk && !failed && !VSP) {
           store_chunk<KB, false>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, kq);
         }
       }
@@ -1054,9 +1061,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         uf2(rr2, ra, rb);
         const float rho = sqrtf(ra + rb) * qk.inv_alpha * (1.0f / kSqrtD);
         if (cur.blk && !failed) {
-          reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
-          reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
-          reinterpret_cast<__half*>(cur.blk + L.kr)[cur.slot] = __float2half_rn(rho);
+          if (VSP) {
+            reinterpret_cast<__half*>(cur.blk + L.vr)[cur.slot] = __float2half_rn(rho);
+          } else {
+            reinterpret_cast<__half*>(cur.blk + L.vn)[cur.slot] = nv16;
+            reinterpret_cast<__half*>(cur.blk + L.kn)[cur.slot] = nk16;
+            reinterpret_cast<__half*>(cur.blk + L.kr)[cur.slot] = __float2half_rn(rho);
+          }
         }
         // the sketch's signs complete the key words
         if (!failed && !bar_wait(&sm.sig_done[g], n & 1)) failed = true;
@@ -1076,8 +1087,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           uint32_t sgw = 0;
           sigma32<kMerged, FK>(sk, w, sgw);
           if (cur.blk && !failed) {
-            store_chunk<KB, kMerged>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, w);
-            if (!kMerged) *reinterpret_cast<uint32_t*>(cur.blk + L.ks + (size_t)cur.slot * 16 + 4 * c) = sgw;
+            if (VSP) {
+              *reinterpret_cast<uint32_t*>(cur.blk + L.vs + (size_t)cur.slot * 16 + 4 * c) = sgw;
+            } else {
+              store_chunk<KB, kMerged>(cur.blk + L.kc, c >> 1, c & 1, cur.slot, w);
+              if (!kMerged) *reinterpret_cast<uint32_t*>(cur.blk + L.ks + (size_t)cur.slot * 16 + 4 * c) = sgw;
+            }
           }
         };
         finish(sk0, kw0, 0);
@@ -1196,13 +1211,21 @@ bool make_tile_map(CUtensorMap* m, const void* base, size_t rows) {
 }
 
 template <int KB, int KQ, int VB>
-cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
-  const int mode = ((a.cache.L.dither || a.key_corr) ? 1 : 0) |
-                   ((a.cache.batch > 1 && a.cache.batch <= kMaxCompact) ? 2 : 0);
-  auto k = mode == 0 ? compress_tc_kernel<KB, KQ, VB, 0>
-           : mode == 1 ? compress_tc_kernel<KB, KQ, VB, 1>
-           : mode == 2 ? compress_tc_kernel<KB, KQ, VB, 2>
-                       : compress_tc_kernel<KB, KQ, VB, 3>;
+cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream,
+                      bool value_sketch = false) {
+  const bool cmp = a.cache.batch > 1 && a.cache.batch <= kMaxCompact;
+  const int mode = ((a.cache.L.dither || a.key_corr) ? 1 : 0) | (cmp ? 2 : 0);
+  void (*k)(CompressArgs, const CUtensorMap, const CUtensorMap);
+  if constexpr (KB == VB && KQ == 1) {
+    if (value_sketch) k = cmp ? compress_tc_kernel<VB, 1, VB, 6> : compress_tc_kernel<VB, 1, VB, 4>;
+  }
+  if (!value_sketch)
+    k = mode == 0 ? compress_tc_kernel<KB, KQ, VB, 0>
+        : mode == 1 ? compress_tc_kernel<KB, KQ, VB, 1>
+        : mode == 2 ? compress_tc_kernel<KB, KQ, VB, 2>
+                    : compress_tc_kernel<KB, KQ, VB, 3>;
+  else if (!(KB == VB && KQ == 1))
+    return cudaErrorInvalidValue;
   // the register hand-over inside the kernel assumes the launch allocation it was built for
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, k) != cudaSuccess || fa.numRegs != kRegsLaunch ||
@@ -1233,8 +1256,11 @@ cudaError_t launch_tc(const CompressArgs& a, const CUtensorMap& mk, const CUtens
 
 bool compress_tc_supported(const CompressArgs& a) {
   const Layout& L = a.cache.L;
-  if (a.in_dtype != TQ_F16 || L.vqjl) return false;
+  if (a.in_dtype != TQ_F16) return false;
   if (a.dense && (L.qjl || a.operands == nullptr)) return false;
+  // values with QJL: a second launch sketches them through the key path (2- or 3-bit
+  // values, the randomized Hadamard rotation, not dithered)
+  if (L.vqjl && (a.dense || L.dither || !(L.vbits == 2 || L.vbits == 3))) return false;
   if ((size_t)a.cache.batch * a.cache.kv_heads * a.max_len >= (1ull << 31)) return false;
   if (L.qjl && !(L.kbits == 2 || L.kbits == 3)) return false;
   if (!L.qjl && !(L.kbits >= 2 && L.kbits <= 4)) return false;
@@ -1262,8 +1288,9 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   if (!make_tile_map(&mk, a.k, rows) || !make_tile_map(&mv, a.v, rows)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaErrorInvalidValue;
 #define TQ_TC(KB, KQ, VB) \
-  if (L.kbits == KB && L.qjl == KQ && L.vbits == VB) return launch_tc<KB, KQ, VB>(a, mk, mv, stream);
+  if (L.kbits == KB && L.qjl == KQ && L.vbits == VB) e = launch_tc<KB, KQ, VB>(a, mk, mv, stream);
 #define TQ_TC_V(KB, KQ) TQ_TC(KB, KQ, 2) TQ_TC(KB, KQ, 3) TQ_TC(KB, KQ, 4)
   TQ_TC_V(3, 1)
   TQ_TC_V(2, 1)
@@ -1272,6 +1299,10 @@ cudaError_t launch_compress_tc(const CompressArgs& a, cudaStream_t stream) {
   TQ_TC_V(4, 0)
 #undef TQ_TC_V
 #undef TQ_TC
+  if (e != cudaSuccess || !L.vqjl) return e;
+  // the value sketch, once every code is stored (a programmatic dependent of the first launch)
+  if (L.vbits == 2) return launch_tc<2, 1, 2>(a, mv, mv, stream, true);
+  if (L.vbits == 3) return launch_tc<3, 1, 3>(a, mv, mv, stream, true);
   return cudaErrorInvalidValue;
 }
 

@@ -227,9 +227,9 @@ tq_status tq_prepare_operands(const tq_config* cfg, const tq_params* params, voi
     e = tqk::launch_prepare_dense(params->pi, operands, reinterpret_cast<cudaStream_t>(stream));
   } else {
     if (!params || !params->signs) return fail(TQ_ERR_INVALID_ARG, "params or params->signs is NULL");
-    if (cfg->key_qjl && !params->s) return fail(TQ_ERR_INVALID_ARG, "params->s is NULL");
-    e = tqk::launch_prepare_operands(params->signs, params->s, cfg->key_qjl, operands,
-                                     reinterpret_cast<cudaStream_t>(stream));
+    const int qjl = cfg->key_qjl || cfg->value_qjl;
+    if (qjl && !params->s) return fail(TQ_ERR_INVALID_ARG, "params->s is NULL");
+    e = tqk::launch_prepare_operands(params->signs, params->s, qjl, operands, reinterpret_cast<cudaStream_t>(stream));
   }
   if (e != cudaSuccess) return cuda_fail(e, "tq_prepare_operands launch");
   return TQ_OK;

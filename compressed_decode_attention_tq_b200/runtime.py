@@ -74,7 +74,7 @@ class PagedKV:
         if rotation == TQ_ROT_DENSE:
             have = t["pi"] is not None
         else:
-            have = t["signs"] is not None and (not key_qjl or t["s"] is not None)
+            have = t["signs"] is not None and (not (key_qjl or value_qjl) or t["s"] is not None)
         if prepared_operands and nops and have:
             t["ops"] = torch.empty(nops, dtype=torch.uint8, device=self.device)
             prepare_operands(self.cfg, make_params(t["signs"], t["pi"], s=t["s"]), t["ops"])

@@ -30,6 +30,9 @@ SMALL = {
                                   name="c2_vqjl"),
     "c3_vqjl_dense": lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=3, value_qjl=True,
                                         name="c3_vqjl_dense"),
+    # 2-bit values with QJL in a two-sequence batch (the value sketch as a second tensor-core launch)
+    "c4_vqjl": lambda: wl.config4(batch=2, kv_heads=2, q_heads=8, max_len=1100, n_splits=5, value_qjl=True,
+                                  name="c4_vqjl"),
     # dithered HD: merged QJL keys and 3-bit values; MSE-only 2-bit keys and 4-bit values
     "c2_dither": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4, dither=True,
                                     name="c2_dither"),
@@ -61,6 +64,8 @@ IN_BLOCK = {
                                                name="c2_in_block_operands"),
     "c4_in_block_operands": lambda: wl.config4(batch=2, kv_heads=2, q_heads=8, max_len=2000, n_splits=8,
                                                name="c4_in_block_operands"),
+    "c2_vqjl_in_block_operands": lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1300, n_splits=4,
+                                                    value_qjl=True, name="c2_vqjl_in_block_operands"),
 }
 
 
