@@ -68,7 +68,8 @@ def workload(n_splits: int = 0, device_index: int = 0):
     import workloads as wl
     from compressed_decode_attention_tq_b200.runtime import splits_for
     w = wl.config2()
-    w.n_splits = n_splits or splits_for(w.batch, w.kv_heads, sm_count(device_index))
+    w.n_splits = n_splits or splits_for(w.batch, w.kv_heads, sm_count(device_index), rows=w.group * w.seq_q,
+                                        max_len=w.max_len)
     return w
 
 
@@ -456,7 +457,10 @@ def config_timings(dev, reps: int = 10):
             K, V = wl.make_kv_device(w, 0, dev)
             q = wl.make_q_device(w, 0, dev)
         seq = torch.as_tensor(lens, dtype=torch.int32, device=dev)
-        ns = default_splits(w.batch, w.kv_heads, dev.index or 0) if c == 2 else w.n_splits
+        # the library's default split count, except where the workload fixes it (64 splits
+        # per head for the long-context workload)
+        ns = (w.n_splits if c == 4 else
+              default_splits(w.batch, w.kv_heads, dev.index or 0, rows=w.group * w.seq_q, max_len=w.max_len))
         out = torch.empty(q.shape, dtype=torch.float32, device=dev)
 
         def timed(fn):

@@ -21,16 +21,22 @@ def _f32(x, device):
     return torch.as_tensor(x, dtype=torch.float32).to(device).contiguous()
 
 
-def splits_for(batch: int, kv_heads: int, sms: int) -> int:
-    """Split count that fills a GPU of `sms` SMs once: the fast decode kernel keeps two CTAs
-    per SM, one CTA per (split, kv head, sequence)."""
-    return max(1, min(1024, (2 * sms) // max(1, batch * kv_heads)))
+def splits_for(batch: int, kv_heads: int, sms: int, rows: int = 1, max_len: Optional[int] = None) -> int:
+    """Split count that fills a GPU of `sms` SMs once: the tensor-core decode kernel keeps two
+    CTAs per SM, one CTA per (split, kv head, sequence, run of query rows); a KV head's
+    rows = G * seq_q query rows are taken four at a time, or eight when there are more than
+    four.  With max_len, no more splits than 128-token units of the longest sequence."""
+    runs = -(-max(1, rows) // (8 if rows > 4 else 4))
+    n = (2 * sms) // max(1, batch * kv_heads * runs)
+    if max_len is not None:
+        n = min(n, -(-max(1, max_len) // 128))
+    return max(1, min(1024, n))
 
 
-def default_splits(batch: int, kv_heads: int, device=None) -> int:
+def default_splits(batch: int, kv_heads: int, device=None, rows: int = 1, max_len: Optional[int] = None) -> int:
     """splits_for on the current (or given) GPU."""
     sms = torch.cuda.get_device_properties(device if device is not None else 0).multi_processor_count
-    return splits_for(batch, kv_heads, sms)
+    return splits_for(batch, kv_heads, sms, rows, max_len)
 
 
 class PagedKV:

@@ -285,3 +285,15 @@ def test_compress_binding_rejects_mismatched_k_and_v(tq):
     for v in (torch.zeros((1, 2, 9, 128), dtype=torch.float16), torch.zeros((1, 2, 8, 128), dtype=torch.float32)):
         with pytest.raises(ValueError, match="same shape and dtype"):
             tq.compress_kv(cfg, params, cache, 0, k, v, None, None, stream=0)
+
+
+def test_default_split_count():
+    # one wave of two thread blocks per SM over (split, kv head, sequence, run of query rows)
+    from compressed_decode_attention_tq_b200.runtime import splits_for
+    assert splits_for(1, 8, 148) == 37                    # 4 query rows per KV head: one run
+    assert splits_for(1, 8, 148, rows=4) == 37
+    assert splits_for(1, 8, 148, rows=32) == 9            # 32 rows: four runs of eight
+    assert splits_for(16, 2, 148, rows=8) == 9            # eight rows: one run
+    assert splits_for(1, 1, 148, max_len=4096) == 32      # no more splits than 128-token units
+    assert splits_for(64, 64, 148) == 1
+    assert splits_for(1, 1, 100000) == 1024

@@ -20,9 +20,9 @@ from parity_util import CompressReport, close, compare_compress_rows, record
 
 pytestmark = pytest.mark.gpu
 
-# the benchmark decodes its workload (configuration 2) with the library's default split
-# count for the GPU; the other configurations use their own
-BENCH_DEFAULT_SPLITS = {2}
+# the benchmark decodes with the library's default split count for the GPU, except the
+# long-context configuration, which fixes 64 splits per head
+BENCH_DEFAULT_SPLITS = {1, 2, 3, 5}
 
 
 def _pages_of(kv, layer, phys, head):
@@ -62,7 +62,8 @@ def full(request):
     kv.compress(0, K, V, seq)
     kv.raise_on_error("compress")
     from compressed_decode_attention_tq_b200.runtime import default_splits
-    ns = default_splits(w.batch, w.kv_heads) if c in BENCH_DEFAULT_SPLITS else w.n_splits
+    ns = (default_splits(w.batch, w.kv_heads, rows=w.group * w.seq_q, max_len=w.max_len)
+          if c in BENCH_DEFAULT_SPLITS else w.n_splits)
     out = kv.decode(0, q, seq, ns)
     kv.raise_on_error("decode")
     ck, kb = ocb.codebook_f32(w.key_bits, 128)
