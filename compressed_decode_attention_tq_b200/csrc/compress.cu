@@ -21,7 +21,7 @@ namespace tqk {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kTokPerBlock = 64;
+constexpr int kTokPerBlockMax = 64;  // tokens per thread block (fewer when the grid would not fill the GPU)
 constexpr int kPad = D + 1;  // padded row stride of S / Pi in shared memory (bank-conflict free)
 
 struct SmemCompress {
@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
   float* stage = sm.stage[warp];
   uint32_t* wbuf = sm.words[warp];
   const float* pis = a.dense ? pi_s : nullptr;
-  for (int tt = warp; tt < kTokPerBlock; tt += kWarps) {
-    const int t = blockIdx.x * kTokPerBlock + tt;
+  for (int tt = warp; tt < a.tok_per_block; tt += kWarps) {
+    const int t = blockIdx.x * a.tok_per_block + tt;
     if (t >= len) break;
     const int phys = a.cache.block_table[(size_t)b * a.cache.max_pages + t / PT];
     if (phys < 0 || phys >= a.cache.num_pages) {
@@ -358,18 +358,28 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t stream) {
     if (e != cudaErrorInvalidValue) return e;  // otherwise fall through to the CUDA-core kernel
   }
   const size_t smem = compress_smem_bytes(a.qjl || a.cache.L.vqjl, a.dense);
-  dim3 grid((a.max_len + kTokPerBlock - 1) / kTokPerBlock, a.cache.kv_heads, a.cache.batch);
+  // tokens per thread block: 64, or fewer (a multiple of the warp count, at least one token
+  // per warp) so that a small input still spreads over about two thread blocks per SM
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long heads = (long long)a.cache.kv_heads * a.cache.batch;
+  long long tpb = heads > 0 ? ((long long)a.max_len * heads + 2LL * sms - 1) / (2LL * sms) : kTokPerBlockMax;
+  tpb = ((tpb + kWarps - 1) / kWarps) * kWarps;
+  CompressArgs b = a;
+  b.tok_per_block = (int)(tpb < kWarps ? kWarps : (tpb > kTokPerBlockMax ? kTokPerBlockMax : tpb));
+  dim3 grid((a.max_len + b.tok_per_block - 1) / b.tok_per_block, a.cache.kv_heads, a.cache.batch);
   if (grid.x == 0) return cudaSuccess;
   if (a.in_dtype == TQ_F16) {
     auto k = compress_kernel<__half>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kWarps * 32, smem, stream>>>(a);
+    k<<<grid, kWarps * 32, smem, stream>>>(b);
   } else {
     auto k = compress_kernel<float>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kWarps * 32, smem, stream>>>(a);
+    k<<<grid, kWarps * 32, smem, stream>>>(b);
   }
   return cudaGetLastError();
 }

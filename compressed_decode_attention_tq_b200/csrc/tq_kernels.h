@@ -14,6 +14,7 @@ struct CompressArgs {
   const void* v;
   int in_dtype, max_len, qjl, dense;
   int key_corr;                  // keys store the corrected norm ||k|| / ||y_hat||
+  int tok_per_block;             // CUDA-core compress: tokens per thread block (set at launch)
   const float *k_off, *v_off;    // dithered: the offsets [batch][kv_heads][max_len], else null
   const int32_t* seq_lens;
   const float *signs, *pi, *s, *k_centroids, *k_boundaries, *v_centroids, *v_boundaries;
