@@ -27,7 +27,10 @@
 // (sign-magnitude nibbles, the signs applied by byte masks), values 3-bit or 2-bit, any R;
 // the randomized Hadamard rotation or a dense Pi (R^T applied in the merge); dithered codes
 // (DT: a key's offset adds xi_k sum_i (R q)_i to its dot product, a value's adds xi_v to
-// every coordinate, carried as one running sum per row next to the accumulator).
+// every coordinate, carried as one running sum per row next to the accumulator); values
+// with QJL for up to four rows (VQ: the value product's four spare columns accumulate the
+// sign-space sums sum_t p_t ||r_v||_t (2 sigma_t - 1) through a second mma per step, and the
+// merge adds sqrt(pi/2)/m S^T of them).
 // Everything else uses decode.cu.
 #include <cuda_fp16.h>
 #include <math_constants.h>
@@ -45,9 +48,9 @@ constexpr int kStages = 3;
 constexpr int kUnit = PT / 2;                  // tokens per copy unit: half a page
 constexpr int kUnitsPerPage = PT / kUnit;
 constexpr int kChunkStride = kUnit * 16 + 32;  // padded so the 4 lanes of a token group hit distinct banks
-constexpr int kNormBytes = 5 * kUnit * 2;      // KN | KR | VN | KD | VD of the unit
+constexpr int kNormBytes = 6 * kUnit * 2;      // KN | KR | VN | KD | VD | VR of the unit
 constexpr int kMaxKChunks = 4;
-constexpr int kMaxVChunks = 3;
+constexpr int kMaxVChunks = 4;  // 3-bit values: 2 crumb chunks + the sign plane; + VS
 constexpr int kStageBytes = kNormBytes + (kMaxKChunks + kMaxVChunks) * kChunkStride;
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // every mbarrier wait gives up after 1 s
 constexpr float kLog2e = 1.4426950408889634f;
@@ -67,6 +70,7 @@ struct SmemFast {
     struct {
       unsigned char stage[kStages][kStageBytes];
       float wacc[kConsumerWarps][kMaxRows][D];
+      float wsig[kConsumerWarps][4][QM];  // values with QJL: the sign-space sums of each warp
     } ring;
     // at the end: the partial accumulators of every split of the (sequence, kv head) being
     // merged, [row][split][D] (the ring and the warp partials are no longer used then)
@@ -78,6 +82,7 @@ struct SmemFast {
   unsigned long long never;  // completed by nothing: the target of the bounded-wait test
   float wm[kConsumerWarps][kMaxRows], wl[kConsumerWarps][kMaxRows], wf[kConsumerWarps][kMaxRows];
   float wx[kConsumerWarps][kMaxRows];  // dithered values: sum_t p_t ||v_t|| xi_t of each warp and row
+  float xsig[4][QM];  // values with QJL, at the merge: each row's sign-space sum / l
   int last;
 };
 
@@ -232,8 +237,9 @@ __device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int
   return (t1 & 0x3u) | ((t2 & 0x3u) << 4) | (t1 & 0x300u) | ((t2 & 0x300u) << 4);
 }
 
-template <int KP, int VP, int NR, bool DT>
+template <int KP, int VP, int NR, bool DT, bool VQ>
 __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
+  static_assert(!VQ || (NR == 4 && !DT), "values with QJL: four rows, not dithered");
   static_assert(NR == 4 || NR == 8, "four or eight rows per CTA");
   constexpr int NT = NR / 4;  // n-tiles of the key and QJL products
   // the next kernel on the stream may be scheduled now; a programmatic dependent waits for
@@ -266,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   constexpr int kVChunks = (VP == V3) ? 3 : 2;
   constexpr bool kQjl = KP != K4;
   // without QJL there is no KR region: its norm slots stay unused
-  const uint32_t unit_bytes =
-      2u * kUnit * (2 + (kQjl ? 1 : 0) + (DT ? 2 : 0)) + 16u * kUnit * (kKChunks + kVChunks);
+  const uint32_t unit_bytes = 2u * kUnit * (2 + (kQjl ? 1 : 0) + (DT ? 2 : 0) + (VQ ? 1 : 0)) +
+                              16u * kUnit * (kKChunks + kVChunks + (VQ ? 1 : 0));
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -325,6 +331,10 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         unsigned char* vc = kc + kMaxKChunks * kChunkStride;
         for (int c = 0; c < kVChunks; ++c)
           bulk_g2s(vc + c * kChunkStride, blk + L.vc + c * PT * 16 + hb16, kUnit * 16, &sm.full[s]);
+        if (VQ) {
+          bulk_g2s(st + kUnit * 10, blk + L.vr + hb2, kUnit * 2, &sm.full[s]);
+          bulk_g2s(vc + kVChunks * kChunkStride, blk + L.vs + hb16, kUnit * 16, &sm.full[s]);
+        }
       }
       // the last copy into each stage has landed (consumers that gave up early did not wait
       // for it) before the ring's space is reused or released; bounded
@@ -802,7 +812,20 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
               x2 = y2;
             }
           }
-          const uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
+          uint32_t b0 = prmt(x1, x2, 0x5410), b1 = prmt(x1, x2, 0x7632);
+          uint32_t b0r = 0, b1r = 0;
+          if (VQ) {
+            // the value product keeps columns 0..3 (rows); columns 4..7 take the sign-space
+            // weights p_t ||r_v||_t of rows 0..3 in a second mma
+            const float rvA = ld_h(st + 10 * kUnit + 2 * ta), rvB = ld_h(st + 10 * kUnit + 2 * tb);
+            const uint32_t pr2 = pack_h2(ta < valid ? p[u][0][0] * rvA : 0.f, tb < valid ? p[u][0][1] * rvB : 0.f);
+            const uint32_t r1 = __shfl_sync(FULL, pr2, src1), r2 = __shfl_sync(FULL, pr2, src2);
+            if (g >= 4) {
+              b0r = prmt(r1, r2, 0x5410);
+              b1r = prmt(r1, r2, 0x7632);
+              b0 = b1 = 0u;
+            }
+          }
             // ---- values: dequantise (pairs of coordinates of one token), transpose, mma
             uint32_t va[16], vb[16];
             {
@@ -828,6 +851,25 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             }
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt) hmma(acc[mt], va[2 * mt], va[2 * mt + 1], vb[2 * mt], vb[2 * mt + 1], b0, b1);
+          if (VQ) {
+            // the signs as fp16 +-1 for the same coordinate pairs, transposed like the values
+            const unsigned char* vsq = vc + kVChunks * kChunkStride;
+            const uint32_t wA = ~*reinterpret_cast<const uint32_t*>(vsq + ta * 16 + 4 * t4);
+            const uint32_t wB = ~*reinterpret_cast<const uint32_t*>(vsq + tb * 16 + 4 * t4);
+            uint32_t qa[16], qb[16];
+#pragma unroll
+            for (int cb = 0; cb < 16; ++cb) {
+              const int pb = pair_base(cb);
+              // bits pb and pb + 4 (a clear sigma means -1) to the two halves' sign bits
+              const uint32_t xa = (((wA >> pb) & 0x11u) * 0x08008000u & 0x80008000u) | 0x3C003C00u;
+              const uint32_t xb = (((wB >> pb) & 0x11u) * 0x08008000u & 0x80008000u) | 0x3C003C00u;
+              qa[cb] = movm_t(xa);
+              qb[cb] = movm_t(xb);
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+              hmma(acc[mt], qa[2 * mt], qa[2 * mt + 1], qb[2 * mt], qb[2 * mt + 1], b0r, b1r);
+          }
         }
       }
       __syncwarp();
@@ -858,7 +900,11 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         const int row = 2 * t4 + (e & 1);
         const int cb = 2 * mt + (e >> 1);
         const int coord = 32 * (g >> 1) + pair_base(cb) + 4 * (g & 1);
-        if (row < R) sm.ring.wacc[warp][row][coord] = acc[mt][e];
+        if (VQ && row >= 4) {
+          if (row - 4 < R) sm.ring.wsig[warp][row - 4][coord] = acc[mt][e];
+        } else if (row < R) {
+          sm.ring.wacc[warp][row][coord] = acc[mt][e];
+        }
       }
     }
   }
@@ -889,6 +935,12 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     for (int w = 0; w < kConsumerWarps; ++w)
       o = fmaf(sm.wf[w][r], DT ? sm.ring.wacc[w][r][j] + sm.wx[w][r] : sm.ring.wacc[w][r][j], o);
     a.part_acc[((row0 + r) * a.n_splits + split) * D + j] = o;
+    if (VQ) {
+      float os = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) os = fmaf(sm.wf[w][r], sm.ring.wsig[w][r][j], os);
+      a.part_sig[((row0 + r) * a.n_splits + split) * QM + j] = os;
+    }
   }
   // ---- the last split of this (sequence, kv head) to finish merges all of them ----
   __syncthreads();
@@ -927,6 +979,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     float* rs = &sm.merge[r * kCap * D];  // row r's region (its partials when in_smem)
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 osg = make_float4(0.f, 0.f, 0.f, 0.f);  // values with QJL: the sign-space sums
+    const float4* ps4 = reinterpret_cast<const float4*>(a.part_sig + (VQ ? rowq * ns * QM : 0)) + c4;
     if (in_smem) {
       for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
 #pragma unroll
@@ -947,6 +1001,13 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         o.y = fmaf(wgt, v.y, o.y);
         o.z = fmaf(wgt, v.z, o.z);
         o.w = fmaf(wgt, v.w, o.w);
+        if (VQ) {
+          const float4 q = ps4[sp * (QM / 4)];
+          osg.x = fmaf(wgt, q.x, osg.x);
+          osg.y = fmaf(wgt, q.y, osg.y);
+          osg.z = fmaf(wgt, q.z, osg.z);
+          osg.w = fmaf(wgt, q.w, osg.w);
+        }
       }
     } else {
       // many splits: the partials in register batches of kMB, the first batch before the
@@ -978,12 +1039,39 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             o.y = fmaf(wgt, v[k].y, o.y);
             o.z = fmaf(wgt, v[k].z, o.z);
             o.w = fmaf(wgt, v[k].w, o.w);
+            if (VQ) {
+              const float4 q = ps4[(size_t)(s0 + k) * (QM / 4)];
+              osg.x = fmaf(wgt, q.x, osg.x);
+              osg.y = fmaf(wgt, q.y, osg.y);
+              osg.z = fmaf(wgt, q.z, osg.z);
+              osg.w = fmaf(wgt, q.w, osg.w);
+            }
           }
         }
       }
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
     float x[4] = {o.x * inv, o.y * inv, o.z * inv, o.w * inv};
+    // values with QJL: + sqrt(pi/2)/m S^T (sign-space sums / l), lane c4 forming outputs
+    // 4 c4 .. 4 c4 + 3 from rows of S (coalesced across c4)
+    float sg[4] = {0.f, 0.f, 0.f, 0.f};
+    if (VQ) {
+      float* xs = sm.xsig[r];
+      *reinterpret_cast<float4*>(xs + 4 * c4) = make_float4(osg.x * inv, osg.y * inv, osg.z * inv, osg.w * inv);
+      __syncwarp();
+      const float4* s4 = reinterpret_cast<const float4*>(a.s) + c4;
+#pragma unroll 8
+      for (int i = 0; i < QM; ++i) {
+        const float4 p = s4[(size_t)i * (D / 4)];
+        const float xi = xs[i];
+        sg[0] = fmaf(p.x, xi, sg[0]);
+        sg[1] = fmaf(p.y, xi, sg[1]);
+        sg[2] = fmaf(p.z, xi, sg[2]);
+        sg[3] = fmaf(p.w, xi, sg[3]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sg[e] *= kQjlScale;
+    }
     if (a.dense) {
       // out = Pi^T (o / l): the row's 128 values through its own region of shared memory
       // (every lane of this warp is past reading it), then lane c4 forms outputs
@@ -1002,7 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         y.z = fmaf(p.z, xi, y.z);
         y.w = fmaf(p.w, xi, y.w);
       }
-      *reinterpret_cast<float4*>(a.out + rowq * D + 4 * c4) = y;
+      *reinterpret_cast<float4*>(a.out + rowq * D + 4 * c4) = make_float4(y.x + sg[0], y.y + sg[1], y.z + sg[2], y.w + sg[3]);
       continue;
     }
     // out = D H (o / l) / sqrt(d): H over coordinates 4 c4 + e, spans 1 and 2 in the
@@ -1023,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       }
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) a.out[rowq * D + 4 * c4 + e] = x[e] * kInvSqrtD * a.signs[4 * c4 + e];
+    for (int e = 0; e < 4; ++e) a.out[rowq * D + 4 * c4 + e] = fmaf(x[e] * kInvSqrtD, a.signs[4 * c4 + e], sg[e]);
   }
 }
 
@@ -1034,7 +1122,9 @@ bool fast_decode_supported(const DecodeArgs& a) {
   // the merge reads Pi as float4
   if (a.dense && (reinterpret_cast<uintptr_t>(a.pi) & 15)) return false;
   const bool kok = (L.kbits == 3 && L.qjl) || (L.kbits == 2 && L.qjl) || (L.kbits == 4 && !L.qjl);
-  const bool vok = (L.vbits == 3 || L.vbits == 2) && !L.vqjl;
+  // values with QJL: up to four query rows per KV head, not dithered, S read as float4
+  const bool vqok = !L.vqjl || (a.rows <= 4 && !L.dither && !(reinterpret_cast<uintptr_t>(a.s) & 15));
+  const bool vok = (L.vbits == 3 || L.vbits == 2) && vqok;
   return kok && vok;
 }
 
@@ -1047,12 +1137,14 @@ cudaError_t launch_fast_split(const DecodeArgs& a, cudaStream_t stream) {
   const int nr = a.rows > 4 ? 8 : 4;
   dim3 grid(a.n_splits, a.cache.kv_heads, a.cache.batch * ((a.rows + nr - 1) / nr));
   void (*k)(DecodeArgs) = nullptr;
-#define TQ_FAST(KB, KPOL, VB, VPOL)                                                         \
-  if (L.kbits == KB && L.vbits == VB) {                                                      \
-    if (L.dither)                                                                            \
-      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, true> : fast_split_kernel<KPOL, VPOL, 4, true>;   \
-    else                                                                                     \
-      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, false> : fast_split_kernel<KPOL, VPOL, 4, false>; \
+#define TQ_FAST(KB, KPOL, VB, VPOL)                                                                   \
+  if (L.kbits == KB && L.vbits == VB) {                                                                \
+    if (L.vqjl)                                                                                        \
+      k = fast_split_kernel<KPOL, VPOL, 4, false, true>;                                               \
+    else if (L.dither)                                                                                 \
+      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, true, false> : fast_split_kernel<KPOL, VPOL, 4, true, false>; \
+    else                                                                                               \
+      k = nr == 8 ? fast_split_kernel<KPOL, VPOL, 8, false, false> : fast_split_kernel<KPOL, VPOL, 4, false, false>; \
   }
   TQ_FAST(3, K3Q, 3, V3)
   TQ_FAST(3, K3Q, 2, V2)
