@@ -231,6 +231,16 @@ __device__ __forceinline__ uint32_t crumb_sel(uint32_t c0, uint32_t c1, int cb) 
   return crumb_t(c0, c1, cb) * 0x11u + 0x4040u;
 }
 
+// The selectors of crumb pairs cb = 8 h + k and 8 h + 4 + k (k < 4) at once, from crumb word
+// w = c0 (h = 0) or c1 (h = 1): one mask keeps both pairs' fields (bits 2k, 2k + 8 and
+// 2k + 16, 2k + 24), one multiply-add turns both into selectors (the low one's product stays
+// below bit 16), and the high one is shifted down.
+__device__ __forceinline__ void crumb_sel2(uint32_t w, int k, uint32_t& lo, uint32_t& hi) {
+  const uint32_t f = ((w >> (2 * k)) & 0x03030303u) * 0x11u + 0x40404040u;
+  lo = f;
+  hi = f >> 16;
+}
+
 // Selector of the int8 residual codes of crumb pairs n and n+1: bytes (a_n, a_n+1, b_n, b_n+1).
 __device__ __forceinline__ uint32_t crumb_pair_sel(uint32_t c0, uint32_t c1, int n) {
   const uint32_t t1 = crumb_t(c0, c1, n), t2 = crumb_t(c0, c1, n + 1);
@@ -670,9 +680,15 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
               const uint32_t sA = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + ta * 16 + 4 * t4);
               const uint32_t sB = *reinterpret_cast<const uint32_t*>(kc + 2 * kChunkStride + tb * 16 + 4 * t4);
     #pragma unroll
-              for (int n = 0; n < 16; ++n) {
-                ha[n] = prmt(kt_lo0, kt_hi0, crumb_sel(ca.x, ca.y, n));
-                hb[n] = prmt(kt_lo0, kt_hi0, crumb_sel(cbv.x, cbv.y, n));
+              for (int hk = 0; hk < 8; ++hk) {
+                const int h = hk >> 2, k = hk & 3;
+                uint32_t sla, sha, slb, shb;
+                crumb_sel2(h ? ca.y : ca.x, k, sla, sha);
+                crumb_sel2(h ? cbv.y : cbv.x, k, slb, shb);
+                ha[8 * h + k] = prmt(kt_lo0, kt_hi0, sla);
+                ha[8 * h + 4 + k] = prmt(kt_lo0, kt_hi0, sha);
+                hb[8 * h + k] = prmt(kt_lo0, kt_hi0, slb);
+                hb[8 * h + 4 + k] = prmt(kt_lo0, kt_hi0, shb);
               }
     #pragma unroll
               for (int n = 0; n < 16; n += 2) {
@@ -838,15 +854,23 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
                 sgB = *reinterpret_cast<const uint32_t*>(vc + 2 * kChunkStride + tb * 16 + 4 * t4);
               }
     #pragma unroll
-              for (int cb = 0; cb < 16; ++cb) {
-                uint32_t xa = prmt(vt_lo, vt_hi, crumb_sel(ca.x, ca.y, cb));
-                uint32_t xb = prmt(vt_lo, vt_hi, crumb_sel(cbv.x, cbv.y, cb));
-                if (VP == V3) {
-                  xa ^= (sgA << (15 - cb)) & 0x80008000u;
-                  xb ^= (sgB << (15 - cb)) & 0x80008000u;
+              for (int hk = 0; hk < 8; ++hk) {
+                const int h = hk >> 2, k = hk & 3;
+                uint32_t sa[2], sb[2];
+                crumb_sel2(h ? ca.y : ca.x, k, sa[0], sa[1]);
+                crumb_sel2(h ? cbv.y : cbv.x, k, sb[0], sb[1]);
+    #pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  const int cb = 8 * h + 4 * q + k;
+                  uint32_t xa = prmt(vt_lo, vt_hi, sa[q]);
+                  uint32_t xb = prmt(vt_lo, vt_hi, sb[q]);
+                  if (VP == V3) {
+                    xa ^= (sgA << (15 - cb)) & 0x80008000u;
+                    xb ^= (sgB << (15 - cb)) & 0x80008000u;
+                  }
+                  va[cb] = movm_t(xa);
+                  vb[cb] = movm_t(xb);
                 }
-                va[cb] = movm_t(xa);
-                vb[cb] = movm_t(xb);
               }
             }
 #pragma unroll
