@@ -735,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             const float nA = ld_h(st + 2 * ta), nB = ld_h(st + 2 * tb);
             const float rA = kQjl ? ld_h(st + 2 * kUnit + 2 * ta) : 0.f;
             const float rB = kQjl ? ld_h(st + 2 * kUnit + 2 * tb) : 0.f;
-            const int s1a = -(dsum[0] + 256 * dsum[1]) / 128, s1b = -(dsum[2] + 256 * dsum[3]) / 128;
+            // every product of the QJL mma is -128 sigma d: the sums are exact multiples of 128
+            const int s1a = -((dsum[0] + 256 * dsum[1]) >> 7), s1b = -((dsum[2] + 256 * dsum[3]) >> 7);
             float dotA = dk[0] + dk[1] + (float)dcor[0] * corr_down[nt];
             float dotB = dk[2] + dk[3] + (float)dcor[2] * corr_down[nt];
             if (DT) {

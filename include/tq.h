@@ -127,13 +127,12 @@ typedef struct tq_config {
   int32_t value_qjl;    /* 1: values carry the 1-bit QJL sketch of their residual and
                            ||r_v|| (TurboQuant_prod on the value cache, [MOBILINT]
                            "Two-Stage Approach": the value is reconstructed as
-                           v_mse + sqrt(pi/2)/m ||r_v|| S^T (2 sigma_v - 1)); served by
-                           the general (CUDA-core) kernels                             */
+                           v_mse + sqrt(pi/2)/m ||r_v|| S^T (2 sigma_v - 1))        */
   int32_t dither;       /* 1: dithered HD ([DITHER]): every key and value is coded as
                            Quant(y - xi) with its own offset xi, stored in KD / VD and added
                            back at reconstruction; needs TQ_ROT_HADAMARD and the uniform
                            grids of tq_dither_codebook; compressed by
-                           tq_compress_kv_dithered; served by the general kernels     */
+                           tq_compress_kv_dithered                                    */
   int32_t key_corrected_norm; /* 1: keys store the corrected norm ([TQKV]
                            compress_single_key returns "corrected_norm"): ||k|| / ||y_hat||
                            with y_hat = c[idx] (+ xi), so that the reconstruction has the
@@ -304,8 +303,8 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int
  *   out        device float [batch][q_heads][seq_q][d]
  * A test of the device's bounded waits: with the environment variable
  * TQ_DEBUG_BOUNDED_WAIT_US set to n (1..1000000) when the call is made, one warp of the
- * tensor-core split kernel (keys 2- or 3-bit with QJL, values 2- or 3-bit, Hadamard
- * rotation) waits n microseconds on a barrier that nothing completes and writes
+ * tensor-core split kernel (keys 2- or 3-bit with QJL or 4-bit without, values 2- or
+ * 3-bit) waits n microseconds on a barrier that nothing completes and writes
  * TQ_ERR_TIMEOUT to dev_status; the results are computed as usual. */
 TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                            int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
