@@ -33,7 +33,7 @@ EXPORTS = ("tq_version", "tq_status_str", "tq_last_error", "tq_check", "tq_valid
            "tq_codebook", "tq_compress_kv", "tq_decode_workspace_bytes", "tq_attend_decode",
            "tq_decode_scores", "tq_decompress", "tq_attend_decode_noalloc", "tq_operand_bytes",
            "tq_prepare_operands", "tq_append_kv", "tq_append_attend_decode", "tq_dither_codebook",
-           "tq_compress_kv_dithered")
+           "tq_compress_kv_dithered", "tq_append_kv_dithered", "tq_append_attend_decode_dithered")
 
 
 class tq_config(ctypes.Structure):
@@ -91,6 +91,9 @@ def _load() -> ctypes.CDLL:
         "tq_append_kv": (I32, [cfgp, parp, cachep, I32, P, P, I32, I32, P, P, P]),
         "tq_append_attend_decode": (I32, [cfgp, parp, cachep, I32, P, P, I32, I32, P, I32, I32, I32, P, I32,
                                           P, SZ, P, P, P]),
+        "tq_append_kv_dithered": (I32, [cfgp, parp, cachep, I32, P, P, P, P, I32, I32, P, P, P]),
+        "tq_append_attend_decode_dithered": (I32, [cfgp, parp, cachep, I32, P, P, P, P, I32, I32, P, I32, I32,
+                                                   I32, P, I32, P, SZ, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -255,6 +258,41 @@ def append_kv(cfg, params, cache, layer, k_new, v_new, seq_lens, status, stream=
     _check(lib.tq_append_kv(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
                             _ptr(k_new), _ptr(v_new), dtype_code(k_new), k_new.shape[2], _ptr(seq_lens),
                             _ptr(status), _stream(stream)), "tq_append_kv")
+
+
+def _check_offsets(k_offsets, v_offsets, shape):
+    import torch
+    for o in (k_offsets, v_offsets):
+        if tuple(o.shape) != tuple(shape) or o.dtype != torch.float32 or not o.is_contiguous():
+            raise ValueError("offsets must be contiguous float32 [batch][kv_heads][n]")
+
+
+def append_kv_dithered(cfg, params, cache, layer, k_new, v_new, k_offsets, v_offsets, seq_lens, status,
+                       stream=None):
+    """append_kv for a dithered configuration; k_offsets, v_offsets: device float32
+    [batch][kv_heads][n_new], the new tokens' offsets."""
+    if v_new.shape != k_new.shape or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    _check_offsets(k_offsets, v_offsets, k_new.shape[:3])
+    _check(lib.tq_append_kv_dithered(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache), layer,
+                                     _ptr(k_new), _ptr(v_new), _ptr(k_offsets), _ptr(v_offsets),
+                                     dtype_code(k_new), k_new.shape[2], _ptr(seq_lens), _ptr(status),
+                                     _stream(stream)), "tq_append_kv_dithered")
+
+
+def append_attend_decode_dithered(cfg, params, cache, layer, k_new, v_new, k_offsets, v_offsets, q, seq_lens,
+                                  n_splits, workspace, out, status, stream=None):
+    """append_attend_decode for a dithered configuration (offsets as for append_kv_dithered)."""
+    if v_new.shape != k_new.shape or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    _check_offsets(k_offsets, v_offsets, k_new.shape[:3])
+    _check(lib.tq_append_attend_decode_dithered(ctypes.byref(cfg), ctypes.byref(params), ctypes.byref(cache),
+                                                layer, _ptr(k_new), _ptr(v_new), _ptr(k_offsets),
+                                                _ptr(v_offsets), dtype_code(k_new), k_new.shape[2], _ptr(q),
+                                                dtype_code(q), q.shape[1], q.shape[2], _ptr(seq_lens), n_splits,
+                                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                _ptr(out), _ptr(status), _stream(stream)),
+           "tq_append_attend_decode_dithered")
 
 
 def append_attend_decode(cfg, params, cache, layer, k_new, v_new, q, seq_lens, n_splits, workspace,

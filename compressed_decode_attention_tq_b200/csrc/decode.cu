@@ -122,21 +122,23 @@ __device__ __forceinline__ void pack_code(int s, int r, int bits, int lane, int 
 }
 
 // Encodes thread i's coordinate of one vector: stored norm, index, (s, r); returns y.
-// cent non-null: store the corrected norm n / ||c[idx]|| ("tq-kv" documentation:
+// xi: the vector's dither offset (0 when not dithered): idx = Quant(y - xi).  cent
+// non-null: store the corrected norm n / ||c[idx] + xi|| ("tq-kv" documentation:
 // corrected_norm) instead of n.
 __device__ __forceinline__ float encode_coord(const DecodeArgs& a, AppendShared& sh, float x, const float* bnd,
                                               int bits, int i, int lane, int warp, __half& nh, int& idx,
-                                              int& s, int& r, const float* cent = nullptr) {
+                                              int& s, int& r, const float* cent = nullptr, float xi = 0.f) {
   const float n = sqrtf(block_sum128(x * x, sh.red, lane, warp));
   const float y = rotate_coord(a, sh, x, n > 0.f ? 1.0f / n : 0.0f, i, lane, warp);
   const int nb = (1 << bits) - 1, h = 1 << (bits - 1);
+  const float yq = y - xi;
   idx = 0;
-  for (int k = 0; k < nb; ++k) idx += (y > bnd[k]) ? 1 : 0;
+  for (int k = 0; k < nb; ++k) idx += (yq > bnd[k]) ? 1 : 0;
   s = idx >= h;
   r = s ? idx - h : h - 1 - idx;
   float stored = n;
   if (cent) {
-    const float c = cent[idx];
+    const float c = cent[idx] + xi;
     const float yn = sqrtf(block_sum128(c * c, sh.red, lane, warp));
     stored = yn > 0.f ? n / yn : 0.f;
   }
@@ -223,6 +225,17 @@ __device__ void append_token(const DecodeArgs& a, int job) {
   uint8_t* blk = a.cache.block(phys, h);
   const int slot = pos % PT;
   const size_t src = (size_t)job * D + i;
+  // dithered: the token's offsets, used and stored as fp16
+  __half kxi16 = __float2half_rn(0.f), vxi16 = kxi16;
+  if (L.dither) {
+    kxi16 = __float2half_rn(a.k_new_off[job]);
+    vxi16 = __float2half_rn(a.v_new_off[job]);
+    if (i == 0) {
+      reinterpret_cast<__half*>(blk + L.kd)[slot] = kxi16;
+      reinterpret_cast<__half*>(blk + L.vd)[slot] = vxi16;
+    }
+  }
+  const float kxi = __half2float(kxi16), vxi = __half2float(vxi16);
   __syncthreads();
 
   // ---- key: norm, rotation, quantisation
@@ -230,11 +243,11 @@ __device__ void append_token(const DecodeArgs& a, int job) {
                                         : ld_new<float>(a.k_new, src);
   __half nh;
   int idx, s, r;
-  encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r, a.key_corr ? sh.tab[0] : nullptr);
+  encode_coord(a, sh, x, sh.tab[1], L.kbits, i, lane, warp, nh, idx, s, r, a.key_corr ? sh.tab[0] : nullptr, kxi);
   if (!L.kmerged) pack_code(s, r, L.kbits, lane, warp, sh.kw);
   if (a.qjl) {
     int sigma;
-    const __half rho = append_qjl(a, sh, x, nh, sh.tab[0][idx], i, lane, warp, sigma);
+    const __half rho = append_qjl(a, sh, x, nh, sh.tab[0][idx] + kxi, i, lane, warp, sigma);
     if (L.kmerged) {
       pack_code(s, r | (s << 2) | (sigma << 3), kMergedNibble, lane, warp, sh.kw);
     } else {
@@ -254,12 +267,12 @@ __device__ void append_token(const DecodeArgs& a, int job) {
   const float xv = a.new_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.v_new)[src])
                                          : ld_new<float>(a.v_new, src);
   __half nv16;
-  encode_coord(a, sh, xv, sh.tab[3], L.vbits, i, lane, warp, nv16, idx, s, r);
+  encode_coord(a, sh, xv, sh.tab[3], L.vbits, i, lane, warp, nv16, idx, s, r, nullptr, vxi);
   pack_code(s, r, L.vbits, lane, warp, sh.vw);
   if (L.vqjl) {
     // values with QJL: the same sketch of the value residual, signs in VS, norm in VR
     int sigma;
-    const __half rho = append_qjl(a, sh, xv, nv16, sh.tab[2][idx], i, lane, warp, sigma);
+    const __half rho = append_qjl(a, sh, xv, nv16, sh.tab[2][idx] + vxi, i, lane, warp, sigma);
     const uint32_t bw = __ballot_sync(FULL, sigma);
     if (lane == 0) sh.vsw[warp] = bw;
     if (i == 0) reinterpret_cast<__half*>(blk + L.vr)[slot] = rho;

@@ -311,14 +311,20 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.n_new = 0;
   a.k_boundaries = params->k_boundaries;
   a.v_boundaries = params->v_boundaries;
+  a.k_new_off = nullptr;
+  a.v_new_off = nullptr;
   a.debug_wait_ns = debug_wait_ns();
   return TQ_OK;
 }
 
 // Checks of the appended tokens' arguments shared by tq_append_kv and tq_append_attend_decode.
 static tq_status check_append(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
-                              const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new) {
-  if (cfg->dither) return fail(TQ_ERR_UNSUPPORTED, "appends take no dither offsets");
+                              const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new,
+                              const float* k_off, const float* v_off, bool dithered_call) {
+  if (cfg->dither && !dithered_call)
+    return fail(TQ_ERR_UNSUPPORTED, "a dithered configuration appends with the _dithered calls (offsets)");
+  if (dithered_call && !cfg->dither) return fail(TQ_ERR_INVALID_ARG, "the _dithered appends need cfg->dither = 1");
+  if (dithered_call && (!k_off || !v_off)) return fail(TQ_ERR_INVALID_ARG, "k_offsets or v_offsets is NULL");
   if (!params->k_boundaries || !params->v_boundaries) return fail(TQ_ERR_INVALID_ARG, "boundary pointer is NULL");
   if (!k_new || !v_new) return fail(TQ_ERR_INVALID_ARG, "k_new or v_new is NULL");
   if (in_dtype != TQ_F16 && in_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "in_dtype must be TQ_F16 or TQ_F32");
@@ -350,24 +356,25 @@ tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params, const 
   return TQ_OK;
 }
 
-tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
-                                  int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
-                                  int32_t n_new, const void* q, int32_t q_dtype, int32_t q_heads,
-                                  int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
-                                  size_t workspace_bytes, float* out, int32_t* dev_status,
-                                  tq_stream_t stream) {
-  CallRange range("tq_append_attend_decode");
-  clear_error();
+static tq_status append_attend_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                      int32_t layer, const void* k_new, const void* v_new, const float* k_off,
+                                      const float* v_off, bool dithered_call, int32_t in_dtype, int32_t n_new,
+                                      const void* q, int32_t q_dtype, int32_t q_heads, int32_t seq_q,
+                                      const int32_t* seq_lens, int32_t n_splits, void* workspace,
+                                      size_t workspace_bytes, float* out, int32_t* dev_status, tq_stream_t stream) {
   tqk::DecodeArgs a;
   tq_status st = decode_common(cfg, params, cache, layer, q, q_dtype, q_heads, seq_q, seq_lens, n_splits,
                                workspace, workspace_bytes, a);
   if (st != TQ_OK) return st;
-  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new)) != TQ_OK) return st;
+  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new, k_off, v_off, dithered_call)) != TQ_OK)
+    return st;
   if (!out) return fail(TQ_ERR_INVALID_ARG, "out is NULL");
   if ((int64_t)cache->batch * q_heads * seq_q + (int64_t)cache->batch * cache->kv_heads * n_new > (int64_t)1 << 30)
     return fail(TQ_ERR_INVALID_ARG, "too many query rows and appended tokens");
   a.k_new = k_new;
   a.v_new = v_new;
+  a.k_new_off = k_off;
+  a.v_new_off = v_off;
   a.new_dtype = in_dtype;
   a.n_new = n_new;
   a.out = out;
@@ -377,17 +384,44 @@ tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params,
   return TQ_OK;
 }
 
-tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
-                       const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new,
-                       const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
-  CallRange range("tq_append_kv");
+tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                  int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
+                                  int32_t n_new, const void* q, int32_t q_dtype, int32_t q_heads,
+                                  int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
+                                  size_t workspace_bytes, float* out, int32_t* dev_status,
+                                  tq_stream_t stream) {
+  CallRange range("tq_append_attend_decode");
   clear_error();
+  return append_attend_common(cfg, params, cache, layer, k_new, v_new, nullptr, nullptr, false, in_dtype, n_new, q,
+                              q_dtype, q_heads, seq_q, seq_lens, n_splits, workspace, workspace_bytes, out,
+                              dev_status, stream);
+}
+
+tq_status tq_append_attend_decode_dithered(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                           int32_t layer, const void* k_new, const void* v_new,
+                                           const float* k_offsets, const float* v_offsets, int32_t in_dtype,
+                                           int32_t n_new, const void* q, int32_t q_dtype, int32_t q_heads,
+                                           int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,
+                                           void* workspace, size_t workspace_bytes, float* out,
+                                           int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_append_attend_decode_dithered");
+  clear_error();
+  return append_attend_common(cfg, params, cache, layer, k_new, v_new, k_offsets, v_offsets, true, in_dtype,
+                              n_new, q, q_dtype, q_heads, seq_q, seq_lens, n_splits, workspace, workspace_bytes,
+                              out, dev_status, stream);
+}
+
+static tq_status append_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
+                               const void* k_new, const void* v_new, const float* k_off, const float* v_off,
+                               bool dithered_call, int32_t in_dtype, int32_t n_new, const int32_t* seq_lens,
+                               int32_t* dev_status, tq_stream_t stream) {
   tq_status st;
   if ((st = check_config(cfg)) != TQ_OK) return st;
   if ((st = check_params(cfg, params, true)) != TQ_OK) return st;
   if ((st = check_cache(cache, layer)) != TQ_OK) return st;
   if (!seq_lens) return fail(TQ_ERR_INVALID_ARG, "seq_lens is NULL");
-  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new)) != TQ_OK) return st;
+  if ((st = check_append(cfg, params, cache, k_new, v_new, in_dtype, n_new, k_off, v_off, dithered_call)) != TQ_OK)
+    return st;
   tqk::DecodeArgs a = {};
   a.cache = cache_ref(cfg, cache, layer);
   a.qjl = cfg->key_qjl;
@@ -403,12 +437,33 @@ tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_c
   a.v_boundaries = params->v_boundaries;
   a.k_new = k_new;
   a.v_new = v_new;
+  a.k_new_off = k_off;
+  a.v_new_off = v_off;
   a.new_dtype = in_dtype;
   a.n_new = n_new;
   a.status = dev_status;
   cudaError_t e = tqk::launch_append(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "tq_append_kv launch");
   return TQ_OK;
+}
+
+tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
+                       const void* k_new, const void* v_new, int32_t in_dtype, int32_t n_new,
+                       const int32_t* seq_lens, int32_t* dev_status, tq_stream_t stream) {
+  CallRange range("tq_append_kv");
+  clear_error();
+  return append_common(cfg, params, cache, layer, k_new, v_new, nullptr, nullptr, false, in_dtype, n_new, seq_lens,
+                       dev_status, stream);
+}
+
+tq_status tq_append_kv_dithered(const tq_config* cfg, const tq_params* params, const tq_cache* cache, int32_t layer,
+                                const void* k_new, const void* v_new, const float* k_offsets, const float* v_offsets,
+                                int32_t in_dtype, int32_t n_new, const int32_t* seq_lens, int32_t* dev_status,
+                                tq_stream_t stream) {
+  CallRange range("tq_append_kv_dithered");
+  clear_error();
+  return append_common(cfg, params, cache, layer, k_new, v_new, k_offsets, v_offsets, true, in_dtype, n_new,
+                       seq_lens, dev_status, stream);
 }
 
 tq_status tq_decode_scores(const tq_config* cfg, const tq_params* params, const tq_cache* cache,

@@ -27,6 +27,7 @@ struct DecodeArgs {
   const void* q;
   int q_dtype, q_heads, seq_q, group, rows, n_splits, qjl, dense;
   int key_corr;  // appended keys store the corrected norm
+  const float *k_new_off, *v_new_off;  // dithered appends: the new tokens' offsets [B][H][n_new]
   const int32_t* seq_lens;
   const float *signs, *pi, *s, *k_centroids, *v_centroids;
   float* qrot;      // [B*Hq*seq_q][D]  workspace

@@ -9,7 +9,8 @@ from typing import Optional
 
 import torch
 
-from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, append_attend_decode, append_kv, attend_decode,
+from . import (TQ_ROT_DENSE, TQ_ROT_HADAMARD, TQError, append_attend_decode, append_attend_decode_dithered,
+               append_kv, append_kv_dithered, attend_decode,
                check_status, codebook, compress_kv, compress_kv_dithered, dither_codebook, last_error,
                decode_scores, decode_workspace_bytes, decompress, make_cache, make_config, make_params,
                operand_bytes, page_bytes, prepare_operands)
@@ -102,10 +103,17 @@ class PagedKV:
             compress_kv(self.cfg, self.params, self.cache, layer, k, v, seq_lens, self.status, stream)
 
     def append(self, layer: int, k_new: torch.Tensor, v_new: torch.Tensor, seq_lens: torch.Tensor,
-               stream=None):
+               stream=None, k_offsets: Optional[torch.Tensor] = None, v_offsets: Optional[torch.Tensor] = None):
         """Compresses k_new, v_new [batch][kv_heads][n_new][d] into positions
-        seq_lens[b] - n_new .. seq_lens[b] - 1 (seq_lens: the lengths after the append)."""
-        append_kv(self.cfg, self.params, self.cache, layer, k_new, v_new, seq_lens, self.status, stream)
+        seq_lens[b] - n_new .. seq_lens[b] - 1 (seq_lens: the lengths after the append); a
+        dithered cache takes the new tokens' offsets [batch][kv_heads][n_new]."""
+        if self.dither:
+            if k_offsets is None or v_offsets is None:
+                raise ValueError("a dithered cache needs k_offsets and v_offsets")
+            append_kv_dithered(self.cfg, self.params, self.cache, layer, k_new, v_new, k_offsets, v_offsets,
+                               seq_lens, self.status, stream)
+        else:
+            append_kv(self.cfg, self.params, self.cache, layer, k_new, v_new, seq_lens, self.status, stream)
 
     def workspace(self, q_heads: int, seq_q: int, n_splits: int) -> torch.Tensor:
         key = (q_heads, seq_q, n_splits)
@@ -116,13 +124,19 @@ class PagedKV:
 
     def decode(self, layer: int, q: torch.Tensor, seq_lens: torch.Tensor, n_splits: int,
                out: Optional[torch.Tensor] = None, stream=None, k_new: Optional[torch.Tensor] = None,
-               v_new: Optional[torch.Tensor] = None) -> torch.Tensor:
+               v_new: Optional[torch.Tensor] = None, k_offsets: Optional[torch.Tensor] = None,
+               v_offsets: Optional[torch.Tensor] = None) -> torch.Tensor:
         """Attention of q over the first seq_lens[b] tokens.  With k_new and v_new the step's
         new tokens are appended first, in the same call (seq_lens count them)."""
         if out is None:
             out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
         ws = self.workspace(q.shape[1], q.shape[2], n_splits)
-        if k_new is not None:
+        if k_new is not None and self.dither:
+            if k_offsets is None or v_offsets is None:
+                raise ValueError("a dithered cache needs k_offsets and v_offsets")
+            append_attend_decode_dithered(self.cfg, self.params, self.cache, layer, k_new, v_new, k_offsets,
+                                          v_offsets, q, seq_lens, n_splits, ws, out, self.status, stream)
+        elif k_new is not None:
             append_attend_decode(self.cfg, self.params, self.cache, layer, k_new, v_new, q, seq_lens,
                                  n_splits, ws, out, self.status, stream)
         else:

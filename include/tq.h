@@ -327,7 +327,8 @@ TQ_API tq_status tq_attend_decode(const tq_config* cfg, const tq_params* params,
  *                 TQ_ERR_OVERFLOW as for tq_compress_kv
  * params.s (with key_qjl) and params.pi (TQ_ROT_DENSE) must be 16-byte aligned; S is
  * used in fp32 as given (no fp16 requirement).  One thread block per new token.
- * Dithered configurations return TQ_ERR_UNSUPPORTED (no offsets are taken here). */
+ * Dithered configurations return TQ_ERR_UNSUPPORTED: their appends take the new tokens'
+ * offsets through tq_append_kv_dithered. */
 TQ_API tq_status tq_append_kv(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                               int32_t layer, const void* k_new, const void* v_new, int32_t in_dtype,
                               int32_t n_new, const int32_t* seq_lens, int32_t* dev_status,
@@ -346,6 +347,27 @@ TQ_API tq_status tq_append_attend_decode(const tq_config* cfg, const tq_params* 
                                          int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,
                                          void* workspace, size_t workspace_bytes, float* out,
                                          int32_t* dev_status, tq_stream_t stream);
+
+/* The two appends for a dithered configuration (cfg->dither = 1, [DITHER]): new token n of
+ * (sequence b, head h) is coded with the offsets xi = fp16(k_offsets[b][h][n]) and
+ * fp16(v_offsets[b][h][n]) exactly as tq_compress_kv_dithered codes it, the offsets stored
+ * in its KD / VD slots.
+ *   k_offsets, v_offsets  device float [batch][kv_heads][n_new]
+ * Everything else as for tq_append_kv and tq_append_attend_decode; TQ_ERR_INVALID_ARG for a
+ * configuration that is not dithered or NULL offsets. */
+TQ_API tq_status tq_append_kv_dithered(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
+                                       int32_t layer, const void* k_new, const void* v_new,
+                                       const float* k_offsets, const float* v_offsets, int32_t in_dtype,
+                                       int32_t n_new, const int32_t* seq_lens, int32_t* dev_status,
+                                       tq_stream_t stream);
+TQ_API tq_status tq_append_attend_decode_dithered(const tq_config* cfg, const tq_params* params,
+                                                  const tq_cache* cache, int32_t layer, const void* k_new,
+                                                  const void* v_new, const float* k_offsets,
+                                                  const float* v_offsets, int32_t in_dtype, int32_t n_new,
+                                                  const void* q, int32_t q_dtype, int32_t q_heads,
+                                                  int32_t seq_q, const int32_t* seq_lens, int32_t n_splits,
+                                                  void* workspace, size_t workspace_bytes, float* out,
+                                                  int32_t* dev_status, tq_stream_t stream);
 
 /* Decode attention for callers that cannot allocate device memory (no counterpart on
  * the source pages; it exists for users of this library).  Same computation, arguments

@@ -120,6 +120,12 @@ def test_dithered_compress_entry_points_check_the_mode(tq):
     cache = tq.tq_cache(p, p, 1, 1, 1, 1, 1)
     st = tq.lib.tq_append_kv(by(dith), by(params), by(cache), 0, p, p, 0, 1, p, None, None)
     assert st == tq.TQ_ERR_UNSUPPORTED and "offsets" in tq.last_error()
+    # ... through the _dithered calls, which a plain cache and missing offsets are refused by
+    st = tq.lib.tq_append_kv_dithered(by(tq.make_config()), by(params), by(cache), 0, p, p, p, p, 0, 1, p, None,
+                                      None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "dither" in tq.last_error()
+    st = tq.lib.tq_append_kv_dithered(by(dith), by(params), by(cache), 0, p, p, None, p, 0, 1, p, None, None)
+    assert st == tq.TQ_ERR_INVALID_ARG and "offsets" in tq.last_error()
 
 
 def test_codebook_argument_errors(tq):

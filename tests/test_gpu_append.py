@@ -50,7 +50,28 @@ CASES = {
                                              key_corrected_norm=True, name="c2_corrected_norm"), (1, 3)),
     "c3_corrected_norm": (lambda: wl.config3(batch=2, max_len=700, min_len=300, n_splits=2,
                                              key_corrected_norm=True, name="c3_corrected_norm"), (2,)),
+    # dithered: the new tokens' offsets through the _dithered calls (MSE-only 2-bit keys too)
+    "c2_dither": (lambda: wl.config2(kv_heads=2, q_heads=8, max_len=1283, n_splits=4, dither=True,
+                                     name="c2_dither"), (1, 3)),
+    "k2v4_dither": (lambda: wl.config2(kv_heads=1, q_heads=4, max_len=520, key_bits=2, key_qjl=False,
+                                       value_bits=4, n_splits=2, dither=True, name="k2v4_dither"), (2,)),
 }
+
+
+def _offsets(run, layer, after, n_new):
+    """Dithered workloads: the offsets of positions after[b] - n_new .. after[b] - 1, as keyword
+    arguments of the append calls (none otherwise)."""
+    if not run.w.dither:
+        return {}
+    B, H = run.w.batch, run.w.kv_heads
+    ko = np.zeros((B, H, n_new))
+    vo = np.zeros((B, H, n_new))
+    for b in range(B):
+        p0 = int(after[b]) - n_new
+        ko[b] = run.KO[layer][b, :, p0:p0 + n_new]
+        vo[b] = run.VO[layer][b, :, p0:p0 + n_new]
+    return dict(k_offsets=torch.as_tensor(ko, dtype=torch.float32, device="cuda").contiguous(),
+                v_offsets=torch.as_tensor(vo, dtype=torch.float32, device="cuda").contiguous())
 
 
 def _new_tokens(run, layer, after, n_new, dt):
@@ -95,7 +116,8 @@ def _check_old_tokens_unchanged(run, before, after, start):
             n = int(start[b])
             u0 = olay.read_sequence(before, run.fmt, 0, h, run.bt[b], n)
             u1 = olay.read_sequence(after, run.fmt, 0, h, run.bt[b], n)
-            for f in ("k_idx", "v_idx", "k_norm", "v_norm", "k_rnorm", "k_sigma", "v_rnorm", "v_sigma"):
+            for f in ("k_idx", "v_idx", "k_norm", "v_norm", "k_rnorm", "k_sigma", "v_rnorm", "v_sigma", "k_offset",
+                      "v_offset"):
                 a0, a1 = getattr(u0, f), getattr(u1, f)
                 if a0 is not None:
                     np.testing.assert_array_equal(a0, a1, err_msg=f"{f} of b={b} h={h} changed")
@@ -110,7 +132,7 @@ def test_append_kv_matches_oracle(name):
     for n_new in steps:
         cur = cur + n_new
         kn, vn = _new_tokens(run, 0, cur, n_new, dt)
-        run.kv.append(0, kn, vn, torch.as_tensor(cur, dtype=torch.int32, device="cuda"))
+        run.kv.append(0, kn, vn, torch.as_tensor(cur, dtype=torch.int32, device="cuda"), **_offsets(run, 0, cur, n_new))
     run.kv.raise_on_error("append")
     assert (cur == run.lens).all()
     pages = run.kv.pages_numpy()
@@ -132,7 +154,7 @@ def test_fused_append_decode_matches_oracle(name):
         cur = cur + n_new
         kn, vn = _new_tokens(run, 0, cur, n_new, dt)
         seq = torch.as_tensor(cur, dtype=torch.int32, device="cuda")
-        out = run.kv.decode(0, qd, seq, run.w.n_splits, k_new=kn, v_new=vn)
+        out = run.kv.decode(0, qd, seq, run.w.n_splits, k_new=kn, v_new=vn, **_offsets(run, 0, cur, n_new))
         run.kv.raise_on_error("append+decode")
         pages = run.kv.pages_numpy()
         run.lens = cur  # the oracle decodes the cache as it stands after this step
