@@ -289,27 +289,47 @@ __device__ void append_token(const DecodeArgs& a, int job) {
 // prologue: one CTA of 128 threads per query row.  Thread i owns coordinate i.
 //   qrot = R q (fp32), q8 = int8 rounding of qrot * 127 / max|qrot| (with its scale),
 //   sq = S q (fp32), sq_int = S q in 16-bit fixed point with a power-of-two scale, sum.
+// A row's terms are published through its ready word: zeroed before the CTA lets the split
+// kernel start, set (release) once every term of the row is written.  The tensor-core split
+// kernel acquires the words of its rows instead of waiting for this whole grid to finish.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_rows) {
-  // Launched as a programmatic dependent of whatever precedes it on the stream: everything
-  // before it has finished once this wait returns.  Then the split kernel may start (its
-  // set-up reads only inputs no kernel of this call writes).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
-  const int row = blockIdx.x;
-  if (row >= total_rows) {
-    // thread blocks past the query rows append the new tokens (none unless a.n_new > 0)
-    if (a.n_new > 0 && row - total_rows < a.cache.batch * a.cache.kv_heads * a.n_new) append_token(a, row - total_rows);
-    return;
+
+// Before launch_dependents: the row's terms of an earlier call are no longer announced (its
+// kQueryParts ready words, threads 0 .. kQueryParts - 1).
+__device__ __forceinline__ void unpublish_row(const DecodeArgs& a, int row) {
+  if (threadIdx.x < kQueryParts) {
+    const unsigned int* rw = a.ready + (size_t)row * kQueryParts + threadIdx.x;
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(rw), "r"(0u) : "memory");
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
   }
+  __syncthreads();
+}
+
+// After every term of the row is written: the barrier orders the block's writes before the
+// release stores that set the ready words.
+__device__ __forceinline__ void publish_row(const DecodeArgs& a, int row) {
+  __syncthreads();
+  if (threadIdx.x < kQueryParts)
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.ready + (size_t)row * kQueryParts + threadIdx.x),
+                 "r"(1u)
+                 : "memory");
+}
+
+// The merge counter of the tensor-core split kernel's run of query rows that starts at this
+// row (runs of four, or eight when a KV head has more than four rows): zero at every call,
+// zeroed before the row's terms are announced
+__device__ __forceinline__ void zero_run_counter(const DecodeArgs& a, int row) {
+  const int nr = a.rows > 4 ? 8 : 4, local = row % a.rows;
+  if (threadIdx.x == 0 && local % nr == 0) a.counter[(row / a.rows) * ((a.rows + nr - 1) / nr) + local / nr] = 0u;
+}
+
+__device__ __forceinline__ void query_row(const DecodeArgs& a, int row) {
   __shared__ __align__(16) float qs[D];
   __shared__ float ys[D];
   __shared__ float red[2][4];
   __shared__ int ired[4];
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
-  // the merge counters of the fused split kernel (one per sequence, kv head and run of up to
-  // four query rows) start every call at zero
-  if (a.counter && i == 0 && row < a.cache.batch * a.cache.kv_heads * ((a.rows + 3) / 4)) a.counter[row] = 0u;
+  zero_run_counter(a, row);
   // the rows of S this warp needs, requested before the query (they do not depend on it)
   float4 p[32];
   if (a.qjl) {
@@ -361,7 +381,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
       t = warp_sum(t);
       if (lane == u) sq = t;
     }
-    a.sq[(size_t)row * QM + 32 * warp + lane] = sq;
+    a.sq[(size_t)row * QM + i] = sq;
   }
   // maxima of |R q| and |S q| over the row
   float my = fabsf(y), ms = fabsf(sq);
@@ -388,7 +408,7 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
       ex -= 1;  // 2^ex <= 32000 / mx
     }
     const int v = __float2int_rn(sq * ldexpf(1.f, ex));
-    a.sq_int[(size_t)row * QM + 32 * warp + lane] = (int16_t)v;
+    a.sq_int[(size_t)row * QM + i] = (int16_t)v;
     int sum = v;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(FULL, sum, o);
@@ -399,6 +419,142 @@ __global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int total_r
       a.sq_sum[row] = ired[0] + ired[1] + ired[2] + ired[3];
     }
   }
+}
+
+// The query terms for the tensor-core split kernel, kQueryParts thread blocks of 128 threads
+// per query row.  Part c forms outputs 32 c .. 32 c + 31 of S q in fp32 (the split kernel
+// takes them to fixed point), 8 per warp; part 0 also R q and its int8 copy with the scale,
+// and zeroes the merge counter of a run that starts at this row.  Each part announces its
+// terms through its own ready word.  Few registers: a block waiting for its predecessor stays
+// resident beside two split-kernel blocks of the previous call.
+// Before launch_dependents: this part's terms of an earlier call are no longer announced.
+__device__ __forceinline__ void unpublish_part(const DecodeArgs& a, int blk) {
+  if (threadIdx.x == 0) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(a.ready + blk), "r"(0u) : "memory");
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  }
+  __syncthreads();
+}
+
+// Part blk % kQueryParts of query row blk / kQueryParts (after unpublish_part and the launch
+// of the dependents).
+__device__ __forceinline__ void query_part(const DecodeArgs& a, int blk) {
+  const int row = blk / kQueryParts, part = blk % kQueryParts;
+  const unsigned int* rw = a.ready + blk;
+  __shared__ __align__(16) float qs[D];
+  __shared__ float ys[D];
+  __shared__ float red[4];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  // the rows of S of this warp's outputs o = 32 part + 8 warp + j, requested before the query
+  // (they do not depend on it); lane l holds entries 4 l .. 4 l + 3 of each
+  const int o0 = 32 * part + 8 * warp;
+  float4 p[8];
+  if (a.qjl) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) p[j] = reinterpret_cast<const float4*>(a.s + (size_t)(o0 + j) * D)[lane];
+  }
+  qs[i] = a.q_dtype == TQ_F16 ? __half2float(reinterpret_cast<const __half*>(a.q)[(size_t)row * D + i])
+                              : reinterpret_cast<const float*>(a.q)[(size_t)row * D + i];
+  if (part == 0) zero_run_counter(a, row);
+  __syncthreads();
+  if (part == 0) {
+    float y;
+    if (!a.dense) {
+      // y = H D q / sqrt(d): the warp-level transform in warp 0
+      if (warp == 0) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = qs[lane + 32 * e] * a.signs[lane + 32 * e];
+        fwht128_warp(v, lane);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ys[lane + 32 * e] = v[e] * kInvSqrtD;
+      }
+      __syncthreads();
+      y = ys[i];
+    } else {
+      const float4* prow = reinterpret_cast<const float4*>(a.pi + (size_t)i * D);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < D / 4; ++k) {
+        const float4 m = prow[k];
+        acc = fmaf(m.x, qs[4 * k], acc);
+        acc = fmaf(m.y, qs[4 * k + 1], acc);
+        acc = fmaf(m.z, qs[4 * k + 2], acc);
+        acc = fmaf(m.w, qs[4 * k + 3], acc);
+      }
+      y = acc;
+    }
+    a.qrot[(size_t)row * D + i] = y;
+    float my = warp_max(fabsf(y));
+    if (lane == 0) red[warp] = my;
+    __syncthreads();
+    my = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float lam = my > 0.f ? 127.f / my : 0.f;
+    a.q8[(size_t)row * D + i] = (int8_t)__float2int_rn(y * lam);
+    if (i == 0) a.q8_scale[row] = lam;
+  }
+  if (a.qjl) {
+    const float4 q4 = reinterpret_cast<const float4*>(qs)[lane];
+    float t[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float v = p[j].x * q4.x;
+      v = fmaf(p[j].y, q4.y, v);
+      v = fmaf(p[j].z, q4.z, v);
+      t[j] = fmaf(p[j].w, q4.w, v);
+    }
+    // sum over the lanes: within each group of eight lanes a reduce-scatter (after the step
+    // over lane bit h a lane keeps the half of its sums whose output index has that bit, plus
+    // the partner's copy of that half), so lane l holds output l & 7 of its group; then the
+    // four groups are added
+#pragma unroll
+    for (int h = 4; h >= 1; h >>= 1) {
+#pragma unroll
+      for (int j = 0; j < h; ++j) {
+        const bool upper = lane & h;
+        const float send = upper ? t[j] : t[j + h];
+        const float keep = upper ? t[j + h] : t[j];
+        t[j] = keep + __shfl_xor_sync(FULL, send, h);
+      }
+    }
+    float v = t[0];
+    v += __shfl_xor_sync(FULL, v, 8);
+    v += __shfl_xor_sync(FULL, v, 16);
+    if (lane < 8) a.sq[(size_t)row * QM + o0 + lane] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(rw), "r"(1u) : "memory");
+}
+
+__global__ void __launch_bounds__(128) query_kernel(DecodeArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  unpublish_part(a, blockIdx.x);
+  asm volatile("griddepcontrol.launch_dependents;");
+  query_part(a, blockIdx.x);
+}
+
+// Query rows (thread blocks 0 .. q_blocks - 1), then one thread block per appended token.
+// With fast_query the query blocks are the tensor-core split kernel's kQueryParts parts per
+// row (as query_kernel), otherwise one block per row with the general kernels' terms.
+__global__ void __launch_bounds__(128) prologue_kernel(DecodeArgs a, int q_blocks) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int blk = blockIdx.x;
+  if (blk < q_blocks) {
+    if (a.fast_query) unpublish_part(a, blk);
+    else unpublish_row(a, blk);
+  }
+  asm volatile("griddepcontrol.launch_dependents;");
+  if (blk >= q_blocks) {
+    // thread blocks past the query rows append the new tokens (none unless a.n_new > 0)
+    if (a.n_new > 0 && blk - q_blocks < a.cache.batch * a.cache.kv_heads * a.n_new) append_token(a, blk - q_blocks);
+    return;
+  }
+  if (a.fast_query) {
+    query_part(a, blk);
+    return;
+  }
+  query_row(a, blk);
+  publish_row(a, blk);
 }
 
 // ---------------------------------------------------------------------------
@@ -743,6 +899,8 @@ DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits
   w.q8_scale = off; off = align256(off + rows * sizeof(float));
   // one counter per (sequence, kv head, run of up to four query rows): at most one per query row
   w.counter = off; off = align256(off + rows * sizeof(unsigned int));
+  // kQueryParts ready words per query row
+  w.ready = off; off = align256(off + rows * kQueryParts * sizeof(unsigned int));
   w.total = off;
   return w;
 }
@@ -801,9 +959,13 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (fast_decode_supported(a)) {
     // query transforms (and zeroed merge counters), then the split kernel, whose last
     // split per (sequence, kv head) merges the partials: two launches
-    cudaError_t e = launch_pdl(prologue_kernel, dim3(blocks), dim3(128), 0, stream, a, total_rows);
+    DecodeArgs f = a;
+    f.fast_query = 1;
+    const int qb = total_rows * kQueryParts;
+    cudaError_t e = a.n_new > 0 ? launch_pdl(prologue_kernel, dim3(qb + blocks - total_rows), dim3(128), 0, stream, f, qb)
+                                : launch_pdl(query_kernel, dim3(qb), dim3(128), 0, stream, f);
     if (e != cudaSuccess) return e;
-    return launch_fast_split(a, stream);
+    return launch_fast_split(f, stream);
   }
   // the split kernel is an ordinary launch: it starts once the prologue (and any append)
   // has finished

@@ -152,6 +152,25 @@ __device__ __forceinline__ bool mbar_wait_sleepy(unsigned long long* bar, uint32
   }
 }
 
+// Wait (bounded by the global timer) until a ready word of the prologue is set.  It is read
+// with acquire semantics, so that what the prologue wrote before setting it is visible to
+// this thread's later reads.  false (and TQ_ERR_TIMEOUT) if it gave up.
+__device__ __forceinline__ bool acquire_ready(const unsigned int* rw, int32_t* status) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(rw) : "memory");
+  if (v) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    __nanosleep(32);
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(rw) : "memory");
+    if (v) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      report(status, TQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -432,10 +451,16 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         else et1 |= v << (8 * (i - 4));
       }
     }
-    // the prologue (our programmatic predecessor) must be done before its outputs are read
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // The prologue (our programmatic predecessor) publishes the query terms of each row in
+    // kQueryParts parts, each with a ready word: acquire those of this CTA's rows (bounded;
+    // the acquires, ordered before the other warps' reads by the barrier, make the terms and
+    // the zeroed merge counter visible), instead of waiting for the whole prologue grid.
+    if (warp == 0 && lane < R * kQueryParts) acquire_ready(a.ready + row0 * kQueryParts + lane, a.status);
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     // B fragments, one n-tile per four rows (tile nt: rows 4 nt .. 4 nt + 3)
     uint32_t bq[NT][8][2], bc[NT][4][2], bs[NT][4][2];
+    int sq_sum_nt[NT];        // of row 4 nt + g/2: the sum of its fixed-point S q
+    float sq_scale_nt[NT];    // and the power of two that scales it
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       // this lane's 32-coordinate slices of row 4 nt + g/2: rotated query, its int8 copy,
@@ -448,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         const size_t rr = row0 + (frow ? fr : 0);
         const float4* qp = reinterpret_cast<const float4*>(a.qrot + rr * D + 32 * t4);
         const int4* q8p = reinterpret_cast<const int4*>(a.q8 + rr * D + 32 * t4);
-        const int4* sqp = reinterpret_cast<const int4*>(a.sq_int + rr * QM + 32 * t4);
+        const float4* sqp = reinterpret_cast<const float4*>(a.sq + rr * QM + 32 * t4);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float4 f = frow ? qp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -463,16 +488,37 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) q8v[16 * k + 4 * u + bb] = (int)(int8_t)((w4[u] >> (8 * bb)) & 255);
         }
+        // S q of the row in 16-bit fixed point: scale 2^ex with 2^ex <= 32000 / max |S q| over
+        // the row (its 128 entries are spread over the four lanes t4 of this group), the sum
+        // of the fixed-point entries with it
+        float mx = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int4 v = (frow && kQjl) ? sqp[k] : make_int4(0, 0, 0, 0);
-          const int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            sqv[8 * k + 2 * u] = (int)(int16_t)(w4[u] & 0xffff);
-            sqv[8 * k + 2 * u + 1] = (int)(int16_t)((uint32_t)w4[u] >> 16);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const float4 f = (frow && kQjl) ? sqp[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+          sqv[4 * k] = __float_as_int(f.x);
+          sqv[4 * k + 1] = __float_as_int(f.y);
+          sqv[4 * k + 2] = __float_as_int(f.z);
+          sqv[4 * k + 3] = __float_as_int(f.w);
         }
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 2));
+        int ex = 0;
+        if (mx > 0.f) {
+          frexpf(32000.f / mx, &ex);
+          ex -= 1;
+        }
+        const float up = ldexpf(1.f, ex);
+        int rs = 0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sqv[c] = __float2int_rn(__int_as_float(sqv[c]) * up);
+          rs += sqv[c];
+        }
+        rs += __shfl_xor_sync(FULL, rs, 1);
+        rs += __shfl_xor_sync(FULL, rs, 2);
+        sq_sum_nt[nt] = rs;
+        sq_scale_nt[nt] = ldexpf(1.f, -ex);
       }
       // the key term: column g = (row 4 nt + g/2, hi or lo half)
 #pragma unroll
@@ -545,12 +591,15 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int rr = t4 + 4 * nt;
+      // row rr's fixed-point sum and scale sit with the lanes g = 2 t4, 2 t4 + 1
+      const int rsum = __shfl_sync(FULL, sq_sum_nt[nt], 8 * t4);
+      const float rscale = __shfl_sync(FULL, sq_scale_nt[nt], 8 * t4);
       T_row[nt] = 0;
       c_row_q[nt] = 0.f;
       corr_down[nt] = 0.f;
       if (rr < R) {
-        T_row[nt] = kQjl ? a.sq_sum[row0 + rr] : 0;
-        c_row_q[nt] = kQjl ? kQjlScale * a.sq_scale[row0 + rr] * kInvSqrtD * kLog2e : 0.f;
+        T_row[nt] = kQjl ? rsum : 0;
+        c_row_q[nt] = kQjl ? kQjlScale * rscale * kInvSqrtD * kLog2e : 0.f;
         const float lam = a.q8_scale[row0 + rr];
         corr_down[nt] = lam > 0.f ? 1.f / (lam * eps_up) : 0.f;
       }

@@ -302,6 +302,8 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.q8 = reinterpret_cast<int8_t*>(ws + w.q8);
   a.q8_scale = reinterpret_cast<float*>(ws + w.q8_scale);
   a.counter = reinterpret_cast<unsigned int*>(ws + w.counter);
+  a.ready = reinterpret_cast<unsigned int*>(ws + w.ready);
+  a.fast_query = 0;
   a.out = nullptr;
   a.scores = nullptr;
   a.max_len = 0;

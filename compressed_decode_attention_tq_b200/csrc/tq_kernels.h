@@ -8,6 +8,10 @@
 
 namespace tqk {
 
+// The prologue of the tensor-core split kernel forms each query row's terms in this many
+// parts (thread blocks), each announced by its own ready word.
+constexpr int kQueryParts = 4;
+
 struct CompressArgs {
   CacheRef cache;
   const void* k;
@@ -42,6 +46,8 @@ struct DecodeArgs {
   float* q8_scale;  // [B*Hq*seq_q] workspace
   unsigned int* counter;  // workspace (sized B*Hq*seq_q): finished splits per (sequence, kv head,
                           // run of up to four query rows)
+  unsigned int* ready;    // workspace [B*Hq*seq_q][kQueryParts]: 1 once the prologue has written that
+                          // part of the row's terms
   float* out;       // [B*Hq*seq_q][D]
   float* scores;    // score-only mode: [B*Hq*seq_q][max_len]
   int max_len;
@@ -55,6 +61,9 @@ struct DecodeArgs {
   // fast split kernel waits this many nanoseconds on a barrier nothing arrives on and
   // reports TQ_ERR_TIMEOUT; the results are computed as usual)
   int debug_wait_ns;
+  // 1: the prologue forms the query terms in kQueryParts parts per row for the tensor-core split
+  // kernel (fp32 S q, ready word per part); 0: one block per row for the general kernels
+  int fast_query;
   int32_t* status;
 };
 
@@ -79,7 +88,7 @@ cudaError_t launch_prepare_dense(const float* pi, void* ops, cudaStream_t stream
 
 // Workspace layout of decode, all offsets 256-byte aligned.
 struct DecodeWorkspace {
-  size_t qrot, sq, part_acc, part_ml, part_sig, sq_int, sq_scale, sq_sum, q8, q8_scale, counter, total;
+  size_t qrot, sq, part_acc, part_ml, part_sig, sq_int, sq_scale, sq_sum, q8, q8_scale, counter, ready, total;
 };
 DecodeWorkspace decode_workspace(int batch, int q_heads, int seq_q, int n_splits, int vqjl);
 
