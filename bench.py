@@ -368,7 +368,7 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": comp_bytes_launch, "achieved_gbs": comp_gbs,
                      "frac": comp_gbs / hbm},
         "decode": {"kernel": "fast_split_kernel", "ms_per_step": dec_ms, "launches_per_step": 2 * L,
-                   "kernels": "prologue_kernel + fast_split_kernel",
+                   "kernels": "query_kernel + fast_split_kernel",
                    "kv_tokens_per_s": L * tok_heads_layer / (dec_ms / 1e3),
                    "algorithmic_bytes_per_launch": dec_bytes_launch, "achieved_gbs": dec_gbs,
                    "frac": dec_gbs / hbm},
