@@ -584,6 +584,31 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         }
       }
     }
+    // With eight rows (two n-tiles) the B fragments (64 registers per lane) live in shared
+    // memory during the page loop, over the warp partials' space (written only after every
+    // consumer warp has left the loop), and are read back per n-tile at each step; every warp
+    // formed the same fragments, warp 0 stores them: [n-tile][8 slots][lane] of 16 bytes
+    constexpr bool kBSmem = NT == 2;
+    uint4* const bfrag = reinterpret_cast<uint4*>(&sm.ring.wacc[0][0][0]);
+    if constexpr (kBSmem) {
+      if (warp == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            bfrag[(nt * 8 + j) * 32 + lane] = make_uint4(bq[nt][2 * j][0], bq[nt][2 * j][1], bq[nt][2 * j + 1][0],
+                                                         bq[nt][2 * j + 1][1]);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            bfrag[(nt * 8 + 4 + j) * 32 + lane] = make_uint4(bc[nt][2 * j][0], bc[nt][2 * j][1],
+                                                             bc[nt][2 * j + 1][0], bc[nt][2 * j + 1][1]);
+            bfrag[(nt * 8 + 6 + j) * 32 + lane] = make_uint4(bs[nt][2 * j][0], bs[nt][2 * j][1],
+                                                             bs[nt][2 * j + 1][0], bs[nt][2 * j + 1][1]);
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    }
     // per-row constants of the lane's own score rows t4 + 4 nt
     int T_row[NT];
     float c_row_q[NT], corr_down[NT];
@@ -753,26 +778,54 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
             }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
+            // this n-tile's B fragments: from shared memory (two n-tiles) or registers
+            uint32_t fq[8][2], fc[4][2], fs[4][2];
+            if constexpr (kBSmem) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint4 v = bfrag[(nt * 8 + j) * 32 + lane];
+                fq[2 * j][0] = v.x; fq[2 * j][1] = v.y; fq[2 * j + 1][0] = v.z; fq[2 * j + 1][1] = v.w;
+              }
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const uint4 c = bfrag[(nt * 8 + 4 + j) * 32 + lane], q = bfrag[(nt * 8 + 6 + j) * 32 + lane];
+                fc[2 * j][0] = c.x; fc[2 * j][1] = c.y; fc[2 * j + 1][0] = c.z; fc[2 * j + 1][1] = c.w;
+                fs[2 * j][0] = q.x; fs[2 * j][1] = q.y; fs[2 * j + 1][0] = q.z; fs[2 * j + 1][1] = q.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                fq[j][0] = bq[nt][j][0];
+                fq[j][1] = bq[nt][j][1];
+              }
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                fc[j][0] = bc[nt][j][0];
+                fc[j][1] = bc[nt][j][1];
+                fs[j][0] = bs[nt][j][0];
+                fs[j][1] = bs[nt][j][1];
+              }
+            }
             // two accumulators per term halve the dependent mma chains
             float dk[4] = {0.f, 0.f, 0.f, 0.f}, dk2[4] = {0.f, 0.f, 0.f, 0.f};
     #pragma unroll
             for (int ks = 0; ks < 8; ks += 2) {
-              hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], bq[nt][ks][0], bq[nt][ks][1]);
-              hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], bq[nt][ks + 1][0],
-                   bq[nt][ks + 1][1]);
+              hmma(dk, ha[2 * ks], hb[2 * ks], ha[2 * ks + 1], hb[2 * ks + 1], fq[ks][0], fq[ks][1]);
+              hmma(dk2, ha[2 * ks + 2], hb[2 * ks + 2], ha[2 * ks + 3], hb[2 * ks + 3], fq[ks + 1][0],
+                   fq[ks + 1][1]);
             }
             int dsum[4] = {0, 0, 0, 0}, dsum2[4] = {0, 0, 0, 0};
             int dcor[4] = {0, 0, 0, 0}, dcor2[4] = {0, 0, 0, 0};
     #pragma unroll
             for (int w = 0; w < 4; w += 2) {
               if (kQjl) {
-                imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], bs[nt][w][0], bs[nt][w][1]);
-                imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], bs[nt][w + 1][0],
-                     bs[nt][w + 1][1]);
+                imma(dsum, sa[2 * w], sb[2 * w], sa[2 * w + 1], sb[2 * w + 1], fs[w][0], fs[w][1]);
+                imma(dsum2, sa[2 * w + 2], sb[2 * w + 2], sa[2 * w + 3], sb[2 * w + 3], fs[w + 1][0],
+                     fs[w + 1][1]);
               }
-              imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], bc[nt][w][0], bc[nt][w][1]);
-              imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], bc[nt][w + 1][0],
-                   bc[nt][w + 1][1]);
+              imma(dcor, ea[2 * w], eb[2 * w], ea[2 * w + 1], eb[2 * w + 1], fc[w][0], fc[w][1]);
+              imma(dcor2, ea[2 * w + 2], eb[2 * w + 2], ea[2 * w + 3], eb[2 * w + 3], fc[w + 1][0],
+                   fc[w + 1][1]);
             }
     #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -949,6 +1002,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
     }
+    // the B fragments in shared memory are read until every consumer warp has left the loop
+    if constexpr (kBSmem) asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     // ---- warp partial: l summed over the 8 lanes of a row, acc scattered by coordinate
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
