@@ -121,3 +121,25 @@ def test_bounded_wait_gives_up_and_the_context_stays_usable(monkeypatch):
     out = r.kv.decode(0, qd, seq, w.n_splits).cpu().numpy()
     assert r.kv.check() == 0
     assert close(out, oracle_decode(r, r.pages, 0, q)).all()
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, 0x01])
+def test_decode_ignores_what_the_workspace_held(fill):
+    """The workspace is scratch: whatever it holds on entry (here every byte `fill`, so that
+    every ready word of the query prologue reads as set, or as clear) the decode output equals
+    the oracle's.  The prologue clears each part's ready word before the split kernel may
+    start, so a stale word can never let the split kernel read query terms early."""
+    import compressed_decode_attention_tq_b200 as tq
+    w = wl.config2(kv_heads=2, q_heads=8, max_len=1500, n_splits=5)
+    r = _run(w)
+    r.kv.raise_on_error("compress")
+    seq = torch.as_tensor(r.lens, dtype=torch.int32, device="cuda")
+    q, qd = q_dev(r)
+    ws = r.kv.workspace(qd.shape[1], qd.shape[2], 5)
+    ref = oracle_decode(r, r.pages, 0, q)
+    for _ in range(2):
+        ws.fill_(fill)
+        out = torch.empty(qd.shape, dtype=torch.float32, device="cuda")
+        tq.attend_decode(r.kv.cfg, r.kv.params, r.kv.cache, 0, qd, seq, 5, ws, out, r.kv.status)
+        r.kv.raise_on_error("decode")
+        assert close(out.cpu().numpy(), ref).all()
