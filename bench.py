@@ -407,7 +407,7 @@ def run_ours(args, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(w, L), "phases": phases, "roofline": roofline,
             "cpu_baseline": cpu, "e2e": e2e, "configs": configs,
-            # per layer: compress_tc_kernel, then prologue_kernel + fast_split_kernel
+            # per layer: compress_tc_kernel, then query_kernel + fast_split_kernel
             "gpu_launches": args.steps * L * 3,
             "clocks": clk.summary(),
         }
