@@ -399,6 +399,7 @@ def run_ours(args, rank, world, local_rank):
     configs = None
     if rank == 0 and not args.no_configs:
         configs = config_timings(dev)
+    quality = reconstruction_quality(kv, w, Ks[0], Vs[0], Qs[0], seq) if rank == 0 else None
 
     if rank == 0:
         line = {
@@ -406,12 +407,56 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(w, L), "phases": phases, "roofline": roofline,
-            "cpu_baseline": cpu, "e2e": e2e, "configs": configs,
+            "cpu_baseline": cpu, "e2e": e2e, "configs": configs, "quality": quality,
             # per layer: compress_tc_kernel, then query_kernel + fast_split_kernel
             "gpu_launches": args.steps * L * 3,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
+
+
+def reconstruction_quality(kv, w, K, V, q, seq):
+    """What the packed cache keeps of layer 0 (outside the timed region): the compression
+    ratio against fp16 K/V; for keys (their MSE stage) and values, the relative squared error
+    of the library's decompression and the mean cosine similarity per vector; the relative
+    RMS error of the score estimator (MSE term + QJL term, from the score-only call) against
+    the exact q.k / sqrt(d); and the cosine similarity of each decode output row with exact
+    softmax attention over the fp16 K/V (PyTorch fp32, for this measurement only)."""
+    import torch
+    T = K.shape[2]
+
+    def recon(x, xh):
+        x = x.float()
+        err = ((x - xh) ** 2).sum(-1)
+        ref = (x ** 2).sum(-1)
+        cos = (x * xh).sum(-1) / (x.norm(dim=-1) * xh.norm(dim=-1)).clamp_min(1e-30)
+        return {"relative_mse": float(err.sum() / ref.sum()), "mean_cosine": float(cos.mean())}
+
+    kh, vh = kv.decompress(0, seq, T)
+    keys, values = recon(K, kh), recon(V, vh)
+    del kh, vh
+    G = w.q_heads // w.kv_heads
+    Kr = K.float().repeat_interleave(G, dim=1)
+    exact = torch.einsum("bhsd,bhtd->bhst", q.float(), Kr) / math.sqrt(128.0)
+    del Kr
+    est = kv.scores(0, q, seq, T)
+    score_err = float(((est - exact) ** 2).mean().sqrt() / (exact ** 2).mean().sqrt())
+    del est
+    out = kv.decode(0, q, seq, w.n_splits)
+    Vr = V.float().repeat_interleave(G, dim=1)
+    ref = torch.einsum("bhst,bhtd->bhsd", torch.softmax(exact, dim=-1), Vr)
+    cos = (out * ref).sum(-1) / (out.norm(dim=-1) * ref.norm(dim=-1)).clamp_min(1e-30)
+    kv.raise_on_error("quality")
+    del Vr, exact, ref
+    torch.cuda.empty_cache()
+    return {
+        "layer": 0,
+        "compression_ratio_vs_fp16": 2 * 128 * 2 / (kv.block_bytes / 256),
+        "keys_mse_stage": keys,
+        "values": values,
+        "score_relative_rms_error": score_err,
+        "decode_output_cosine": {"min": float(cos.min()), "mean": float(cos.mean())},
+    }
 
 
 def config_timings(dev, reps: int = 10):

@@ -64,10 +64,16 @@ class TQError(RuntimeError):
         super().__init__(f"{where}: {status_str(status)}" + (f" ({detail})" if detail else ""))
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libtq.so not built at {LIB_PATH}; run __graft_entry__.build()")
-    lib = ctypes.CDLL(LIB_PATH)
+# The same library with the kernels' index checks compiled in (built beside libtq.so): a
+# failed check records TQ_ERR_BOUNDS in dev_status.
+DEBUG_LIB_PATH = os.path.join(PKG, "libtq_debug.so")
+
+
+def _load(path: Optional[str] = None) -> ctypes.CDLL:
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not built at {path}; run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
     P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     cfgp, parp, cachep = ctypes.POINTER(tq_config), ctypes.POINTER(tq_params), ctypes.POINTER(tq_cache)
     sig = {

@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(kWarps * 32) compress_kernel(CompressArgs a) {
     uint8_t* blk = a.cache.block(phys, h);
     const int slot = t % PT;
     const size_t row = (head_off + t) * D;
+    TQ_DCHECK(a.status, t < a.max_len && t / PT < a.cache.max_pages);
     // dithered: the vectors' offsets, used and stored as fp16
     __half kxi = __float2half_rn(0.f), vxi = kxi;
     if (L.dither) {

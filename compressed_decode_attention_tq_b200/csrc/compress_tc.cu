@@ -892,6 +892,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (bad_len && row == 0 && l.t0 == 0) report(a.status, TQ_ERR_BOUNDS);
       TokRef r{nullptr, tok % PT};
       if (!bad_len && tok < l.len) {
+        TQ_DCHECK(a.status, tok < a.max_len && tok / PT < a.cache.max_pages && l.h < a.cache.kv_heads);
         if (l.phys < 0 || l.phys >= a.cache.num_pages) {
           report(a.status, TQ_ERR_BOUNDS);
         } else {

@@ -320,6 +320,7 @@ __device__ __forceinline__ void publish_row(const DecodeArgs& a, int row) {
 // zeroed before the row's terms are announced
 __device__ __forceinline__ void zero_run_counter(const DecodeArgs& a, int row) {
   const int nr = a.rows > 4 ? 8 : 4, local = row % a.rows;
+  TQ_DCHECK(a.status, (row / a.rows) * ((a.rows + nr - 1) / nr) + local / nr < a.cache.batch * a.q_heads * a.seq_q);
   if (threadIdx.x == 0 && local % nr == 0) a.counter[(row / a.rows) * ((a.rows + nr - 1) / nr) + local / nr] = 0u;
 }
 
@@ -440,6 +441,7 @@ __device__ __forceinline__ void unpublish_part(const DecodeArgs& a, int blk) {
 // of the dependents).
 __device__ __forceinline__ void query_part(const DecodeArgs& a, int blk) {
   const int row = blk / kQueryParts, part = blk % kQueryParts;
+  TQ_DCHECK(a.status, row < a.cache.batch * a.q_heads * a.seq_q);
   const unsigned int* rw = a.ready + blk;
   __shared__ __align__(16) float qs[D];
   __shared__ float ys[D];
@@ -617,6 +619,7 @@ __global__ void __launch_bounds__(128) split_kernel(DecodeArgs a) {
   const int n_eff = bad_len ? 0 : len;
   const int npages = (n_eff + PT - 1) / PT;
   const int cp = (npages + a.n_splits - 1) / a.n_splits;
+  TQ_DCHECK(a.status, R >= 1 && R <= kRowsMax && split < a.n_splits);
   const int t_begin = min(n_eff, split * cp * PT);
   const int t_end = min(n_eff, (split + 1) * cp * PT);
   float acc[RB];
@@ -832,6 +835,7 @@ __global__ void __launch_bounds__(128) combine_kernel(DecodeArgs a, int total_ro
   const int row = blockIdx.x;
   if (row >= total_rows) return;
   const bool vqjl = a.cache.L.vqjl != 0;
+  TQ_DCHECK(a.status, row < a.cache.batch * a.q_heads * a.seq_q);
   const float* ml = a.part_ml + (size_t)row * a.n_splits * 2;
   const float* pa = a.part_acc + (size_t)row * a.n_splits * D;
   const float* ps = vqjl ? a.part_sig + (size_t)row * a.n_splits * QM : nullptr;

@@ -284,6 +284,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   const Layout& L = a.cache.L;
   const int R = min(NR, a.rows - NR * chunk);
   const size_t row0 = ((size_t)b * a.q_heads + (size_t)gh * a.group) * a.seq_q + NR * chunk;
+  TQ_DCHECK(a.status, R >= 1 && R <= NR && row0 + R <= (size_t)a.cache.batch * a.q_heads * a.seq_q);
 
   const int len = a.seq_lens[b];
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
@@ -331,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
         }
         issued = i + 1;
         const int u = u_begin + i, half = u % kUnitsPerPage;
+        TQ_DCHECK(a.status, u >= 0 && u < units_all && u / kUnitsPerPage < a.cache.max_pages);
+        TQ_DCHECK(a.status, unit_bytes <= (uint32_t)kStageBytes);
         if (a.n_new > 0 && !prologue_done && (u + 1) * kUnit > t_new) {
           asm volatile("griddepcontrol.wait;" ::: "memory");
           asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -682,6 +685,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       const unsigned char* vc = kc + kMaxKChunks * kChunkStride;
       const int tok0 = (u_begin + i) * kUnit;
       const int valid = min(kUnit, t_end - tok0);
+      TQ_DCHECK(a.status, valid >= 1 && valid <= kUnit && tok0 + valid <= n_eff);
       // two 16-token steps per iteration: their key and value work interleave, and one
       // joint running maximum (one rescale) serves both
       for (int pr = warp; pr * 32 < valid; pr += kConsumerWarps) {
@@ -1053,6 +1057,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       l = fmaf(f, sm.wl[w][tid], l);
     }
     const size_t pr = (row0 + tid) * a.n_splits + split;
+    TQ_DCHECK(a.status, split < a.n_splits);
     a.part_ml[pr * 2] = (M == -CUDART_INF_F) ? M : M / kLog2e;
     a.part_ml[pr * 2 + 1] = l;
   }
@@ -1091,6 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   // (m, l) pairs; otherwise register batches from L2
   constexpr int kCap = kMergeFloats / (NR * D);
   const bool in_smem = ns <= kCap;
+  TQ_DCHECK(a.status, ns >= 1 && (size_t)R * kCap * D <= (size_t)kMergeFloats);
   if (in_smem && tid == 0) {
     // the other splits' partials were made visible to this thread by the acquire above;
     // order them before this thread's async-proxy reads

@@ -83,6 +83,7 @@ __global__ void decompress_kernel(DecompressArgs a) {
   }
   const uint8_t* blk = a.cache.block(phys, h);
   const int slot = t % PT;
+  TQ_DCHECK(a.status, t < a.max_len && t / PT < a.cache.max_pages && slot < PT);
   const size_t row = (((size_t)b * a.cache.kv_heads + h) * a.max_len + t) * D;
   const Layout& L = a.cache.L;
   const float* pi = a.dense ? a.pi : nullptr;

@@ -73,6 +73,20 @@ __device__ __forceinline__ void report(int32_t* st, int code) {
   if (st) atomicCAS(st, 0, code);
 }
 
+// Index checks of the debug build (compiled with -DTQ_DEBUG, libtq_debug.so): a check that
+// fails records TQ_ERR_BOUNDS in the status word and the kernel carries on (no trap, so the
+// context stays usable); the release build compiles them away.
+#ifdef TQ_DEBUG
+#define TQ_DCHECK(status, cond)                    \
+  do {                                             \
+    if (!(cond)) report((status), TQ_ERR_BOUNDS);  \
+  } while (0)
+#else
+#define TQ_DCHECK(status, cond) \
+  do {                          \
+  } while (0)
+#endif
+
 // Stored-code magnitude table: mag[r] = c[h + r] with h = 2^(b-1).
 // Value of stored (s, r): s ? mag[r] : -mag[r].
 

@@ -34,6 +34,17 @@ def test_every_declared_symbol_is_exported(tq):
     assert exported == set(declared)
 
 
+def test_debug_library_exports_the_same_symbols(tq):
+    """libtq_debug.so (the kernels' index checks compiled in) is built beside libtq.so and
+    exports exactly the calls tq.h declares."""
+    assert os.path.exists(tq.DEBUG_LIB_PATH), "build() makes libtq_debug.so as well"
+    out = subprocess.run(["nm", "-D", "--defined-only", tq.DEBUG_LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    assert set(re.findall(r"\b(tq_[a-z_0-9]+)\b", out)) == set(_declared_functions())
+    dbg = tq._load(tq.DEBUG_LIB_PATH)
+    assert dbg.tq_version() == tq.lib.tq_version()
+
+
 def test_version_and_status_strings(tq):
     assert tq.lib.tq_version() >= 100
     assert tq.status_str(0) == "TQ_OK"
