@@ -1,7 +1,7 @@
 """Shared pieces of the GPU parity tests: run the library on a workload, run the oracle on
 the same seeded inputs, compare with the stated tolerances.
 
-Tolerances (spec contract):
+Tolerances (the acceptance contract of this library):
   * packed indices and QJL sign bits bit-exact, except coordinates whose rotated value
     lies within 1e-6 of a codebook boundary, and sign bits whose projection (S r)_i lies
     within 1e-6 * sum_j |S_ij r_j| of zero (both counted and reported);
