@@ -32,6 +32,7 @@
 // sign-space sums sum_t p_t ||r_v||_t (2 sigma_t - 1) through a second mma per step, and the
 // merge adds sqrt(pi/2)/m S^T of them).
 // Everything else uses decode.cu.
+#include <climits>
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -83,6 +84,7 @@ struct SmemFast {
   float wm[kConsumerWarps][kMaxRows], wl[kConsumerWarps][kMaxRows], wf[kConsumerWarps][kMaxRows];
   float wx[kConsumerWarps][kMaxRows];  // dithered values: sum_t p_t ||v_t|| xi_t of each warp and row
   float xsig[4][QM];  // values with QJL, at the merge: each row's sign-space sum / l
+  int cu;  // units per split
   int last;
 };
 
@@ -290,13 +292,9 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
   const bool bad_len = len < 0 || len > a.cache.max_pages * PT;
   if (bad_len && tid == 0 && split == 0) report(a.status, TQ_ERR_BOUNDS);
   const int n_eff = bad_len ? 0 : len;
-  // the sequence in half-page units, dealt to the splits in contiguous runs
+  // the sequence in half-page units, dealt to the splits in contiguous runs of sm.cu units
+  // (formed below, before the first barrier)
   const int units_all = (n_eff + kUnit - 1) / kUnit;
-  const int cu = (units_all + a.n_splits - 1) / a.n_splits;
-  const int u_begin = min(units_all, split * cu);
-  const int u_end = min(units_all, (split + 1) * cu);
-  const int nunits = u_end - u_begin;
-  const int t_end = min(n_eff, u_end * kUnit);
 
   constexpr int kKChunks = (KP == K2Q) ? 3 : 4;  // K2Q: 2 code chunks + the KS chunk
   constexpr int kVChunks = (VP == V3) ? 3 : 2;
@@ -314,7 +312,47 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     mbar_init(&sm.never, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (warp == 0) {
+    // Units per split.  Sequences of one length: the longest's units over the n_splits splits
+    // (every sequence takes all of them).  Sequences of different lengths: no longer than the
+    // batch's mean share of one wave of target_ctas thread blocks, so that the longest
+    // sequence is cut into more splits and the shorter ones into fewer (each stream of u
+    // units takes ceil(u / cu) of the n_splits), instead of every sequence taking n_splits
+    // splits and the longest ones' setting the pace.
+    const int cap = a.cache.max_pages * PT;
+    int maxu = 0, minu = INT_MAX;
+    long long total = 0;
+    for (int bb = lane; bb < a.cache.batch; bb += 32) {
+      const int l = a.seq_lens[bb];
+      const int u = (l < 0 || l > cap) ? 0 : (l + kUnit - 1) / kUnit;
+      maxu = max(maxu, u);
+      minu = min(minu, u);
+      total += u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      maxu = max(maxu, __shfl_xor_sync(FULL, maxu, o));
+      minu = min(minu, __shfl_xor_sync(FULL, minu, o));
+      total += __shfl_xor_sync(FULL, total, o);
+    }
+    int c = (maxu + a.n_splits - 1) / a.n_splits;
+    const long long streams = (long long)a.cache.batch * a.cache.kv_heads * nchunk;
+    if (minu != maxu && a.target_ctas > streams) {
+      const long long work = total * a.cache.kv_heads * nchunk;
+      c = max(c, (int)((work + (a.target_ctas - streams) - 1) / (a.target_ctas - streams)));
+    }
+    if (lane == 0) sm.cu = max(1, c);
+  }
   __syncthreads();
+  const int cu = sm.cu;
+  // this stream's splits (at most n_splits: cu is at least the longest's share); thread
+  // blocks past them have nothing to do (uniform per block)
+  const int n_split_b = max(1, (units_all + cu - 1) / cu);
+  if (split >= n_split_b) return;
+  const int u_begin = min(units_all, split * cu);
+  const int u_end = min(units_all, (split + 1) * cu);
+  const int nunits = u_end - u_begin;
+  const int t_end = min(n_eff, u_end * kUnit);
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
@@ -1086,11 +1124,12 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
                  : "=r"(done)
                  : "l"(&a.counter[((size_t)b * a.cache.kv_heads + gh) * nchunk + chunk])
                  : "memory");
-    sm.last = done == (unsigned int)a.n_splits - 1;
+    sm.last = done == (unsigned int)n_split_b - 1;
   }
   __syncthreads();
   if (!sm.last) return;
-  const int ns = a.n_splits;
+  const int ns = n_split_b;      // the partials to merge
+  const size_t nst = a.n_splits;  // their row stride in the workspace
   // every split's accumulators of every row in one round trip when they fit: a bulk copy per
   // row (the rows' partials are contiguous), landing while the maxima are formed from the
   // (m, l) pairs; otherwise register batches from L2
@@ -1103,19 +1142,19 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
     asm volatile("fence.proxy.async.global;" ::: "memory");
     mbar_expect_tx(&sm.mbar, (uint32_t)(R * ns * D * sizeof(float)));
     for (int rr = 0; rr < R; ++rr)
-      bulk_g2s(&sm.merge[rr * kCap * D], a.part_acc + (row0 + rr) * ns * D, (uint32_t)(ns * D * sizeof(float)),
+      bulk_g2s(&sm.merge[rr * kCap * D], a.part_acc + (row0 + rr) * nst * D, (uint32_t)(ns * D * sizeof(float)),
                &sm.mbar);
   }
   // warp w merges rows w, w + 5, ...; lane c4 owns coordinates 4 c4 .. 4 c4 + 3
   for (int r = warp; r < R; r += kThreads / 32) {
     const int c4 = lane;
     const size_t rowq = row0 + r;
-    const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * ns * 2);
+    const float2* ml2 = reinterpret_cast<const float2*>(a.part_ml + rowq * nst * 2);
     float* rs = &sm.merge[r * kCap * D];  // row r's region (its partials when in_smem)
     float M = -CUDART_INF_F, l = 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 osg = make_float4(0.f, 0.f, 0.f, 0.f);  // values with QJL: the sign-space sums
-    const float4* ps4 = reinterpret_cast<const float4*>(a.part_sig + (VQ ? rowq * ns * QM : 0)) + c4;
+    const float4* ps4 = reinterpret_cast<const float4*>(a.part_sig + (VQ ? rowq * nst * QM : 0)) + c4;
     if (in_smem) {
       for (int sp = c4; sp < ns; sp += 32) M = fmaxf(M, ml2[sp].x);
 #pragma unroll
@@ -1148,7 +1187,7 @@ __global__ void __launch_bounds__(kThreads, 2) fast_split_kernel(DecodeArgs a) {
       // many splits: the partials in register batches of kMB, the first batch before the
       // maximum is formed (about ns / kMB round trips to L2)
       constexpr int kMB = 20;
-      const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * ns * D) + c4;
+      const float4* pa4 = reinterpret_cast<const float4*>(a.part_acc + rowq * nst * D) + c4;
       for (int s0 = 0; s0 < ns; s0 += kMB) {
         float4 v[kMB];
         float2 m2[kMB];

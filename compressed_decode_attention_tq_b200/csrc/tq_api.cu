@@ -253,6 +253,18 @@ static int debug_wait_ns() {
   return (int)(us * 1000);
 }
 
+// SMs of the current device (looked up once per device)
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
 static tq_status decode_common(const tq_config* cfg, const tq_params* params, const tq_cache* cache,
                                int32_t layer, const void* q, int32_t q_dtype, int32_t q_heads,
                                int32_t seq_q, const int32_t* seq_lens, int32_t n_splits, void* workspace,
@@ -304,6 +316,7 @@ static tq_status decode_common(const tq_config* cfg, const tq_params* params, co
   a.counter = reinterpret_cast<unsigned int*>(ws + w.counter);
   a.ready = reinterpret_cast<unsigned int*>(ws + w.ready);
   a.fast_query = 0;
+  a.target_ctas = 2 * sm_count();
   a.out = nullptr;
   a.scores = nullptr;
   a.max_len = 0;

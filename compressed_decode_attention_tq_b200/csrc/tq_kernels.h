@@ -61,6 +61,9 @@ struct DecodeArgs {
   // fast split kernel waits this many nanoseconds on a barrier nothing arrives on and
   // reports TQ_ERR_TIMEOUT; the results are computed as usual)
   int debug_wait_ns;
+  // the tensor-core split kernel's wave: thread blocks resident at once (two per SM); a batch
+  // of different lengths sizes its splits from it
+  int target_ctas;
   // 1: the prologue forms the query terms in kQueryParts parts per row for the tensor-core split
   // kernel (fp32 S q, ready word per part); 0: one block per row for the general kernels
   int fast_query;

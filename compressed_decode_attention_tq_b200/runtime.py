@@ -26,9 +26,13 @@ def splits_for(batch: int, kv_heads: int, sms: int, rows: int = 1, max_len: Opti
     """Split count that fills a GPU of `sms` SMs once: the tensor-core decode kernel keeps two
     CTAs per SM, one CTA per (split, kv head, sequence, run of query rows); a KV head's
     rows = G * seq_q query rows are taken four at a time, or eight when there are more than
-    four.  With max_len, no more splits than 128-token units of the longest sequence."""
+    four.  A batch of several sequences gets twice that: when their lengths differ the kernel
+    cuts the longest into more splits and the shorter ones into fewer (at most this count).
+    With max_len, no more splits than 128-token units of the longest sequence."""
     runs = -(-max(1, rows) // (8 if rows > 4 else 4))
     n = (2 * sms) // max(1, batch * kv_heads * runs)
+    if batch > 1:
+        n *= 2
     if max_len is not None:
         n = min(n, -(-max(1, max_len) // 128))
     return max(1, min(1024, n))

@@ -310,7 +310,7 @@ def test_default_split_count():
     assert splits_for(1, 8, 148) == 37                    # 4 query rows per KV head: one run
     assert splits_for(1, 8, 148, rows=4) == 37
     assert splits_for(1, 8, 148, rows=32) == 9            # 32 rows: four runs of eight
-    assert splits_for(16, 2, 148, rows=8) == 9            # eight rows: one run
+    assert splits_for(16, 2, 148, rows=8) == 18           # eight rows: one run; twice the share for a batch
     assert splits_for(1, 1, 148, max_len=4096) == 32      # no more splits than 128-token units
     assert splits_for(64, 64, 148) == 1
     assert splits_for(1, 1, 100000) == 1024
