@@ -293,8 +293,10 @@ TQ_API size_t tq_decode_workspace_bytes(const tq_config* cfg, int32_t batch, int
  *   out     = R^T sum_t softmax(score)_t ||v||_t c_v[idx_v,t]
  *             [+ with value_qjl: sqrt(pi/2)/m S^T sum_t softmax(score)_t ||r_v||_t (2 sigma_v,t - 1)]
  * over t < seq_lens[b] (no causal mask between the seq_q rows; an empty sequence
- * gives 0).  The sequence is cut into n_splits contiguous ranges processed in
- * parallel and merged by their log-sum-exp.
+ * gives 0).  The sequence is cut into at most n_splits contiguous ranges processed in
+ * parallel and merged by their log-sum-exp: n_splits when every sequence of the batch
+ * has the same length; when the lengths differ, the tensor-core kernel sizes the ranges
+ * from the batch's total work, so that shorter sequences take fewer of them.
  *   q          device [batch][q_heads][seq_q][d], element type q_dtype
  *   q_heads    multiple of kv_heads; q_heads/kv_heads * seq_q <= 32
  *   n_splits   1..1024
