@@ -422,12 +422,6 @@ __device__ __forceinline__ void query_row(const DecodeArgs& a, int row) {
   }
 }
 
-// The query terms for the tensor-core split kernel, kQueryParts thread blocks of 128 threads
-// per query row.  Part c forms outputs 32 c .. 32 c + 31 of S q in fp32 (the split kernel
-// takes them to fixed point), 8 per warp; part 0 also R q and its int8 copy with the scale,
-// and zeroes the merge counter of a run that starts at this row.  Each part announces its
-// terms through its own ready word.  Few registers: a block waiting for its predecessor stays
-// resident beside two split-kernel blocks of the previous call.
 // Before launch_dependents: this part's terms of an earlier call are no longer announced.
 __device__ __forceinline__ void unpublish_part(const DecodeArgs& a, int blk) {
   if (threadIdx.x == 0) {
@@ -528,6 +522,12 @@ __device__ __forceinline__ void query_part(const DecodeArgs& a, int blk) {
   if (threadIdx.x == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(rw), "r"(1u) : "memory");
 }
 
+// The query terms for the tensor-core split kernel, kQueryParts thread blocks of 128 threads
+// per query row.  Part c forms outputs 32 c .. 32 c + 31 of S q in fp32 (the split kernel
+// takes them to fixed point), 8 per warp; part 0 also R q and its int8 copy with the scale,
+// and zeroes the merge counter of a run that starts at this row.  Each part announces its
+// terms through its own ready word.  Few registers: a block waiting for its predecessor stays
+// resident beside two split-kernel blocks of the previous call.
 __global__ void __launch_bounds__(128) query_kernel(DecodeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   unpublish_part(a, blockIdx.x);
